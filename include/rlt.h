@@ -1,0 +1,267 @@
+/*
+ * rlt.h -- C ABI of librlt.so, the B200 (sm_100a) implementation of the
+ * Recurrent Looped Transformer (RLT) hot path: the batched recurrent decoder
+ * state transition, the token-parallel causal encoder and the encoder KV
+ * memory that feeds it.
+ *
+ * Definitions follow "Recurrent Looped Transformer" (Y. Zhang, technical
+ * report, Sept. 2026) and its project page:
+ *   §2.1      sequence, state H_t = (s_t, C^D_t), window W includes the current
+ *             token, at most W-1 retained positions per layer
+ *   §2.2      eq. 2.1 causal encoder, eq. 2.2 memory groups (G = 1 or L_D)
+ *   §2.3      eqs. 2.3-2.7 H_0 = (s_*, empty), Merge, D_phi, readout
+ *   §2.4      eq. 2.8 encoder step form, prefix-restricted memory
+ *   §2.5      eqs. 2.9-2.11 gated merge, eqs. 2.12-2.16 decoder block
+ *   §2.6      tied configuration
+ *   §5.3      behaviour log-probabilities under the actual sampler
+ *   App. A    execution schedules (A.1 prefill, A.2 generation, A.4 replay)
+ * Readings where the pages leave a step open: FFN = SwiGLU; rotate-half RoPE
+ * (base rope_base) at position p = t-1 on every query and key; one pre-norm
+ * RMSNorm per sublayer; multi-head attention scaled by 1/sqrt(d/n_heads); no
+ * final encoder norm; BOS id bos_id.
+ *
+ * Conventions for every entry point
+ *  - Every function returns an int32 status: RLT_OK (0) or a negative code.
+ *    Nothing throws across the ABI.  rlt_last_error() returns the text of the
+ *    calling thread's last error.
+ *  - Arguments and capacities are validated synchronously before any work is
+ *    enqueued; a rejected call leaves model and state unchanged.
+ *  - "_dev" pointers are device pointers owned by the caller, ordered on the
+ *    CUDA stream passed as `stream` (a cudaStream_t; NULL = legacy default
+ *    stream).  Host pointers are read/written synchronously.
+ *  - The library owns all model and state device memory.  Kernel errors are
+ *    asynchronous: they surface as RLT_E_CUDA on a later call.
+ *  - A state remembers the model version it was built under.  Loading weights
+ *    bumps the version; using an older state then fails with RLT_E_STALE
+ *    (report §5.4 and App. C: caches built under other weights are invalid).
+ *  - All sequences of one state advance in lock step (report §4.1 batching of
+ *    ready transitions): they share positions n_enc and n_dec.
+ */
+#ifndef RLT_H_
+#define RLT_H_
+
+#include <stddef.h>
+#include <stdint.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+#define RLT_OK 0
+#define RLT_E_INVAL (-1)       /* bad argument or unsupported shape */
+#define RLT_E_CAPACITY (-2)    /* position would pass max_len, or batch > capacity */
+#define RLT_E_OOM (-3)         /* device allocation failed */
+#define RLT_E_CUDA (-4)        /* a CUDA call or kernel failed */
+#define RLT_E_STALE (-5)       /* state built under older weights */
+#define RLT_E_STATE (-6)       /* call not valid in the state's current phase */
+
+#define RLT_MERGE_PAPER 0      /* eqs. 2.9-2.11: u = e + alpha g*(W_s r), g = sig(W_g[e;r]+b_g), r = RMSNorm_s(s) */
+#define RLT_MERGE_CONVEX 1     /* u = g*e + (1-g)*s, g = sig(W_g[e;s]) */
+
+#define RLT_DTYPE_F32 0        /* fp32 weights, caches and arithmetic */
+#define RLT_DTYPE_BF16 1       /* bf16 weights/caches/GEMM inputs, fp32 accumulation and residual stream */
+
+typedef struct rlt_config {
+  int32_t d_model;     /* residual width d */
+  int32_t n_heads;     /* heads; head size d/n_heads must be even */
+  int32_t n_layers;    /* L_E = L_D = L */
+  int32_t window;      /* SWA window W >= 1, includes the current token */
+  int32_t groups;      /* memory groups G: 1 (shared) or n_layers (per layer) */
+  int32_t ffn;         /* SwiGLU hidden width F */
+  int32_t vocab;       /* V */
+  int32_t tied;        /* 1: decoder SWA/FFN reuse encoder layer weights (§2.6); 0: untied */
+  int32_t merge_kind;  /* RLT_MERGE_* */
+  int32_t dtype;       /* RLT_DTYPE_* */
+  float alpha;         /* feedback scale of eq. 2.11 */
+  float rms_eps;       /* epsilon inside every RMSNorm */
+  float rope_base;     /* rotary base */
+  float init_std;      /* std of random initialisation */
+  int32_t bos_id;      /* token id of BOS */
+} rlt_config;
+
+typedef struct rlt_model rlt_model;
+typedef struct rlt_state rlt_state;
+
+/* Behaviour sampler (report §5.3): the top_k largest raw logits, ordered by
+ * (value desc, id asc), tempered by 1/temperature and renormalised; the
+ * uniform is (Philox4x32-10(counter = (t, b, 0, 0), key = seed).x0 >> 8) *
+ * 2^-24 where t is the position of the state s_t that predicts the token and
+ * b the sequence's batch index.  1 <= top_k <= 256, temperature > 0. */
+typedef struct rlt_sampling {
+  float temperature;
+  int32_t top_k;
+  uint64_t seed;
+} rlt_sampling;
+
+/* Outputs of one readout.  Every pointer is a caller-owned device array or
+ * NULL (not wanted). */
+typedef struct rlt_readout_out {
+  float* logp;          /* [B] log p(next[b] | x_1..t), needs next_dev */
+  int32_t* sampled;     /* [B] sampled x_{t+1}, needs a sampler */
+  float* logp_sampled;  /* [B] raw log p of the sampled token */
+  float* logmu;         /* [B] behaviour log-prob of the sampled token (tempered, truncated) */
+  float* logits;        /* [B, V] raw logits */
+} rlt_readout_out;
+
+/* State inspection (test hooks, report §6 snapshot contents). */
+typedef struct rlt_state_info {
+  int32_t batch, max_len;
+  int32_t n_enc;        /* tokens encoded: e_1..e_n_enc and M_<=n_enc exist */
+  int32_t n_dec;        /* decoder transitions applied: the state is H_n_dec */
+  int32_t ring_valid;   /* retained SWA entries per layer: min(n_dec, W-1) */
+  int32_t ring_head;    /* slot the next transition writes: n_dec mod (W-1), 0 if W = 1 */
+  int32_t has_encoder_cache;
+  uint64_t model_version;
+} rlt_state_info;
+
+#define RLT_STATE_ENCODER_CACHE 1   /* keep C^E (needed for incremental encoding, eq. 2.8) */
+
+/* what for rlt_state_read: */
+#define RLT_READ_S 0        /* [B][d] fp32 recurrent output s_t */
+#define RLT_READ_E 1        /* [B][max_len][d] fp32 encoder outputs */
+#define RLT_READ_RING_K 2   /* layer `index`: [B][H][W-1][hd] keys (model dtype), slot of position j = (j-1) mod (W-1) */
+#define RLT_READ_RING_V 3   /* layer `index`: values, same layout */
+#define RLT_READ_MEM_K 4    /* group `index`: [B][H][max_len][hd] memory keys (rotated) */
+#define RLT_READ_MEM_V 5    /* group `index`: memory values */
+#define RLT_READ_ENC_K 6    /* layer `index`: [B][H][max_len][hd] encoder cache keys (needs the encoder cache) */
+#define RLT_READ_ENC_V 7
+
+/* ---------------------------------------------------------------- model */
+
+/* Allocates a model on the current device and fills every weight from the
+ * counter-based generator: element i of the tensor with stream id s is
+ * init_std * (sum of the twelve 32-bit words of Philox4x32-10 with counters
+ * (i_lo, i_hi, s, j), j = 0..2, key = seed, times 2^-32, minus 6), rounded to
+ * fp32 and then (bf16 models) to bf16 by round-to-nearest-even.  Gains are 1
+ * and b_gate is 0.  Tensor names, shapes and stream ids: see rlt_tensor_info.
+ * Errors: RLT_E_INVAL (config), RLT_E_OOM, RLT_E_CUDA. */
+int32_t rlt_init_weights(const rlt_config* cfg, uint64_t seed, rlt_model** out);
+
+/* Copies a whole tensor from host memory in the model's storage format (fp32,
+ * or bf16 bit patterns) and bumps the model version.  bytes must equal
+ * rows*cols*element size.  Errors: RLT_E_INVAL (unknown name, size). */
+int32_t rlt_load_weights(rlt_model* m, const char* name, const void* host, size_t bytes);
+
+/* Copies a whole tensor to host memory (storage format). */
+int32_t rlt_get_weights(const rlt_model* m, const char* name, void* host, size_t bytes);
+
+/* Shape and generator stream id of a tensor: names are emb [V,d], s_star [d],
+ * g_mem [d], g_merge [d], w_gate [d,2d], b_gate [d], w_state [d,d], g_out [d],
+ * w_out [V,d], wk_mem.g / wv_mem.g [d,d], and per layer l: wq.l wk.l wv.l
+ * wo.l [d,d], w1.l w3.l [F,d], w2.l [d,F], g_ea.l g_ef.l g_dsa.l g_dmem.l
+ * g_dffn.l [d], wq_mem.l wo_mem.l [d,d], and when untied dwq.l dwk.l dwv.l
+ * dwo.l dw1.l dw2.l dw3.l.  Stream ids: emb 0, s_star 1, g_mem 2, g_merge 3,
+ * w_gate 4, b_gate 5, w_state 6, g_out 7, w_out 8, wk_mem.g 16+2g,
+ * wv_mem.g 17+2g, layer slot k of layer l 1024+32l+k in the order listed. */
+int32_t rlt_tensor_info(const rlt_model* m, const char* name, int64_t* rows, int64_t* cols, int32_t* stream_id);
+
+int32_t rlt_model_free(rlt_model* m);
+
+/* ---------------------------------------------------------------- state */
+
+/* Creates the state of `batch` independent sequences of up to max_len tokens,
+ * at H_0 = (s_*, empty) with empty encoder caches (eq. 2.3).  Device memory:
+ * encoder outputs [B][max_len][d] fp32, memory 2*G*B*max_len*d elements, SWA
+ * ring 2*L*B*(W-1)*d elements, plus (flag RLT_STATE_ENCODER_CACHE) the encoder
+ * cache 2*L*B*max_len*d elements, plus step workspace.
+ * Errors: RLT_E_INVAL, RLT_E_OOM. */
+int32_t rlt_state_create(rlt_model* m, int32_t batch, int32_t max_len, int32_t flags, rlt_state** out);
+int32_t rlt_state_free(rlt_state* s);
+
+/* Returns the state to H_0 with empty caches (positions 0) under the model's
+ * current weights. */
+int32_t rlt_state_reset(rlt_state* s, void* stream);
+
+int32_t rlt_state_info_get(const rlt_state* s, rlt_state_info* out);
+
+/* Copies one state component to host memory (synchronous); layouts above. */
+int32_t rlt_state_read(const rlt_state* s, int32_t what, int32_t index, void* host, size_t bytes);
+
+/* ---------------------------------------------------------------- schedules */
+
+/* Token-parallel causal encoder (eq. 2.1) and memory projection (eq. 2.2) for
+ * T tokens per sequence, tok_dev [B][T] int32 (row-major), placed at positions
+ * n_enc+1..n_enc+T.  Only an empty encoder (n_enc == 0) is supported by this
+ * schedule; later tokens are encoded by rlt_decoder_step.  Does not advance
+ * the decoder.  Errors: RLT_E_CAPACITY (n_enc+T > max_len), RLT_E_STATE
+ * (n_enc != 0), RLT_E_STALE, RLT_E_INVAL. */
+int32_t rlt_encode_prefix(rlt_model* m, rlt_state* s, const int32_t* tok_dev, int32_t T, void* stream);
+
+/* Readout of the current s_t (eq. 2.6): log p of next_dev [B] (may be NULL),
+ * and/or a sample from the behaviour sampler (samp may be NULL).  Requires
+ * n_dec >= 1. */
+int32_t rlt_readout(rlt_model* m, rlt_state* s, const int32_t* next_dev, const rlt_sampling* samp,
+                    const rlt_readout_out* out, void* stream);
+
+/* Consumes x_t for every sequence, t = n_dec+1 (App. A.2): if x_t is not yet
+ * encoded (n_enc < t), runs the encoder step (eq. 2.8, needs the encoder
+ * cache) and the memory append; then the merge and the L_D decoder blocks
+ * (eqs. 2.4, 2.5, 2.12-2.16) with one SWA insert per layer; then the readout
+ * as rlt_readout does (skipped when next_dev, samp and out are all NULL).
+ * tok_dev [B] int32 is read only when the token is encoded here.
+ * Errors: RLT_E_CAPACITY (t > max_len), RLT_E_STATE (no encoder cache and x_t
+ * not encoded), RLT_E_STALE, RLT_E_INVAL. */
+int32_t rlt_decoder_step(rlt_model* m, rlt_state* s, const int32_t* tok_dev, const int32_t* next_dev,
+                         const rlt_sampling* samp, const rlt_readout_out* out, void* stream);
+
+/* Prompt prefill (App. A.1): rlt_encode_prefix over tok_dev [B][T], then T
+ * decoder transitions.  If logp_dev != NULL it receives [B][T-1] teacher
+ * log-probs log p(x_{t+1} | x_1..t), t = 1..T-1.  The state ends at H_T; call
+ * rlt_readout to sample the first response token. */
+int32_t rlt_prefill(rlt_model* m, rlt_state* s, const int32_t* tok_dev, int32_t T, float* logp_dev, void* stream);
+
+/* Current-policy replay (App. A.4): from a fresh H_0 under the current
+ * weights, encode tok_dev [B][S] token-parallel, run the S-1 transitions and
+ * write logp_dev [B][S-1] = log p(x_{t+1} | x_1..t).  Uses a state the model
+ * keeps for replay (allocated on first use or growth).  S >= 2. */
+int32_t rlt_replay_logprobs(rlt_model* m, const int32_t* tok_dev, int32_t B, int32_t S, float* logp_dev,
+                            void* stream);
+
+/* ---------------------------------------------------------------- ops */
+
+/* Kernel-level check of the step's contraction: y_dev [N][M] fp32 =
+ * x_dev [N][K] . w_dev [M][K]^T, both operands row-major in `dtype`
+ * (RLT_DTYPE_BF16: bf16, RLT_DTYPE_F32: fp32).  use_tensor_cores = 1 runs the
+ * tcgen05 kernel (bf16 only; M % 128 == 0, K % 64 == 0), 0 the CUDA-core
+ * kernel.  Split-K workspace is allocated and freed inside the call.
+ * Errors: RLT_E_INVAL (shape/dtype), RLT_E_OOM, RLT_E_CUDA. */
+int32_t rlt_op_linear(const void* w_dev, const void* x_dev, float* y_dev, int32_t M, int32_t N, int32_t K,
+                      int32_t dtype, int32_t use_tensor_cores, void* stream);
+
+/* Behaviour sampler (see rlt_sampling) on caller-given logits_dev [B][V]
+ * fp32, as position t: writes token_dev [B] int32, logp_dev [B] (raw
+ * log-softmax of the token, may be NULL) and logmu_dev [B] (tempered and
+ * truncated log-prob, may be NULL).  Errors: RLT_E_INVAL. */
+int32_t rlt_op_sample(const float* logits_dev, int32_t B, int32_t V, const rlt_sampling* samp, uint32_t t,
+                      int32_t* token_dev, float* logp_dev, float* logmu_dev, void* stream);
+
+/* ---------------------------------------------------------------- misc */
+
+/* Copies the calling thread's last error text (NUL-terminated, truncated to
+ * n) and returns its status code. */
+int32_t rlt_last_error(char* buf, size_t n);
+
+/* Checks the device-side error word that bounded waits inside the kernels
+ * set when a wait runs out (never expected); returns RLT_E_CUDA and clears it
+ * if set.  Synchronises the device. */
+int32_t rlt_check_device(void);
+
+/* Kernel timing hook for measurement: when enabled, the library records CUDA
+ * events on the launching stream around every launch of the decode-attention
+ * kernels.  Enabling (or disabling) clears the record.  rlt_profile_read
+ * synchronises the device and, for kind 0 (prefix attention: cross-attention
+ * to the memory and the encoder step) or kind 1 (SWA attention), returns the
+ * summed event intervals in milliseconds, the launch count and the
+ * algorithmic KV bytes those launches read and wrote (keys and values of
+ * every attended position, plus the SWA insert). */
+int32_t rlt_profile_enable(rlt_model* m, int32_t on);
+
+/* Number of kernel launches the library has issued since it was loaded
+ * (host-side counter, all devices and threads). */
+int32_t rlt_kernel_launches(int64_t* count);
+int32_t rlt_profile_read(rlt_model* m, int32_t kind, double* ms, int64_t* launches, double* bytes);
+
+#ifdef __cplusplus
+}
+#endif
+#endif /* RLT_H_ */

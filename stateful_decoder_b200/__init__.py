@@ -1,0 +1,324 @@
+"""Python binding of librlt.so, the sm_100a implementation of the Recurrent
+Looped Transformer hot path (C ABI in include/rlt.h).
+
+Argument marshalling only: every step of the computation runs in the CUDA
+kernels of the library.  Device arrays are torch CUDA tensors (their
+``data_ptr()`` is handed to the library); host arrays are numpy arrays.  The
+library must have been built (``stateful_decoder_b200.build.build()``); if it
+is missing this module raises at import -- there is no fallback.
+"""
+from __future__ import annotations
+
+import ctypes
+import os
+
+import numpy as np
+
+_HERE = os.path.dirname(os.path.abspath(__file__))
+LIB_PATH = os.path.join(_HERE, "librlt.so")
+
+if not os.path.exists(LIB_PATH):
+    raise ImportError(f"{LIB_PATH} is missing: build it with `python -m stateful_decoder_b200.build`")
+
+_lib = ctypes.CDLL(LIB_PATH)
+
+RLT_OK = 0
+RLT_E_INVAL = -1
+RLT_E_CAPACITY = -2
+RLT_E_OOM = -3
+RLT_E_CUDA = -4
+RLT_E_STALE = -5
+RLT_E_STATE = -6
+
+MERGE_PAPER = 0
+MERGE_CONVEX = 1
+DTYPE_F32 = 0
+DTYPE_BF16 = 1
+STATE_ENCODER_CACHE = 1
+
+READ_S, READ_E, READ_RING_K, READ_RING_V, READ_MEM_K, READ_MEM_V, READ_ENC_K, READ_ENC_V = range(8)
+
+EXPORTED = (
+    "rlt_init_weights", "rlt_load_weights", "rlt_get_weights", "rlt_tensor_info", "rlt_model_free",
+    "rlt_state_create", "rlt_state_free", "rlt_state_reset", "rlt_state_info_get", "rlt_state_read",
+    "rlt_encode_prefix", "rlt_readout", "rlt_decoder_step", "rlt_prefill", "rlt_replay_logprobs",
+    "rlt_last_error", "rlt_check_device", "rlt_profile_enable", "rlt_profile_read", "rlt_op_linear",
+    "rlt_op_sample", "rlt_kernel_launches",
+)
+
+
+class RltError(RuntimeError):
+    def __init__(self, code: int, msg: str):
+        super().__init__(f"rlt error {code}: {msg}")
+        self.code = code
+
+
+class Config(ctypes.Structure):
+    _fields_ = [
+        ("d_model", ctypes.c_int32), ("n_heads", ctypes.c_int32), ("n_layers", ctypes.c_int32),
+        ("window", ctypes.c_int32), ("groups", ctypes.c_int32), ("ffn", ctypes.c_int32), ("vocab", ctypes.c_int32),
+        ("tied", ctypes.c_int32), ("merge_kind", ctypes.c_int32), ("dtype", ctypes.c_int32),
+        ("alpha", ctypes.c_float), ("rms_eps", ctypes.c_float), ("rope_base", ctypes.c_float),
+        ("init_std", ctypes.c_float), ("bos_id", ctypes.c_int32),
+    ]
+
+
+class Sampling(ctypes.Structure):
+    _fields_ = [("temperature", ctypes.c_float), ("top_k", ctypes.c_int32), ("seed", ctypes.c_uint64)]
+
+
+class ReadoutOut(ctypes.Structure):
+    _fields_ = [("logp", ctypes.c_void_p), ("sampled", ctypes.c_void_p), ("logp_sampled", ctypes.c_void_p),
+                ("logmu", ctypes.c_void_p), ("logits", ctypes.c_void_p)]
+
+
+class StateInfo(ctypes.Structure):
+    _fields_ = [("batch", ctypes.c_int32), ("max_len", ctypes.c_int32), ("n_enc", ctypes.c_int32),
+                ("n_dec", ctypes.c_int32), ("ring_valid", ctypes.c_int32), ("ring_head", ctypes.c_int32),
+                ("has_encoder_cache", ctypes.c_int32), ("model_version", ctypes.c_uint64)]
+
+
+_vp = ctypes.c_void_p
+_i32 = ctypes.c_int32
+_sig = {
+    "rlt_init_weights": [ctypes.POINTER(Config), ctypes.c_uint64, ctypes.POINTER(_vp)],
+    "rlt_load_weights": [_vp, ctypes.c_char_p, _vp, ctypes.c_size_t],
+    "rlt_get_weights": [_vp, ctypes.c_char_p, _vp, ctypes.c_size_t],
+    "rlt_tensor_info": [_vp, ctypes.c_char_p, ctypes.POINTER(ctypes.c_int64), ctypes.POINTER(ctypes.c_int64),
+                        ctypes.POINTER(_i32)],
+    "rlt_model_free": [_vp],
+    "rlt_state_create": [_vp, _i32, _i32, _i32, ctypes.POINTER(_vp)],
+    "rlt_state_free": [_vp],
+    "rlt_state_reset": [_vp, _vp],
+    "rlt_state_info_get": [_vp, ctypes.POINTER(StateInfo)],
+    "rlt_state_read": [_vp, _i32, _i32, _vp, ctypes.c_size_t],
+    "rlt_encode_prefix": [_vp, _vp, _vp, _i32, _vp],
+    "rlt_readout": [_vp, _vp, _vp, ctypes.POINTER(Sampling), ctypes.POINTER(ReadoutOut), _vp],
+    "rlt_decoder_step": [_vp, _vp, _vp, _vp, ctypes.POINTER(Sampling), ctypes.POINTER(ReadoutOut), _vp],
+    "rlt_prefill": [_vp, _vp, _vp, _i32, _vp, _vp],
+    "rlt_replay_logprobs": [_vp, _vp, _i32, _i32, _vp, _vp],
+    "rlt_op_linear": [_vp, _vp, _vp, _i32, _i32, _i32, _i32, _i32, _vp],
+    "rlt_op_sample": [_vp, _i32, _i32, ctypes.POINTER(Sampling), ctypes.c_uint32, _vp, _vp, _vp, _vp],
+    "rlt_last_error": [ctypes.c_char_p, ctypes.c_size_t],
+    "rlt_check_device": [],
+    "rlt_kernel_launches": [ctypes.POINTER(ctypes.c_int64)],
+    "rlt_profile_enable": [_vp, _i32],
+    "rlt_profile_read": [_vp, _i32, ctypes.POINTER(ctypes.c_double), ctypes.POINTER(ctypes.c_int64),
+                         ctypes.POINTER(ctypes.c_double)],
+}
+for _name, _args in _sig.items():
+    _f = getattr(_lib, _name)
+    _f.argtypes = _args
+    _f.restype = ctypes.c_int32
+
+
+def rlt_last_error() -> tuple[int, str]:
+    buf = ctypes.create_string_buffer(1024)
+    code = _lib.rlt_last_error(buf, 1024)
+    return code, buf.value.decode(errors="replace")
+
+
+def _check(code: int) -> None:
+    if code != RLT_OK:
+        _, msg = rlt_last_error()
+        raise RltError(code, msg)
+
+
+def _stream(stream):
+    if stream is None:
+        import torch
+        return ctypes.c_void_p(torch.cuda.current_stream().cuda_stream)
+    if isinstance(stream, int):
+        return ctypes.c_void_p(stream)
+    return ctypes.c_void_p(stream.cuda_stream)
+
+
+def _dev(t, dtype_name: str | None = None):
+    """Device pointer of a contiguous CUDA tensor (or None)."""
+    if t is None:
+        return None
+    if not t.is_cuda or not t.is_contiguous():
+        raise ValueError("expected a contiguous CUDA tensor")
+    if dtype_name is not None and str(t.dtype) != dtype_name:
+        raise ValueError(f"expected {dtype_name}, got {t.dtype}")
+    return ctypes.c_void_p(t.data_ptr())
+
+
+def make_config(**kw) -> Config:
+    return Config(d_model=kw["d"], n_heads=kw["n_heads"], n_layers=kw["n_layers"], window=kw["window"],
+                  groups=kw["groups"], ffn=kw["ffn"], vocab=kw["vocab"], tied=kw.get("tied", 1),
+                  merge_kind=kw.get("merge_kind", 0), dtype=kw["dtype"], alpha=kw.get("alpha", 1.0),
+                  rms_eps=kw.get("rms_eps", 1e-6), rope_base=kw.get("rope_base", 10000.0),
+                  init_std=kw.get("init_std", 0.02), bos_id=kw.get("bos_id", 0))
+
+
+class Model:
+    """Owner of an ``rlt_model*``."""
+
+    def __init__(self, handle: ctypes.c_void_p, cfg: dict):
+        self.h = handle
+        self.cfg = dict(cfg)
+
+    def __del__(self):
+        self.free()
+
+    def free(self):
+        if getattr(self, "h", None):
+            _lib.rlt_model_free(self.h)
+            self.h = None
+
+    @property
+    def storage_dtype(self):
+        return np.float32 if self.cfg["dtype"] == DTYPE_F32 else np.uint16
+
+    def tensor_info(self, name: str):
+        r, c, s = ctypes.c_int64(), ctypes.c_int64(), ctypes.c_int32()
+        _check(_lib.rlt_tensor_info(self.h, name.encode(), ctypes.byref(r), ctypes.byref(c), ctypes.byref(s)))
+        return r.value, c.value, s.value
+
+    def load_weights(self, name: str, raw: np.ndarray) -> None:
+        raw = np.ascontiguousarray(raw, dtype=self.storage_dtype)
+        _check(_lib.rlt_load_weights(self.h, name.encode(), raw.ctypes.data, raw.nbytes))
+
+    def get_weights(self, name: str) -> np.ndarray:
+        r, c, _ = self.tensor_info(name)
+        out = np.zeros((r, c), dtype=self.storage_dtype)
+        _check(_lib.rlt_get_weights(self.h, name.encode(), out.ctypes.data, out.nbytes))
+        return out
+
+
+class State:
+    """Owner of an ``rlt_state*``."""
+
+    def __init__(self, handle: ctypes.c_void_p, model: Model, batch: int, max_len: int):
+        self.h = handle
+        self.model = model
+        self.batch = batch
+        self.max_len = max_len
+
+    def __del__(self):
+        self.free()
+
+    def free(self):
+        if getattr(self, "h", None):
+            _lib.rlt_state_free(self.h)
+            self.h = None
+
+    def info(self) -> dict:
+        i = StateInfo()
+        _check(_lib.rlt_state_info_get(self.h, ctypes.byref(i)))
+        return {f: getattr(i, f) for f, _ in StateInfo._fields_}
+
+    def read(self, what: int, index: int = 0) -> np.ndarray:
+        c = self.model.cfg
+        d, B, L = c["d"], self.batch, self.max_len
+        H = c["n_heads"]
+        hd = d // H
+        sd = self.model.storage_dtype
+        if what == READ_S:
+            out = np.zeros((B, d), np.float32)
+        elif what == READ_E:
+            out = np.zeros((B, L, d), np.float32)
+        elif what in (READ_RING_K, READ_RING_V):
+            out = np.zeros((B, H, c["window"] - 1, hd), sd)
+        else:
+            out = np.zeros((B, H, L, hd), sd)
+        _check(_lib.rlt_state_read(self.h, what, index, out.ctypes.data, out.nbytes))
+        return out
+
+
+# ------------------------------------------------------------------ entry points
+def rlt_init_weights(cfg: dict, seed: int) -> Model:
+    c = make_config(**cfg)
+    h = ctypes.c_void_p()
+    _check(_lib.rlt_init_weights(ctypes.byref(c), seed, ctypes.byref(h)))
+    return Model(h, cfg)
+
+
+def rlt_state_create(model: Model, batch: int, max_len: int, flags: int = 0) -> State:
+    h = ctypes.c_void_p()
+    _check(_lib.rlt_state_create(model.h, batch, max_len, flags, ctypes.byref(h)))
+    return State(h, model, batch, max_len)
+
+
+def rlt_state_reset(state: State, stream=None) -> None:
+    _check(_lib.rlt_state_reset(state.h, _stream(stream)))
+
+
+def rlt_encode_prefix(model: Model, state: State, tokens, stream=None) -> None:
+    """tokens: int32 CUDA tensor [B, T]."""
+    _check(_lib.rlt_encode_prefix(model.h, state.h, _dev(tokens, "torch.int32"), tokens.shape[1], _stream(stream)))
+
+
+def _readout_out(logp=None, sampled=None, logp_sampled=None, logmu=None, logits=None):
+    return ReadoutOut(logp=_dev(logp, "torch.float32"), sampled=_dev(sampled, "torch.int32"),
+                      logp_sampled=_dev(logp_sampled, "torch.float32"), logmu=_dev(logmu, "torch.float32"),
+                      logits=_dev(logits, "torch.float32"))
+
+
+def _sampling(sampling):
+    if sampling is None:
+        return None
+    return ctypes.byref(Sampling(temperature=sampling["temperature"], top_k=sampling["top_k"], seed=sampling["seed"]))
+
+
+def rlt_readout(model: Model, state: State, next_tokens=None, sampling: dict | None = None, stream=None,
+                **outs) -> None:
+    o = _readout_out(**outs)
+    _check(_lib.rlt_readout(model.h, state.h, _dev(next_tokens, "torch.int32"), _sampling(sampling),
+                            ctypes.byref(o), _stream(stream)))
+
+
+def rlt_decoder_step(model: Model, state: State, tokens=None, next_tokens=None, sampling: dict | None = None,
+                     stream=None, **outs) -> None:
+    o = _readout_out(**outs)
+    _check(_lib.rlt_decoder_step(model.h, state.h, _dev(tokens, "torch.int32"), _dev(next_tokens, "torch.int32"),
+                                 _sampling(sampling), ctypes.byref(o), _stream(stream)))
+
+
+def rlt_prefill(model: Model, state: State, tokens, logp=None, stream=None) -> None:
+    _check(_lib.rlt_prefill(model.h, state.h, _dev(tokens, "torch.int32"), tokens.shape[1],
+                            _dev(logp, "torch.float32"), _stream(stream)))
+
+
+def rlt_replay_logprobs(model: Model, tokens, logp, stream=None) -> None:
+    """tokens int32 [B, S] and logp float32 [B, S-1], both CUDA tensors."""
+    B, S = tokens.shape
+    _check(_lib.rlt_replay_logprobs(model.h, _dev(tokens, "torch.int32"), B, S, _dev(logp, "torch.float32"),
+                                    _stream(stream)))
+
+
+def rlt_op_linear(w, x, y, use_tensor_cores: bool = True, stream=None) -> None:
+    """y [N, M] fp32 = x [N, K] @ w [M, K]^T (CUDA tensors, bf16 or fp32)."""
+    M, K = w.shape
+    N = x.shape[0]
+    dt = DTYPE_BF16 if str(w.dtype) == "torch.bfloat16" else DTYPE_F32
+    _check(_lib.rlt_op_linear(_dev(w), _dev(x), _dev(y, "torch.float32"), M, N, K, dt, int(use_tensor_cores),
+                              _stream(stream)))
+
+
+def rlt_op_sample(logits, sampling: dict, t: int, token, logp=None, logmu=None, stream=None) -> None:
+    """Sample from fp32 logits [B, V] (CUDA) as position t."""
+    B, V = logits.shape
+    _check(_lib.rlt_op_sample(_dev(logits, "torch.float32"), B, V, _sampling(sampling), t, _dev(token, "torch.int32"),
+                              _dev(logp, "torch.float32"), _dev(logmu, "torch.float32"), _stream(stream)))
+
+
+def rlt_check_device() -> None:
+    _check(_lib.rlt_check_device())
+
+
+def rlt_kernel_launches() -> int:
+    n = ctypes.c_int64()
+    _check(_lib.rlt_kernel_launches(ctypes.byref(n)))
+    return n.value
+
+
+def rlt_profile_enable(model: Model, on: bool) -> None:
+    _check(_lib.rlt_profile_enable(model.h, int(on)))
+
+
+def rlt_profile_read(model: Model, kind: int) -> tuple[float, int, float]:
+    ms, n, by = ctypes.c_double(), ctypes.c_int64(), ctypes.c_double()
+    _check(_lib.rlt_profile_read(model.h, kind, ctypes.byref(ms), ctypes.byref(n), ctypes.byref(by)))
+    return ms.value, n.value, by.value

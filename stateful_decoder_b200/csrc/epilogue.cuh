@@ -1,0 +1,80 @@
+// epilogue.cuh -- fused GEMM epilogues.  Every GEMM here computes
+// C[n][m] = sum_k X[n][k] * W[m][k] (W = weight rows, X = activation rows) and
+// hands each accumulator to one of these functors, which fold the elementwise
+// step that follows the contraction in "Recurrent Looped Transformer":
+//   STORE   plain store (fp32 or the activation type)
+//   RESID   residual add into the fp32 stream (eqs. 2.14-2.16 and the encoder)
+//   SWIGLU  silu(gate) * up on interleaved W1/W3 rows (row 2i = W1 row i,
+//           row 2i+1 = W3 row i); writes column i
+//   GATE    sigmoid(acc + b_g) (eq. 2.10)
+//   MERGE   u = e + alpha * g * acc with acc = W_s r (eq. 2.11)
+//   CONVEX  g = sigmoid(acc), u = g*e + (1-g)*s (convex merge, in place on s)
+#pragma once
+#include "common.cuh"
+
+namespace rlt {
+
+enum EpiKind : int {
+  EPI_STORE = 0,
+  EPI_RESID = 1,
+  EPI_SWIGLU = 2,
+  EPI_GATE = 3,
+  EPI_MERGE = 4,
+  EPI_CONVEX = 5,
+};
+
+struct EpiParams {
+  void* out;            // output base
+  RowMap out_map;       // row addressing of the output
+  int out_bf16;         // STORE/SWIGLU: 1 = bf16 output, 0 = fp32
+  const float* aux0;    // MERGE/CONVEX: e_t rows
+  RowMap aux0_map;
+  const float* aux1;    // MERGE: gate rows
+  int64_t ld_aux1;
+  const void* bias;     // GATE: b_g [M], model storage type
+  int bias_bf16;
+  float alpha;          // MERGE: feedback scale
+};
+
+__device__ __forceinline__ float sigmoidf_(float x) { return 1.0f / (1.0f + __expf(-x)); }
+__device__ __forceinline__ float siluf_(float x) { return x / (1.0f + __expf(-x)); }
+
+__device__ __forceinline__ float load_bias(const EpiParams& p, int m) {
+  return p.bias_bf16 ? __bfloat162float(reinterpret_cast<const bf16*>(p.bias)[m])
+                     : reinterpret_cast<const float*>(p.bias)[m];
+}
+
+// Non-pair epilogues: one accumulator for output (n, m).
+template <int EPI>
+__device__ __forceinline__ void epi_apply(const EpiParams& p, int64_t n, int m, float acc) {
+  if constexpr (EPI == EPI_STORE) {
+    const int64_t o = p.out_map.off(n) + m;
+    if (p.out_bf16) reinterpret_cast<bf16*>(p.out)[o] = __float2bfloat16_rn(acc);
+    else reinterpret_cast<float*>(p.out)[o] = acc;
+  } else if constexpr (EPI == EPI_RESID) {
+    float* o = reinterpret_cast<float*>(p.out) + p.out_map.off(n) + m;
+    *o = *o + acc;
+  } else if constexpr (EPI == EPI_GATE) {
+    reinterpret_cast<float*>(p.out)[p.out_map.off(n) + m] = sigmoidf_(acc + load_bias(p, m));
+  } else if constexpr (EPI == EPI_MERGE) {
+    const float e = p.aux0[p.aux0_map.off(n) + m];
+    const float g = p.aux1[n * p.ld_aux1 + m];
+    reinterpret_cast<float*>(p.out)[p.out_map.off(n) + m] = e + p.alpha * g * acc;
+  } else if constexpr (EPI == EPI_CONVEX) {
+    const float e = p.aux0[p.aux0_map.off(n) + m];
+    float* o = reinterpret_cast<float*>(p.out) + p.out_map.off(n) + m;
+    const float g = sigmoidf_(acc);
+    *o = g * e + (1.0f - g) * (*o);
+  }
+}
+
+// SWIGLU pair epilogue: gate accumulator of row 2i and up accumulator of row
+// 2i+1 give hidden column i.
+__device__ __forceinline__ void epi_swiglu(const EpiParams& p, int64_t n, int i, float gate, float up) {
+  const float h = siluf_(gate) * up;
+  const int64_t o = p.out_map.off(n) + i;
+  if (p.out_bf16) reinterpret_cast<bf16*>(p.out)[o] = __float2bfloat16_rn(h);
+  else reinterpret_cast<float*>(p.out)[o] = h;
+}
+
+}  // namespace rlt

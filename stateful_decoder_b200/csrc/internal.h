@@ -1,0 +1,100 @@
+// internal.h -- launchers of librlt's kernels (host side, not exported).
+#pragma once
+#include <cuda_bf16.h>
+#include <cuda_runtime.h>
+#include <stdint.h>
+
+#include "common.cuh"
+#include "epilogue.cuh"
+
+namespace rlt {
+
+constexpr int kSmCount = 148;  // B200 streaming multiprocessors
+
+// Host-side count of kernel launches issued by the library (every launcher
+// calls note_launch once per <<<>>>).
+void note_launch();
+int64_t launch_count();
+
+// ---------------------------------------------------------------- GEMMs
+// C[n][m] = sum_k X[n][k] W[m][k] with a fused epilogue (epilogue.cuh).
+// bf16 on tcgen05: M % 128 == 0, K % 64 == 0, ld* % 8 == 0, 16-byte aligned
+// bases.  `workspace` holds split-K partials (gemm_tc_workspace_floats).
+cudaError_t gemm_tc(const bf16* W, int64_t ldw, const bf16* X, int64_t ldx, int M, int N, int K, int epi,
+                    const EpiParams& ep, float* workspace, size_t workspace_floats, cudaStream_t st);
+size_t gemm_tc_workspace_floats(int M, int K, int N);
+int gemm_tc_splits(int M, int K, int N);
+int gemm_tc_bn(int N);
+
+// CUDA-core GEMM (fp32 models; also a cross-check for the tensor-core path).
+template <typename WT, typename XT>
+cudaError_t gemm_simt(const WT* W, int64_t ldw, const XT* X, int64_t ldx, int M, int N, int K, int epi,
+                      const EpiParams& ep, cudaStream_t st);
+
+// ---------------------------------------------------------------- attention
+// SWA decode attention of one decoder layer (eq. 2.14) over the ring of
+// retained entries plus the current key/value, then the ring insert.
+template <typename KT>
+cudaError_t swa_attn(const float* qkv, int64_t ld_qkv, KT* ring_k, KT* ring_v, int B, int H, int hd, int t, int W,
+                     const float* rope_cs, KT* out, int64_t ld_out, cudaStream_t st);
+
+// Decode attention of one query per (sequence, head) over key/value rows
+// 0..n-1 of a [B][H][ld_t][hd] cache; the query is rotated at position
+// qpos (0-based) first.  Split over fixed chunks of keys when n is large.
+template <typename KT>
+cudaError_t prefix_attn(const float* q, int64_t ld_q, const KT* k, const KT* v, int64_t ld_t, int B, int H, int hd,
+                        int n, int qpos, const float* rope_cs, KT* out, int64_t ld_out, float* ws, size_t ws_floats,
+                        cudaStream_t st);
+size_t prefix_attn_workspace_floats(int B, int H, int hd, int n);
+constexpr int kPrefixChunk = 256;
+
+// Token-parallel causal attention for the encoder (eq. 2.1): Q, K, V are
+// [B][H][ld_t][hd] (rows 0..T-1 used); out row b*T+i, columns h*hd.
+template <typename KT>
+cudaError_t causal_attn(const KT* q, const KT* k, const KT* v, int64_t ld_tq, int64_t ld_tkv, int B, int H, int hd,
+                        int T, KT* out, int64_t ld_out, cudaStream_t st);
+
+// ---------------------------------------------------------------- elementwise
+// Generator fill of a [rows][cols] view (rows `pitch` elements apart).
+template <typename WT>
+cudaError_t init_normal(WT* dst, int64_t rows, int64_t cols, int64_t pitch, uint64_t seed, uint32_t stream_id,
+                        float std, cudaStream_t st);
+template <typename WT>
+cudaError_t init_const(WT* dst, int64_t rows, int64_t cols, int64_t pitch, float value, cudaStream_t st);
+
+// e rows (RowMap) = Emb[tok]
+template <typename WT>
+cudaError_t embed(const int32_t* tok, int64_t n_rows, int tok_per_seq, int64_t tok_seq_stride, const WT* emb, int d,
+                  int vocab, float* out, RowMap out_map, cudaStream_t st);
+
+// out[r] = gamma * x[r] / sqrt(mean(x[r]^2) + eps), x fp32 rows via RowMap
+template <typename WT, typename OT>
+cudaError_t rmsnorm(const float* x, RowMap x_map, const WT* gamma, int64_t rows, int d, float eps, OT* out,
+                    int64_t ld_out, cudaStream_t st);
+
+// Merge operand: xb[b] = [e_t ; RMSNorm_s(s)] (kind 0) or [e_t ; s] (kind 1)
+template <typename WT, typename OT>
+cudaError_t merge_prep(const float* e, RowMap e_map, const float* s, const WT* gamma, int B, int d, float eps,
+                       int kind, OT* out, cudaStream_t st);
+
+// Scatter head-split rows into a [B][H][ld_t][hd] store at positions
+// pos0 + (r % rows_per_seq), rotating (rope != 0) at that position.
+template <typename XT, typename KT>
+cudaError_t head_scatter(const XT* x, int64_t ld_x, int64_t col0, int64_t rows, int rows_per_seq, int pos0, int H,
+                         int hd, int rope, const float* rope_cs, KT* dst, int64_t ld_t, cudaStream_t st);
+
+// logp[b*ld_logp] = logits[b][next[b*next_stride]] - logsumexp(logits[b])
+cudaError_t logp_gather(const float* logits, int B, int V, const int32_t* next, int64_t next_stride, float* logp,
+                        int64_t ld_logp, cudaStream_t st);
+
+// Top-k / temperature behaviour sampler (report §5.3).
+cudaError_t sample_topk(const float* logits, int B, int V, float temperature, int top_k, uint64_t seed, uint32_t t,
+                        int32_t* token, float* logp_tok, float* logmu, cudaStream_t st);
+
+cudaError_t copy_f32(float* dst, const float* src, int64_t n, cudaStream_t st);
+
+// dst[b][:] = src[:] (fp32) for b < B
+template <typename WT>
+cudaError_t broadcast_row(const WT* src, int d, float* dst, int B, cudaStream_t st);
+
+}  // namespace rlt

@@ -1,0 +1,417 @@
+// ops.cu -- elementwise and row kernels of the RLT step: weight generator,
+// embedding gather, RMSNorm, merge operand, head scatter with rotary map,
+// readout log-probabilities and the behaviour sampler.
+#include <float.h>
+
+#include <atomic>
+
+#include "common.cuh"
+#include "internal.h"
+
+namespace rlt {
+
+__device__ int g_device_error = 0;
+
+namespace {
+std::atomic<int64_t> g_launches{0};
+}
+void note_launch() { g_launches.fetch_add(1, std::memory_order_relaxed); }
+int64_t launch_count() { return g_launches.load(std::memory_order_relaxed); }
+
+namespace {
+
+// ------------------------------------------------------------------ init
+// Element i of generator stream `sid`: init_std * (Irwin-Hall(12) - 6), the
+// twelve uniforms being the words of three Philox4x32-10 blocks with counters
+// (i_lo, i_hi, sid, j), key = seed.  Integer sum, exact double arithmetic,
+// then fp32 and (bf16 storage) round-to-nearest-even.
+template <typename WT>
+__global__ void init_normal_kernel(WT* dst, int64_t rows, int64_t cols, int64_t pitch, uint32_t k0, uint32_t k1,
+                                   uint32_t sid, float std) {
+  const int64_t n = rows * cols;
+  for (int64_t i = (int64_t)blockIdx.x * blockDim.x + threadIdx.x; i < n; i += (int64_t)gridDim.x * blockDim.x) {
+    uint64_t sum = 0;
+#pragma unroll
+    for (uint32_t j = 0; j < 3; ++j) {
+      uint32_t c[4] = {(uint32_t)i, (uint32_t)((uint64_t)i >> 32), sid, j};
+      philox4x32_10(c, k0, k1);
+      sum += (uint64_t)c[0] + c[1] + c[2] + c[3];
+    }
+    const double z = (double)sum * (1.0 / 4294967296.0) - 6.0;
+    const float f = __double2float_rn((double)std * z);
+    dst[(i / cols) * pitch + (i % cols)] = from_f32<WT>(f);
+  }
+}
+
+template <typename WT>
+__global__ void init_const_kernel(WT* dst, int64_t rows, int64_t cols, int64_t pitch, float value) {
+  const int64_t n = rows * cols;
+  for (int64_t i = (int64_t)blockIdx.x * blockDim.x + threadIdx.x; i < n; i += (int64_t)gridDim.x * blockDim.x)
+    dst[(i / cols) * pitch + (i % cols)] = from_f32<WT>(value);
+}
+
+// ------------------------------------------------------------------ embed
+template <typename WT>
+__global__ void embed_kernel(const int32_t* __restrict__ tok, int tok_per_seq, int64_t tok_seq_stride,
+                             const WT* __restrict__ emb, int d, int vocab, float* out, RowMap out_map) {
+  const int64_t r = blockIdx.x;
+  int32_t id = tok[(r / tok_per_seq) * tok_seq_stride + (r % tok_per_seq)];
+  if (id < 0 || id >= vocab) {
+    if (threadIdx.x == 0) atomicExch(&g_device_error, 2);
+    id = 0;
+  }
+  float* o = out + out_map.off(r);
+  const WT* e = emb + (int64_t)id * d;
+  for (int i = threadIdx.x; i < d; i += blockDim.x) o[i] = to_f32(e[i]);
+}
+
+// ------------------------------------------------------------------ rmsnorm
+template <typename WT, typename OT>
+__global__ void rmsnorm_kernel(const float* __restrict__ x, RowMap x_map, const WT* __restrict__ gamma, int d,
+                               float eps, OT* out, int64_t ld_out) {
+  __shared__ float red[32];
+  const int64_t r = blockIdx.x;
+  const float* xr = x + x_map.off(r);
+  float ss = 0.f;
+  for (int i = threadIdx.x; i < d; i += blockDim.x) ss = fmaf(xr[i], xr[i], ss);
+  ss = block_sum(ss, red);
+  const float inv = rsqrtf(ss / (float)d + eps);
+  OT* o = out + r * ld_out;
+  for (int i = threadIdx.x; i < d; i += blockDim.x) o[i] = from_f32<OT>(to_f32(gamma[i]) * xr[i] * inv);
+}
+
+// Merge operand (eqs. 2.9-2.10): row b = [e_t ; RMSNorm_s(s_{t-1})] for the
+// report's merge, [e_t ; s_{t-1}] for the convex gate.
+template <typename WT, typename OT>
+__global__ void merge_prep_kernel(const float* __restrict__ e, RowMap e_map, const float* __restrict__ s,
+                                  const WT* __restrict__ gamma, int d, float eps, int kind, OT* out) {
+  __shared__ float red[32];
+  const int b = blockIdx.x;
+  const float* er = e + e_map.off(b);
+  const float* sr = s + (int64_t)b * d;
+  OT* o = out + (int64_t)b * 2 * d;
+  float ss = 0.f;
+  for (int i = threadIdx.x; i < d; i += blockDim.x) ss = fmaf(sr[i], sr[i], ss);
+  ss = block_sum(ss, red);
+  const float inv = rsqrtf(ss / (float)d + eps);
+  for (int i = threadIdx.x; i < d; i += blockDim.x) {
+    o[i] = from_f32<OT>(er[i]);
+    o[d + i] = from_f32<OT>(kind == 0 ? to_f32(gamma[i]) * sr[i] * inv : sr[i]);
+  }
+}
+
+// ------------------------------------------------------------------ scatter
+// Row r of x (columns col0 + h*hd + i) goes to dst[b][h][pos][i] with
+// b = r / rows_per_seq, pos = pos0 + r % rows_per_seq, rotating the pair
+// (i, i+hd/2) by pos * base^(-2i/hd) when rope != 0.
+template <typename XT, typename KT>
+__global__ void head_scatter_kernel(const XT* __restrict__ x, int64_t ld_x, int64_t col0, int64_t rows,
+                                    int rows_per_seq, int pos0, int H, int hd, int rope,
+                                    const float* __restrict__ rope_cs, KT* dst, int64_t ld_t) {
+  const int half = hd / 2;
+  const int64_t n = rows * H * half;
+  for (int64_t idx = (int64_t)blockIdx.x * blockDim.x + threadIdx.x; idx < n; idx += (int64_t)gridDim.x * blockDim.x) {
+    const int i = (int)(idx % half);
+    const int h = (int)((idx / half) % H);
+    const int64_t r = idx / ((int64_t)half * H);
+    const int64_t b = r / rows_per_seq;
+    const int pos = pos0 + (int)(r % rows_per_seq);
+    const XT* xr = x + r * ld_x + col0 + (int64_t)h * hd;
+    float a = to_f32(xr[i]), c = to_f32(xr[i + half]);
+    if (rope) {
+      const float* cs = rope_cs + ((int64_t)pos * half + i) * 2;
+      const float ra = a * cs[0] - c * cs[1];
+      const float rc = a * cs[1] + c * cs[0];
+      a = ra;
+      c = rc;
+    }
+    KT* o = dst + ((b * H + h) * ld_t + pos) * hd;
+    o[i] = from_f32<KT>(a);
+    o[i + half] = from_f32<KT>(c);
+  }
+}
+
+// ------------------------------------------------------------------ readout
+__global__ void logp_gather_kernel(const float* __restrict__ logits, int V, const int32_t* __restrict__ next,
+                                   int64_t next_stride, float* logp, int64_t ld_logp) {
+  __shared__ float red[32];
+  const int b = blockIdx.x;
+  const float* l = logits + (int64_t)b * V;
+  float mx = -INFINITY;
+  for (int i = threadIdx.x; i < V; i += blockDim.x) mx = fmaxf(mx, l[i]);
+  mx = block_max(mx, red);
+  float s = 0.f;
+  for (int i = threadIdx.x; i < V; i += blockDim.x) s += __expf(l[i] - mx);
+  s = block_sum(s, red);
+  if (threadIdx.x == 0) {
+    int32_t id = next[(int64_t)b * next_stride];
+    if (id < 0 || id >= V) {
+      atomicExch(&g_device_error, 2);
+      id = 0;
+    }
+    logp[(int64_t)b * ld_logp] = l[id] - (mx + logf(s));
+  }
+}
+
+// order-preserving key of a float (larger float -> larger key); -0 and +0
+// share a key so equal values compare equal as floats do
+__device__ __forceinline__ uint32_t fkey(float f) {
+  if (f == 0.0f) f = 0.0f;
+  const uint32_t u = __float_as_uint(f);
+  return (u & 0x80000000u) ? ~u : (u | 0x80000000u);
+}
+
+constexpr int kSampleThreads = 1024;
+constexpr int kMaxTopK = 256;
+
+// One block per sequence.  (1) radix-select the key of the top_k-th largest
+// logit; (2) gather every logit above it plus the lowest-id ones equal to it;
+// (3) sort the candidates by (value desc, id asc); (4) thread 0 forms the
+// tempered weights, their running sums in that order, draws the Philox
+// uniform for counter (t, b, 0, 0) and picks the first candidate whose
+// running sum exceeds u * total.
+__global__ void __launch_bounds__(kSampleThreads)
+    sample_kernel(const float* __restrict__ logits, int V, float temperature, int top_k, uint32_t k0, uint32_t k1,
+                  uint32_t t, int32_t* token, float* logp_tok, float* logmu) {
+  __shared__ uint32_t hist[256];
+  __shared__ uint32_t s_sel[2];
+  __shared__ float red[32];
+  __shared__ uint32_t cand_key[kMaxTopK];
+  __shared__ int32_t cand_id[kMaxTopK];
+  __shared__ uint32_t scan[kSampleThreads];
+  __shared__ uint32_t n_gt;
+  const int b = blockIdx.x, tid = threadIdx.x;
+  const float* l = logits + (int64_t)b * V;
+  const int k = top_k < V ? top_k : V;
+
+  uint32_t prefix = 0, mask = 0, need = (uint32_t)k;
+  for (int shift = 24; shift >= 0; shift -= 8) {
+    for (int i = tid; i < 256; i += kSampleThreads) hist[i] = 0;
+    __syncthreads();
+    for (int i = tid; i < V; i += kSampleThreads) {
+      const uint32_t u = fkey(l[i]);
+      if ((u & mask) == prefix) atomicAdd(&hist[(u >> shift) & 255u], 1u);
+    }
+    __syncthreads();
+    if (tid == 0) {
+      uint32_t cum = 0, sel = 0;
+      for (int dg = 255; dg >= 0; --dg) {
+        if (cum + hist[dg] >= need) { sel = (uint32_t)dg; break; }
+        cum += hist[dg];
+      }
+      s_sel[0] = sel;
+      s_sel[1] = need - cum;
+    }
+    __syncthreads();
+    prefix |= s_sel[0] << shift;
+    mask |= 255u << shift;
+    need = s_sel[1];
+    __syncthreads();
+  }
+  const uint32_t thr = prefix;  // key of the k-th largest logit; `need` ties at it are taken
+
+  // ordered pass over contiguous id ranges so ties are taken by ascending id
+  const int per = (V + kSampleThreads - 1) / kSampleThreads;
+  const int lo = tid * per, hi = min(V, lo + per);
+  uint32_t my_eq = 0;
+  for (int i = lo; i < hi; ++i) my_eq += fkey(l[i]) == thr;
+  scan[tid] = my_eq;
+  if (tid == 0) n_gt = 0;
+  __syncthreads();
+  for (int off = 1; off < kSampleThreads; off <<= 1) {  // inclusive scan
+    const uint32_t v = tid >= off ? scan[tid - off] : 0u;
+    __syncthreads();
+    scan[tid] += v;
+    __syncthreads();
+  }
+  uint32_t eq_rank = scan[tid] - my_eq;
+  const uint32_t n_above = (uint32_t)k - need;
+  for (int i = lo; i < hi; ++i) {
+    const uint32_t u = fkey(l[i]);
+    if (u > thr) {
+      const uint32_t slot = atomicAdd(&n_gt, 1u);
+      cand_key[slot] = u;
+      cand_id[slot] = i;
+    } else if (u == thr) {
+      if (eq_rank < need) {
+        cand_key[n_above + eq_rank] = u;
+        cand_id[n_above + eq_rank] = i;
+      }
+      ++eq_rank;
+    }
+  }
+  __syncthreads();
+  // bitonic sort of kMaxTopK entries (padding sorts last)
+  for (int i = tid; i < kMaxTopK; i += kSampleThreads)
+    if (i >= k) { cand_key[i] = 0u; cand_id[i] = 0x7FFFFFFF; }
+  __syncthreads();
+  for (int size = 2; size <= kMaxTopK; size <<= 1) {
+    for (int stride = size >> 1; stride > 0; stride >>= 1) {
+      if (tid < kMaxTopK) {
+        const int j = tid ^ stride;
+        if (j > tid) {
+          // "a before b": larger key, or equal key and smaller id
+          const bool asc = (tid & size) == 0;
+          const uint32_t ka = cand_key[tid], kb = cand_key[j];
+          const int32_t ia = cand_id[tid], ib = cand_id[j];
+          const bool a_first = ka > kb || (ka == kb && ia < ib);
+          if (asc ? !a_first : a_first) {
+            cand_key[tid] = kb; cand_key[j] = ka;
+            cand_id[tid] = ib; cand_id[j] = ia;
+          }
+        }
+      }
+      __syncthreads();
+    }
+  }
+  // raw log-softmax normaliser over the whole vocabulary
+  const float mx = l[cand_id[0]];
+  float s = 0.f;
+  for (int i = tid; i < V; i += kSampleThreads) s += __expf(l[i] - mx);
+  s = block_sum(s, red);
+  if (tid == 0) {
+    const float z0 = l[cand_id[0]] / temperature;
+    float w[kMaxTopK];
+    float total = 0.f;
+    for (int r = 0; r < k; ++r) {
+      w[r] = expf(l[cand_id[r]] / temperature - z0);
+      total += w[r];
+    }
+    uint32_t c[4] = {t, (uint32_t)b, 0u, 0u};
+    philox4x32_10(c, k0, k1);
+    const float u = (float)(c[0] >> 8) * (1.0f / 16777216.0f);
+    const float target = u * total;
+    float run = 0.f;
+    int pick = k - 1;
+    for (int r = 0; r < k; ++r) {
+      run += w[r];
+      if (run > target) { pick = r; break; }
+    }
+    const int32_t id = cand_id[pick];
+    if (token) token[b] = id;
+    if (logmu) logmu[b] = (l[id] / temperature - z0) - logf(total);
+    if (logp_tok) logp_tok[b] = l[id] - (mx + logf(s));
+  }
+}
+
+template <typename WT>
+__global__ void broadcast_kernel(const WT* __restrict__ src, int d, float* dst, int B) {
+  const int64_t n = (int64_t)B * d;
+  for (int64_t i = (int64_t)blockIdx.x * blockDim.x + threadIdx.x; i < n; i += (int64_t)gridDim.x * blockDim.x)
+    dst[i] = to_f32(src[i % d]);
+}
+
+__global__ void copy_kernel(float* dst, const float* src, int64_t n) {
+  for (int64_t i = (int64_t)blockIdx.x * blockDim.x + threadIdx.x; i < n; i += (int64_t)gridDim.x * blockDim.x)
+    dst[i] = src[i];
+}
+
+inline unsigned grid_for(int64_t n, int threads, int cap = 148 * 16) {
+  int64_t g = (n + threads - 1) / threads;
+  if (g > cap) g = cap;
+  if (g < 1) g = 1;
+  return (unsigned)g;
+}
+
+}  // namespace
+
+template <typename WT>
+cudaError_t init_normal(WT* dst, int64_t rows, int64_t cols, int64_t pitch, uint64_t seed, uint32_t sid, float std,
+                        cudaStream_t st) {
+  const int64_t n = rows * cols;
+  init_normal_kernel<WT><<<grid_for(n, 256, 148 * 64), 256, 0, st>>>(dst, rows, cols, pitch, (uint32_t)seed,
+                                                                     (uint32_t)(seed >> 32), sid, std);
+  note_launch();
+  return cudaGetLastError();
+}
+
+template <typename WT>
+cudaError_t init_const(WT* dst, int64_t rows, int64_t cols, int64_t pitch, float value, cudaStream_t st) {
+  init_const_kernel<WT><<<grid_for(rows * cols, 256), 256, 0, st>>>(dst, rows, cols, pitch, value);
+  note_launch();
+  return cudaGetLastError();
+}
+
+template <typename WT>
+cudaError_t embed(const int32_t* tok, int64_t n_rows, int tok_per_seq, int64_t tok_seq_stride, const WT* emb, int d,
+                  int vocab, float* out, RowMap out_map, cudaStream_t st) {
+  embed_kernel<WT><<<(unsigned)n_rows, 128, 0, st>>>(tok, tok_per_seq, tok_seq_stride, emb, d, vocab, out, out_map);
+  note_launch();
+  return cudaGetLastError();
+}
+
+template <typename WT, typename OT>
+cudaError_t rmsnorm(const float* x, RowMap x_map, const WT* gamma, int64_t rows, int d, float eps, OT* out,
+                    int64_t ld_out, cudaStream_t st) {
+  const int threads = d >= 1024 ? 256 : 128;
+  rmsnorm_kernel<WT, OT><<<(unsigned)rows, threads, 0, st>>>(x, x_map, gamma, d, eps, out, ld_out);
+  note_launch();
+  return cudaGetLastError();
+}
+
+template <typename WT, typename OT>
+cudaError_t merge_prep(const float* e, RowMap e_map, const float* s, const WT* gamma, int B, int d, float eps,
+                       int kind, OT* out, cudaStream_t st) {
+  merge_prep_kernel<WT, OT><<<B, d >= 1024 ? 256 : 128, 0, st>>>(e, e_map, s, gamma, d, eps, kind, out);
+  note_launch();
+  return cudaGetLastError();
+}
+
+template <typename XT, typename KT>
+cudaError_t head_scatter(const XT* x, int64_t ld_x, int64_t col0, int64_t rows, int rows_per_seq, int pos0, int H,
+                         int hd, int rope, const float* rope_cs, KT* dst, int64_t ld_t, cudaStream_t st) {
+  const int64_t n = rows * H * (hd / 2);
+  head_scatter_kernel<XT, KT><<<grid_for(n, 256, 148 * 32), 256, 0, st>>>(x, ld_x, col0, rows, rows_per_seq, pos0, H,
+                                                                          hd, rope, rope_cs, dst, ld_t);
+  note_launch();
+  return cudaGetLastError();
+}
+
+cudaError_t logp_gather(const float* logits, int B, int V, const int32_t* next, int64_t next_stride, float* logp,
+                        int64_t ld_logp, cudaStream_t st) {
+  logp_gather_kernel<<<B, 1024, 0, st>>>(logits, V, next, next_stride, logp, ld_logp);
+  note_launch();
+  return cudaGetLastError();
+}
+
+cudaError_t sample_topk(const float* logits, int B, int V, float temperature, int top_k, uint64_t seed, uint32_t t,
+                        int32_t* token, float* logp_tok, float* logmu, cudaStream_t st) {
+  if (top_k < 1 || top_k > kMaxTopK || !(temperature > 0.f)) return cudaErrorInvalidValue;
+  sample_kernel<<<B, kSampleThreads, 0, st>>>(logits, V, temperature, top_k, (uint32_t)seed, (uint32_t)(seed >> 32), t,
+                                             token, logp_tok, logmu);
+  note_launch();
+  return cudaGetLastError();
+}
+
+template <typename WT>
+cudaError_t broadcast_row(const WT* src, int d, float* dst, int B, cudaStream_t st) {
+  broadcast_kernel<WT><<<grid_for((int64_t)B * d, 256), 256, 0, st>>>(src, d, dst, B);
+  note_launch();
+  return cudaGetLastError();
+}
+
+cudaError_t copy_f32(float* dst, const float* src, int64_t n, cudaStream_t st) {
+  copy_kernel<<<grid_for(n, 256), 256, 0, st>>>(dst, src, n);
+  note_launch();
+  return cudaGetLastError();
+}
+
+#define RLT_INST_W(WT)                                                                                              \
+  template cudaError_t init_normal<WT>(WT*, int64_t, int64_t, int64_t, uint64_t, uint32_t, float, cudaStream_t);  \
+  template cudaError_t init_const<WT>(WT*, int64_t, int64_t, int64_t, float, cudaStream_t);                      \
+  template cudaError_t embed<WT>(const int32_t*, int64_t, int, int64_t, const WT*, int, int, float*, RowMap,     \
+                                 cudaStream_t);                                                                   \
+  template cudaError_t rmsnorm<WT, WT>(const float*, RowMap, const WT*, int64_t, int, float, WT*, int64_t,        \
+                                       cudaStream_t);                                                             \
+  template cudaError_t merge_prep<WT, WT>(const float*, RowMap, const float*, const WT*, int, int, float, int,    \
+                                          WT*, cudaStream_t);                                                     \
+  template cudaError_t head_scatter<float, WT>(const float*, int64_t, int64_t, int64_t, int, int, int, int, int,   \
+                                               const float*, WT*, int64_t, cudaStream_t);                         \
+  template cudaError_t broadcast_row<WT>(const WT*, int, float*, int, cudaStream_t);
+
+RLT_INST_W(float)
+RLT_INST_W(bf16)
+template cudaError_t head_scatter<bf16, bf16>(const bf16*, int64_t, int64_t, int64_t, int, int, int, int, int,
+                                              const float*, bf16*, int64_t, cudaStream_t);
+
+}  // namespace rlt

@@ -1,0 +1,1005 @@
+// rlt_api.cu -- host engine and C ABI of librlt (include/rlt.h).
+//
+// Owns model weights and per-batch state in device memory and schedules the
+// kernels of one lock-step transition for B independent sequences
+// ("Recurrent Looped Transformer" §4.1: ready decoder transitions of
+// independent sequences are batched).  Schedules follow App. A: encoder
+// prefill (A.1, eq. 2.1), incremental generation (A.2, eq. 2.8), replay
+// (A.4).
+//
+// Weight storage.  Every tensor is kept in the model dtype.  Matrices that
+// feed one contraction are stored together so one GEMM covers them:
+//   wq/wk/wv of a layer  -> rows [0,d), [d,2d), [2d,3d) of a [3d][d] block
+//   w1/w3 of a layer     -> interleaved rows of a [2F][d] block (row 2i = w1
+//                           row i, row 2i+1 = w3 row i; SwiGLU pairs meet in
+//                           adjacent accumulator lanes)
+//   wk_mem.g/wv_mem.g    -> rows [2dg, 2dg+d) and [2dg+d, 2d(g+1)) of [2dG][d]
+// The named tensors of rlt.h are views into these blocks.
+#include <cuda_runtime.h>
+
+#include <cmath>
+#include <cstdio>
+#include <cstring>
+#include <map>
+#include <string>
+#include <vector>
+
+#include "internal.h"
+#include "rlt.h"
+
+using namespace rlt;
+
+// ------------------------------------------------------------------ errors
+namespace {
+thread_local std::string t_err = "";
+thread_local int32_t t_err_code = RLT_OK;
+
+int32_t fail(int32_t code, const std::string& msg) {
+  t_err = msg;
+  t_err_code = code;
+  return code;
+}
+int32_t ok() { return RLT_OK; }
+}  // namespace
+
+#define RLT_CUDA(...)                                                                                          \
+  do {                                                                                                         \
+    cudaError_t e_ = (__VA_ARGS__);                                                                            \
+    if (e_ != cudaSuccess) return fail(RLT_E_CUDA, std::string(#__VA_ARGS__) + ": " + cudaGetErrorString(e_)); \
+  } while (0)
+#define RLT_TRY(...)                 \
+  do {                               \
+    int32_t r_ = (__VA_ARGS__);      \
+    if (r_ != RLT_OK) return r_;     \
+  } while (0)
+
+// ------------------------------------------------------------------ model
+struct View {
+  void* base;       // first element
+  int64_t rows, cols, pitch;  // pitch in elements between logical rows
+  int32_t sid;      // generator stream id
+  int32_t kind;     // 0 random, 1 ones, 2 zeros
+};
+
+struct LayerW {
+  void* qkv;   // [3d][d]
+  void* wo;    // [d][d]
+  void* w13;   // [2F][d] interleaved
+  void* w2;    // [d][F]
+  void* wq_mem;
+  void* wo_mem;
+  void* g_ea; void* g_ef; void* g_dsa; void* g_dmem; void* g_dffn;
+  void* dqkv; void* dwo; void* dw13; void* dw2;  // decoder weights (== encoder ones when tied)
+};
+
+struct ProfileRec {
+  bool on = false;
+  std::vector<cudaEvent_t> ev;
+  size_t used = 0;
+  double bytes[2] = {0, 0};
+  int64_t launches[2] = {0, 0};
+  std::vector<int> kind;  // per event pair
+};
+
+struct rlt_model {
+  rlt_config cfg;
+  int hd = 0;
+  size_t esz = 0;
+  int device = 0;
+  uint64_t version = 1;
+  std::vector<void*> allocs;
+  void* emb = nullptr; void* s_star = nullptr; void* g_mem = nullptr; void* g_merge = nullptr;
+  void* w_gate = nullptr; void* b_gate = nullptr; void* w_state = nullptr; void* g_out = nullptr;
+  void* w_out = nullptr; void* w_kvm = nullptr;
+  std::vector<LayerW> layers;
+  std::map<std::string, View> views;
+  float* rope_cs = nullptr;
+  int rope_len = 0;
+  rlt_state* replay = nullptr;
+  ProfileRec prof;
+};
+
+struct rlt_state {
+  rlt_model* m = nullptr;
+  int32_t B = 0, max_len = 0, flags = 0;
+  uint64_t version = 0;
+  int32_t n_enc = 0, n_dec = 0;
+  std::vector<void*> allocs;
+  float* e = nullptr;          // [B][max_len][d]
+  void* mem_k = nullptr; void* mem_v = nullptr;  // [G][B][H][max_len][hd]
+  void* ce_k = nullptr; void* ce_v = nullptr;    // [L][B][H][max_len][hd]
+  void* ring_k = nullptr; void* ring_v = nullptr;  // [L][B][H][W-1][hd]
+  float* s = nullptr;          // [B][d]
+  void* xb = nullptr;          // [B][2d] GEMM operand (model dtype)
+  float* qkv = nullptr;        // [B][max(3d, 2dG)]
+  int64_t ld_qkv = 0;
+  void* attn = nullptr;        // [B][d]
+  void* hbuf = nullptr;        // [B][F]
+  float* gate = nullptr;       // [B][d]
+  float* logits = nullptr;     // [B][V]
+  float* gemm_ws = nullptr; size_t gemm_ws_floats = 0;
+  float* attn_ws = nullptr; size_t attn_ws_floats = 0;
+  // encoder-prefill workspace, rows = sequences x tokens of one chunk
+  int64_t pf_rows = 0;
+  void* pf_x = nullptr; void* pf_big = nullptr; void* pf_q = nullptr; void* pf_k = nullptr; void* pf_v = nullptr;
+  void* pf_attn = nullptr;
+  int64_t pf_big_cols = 0;
+  float* pf_ws = nullptr; size_t pf_ws_floats = 0;
+};
+
+namespace {
+
+int32_t dev_alloc(std::vector<void*>& list, void** p, size_t bytes) {
+  *p = nullptr;
+  if (bytes == 0) return RLT_OK;
+  cudaError_t e = cudaMalloc(p, bytes);
+  if (e != cudaSuccess) {
+    cudaGetLastError();
+    *p = nullptr;
+    return fail(RLT_E_OOM, "cudaMalloc of " + std::to_string(bytes) + " bytes failed: " + cudaGetErrorString(e));
+  }
+  list.push_back(*p);
+  return RLT_OK;
+}
+
+void free_all(std::vector<void*>& list) {
+  for (void* p : list) cudaFree(p);
+  list.clear();
+}
+
+char* off(void* base, int64_t elems, size_t esz) { return static_cast<char*>(base) + elems * (int64_t)esz; }
+
+int32_t validate(const rlt_config* c) {
+  if (!c) return fail(RLT_E_INVAL, "null config");
+  if (c->d_model <= 0 || c->n_heads <= 0 || c->d_model % c->n_heads) return fail(RLT_E_INVAL, "d_model % n_heads != 0");
+  const int hd = c->d_model / c->n_heads;
+  if (!(hd == 16 || hd == 32 || hd == 64 || hd == 128)) return fail(RLT_E_INVAL, "head size must be 16, 32, 64 or 128");
+  if (c->n_layers <= 0 || c->window < 1 || c->ffn <= 0 || c->vocab <= 1) return fail(RLT_E_INVAL, "bad sizes");
+  if (!(c->groups == 1 || c->groups == c->n_layers)) return fail(RLT_E_INVAL, "groups must be 1 or n_layers");
+  if (c->tied != 0 && c->tied != 1) return fail(RLT_E_INVAL, "tied must be 0 or 1");
+  if (c->merge_kind != RLT_MERGE_PAPER && c->merge_kind != RLT_MERGE_CONVEX) return fail(RLT_E_INVAL, "merge_kind");
+  if (c->dtype != RLT_DTYPE_F32 && c->dtype != RLT_DTYPE_BF16) return fail(RLT_E_INVAL, "dtype");
+  if (c->bos_id < 0 || c->bos_id >= c->vocab) return fail(RLT_E_INVAL, "bos_id");
+  if (!(c->rms_eps >= 0.f) || !(c->rope_base > 1.f) || !(c->init_std >= 0.f)) return fail(RLT_E_INVAL, "eps/base/std");
+  if (c->dtype == RLT_DTYPE_BF16) {
+    // tensor-core contraction shapes: 128-row weight tiles, 64-deep K steps
+    if (c->d_model % 128 || c->ffn % 64 || c->vocab % 128)
+      return fail(RLT_E_INVAL, "bf16 models need d_model % 128 == 0, ffn % 64 == 0, vocab % 128 == 0");
+  }
+  return RLT_OK;
+}
+
+int32_t ensure_rope(rlt_model* m, int len) {
+  if (len <= m->rope_len) return RLT_OK;
+  int n = m->rope_len > 0 ? m->rope_len : 4096;
+  while (n < len) n *= 2;
+  const int half = m->hd / 2;
+  std::vector<float> h((size_t)n * half * 2);
+  for (int p = 0; p < n; ++p)
+    for (int i = 0; i < half; ++i) {
+      const double th = (double)p * std::pow((double)m->cfg.rope_base, -2.0 * i / m->hd);
+      h[((size_t)p * half + i) * 2] = (float)std::cos(th);
+      h[((size_t)p * half + i) * 2 + 1] = (float)std::sin(th);
+    }
+  void* p = nullptr;
+  RLT_TRY(dev_alloc(m->allocs, &p, h.size() * sizeof(float)));
+  RLT_CUDA(cudaMemcpy(p, h.data(), h.size() * sizeof(float), cudaMemcpyHostToDevice));
+  m->rope_cs = static_cast<float*>(p);
+  m->rope_len = n;
+  return RLT_OK;
+}
+
+void add_view(rlt_model* m, const std::string& name, void* base, int64_t rows, int64_t cols, int64_t pitch, int sid,
+              int kind) {
+  m->views[name] = View{base, rows, cols, pitch, sid, kind};
+}
+
+int32_t build_model(rlt_model* m) {
+  const rlt_config& c = m->cfg;
+  const int64_t d = c.d_model, F = c.ffn, V = c.vocab, L = c.n_layers, G = c.groups;
+  const size_t es = m->esz;
+  auto A = [&](void** p, int64_t elems) { return dev_alloc(m->allocs, p, (size_t)elems * es); };
+  RLT_TRY(A(&m->emb, V * d));
+  RLT_TRY(A(&m->s_star, d));
+  RLT_TRY(A(&m->g_mem, d));
+  RLT_TRY(A(&m->g_merge, d));
+  RLT_TRY(A(&m->w_gate, d * 2 * d));
+  RLT_TRY(A(&m->b_gate, d));
+  RLT_TRY(A(&m->w_state, d * d));
+  RLT_TRY(A(&m->g_out, d));
+  RLT_TRY(A(&m->w_out, V * d));
+  RLT_TRY(A(&m->w_kvm, G * 2 * d * d));
+  add_view(m, "emb", m->emb, V, d, d, 0, 0);
+  add_view(m, "s_star", m->s_star, 1, d, d, 1, 0);
+  add_view(m, "g_mem", m->g_mem, 1, d, d, 2, 1);
+  add_view(m, "g_merge", m->g_merge, 1, d, d, 3, 1);
+  add_view(m, "w_gate", m->w_gate, d, 2 * d, 2 * d, 4, 0);
+  add_view(m, "b_gate", m->b_gate, 1, d, d, 5, 2);
+  add_view(m, "w_state", m->w_state, d, d, d, 6, 0);
+  add_view(m, "g_out", m->g_out, 1, d, d, 7, 1);
+  add_view(m, "w_out", m->w_out, V, d, d, 8, 0);
+  for (int g = 0; g < G; ++g) {
+    add_view(m, "wk_mem." + std::to_string(g), off(m->w_kvm, (int64_t)g * 2 * d * d, es), d, d, d, 16 + 2 * g, 0);
+    add_view(m, "wv_mem." + std::to_string(g), off(m->w_kvm, ((int64_t)g * 2 + 1) * d * d, es), d, d, d, 17 + 2 * g, 0);
+  }
+  m->layers.resize(L);
+  for (int l = 0; l < L; ++l) {
+    LayerW& w = m->layers[l];
+    const std::string sfx = "." + std::to_string(l);
+    const int sid0 = 1024 + 32 * l;
+    RLT_TRY(A(&w.qkv, 3 * d * d));
+    RLT_TRY(A(&w.wo, d * d));
+    RLT_TRY(A(&w.w13, 2 * F * d));
+    RLT_TRY(A(&w.w2, d * F));
+    RLT_TRY(A(&w.wq_mem, d * d));
+    RLT_TRY(A(&w.wo_mem, d * d));
+    RLT_TRY(A(&w.g_ea, d));
+    RLT_TRY(A(&w.g_ef, d));
+    RLT_TRY(A(&w.g_dsa, d));
+    RLT_TRY(A(&w.g_dmem, d));
+    RLT_TRY(A(&w.g_dffn, d));
+    add_view(m, "wq" + sfx, w.qkv, d, d, d, sid0 + 0, 0);
+    add_view(m, "wk" + sfx, off(w.qkv, d * d, es), d, d, d, sid0 + 1, 0);
+    add_view(m, "wv" + sfx, off(w.qkv, 2 * d * d, es), d, d, d, sid0 + 2, 0);
+    add_view(m, "wo" + sfx, w.wo, d, d, d, sid0 + 3, 0);
+    add_view(m, "w1" + sfx, w.w13, F, d, 2 * d, sid0 + 4, 0);
+    add_view(m, "w2" + sfx, w.w2, d, F, F, sid0 + 5, 0);
+    add_view(m, "w3" + sfx, off(w.w13, d, es), F, d, 2 * d, sid0 + 6, 0);
+    add_view(m, "g_ea" + sfx, w.g_ea, 1, d, d, sid0 + 7, 1);
+    add_view(m, "g_ef" + sfx, w.g_ef, 1, d, d, sid0 + 8, 1);
+    add_view(m, "g_dsa" + sfx, w.g_dsa, 1, d, d, sid0 + 9, 1);
+    add_view(m, "g_dmem" + sfx, w.g_dmem, 1, d, d, sid0 + 10, 1);
+    add_view(m, "g_dffn" + sfx, w.g_dffn, 1, d, d, sid0 + 11, 1);
+    add_view(m, "wq_mem" + sfx, w.wq_mem, d, d, d, sid0 + 12, 0);
+    add_view(m, "wo_mem" + sfx, w.wo_mem, d, d, d, sid0 + 13, 0);
+    if (c.tied) {
+      w.dqkv = w.qkv; w.dwo = w.wo; w.dw13 = w.w13; w.dw2 = w.w2;
+    } else {
+      RLT_TRY(A(&w.dqkv, 3 * d * d));
+      RLT_TRY(A(&w.dwo, d * d));
+      RLT_TRY(A(&w.dw13, 2 * F * d));
+      RLT_TRY(A(&w.dw2, d * F));
+      add_view(m, "dwq" + sfx, w.dqkv, d, d, d, sid0 + 14, 0);
+      add_view(m, "dwk" + sfx, off(w.dqkv, d * d, es), d, d, d, sid0 + 15, 0);
+      add_view(m, "dwv" + sfx, off(w.dqkv, 2 * d * d, es), d, d, d, sid0 + 16, 0);
+      add_view(m, "dwo" + sfx, w.dwo, d, d, d, sid0 + 17, 0);
+      add_view(m, "dw1" + sfx, w.dw13, F, d, 2 * d, sid0 + 18, 0);
+      add_view(m, "dw2" + sfx, w.dw2, d, F, F, sid0 + 19, 0);
+      add_view(m, "dw3" + sfx, off(w.dw13, d, es), F, d, 2 * d, sid0 + 20, 0);
+    }
+  }
+  return RLT_OK;
+}
+
+template <typename T>
+int32_t init_views(rlt_model* m, uint64_t seed) {
+  for (auto& kv : m->views) {
+    const View& v = kv.second;
+    cudaError_t e;
+    if (v.kind == 0)
+      e = init_normal<T>(static_cast<T*>(v.base), v.rows, v.cols, v.pitch, seed, (uint32_t)v.sid, m->cfg.init_std, 0);
+    else
+      e = init_const<T>(static_cast<T*>(v.base), v.rows, v.cols, v.pitch, v.kind == 1 ? 1.0f : 0.0f, 0);
+    if (e != cudaSuccess) return fail(RLT_E_CUDA, "init " + kv.first + ": " + cudaGetErrorString(e));
+  }
+  RLT_CUDA(cudaDeviceSynchronize());
+  return RLT_OK;
+}
+
+// ------------------------------------------------------------------ GEMM dispatch
+template <typename T>
+int32_t gemm(rlt_state* S, const void* W, int64_t ldw, const void* X, int64_t ldx, int M, int N, int K, int epi,
+             const EpiParams& ep, float* ws, size_t ws_floats, cudaStream_t st);
+
+template <>
+int32_t gemm<bf16>(rlt_state*, const void* W, int64_t ldw, const void* X, int64_t ldx, int M, int N, int K, int epi,
+                   const EpiParams& ep, float* ws, size_t ws_floats, cudaStream_t st) {
+  RLT_CUDA(gemm_tc(static_cast<const bf16*>(W), ldw, static_cast<const bf16*>(X), ldx, M, N, K, epi, ep, ws, ws_floats,
+                   st));
+  return RLT_OK;
+}
+
+template <>
+int32_t gemm<float>(rlt_state*, const void* W, int64_t ldw, const void* X, int64_t ldx, int M, int N, int K, int epi,
+                    const EpiParams& ep, float*, size_t, cudaStream_t st) {
+  RLT_CUDA(gemm_simt<float, float>(static_cast<const float*>(W), ldw, static_cast<const float*>(X), ldx, M, N, K, epi,
+                                   ep, st));
+  return RLT_OK;
+}
+
+EpiParams epi_out(void* out, RowMap map, int out_bf16) {
+  EpiParams p{};
+  p.out = out;
+  p.out_map = map;
+  p.out_bf16 = out_bf16;
+  p.aux0_map = plain_rows(0);
+  return p;
+}
+
+// ------------------------------------------------------------------ profiling
+// Records an event before (prof_begin) and after (prof_end) one kernel launch
+// on the launching stream; kind 0 = prefix attention, 1 = SWA attention.
+void prof_begin(rlt_model* m, cudaStream_t st) {
+  ProfileRec& p = m->prof;
+  if (!p.on) return;
+  if (p.used + 2 > p.ev.size()) {
+    for (int i = 0; i < 1024; ++i) {
+      cudaEvent_t e;
+      if (cudaEventCreate(&e) != cudaSuccess) break;
+      p.ev.push_back(e);
+    }
+  }
+  if (p.used + 2 <= p.ev.size()) cudaEventRecord(p.ev[p.used], st);
+}
+void prof_end(rlt_model* m, cudaStream_t st, int kind, double bytes) {
+  ProfileRec& p = m->prof;
+  if (!p.on || p.used + 2 > p.ev.size()) return;
+  cudaEventRecord(p.ev[p.used + 1], st);
+  p.kind.push_back(kind);
+  p.bytes[kind] += bytes;
+  p.launches[kind] += 1;
+  p.used += 2;
+}
+
+// ------------------------------------------------------------------ state
+int32_t make_state(rlt_model* m, int32_t B, int32_t max_len, int32_t flags, rlt_state** out) {
+  const rlt_config& c = m->cfg;
+  if (B <= 0 || max_len <= 0) return fail(RLT_E_INVAL, "batch and max_len must be positive");
+  RLT_TRY(ensure_rope(m, max_len + 1));
+  rlt_state* S = new rlt_state();
+  S->m = m;
+  S->B = B;
+  S->max_len = max_len;
+  S->flags = flags;
+  S->version = m->version;
+  const int64_t d = c.d_model, L = c.n_layers, G = c.groups, F = c.ffn, V = c.vocab, Wm1 = c.window - 1;
+  const size_t es = m->esz;
+  auto A = [&](void** p, int64_t bytes) { return dev_alloc(S->allocs, p, (size_t)bytes); };
+  int32_t r = RLT_OK;
+  void* p = nullptr;
+  if ((r = A(&p, (int64_t)B * max_len * d * 4))) goto fail_;
+  S->e = static_cast<float*>(p);
+  if ((r = A(&S->mem_k, G * B * max_len * d * (int64_t)es))) goto fail_;
+  if ((r = A(&S->mem_v, G * B * max_len * d * (int64_t)es))) goto fail_;
+  if (flags & RLT_STATE_ENCODER_CACHE) {
+    if ((r = A(&S->ce_k, L * B * max_len * d * (int64_t)es))) goto fail_;
+    if ((r = A(&S->ce_v, L * B * max_len * d * (int64_t)es))) goto fail_;
+  }
+  if (Wm1 > 0) {
+    if ((r = A(&S->ring_k, L * B * Wm1 * d * (int64_t)es))) goto fail_;
+    if ((r = A(&S->ring_v, L * B * Wm1 * d * (int64_t)es))) goto fail_;
+  }
+  if ((r = A(&p, (int64_t)B * d * 4))) goto fail_;
+  S->s = static_cast<float*>(p);
+  if ((r = A(&S->xb, (int64_t)B * 2 * d * es))) goto fail_;
+  S->ld_qkv = std::max<int64_t>(3 * d, 2 * d * G);
+  if ((r = A(&p, (int64_t)B * S->ld_qkv * 4))) goto fail_;
+  S->qkv = static_cast<float*>(p);
+  if ((r = A(&S->attn, (int64_t)B * d * es))) goto fail_;
+  if ((r = A(&S->hbuf, (int64_t)B * F * es))) goto fail_;
+  if ((r = A(&p, (int64_t)B * d * 4))) goto fail_;
+  S->gate = static_cast<float*>(p);
+  if ((r = A(&p, (int64_t)B * V * 4))) goto fail_;
+  S->logits = static_cast<float*>(p);
+  if (c.dtype == RLT_DTYPE_BF16) {
+    size_t w = 0;
+    const int Ms[] = {(int)(3 * d), (int)d, (int)(2 * F), (int)(2 * d * G), (int)V};
+    const int Ks[] = {(int)d, (int)F, (int)(2 * d)};
+    for (int M : Ms)
+      for (int K : Ks) w = std::max(w, gemm_tc_workspace_floats(M, K, B));
+    S->gemm_ws_floats = w;
+    if ((r = A(&p, (int64_t)w * 4))) goto fail_;
+    S->gemm_ws = static_cast<float*>(p);
+  }
+  S->attn_ws_floats = prefix_attn_workspace_floats(B, c.n_heads, (int)(d / c.n_heads), max_len);
+  if ((r = A(&p, (int64_t)S->attn_ws_floats * 4))) goto fail_;
+  S->attn_ws = static_cast<float*>(p);
+  *out = S;
+  return RLT_OK;
+fail_:
+  free_all(S->allocs);
+  delete S;
+  return r;
+}
+
+template <typename T>
+int32_t reset_state(rlt_state* S, cudaStream_t st) {
+  RLT_CUDA(broadcast_row<T>(static_cast<const T*>(S->m->s_star), S->m->cfg.d_model, S->s, S->B, st));
+  S->n_enc = 0;
+  S->n_dec = 0;
+  S->version = S->m->version;
+  return RLT_OK;
+}
+
+int32_t ensure_prefill_ws(rlt_state* S, int T) {
+  const rlt_config& c = S->m->cfg;
+  const int64_t d = c.d_model, G = c.groups, F = c.ffn;
+  const size_t es = S->m->esz;
+  const int64_t big_cols = std::max<int64_t>(std::max<int64_t>(3 * d, F), 2 * d * G);
+  const bool cache = (S->flags & RLT_STATE_ENCODER_CACHE) != 0;
+  // bytes per token row of the prefill workspace
+  const int64_t per_row = (int64_t)es * (d /*x*/ + big_cols + d /*q*/ + d /*attn*/ + (cache ? 0 : 2 * d));
+  const int64_t budget = (int64_t)4 << 30;
+  int64_t seqs = std::max<int64_t>(1, std::min<int64_t>(S->B, budget / (per_row * T)));
+  const int64_t rows = seqs * T;
+  if (rows <= S->pf_rows && S->pf_big_cols == big_cols) return RLT_OK;
+  for (void* p : {S->pf_x, S->pf_big, S->pf_q, S->pf_k, S->pf_v, S->pf_attn, (void*)S->pf_ws}) {
+    if (!p) continue;
+    cudaFree(p);
+    for (auto it = S->allocs.begin(); it != S->allocs.end(); ++it)
+      if (*it == p) { S->allocs.erase(it); break; }
+  }
+  S->pf_x = S->pf_big = S->pf_q = S->pf_k = S->pf_v = S->pf_attn = nullptr;
+  S->pf_ws = nullptr;
+  S->pf_rows = 0;
+  auto A = [&](void** p, int64_t bytes) { return dev_alloc(S->allocs, p, (size_t)bytes); };
+  RLT_TRY(A(&S->pf_x, rows * d * (int64_t)es));
+  RLT_TRY(A(&S->pf_big, rows * big_cols * (int64_t)es));
+  RLT_TRY(A(&S->pf_q, rows * d * (int64_t)es));
+  RLT_TRY(A(&S->pf_attn, rows * d * (int64_t)es));
+  if (!cache) {
+    RLT_TRY(A(&S->pf_k, rows * d * (int64_t)es));
+    RLT_TRY(A(&S->pf_v, rows * d * (int64_t)es));
+  }
+  if (c.dtype == RLT_DTYPE_BF16) {
+    size_t w = 0;
+    for (int M : {(int)(3 * d), (int)d, (int)(2 * F), (int)(2 * d * G)})
+      for (int K : {(int)d, (int)F}) w = std::max(w, gemm_tc_workspace_floats(M, K, (int)rows));
+    S->pf_ws_floats = w;
+    void* p = nullptr;
+    RLT_TRY(A(&p, (int64_t)w * 4));
+    S->pf_ws = static_cast<float*>(p);
+  }
+  S->pf_rows = rows;
+  S->pf_big_cols = big_cols;
+  return RLT_OK;
+}
+
+int32_t check_state(rlt_model* m, rlt_state* S) {
+  if (!m || !S) return fail(RLT_E_INVAL, "null model or state");
+  if (S->m != m) return fail(RLT_E_INVAL, "state belongs to another model");
+  if (S->version != m->version) return fail(RLT_E_STALE, "state was built under older weights");
+  RLT_CUDA(cudaSetDevice(m->device));
+  return RLT_OK;
+}
+
+// ------------------------------------------------------------------ schedules
+// Token-parallel encoder over T tokens of every sequence (eq. 2.1) and the
+// memory projection of eq. 2.2, chunked over sequences.
+template <typename T>
+int32_t encode_prefix_impl(rlt_model* m, rlt_state* S, const int32_t* tok, int32_t Tn, cudaStream_t st) {
+  const rlt_config& c = m->cfg;
+  const int d = c.d_model, H = c.n_heads, hd = m->hd, F = c.ffn, G = c.groups, L = c.n_layers;
+  const int is_bf16 = c.dtype == RLT_DTYPE_BF16;
+  const bool cache = (S->flags & RLT_STATE_ENCODER_CACHE) != 0;
+  RLT_TRY(ensure_prefill_ws(S, Tn));
+  const int64_t seqs_per_chunk = S->pf_rows / Tn;
+  for (int64_t b0 = 0; b0 < S->B; b0 += seqs_per_chunk) {
+    const int Bc = (int)std::min<int64_t>(seqs_per_chunk, S->B - b0);
+    const int64_t rows = (int64_t)Bc * Tn;
+    float* e0 = S->e + b0 * S->max_len * d;
+    const RowMap emap{d, Tn, (int64_t)S->max_len * d};
+    RLT_CUDA(embed<T>(tok + b0 * Tn, rows, Tn, Tn, static_cast<const T*>(m->emb), d, c.vocab, e0, emap, st));
+    for (int l = 0; l < L; ++l) {
+      const LayerW& w = m->layers[l];
+      RLT_CUDA(rmsnorm<T, T>(e0, emap, static_cast<const T*>(w.g_ea), rows, d, c.rms_eps, static_cast<T*>(S->pf_x), d, st));
+      RLT_TRY(gemm<T>(S, w.qkv, d, S->pf_x, d, 3 * d, (int)rows, d, EPI_STORE, epi_out(S->pf_big, plain_rows(3 * d), is_bf16),
+                      S->pf_ws, S->pf_ws_floats, st));
+      T* kdst;
+      T* vdst;
+      int64_t ld_tk;
+      if (cache) {
+        const int64_t lay = (int64_t)l * S->B * H * S->max_len * hd;
+        kdst = static_cast<T*>(S->ce_k) + lay + b0 * H * S->max_len * hd;
+        vdst = static_cast<T*>(S->ce_v) + lay + b0 * H * S->max_len * hd;
+        ld_tk = S->max_len;
+      } else {
+        kdst = static_cast<T*>(S->pf_k);
+        vdst = static_cast<T*>(S->pf_v);
+        ld_tk = Tn;
+      }
+      const T* qkv = static_cast<const T*>(S->pf_big);
+      RLT_CUDA((head_scatter<T, T>(qkv, 3 * d, 0, rows, Tn, 0, H, hd, 1, m->rope_cs, static_cast<T*>(S->pf_q), Tn, st)));
+      RLT_CUDA((head_scatter<T, T>(qkv, 3 * d, d, rows, Tn, 0, H, hd, 1, m->rope_cs, kdst, ld_tk, st)));
+      RLT_CUDA((head_scatter<T, T>(qkv, 3 * d, 2 * d, rows, Tn, 0, H, hd, 0, m->rope_cs, vdst, ld_tk, st)));
+      RLT_CUDA(causal_attn<T>(static_cast<const T*>(S->pf_q), kdst, vdst, Tn, ld_tk, Bc, H, hd, Tn,
+                              static_cast<T*>(S->pf_attn), d, st));
+      RLT_TRY(gemm<T>(S, w.wo, d, S->pf_attn, d, d, (int)rows, d, EPI_RESID, epi_out(e0, emap, 0), S->pf_ws,
+                      S->pf_ws_floats, st));
+      RLT_CUDA(rmsnorm<T, T>(e0, emap, static_cast<const T*>(w.g_ef), rows, d, c.rms_eps, static_cast<T*>(S->pf_x), d, st));
+      RLT_TRY(gemm<T>(S, w.w13, d, S->pf_x, d, 2 * F, (int)rows, d, EPI_SWIGLU, epi_out(S->pf_big, plain_rows(F), is_bf16),
+                      S->pf_ws, S->pf_ws_floats, st));
+      RLT_TRY(gemm<T>(S, w.w2, F, S->pf_big, F, d, (int)rows, F, EPI_RESID, epi_out(e0, emap, 0), S->pf_ws,
+                      S->pf_ws_floats, st));
+    }
+    // memory projection (eq. 2.2): n = RMSNorm_E(e); k^g = RoPE(W_K^g n), v^g = W_V^g n
+    RLT_CUDA(rmsnorm<T, T>(e0, emap, static_cast<const T*>(m->g_mem), rows, d, c.rms_eps, static_cast<T*>(S->pf_x), d, st));
+    RLT_TRY(gemm<T>(S, m->w_kvm, d, S->pf_x, d, 2 * d * G, (int)rows, d, EPI_STORE,
+                    epi_out(S->pf_big, plain_rows(2 * d * G), is_bf16), S->pf_ws, S->pf_ws_floats, st));
+    for (int g = 0; g < G; ++g) {
+      const int64_t grp = ((int64_t)g * S->B + b0) * H * S->max_len * hd;
+      const T* kv = static_cast<const T*>(S->pf_big);
+      RLT_CUDA((head_scatter<T, T>(kv, 2 * d * G, (int64_t)2 * d * g, rows, Tn, 0, H, hd, 1, m->rope_cs,
+                                   static_cast<T*>(S->mem_k) + grp, S->max_len, st)));
+      RLT_CUDA((head_scatter<T, T>(kv, 2 * d * G, (int64_t)2 * d * g + d, rows, Tn, 0, H, hd, 0, m->rope_cs,
+                                   static_cast<T*>(S->mem_v) + grp, S->max_len, st)));
+    }
+  }
+  S->n_enc = Tn;
+  return RLT_OK;
+}
+
+// Encoder step (eq. 2.8) for x_t, t = n_enc + 1, and the memory append.
+template <typename T>
+int32_t encode_step_impl(rlt_model* m, rlt_state* S, const int32_t* tok, cudaStream_t st) {
+  const rlt_config& c = m->cfg;
+  const int d = c.d_model, H = c.n_heads, hd = m->hd, F = c.ffn, G = c.groups, L = c.n_layers, B = S->B;
+  const int is_bf16 = c.dtype == RLT_DTYPE_BF16;
+  const int t = S->n_enc + 1;
+  float* et = S->e + (int64_t)(t - 1) * d;
+  const RowMap emap = plain_rows((int64_t)S->max_len * d);
+  RLT_CUDA(embed<T>(tok, B, 1, 1, static_cast<const T*>(m->emb), d, c.vocab, et, emap, st));
+  for (int l = 0; l < L; ++l) {
+    const LayerW& w = m->layers[l];
+    const int64_t lay = (int64_t)l * B * H * S->max_len * hd;
+    T* ck = static_cast<T*>(S->ce_k) + lay;
+    T* cv = static_cast<T*>(S->ce_v) + lay;
+    RLT_CUDA(rmsnorm<T, T>(et, emap, static_cast<const T*>(w.g_ea), B, d, c.rms_eps, static_cast<T*>(S->xb), d, st));
+    RLT_TRY(gemm<T>(S, w.qkv, d, S->xb, d, 3 * d, B, d, EPI_STORE, epi_out(S->qkv, plain_rows(S->ld_qkv), 0), S->gemm_ws,
+                    S->gemm_ws_floats, st));
+    RLT_CUDA((head_scatter<float, T>(S->qkv, S->ld_qkv, d, B, 1, t - 1, H, hd, 1, m->rope_cs, ck, S->max_len, st)));
+    RLT_CUDA((head_scatter<float, T>(S->qkv, S->ld_qkv, 2 * d, B, 1, t - 1, H, hd, 0, m->rope_cs, cv, S->max_len, st)));
+    prof_begin(m, st);
+    RLT_CUDA(prefix_attn<T>(S->qkv, S->ld_qkv, ck, cv, S->max_len, B, H, hd, t, t - 1, m->rope_cs,
+                            static_cast<T*>(S->attn), d, S->attn_ws, S->attn_ws_floats, st));
+    prof_end(m, st, 0, (double)B * H * t * hd * 2 * m->esz);
+    RLT_TRY(gemm<T>(S, w.wo, d, S->attn, d, d, B, d, EPI_RESID, epi_out(et, emap, 0), S->gemm_ws, S->gemm_ws_floats, st));
+    RLT_CUDA(rmsnorm<T, T>(et, emap, static_cast<const T*>(w.g_ef), B, d, c.rms_eps, static_cast<T*>(S->xb), d, st));
+    RLT_TRY(gemm<T>(S, w.w13, d, S->xb, d, 2 * F, B, d, EPI_SWIGLU, epi_out(S->hbuf, plain_rows(F), is_bf16), S->gemm_ws,
+                    S->gemm_ws_floats, st));
+    RLT_TRY(gemm<T>(S, w.w2, F, S->hbuf, F, d, B, F, EPI_RESID, epi_out(et, emap, 0), S->gemm_ws, S->gemm_ws_floats, st));
+  }
+  RLT_CUDA(rmsnorm<T, T>(et, emap, static_cast<const T*>(m->g_mem), B, d, c.rms_eps, static_cast<T*>(S->xb), d, st));
+  RLT_TRY(gemm<T>(S, m->w_kvm, d, S->xb, d, 2 * d * G, B, d, EPI_STORE, epi_out(S->qkv, plain_rows(S->ld_qkv), 0),
+                  S->gemm_ws, S->gemm_ws_floats, st));
+  for (int g = 0; g < G; ++g) {
+    const int64_t grp = (int64_t)g * B * H * S->max_len * hd;
+    RLT_CUDA((head_scatter<float, T>(S->qkv, S->ld_qkv, (int64_t)2 * d * g, B, 1, t - 1, H, hd, 1, m->rope_cs,
+                                     static_cast<T*>(S->mem_k) + grp, S->max_len, st)));
+    RLT_CUDA((head_scatter<float, T>(S->qkv, S->ld_qkv, (int64_t)2 * d * g + d, B, 1, t - 1, H, hd, 0, m->rope_cs,
+                                     static_cast<T*>(S->mem_v) + grp, S->max_len, st)));
+  }
+  S->n_enc = t;
+  return RLT_OK;
+}
+
+// One decoder transition H_t = D_phi(Merge(e_t, s_{t-1}); M_<=t, C^D_{t-1}, t)
+// (eqs. 2.4-2.5, 2.9-2.16) for t = n_dec + 1.  s is updated in place: it
+// holds u_t after the merge, then z^l after every block, and s_t at the end.
+template <typename T>
+int32_t transition_impl(rlt_model* m, rlt_state* S, cudaStream_t st) {
+  const rlt_config& c = m->cfg;
+  const int d = c.d_model, H = c.n_heads, hd = m->hd, F = c.ffn, L = c.n_layers, B = S->B, W = c.window;
+  const int is_bf16 = c.dtype == RLT_DTYPE_BF16;
+  const int t = S->n_dec + 1;
+  const float* et = S->e + (int64_t)(t - 1) * d;
+  const RowMap emap = plain_rows((int64_t)S->max_len * d);
+  const RowMap srow = plain_rows(d);
+  // merge
+  RLT_CUDA((merge_prep<T, T>(et, emap, S->s, static_cast<const T*>(m->g_merge), B, d, c.rms_eps, c.merge_kind,
+                             static_cast<T*>(S->xb), st)));
+  if (c.merge_kind == RLT_MERGE_PAPER) {
+    EpiParams g = epi_out(S->gate, srow, 0);
+    g.bias = m->b_gate;
+    g.bias_bf16 = is_bf16;
+    RLT_TRY(gemm<T>(S, m->w_gate, 2 * d, S->xb, 2 * d, d, B, 2 * d, EPI_GATE, g, S->gemm_ws, S->gemm_ws_floats, st));
+    EpiParams u = epi_out(S->s, srow, 0);
+    u.aux0 = et;
+    u.aux0_map = emap;
+    u.aux1 = S->gate;
+    u.ld_aux1 = d;
+    u.alpha = c.alpha;
+    RLT_TRY(gemm<T>(S, m->w_state, d, off(S->xb, d, m->esz), 2 * d, d, B, d, EPI_MERGE, u, S->gemm_ws,
+                    S->gemm_ws_floats, st));
+  } else {
+    EpiParams u = epi_out(S->s, srow, 0);
+    u.aux0 = et;
+    u.aux0_map = emap;
+    RLT_TRY(gemm<T>(S, m->w_gate, 2 * d, S->xb, 2 * d, d, B, 2 * d, EPI_CONVEX, u, S->gemm_ws, S->gemm_ws_floats, st));
+  }
+  const int n_ring = std::min(t - 1, W - 1);
+  for (int l = 0; l < L; ++l) {
+    const LayerW& w = m->layers[l];
+    const int grp = c.groups == 1 ? 0 : l;
+    // SWA sublayer (eqs. 2.12-2.14)
+    RLT_CUDA(rmsnorm<T, T>(S->s, srow, static_cast<const T*>(w.g_dsa), B, d, c.rms_eps, static_cast<T*>(S->xb), d, st));
+    RLT_TRY(gemm<T>(S, w.dqkv, d, S->xb, d, 3 * d, B, d, EPI_STORE, epi_out(S->qkv, plain_rows(3 * d), 0), S->gemm_ws,
+                    S->gemm_ws_floats, st));
+    const int64_t rlay = (int64_t)l * B * H * (W > 1 ? W - 1 : 0) * hd;
+    T* rk = W > 1 ? static_cast<T*>(S->ring_k) + rlay : nullptr;
+    T* rv = W > 1 ? static_cast<T*>(S->ring_v) + rlay : nullptr;
+    prof_begin(m, st);
+    RLT_CUDA(swa_attn<T>(S->qkv, 3 * d, rk, rv, B, H, hd, t, W, m->rope_cs, static_cast<T*>(S->attn), d, st));
+    prof_end(m, st, 1, (double)B * H * hd * m->esz * (2.0 * n_ring + (W > 1 ? 2.0 : 0.0)));
+    RLT_TRY(gemm<T>(S, w.dwo, d, S->attn, d, d, B, d, EPI_RESID, epi_out(S->s, srow, 0), S->gemm_ws, S->gemm_ws_floats, st));
+    // cross-attention to M^{g(l)}_{<=t} (eq. 2.15)
+    RLT_CUDA(rmsnorm<T, T>(S->s, srow, static_cast<const T*>(w.g_dmem), B, d, c.rms_eps, static_cast<T*>(S->xb), d, st));
+    RLT_TRY(gemm<T>(S, w.wq_mem, d, S->xb, d, d, B, d, EPI_STORE, epi_out(S->qkv, plain_rows(d), 0), S->gemm_ws,
+                    S->gemm_ws_floats, st));
+    const int64_t mg = (int64_t)grp * B * H * S->max_len * hd;
+    prof_begin(m, st);
+    RLT_CUDA(prefix_attn<T>(S->qkv, d, static_cast<const T*>(S->mem_k) + mg, static_cast<const T*>(S->mem_v) + mg,
+                            S->max_len, B, H, hd, t, t - 1, m->rope_cs, static_cast<T*>(S->attn), d, S->attn_ws,
+                            S->attn_ws_floats, st));
+    prof_end(m, st, 0, (double)B * H * t * hd * 2 * m->esz);
+    RLT_TRY(gemm<T>(S, w.wo_mem, d, S->attn, d, d, B, d, EPI_RESID, epi_out(S->s, srow, 0), S->gemm_ws,
+                    S->gemm_ws_floats, st));
+    // FFN (eq. 2.16)
+    RLT_CUDA(rmsnorm<T, T>(S->s, srow, static_cast<const T*>(w.g_dffn), B, d, c.rms_eps, static_cast<T*>(S->xb), d, st));
+    RLT_TRY(gemm<T>(S, w.dw13, d, S->xb, d, 2 * F, B, d, EPI_SWIGLU, epi_out(S->hbuf, plain_rows(F), is_bf16),
+                    S->gemm_ws, S->gemm_ws_floats, st));
+    RLT_TRY(gemm<T>(S, w.dw2, F, S->hbuf, F, d, B, F, EPI_RESID, epi_out(S->s, srow, 0), S->gemm_ws, S->gemm_ws_floats, st));
+  }
+  S->n_dec = t;
+  return RLT_OK;
+}
+
+// Readout (eq. 2.6) of s_t: logits = W_o RMSNorm_o(s_t), then the teacher
+// log-prob and/or the behaviour sample.
+template <typename T>
+int32_t readout_impl(rlt_model* m, rlt_state* S, const int32_t* next, int64_t next_stride, float* logp, int64_t ld_logp,
+                     const rlt_sampling* samp, const rlt_readout_out* out, cudaStream_t st) {
+  const rlt_config& c = m->cfg;
+  const int d = c.d_model, V = c.vocab, B = S->B;
+  RLT_CUDA(rmsnorm<T, T>(S->s, plain_rows(d), static_cast<const T*>(m->g_out), B, d, c.rms_eps, static_cast<T*>(S->xb), d, st));
+  RLT_TRY(gemm<T>(S, m->w_out, d, S->xb, d, V, B, d, EPI_STORE, epi_out(S->logits, plain_rows(V), 0), S->gemm_ws,
+                  S->gemm_ws_floats, st));
+  if (next && logp) RLT_CUDA(logp_gather(S->logits, B, V, next, next_stride, logp, ld_logp, st));
+  if (samp)
+    RLT_CUDA(sample_topk(S->logits, B, V, samp->temperature, samp->top_k, samp->seed, (uint32_t)S->n_dec,
+                         out ? out->sampled : nullptr, out ? out->logp_sampled : nullptr, out ? out->logmu : nullptr, st));
+  if (out && out->logits) RLT_CUDA(copy_f32(out->logits, S->logits, (int64_t)B * V, st));
+  return RLT_OK;
+}
+
+#define RLT_DISPATCH(m, fn, ...) \
+  ((m)->cfg.dtype == RLT_DTYPE_BF16 ? fn<bf16>(__VA_ARGS__) : fn<float>(__VA_ARGS__))
+
+int32_t check_sampling(const rlt_sampling* samp, const rlt_readout_out* out) {
+  if (!samp) return RLT_OK;
+  if (!(samp->temperature > 0.f) || samp->top_k < 1 || samp->top_k > 256)
+    return fail(RLT_E_INVAL, "sampler needs temperature > 0 and 1 <= top_k <= 256");
+  if (!out || !(out->sampled || out->logmu || out->logp_sampled)) return fail(RLT_E_INVAL, "sampler without outputs");
+  return RLT_OK;
+}
+
+}  // namespace
+
+// ====================================================================== C ABI
+extern "C" {
+
+int32_t rlt_init_weights(const rlt_config* cfg, uint64_t seed, rlt_model** out) {
+  if (!out) return fail(RLT_E_INVAL, "null output");
+  *out = nullptr;
+  RLT_TRY(validate(cfg));
+  rlt_model* m = new rlt_model();
+  m->cfg = *cfg;
+  m->hd = cfg->d_model / cfg->n_heads;
+  m->esz = cfg->dtype == RLT_DTYPE_BF16 ? 2 : 4;
+  cudaGetDevice(&m->device);
+  int32_t r = build_model(m);
+  if (r == RLT_OK) r = ensure_rope(m, 4096);
+  if (r == RLT_OK) r = RLT_DISPATCH(m, init_views, m, seed);
+  if (r != RLT_OK) {
+    free_all(m->allocs);
+    delete m;
+    return r;
+  }
+  *out = m;
+  return ok();
+}
+
+int32_t rlt_tensor_info(const rlt_model* m, const char* name, int64_t* rows, int64_t* cols, int32_t* sid) {
+  if (!m || !name) return fail(RLT_E_INVAL, "null argument");
+  auto it = m->views.find(name);
+  if (it == m->views.end()) return fail(RLT_E_INVAL, std::string("unknown tensor ") + name);
+  if (rows) *rows = it->second.rows;
+  if (cols) *cols = it->second.cols;
+  if (sid) *sid = it->second.sid;
+  return ok();
+}
+
+int32_t rlt_load_weights(rlt_model* m, const char* name, const void* host, size_t bytes) {
+  if (!m || !name || !host) return fail(RLT_E_INVAL, "null argument");
+  auto it = m->views.find(name);
+  if (it == m->views.end()) return fail(RLT_E_INVAL, std::string("unknown tensor ") + name);
+  const View& v = it->second;
+  if (bytes != (size_t)(v.rows * v.cols) * m->esz) return fail(RLT_E_INVAL, "size mismatch for " + std::string(name));
+  RLT_CUDA(cudaSetDevice(m->device));
+  RLT_CUDA(cudaMemcpy2D(v.base, v.pitch * m->esz, host, v.cols * m->esz, v.cols * m->esz, v.rows, cudaMemcpyHostToDevice));
+  m->version += 1;
+  return ok();
+}
+
+int32_t rlt_get_weights(const rlt_model* m, const char* name, void* host, size_t bytes) {
+  if (!m || !name || !host) return fail(RLT_E_INVAL, "null argument");
+  auto it = m->views.find(name);
+  if (it == m->views.end()) return fail(RLT_E_INVAL, std::string("unknown tensor ") + name);
+  const View& v = it->second;
+  if (bytes != (size_t)(v.rows * v.cols) * m->esz) return fail(RLT_E_INVAL, "size mismatch for " + std::string(name));
+  RLT_CUDA(cudaSetDevice(m->device));
+  RLT_CUDA(cudaMemcpy2D(host, v.cols * m->esz, v.base, v.pitch * m->esz, v.cols * m->esz, v.rows, cudaMemcpyDeviceToHost));
+  return ok();
+}
+
+int32_t rlt_state_free(rlt_state* s);
+
+int32_t rlt_model_free(rlt_model* m) {
+  if (!m) return ok();
+  cudaSetDevice(m->device);
+  cudaDeviceSynchronize();
+  if (m->replay) rlt_state_free(m->replay);
+  for (cudaEvent_t e : m->prof.ev) cudaEventDestroy(e);
+  free_all(m->allocs);
+  delete m;
+  return ok();
+}
+
+int32_t rlt_state_create(rlt_model* m, int32_t batch, int32_t max_len, int32_t flags, rlt_state** out) {
+  if (!m || !out) return fail(RLT_E_INVAL, "null argument");
+  *out = nullptr;
+  if (flags & ~RLT_STATE_ENCODER_CACHE) return fail(RLT_E_INVAL, "unknown flags");
+  RLT_CUDA(cudaSetDevice(m->device));
+  rlt_state* S = nullptr;
+  RLT_TRY(make_state(m, batch, max_len, flags, &S));
+  int32_t r = RLT_DISPATCH(m, reset_state, S, (cudaStream_t)0);
+  if (r == RLT_OK) {
+    cudaError_t e = cudaStreamSynchronize(0);
+    if (e != cudaSuccess) r = fail(RLT_E_CUDA, cudaGetErrorString(e));
+  }
+  if (r != RLT_OK) {
+    free_all(S->allocs);
+    delete S;
+    return r;
+  }
+  *out = S;
+  return ok();
+}
+
+int32_t rlt_state_free(rlt_state* s) {
+  if (!s) return ok();
+  cudaSetDevice(s->m->device);
+  cudaDeviceSynchronize();
+  free_all(s->allocs);
+  delete s;
+  return ok();
+}
+
+int32_t rlt_state_reset(rlt_state* s, void* stream) {
+  if (!s) return fail(RLT_E_INVAL, "null state");
+  RLT_CUDA(cudaSetDevice(s->m->device));
+  return RLT_DISPATCH(s->m, reset_state, s, (cudaStream_t)stream);
+}
+
+int32_t rlt_state_info_get(const rlt_state* s, rlt_state_info* out) {
+  if (!s || !out) return fail(RLT_E_INVAL, "null argument");
+  const int Wm1 = s->m->cfg.window - 1;
+  out->batch = s->B;
+  out->max_len = s->max_len;
+  out->n_enc = s->n_enc;
+  out->n_dec = s->n_dec;
+  out->ring_valid = std::min(s->n_dec, Wm1);
+  out->ring_head = Wm1 > 0 ? s->n_dec % Wm1 : 0;
+  out->has_encoder_cache = (s->flags & RLT_STATE_ENCODER_CACHE) ? 1 : 0;
+  out->model_version = s->version;
+  return ok();
+}
+
+int32_t rlt_state_read(const rlt_state* s, int32_t what, int32_t index, void* host, size_t bytes) {
+  if (!s || !host) return fail(RLT_E_INVAL, "null argument");
+  const rlt_model* m = s->m;
+  const rlt_config& c = m->cfg;
+  const int64_t d = c.d_model, B = s->B, Wm1 = c.window - 1;
+  const void* src = nullptr;
+  size_t n = 0;
+  switch (what) {
+    case RLT_READ_S: src = s->s; n = (size_t)(B * d) * 4; break;
+    case RLT_READ_E: src = s->e; n = (size_t)(B * s->max_len * d) * 4; break;
+    case RLT_READ_RING_K:
+    case RLT_READ_RING_V:
+      if (index < 0 || index >= c.n_layers || Wm1 == 0) return fail(RLT_E_INVAL, "bad layer or empty ring");
+      n = (size_t)(B * Wm1 * d) * m->esz;
+      src = off(what == RLT_READ_RING_K ? s->ring_k : s->ring_v, (int64_t)index * B * Wm1 * d, m->esz);
+      break;
+    case RLT_READ_MEM_K:
+    case RLT_READ_MEM_V:
+      if (index < 0 || index >= c.groups) return fail(RLT_E_INVAL, "bad group");
+      n = (size_t)(B * s->max_len * d) * m->esz;
+      src = off(what == RLT_READ_MEM_K ? s->mem_k : s->mem_v, (int64_t)index * B * s->max_len * d, m->esz);
+      break;
+    case RLT_READ_ENC_K:
+    case RLT_READ_ENC_V:
+      if (!(s->flags & RLT_STATE_ENCODER_CACHE) || index < 0 || index >= c.n_layers)
+        return fail(RLT_E_INVAL, "no encoder cache or bad layer");
+      n = (size_t)(B * s->max_len * d) * m->esz;
+      src = off(what == RLT_READ_ENC_K ? s->ce_k : s->ce_v, (int64_t)index * B * s->max_len * d, m->esz);
+      break;
+    default: return fail(RLT_E_INVAL, "unknown component");
+  }
+  if (bytes != n) return fail(RLT_E_INVAL, "size mismatch: need " + std::to_string(n));
+  RLT_CUDA(cudaSetDevice(m->device));
+  RLT_CUDA(cudaDeviceSynchronize());
+  RLT_CUDA(cudaMemcpy(host, src, n, cudaMemcpyDeviceToHost));
+  return ok();
+}
+
+int32_t rlt_encode_prefix(rlt_model* m, rlt_state* s, const int32_t* tok_dev, int32_t T, void* stream) {
+  RLT_TRY(check_state(m, s));
+  if (!tok_dev || T <= 0) return fail(RLT_E_INVAL, "need tokens and T > 0");
+  if (s->n_enc != 0) return fail(RLT_E_STATE, "token-parallel encoding starts from an empty encoder");
+  if (T > s->max_len) return fail(RLT_E_CAPACITY, "T exceeds max_len");
+  return RLT_DISPATCH(m, encode_prefix_impl, m, s, tok_dev, T, (cudaStream_t)stream);
+}
+
+int32_t rlt_readout(rlt_model* m, rlt_state* s, const int32_t* next_dev, const rlt_sampling* samp,
+                    const rlt_readout_out* out, void* stream) {
+  RLT_TRY(check_state(m, s));
+  if (s->n_dec < 1) return fail(RLT_E_STATE, "readout needs at least one transition");
+  RLT_TRY(check_sampling(samp, out));
+  return RLT_DISPATCH(m, readout_impl, m, s, next_dev, (int64_t)1, out ? out->logp : nullptr, (int64_t)1, samp, out,
+                      (cudaStream_t)stream);
+}
+
+int32_t rlt_decoder_step(rlt_model* m, rlt_state* s, const int32_t* tok_dev, const int32_t* next_dev,
+                         const rlt_sampling* samp, const rlt_readout_out* out, void* stream) {
+  RLT_TRY(check_state(m, s));
+  RLT_TRY(check_sampling(samp, out));
+  const int t = s->n_dec + 1;
+  if (t > s->max_len) return fail(RLT_E_CAPACITY, "position would pass max_len");
+  cudaStream_t st = (cudaStream_t)stream;
+  if (s->n_enc < t) {
+    if (!(s->flags & RLT_STATE_ENCODER_CACHE)) return fail(RLT_E_STATE, "x_t not encoded and the state has no encoder cache");
+    if (!tok_dev) return fail(RLT_E_INVAL, "x_t must be given when it is not yet encoded");
+    RLT_TRY(RLT_DISPATCH(m, encode_step_impl, m, s, tok_dev, st));
+  }
+  RLT_TRY(RLT_DISPATCH(m, transition_impl, m, s, st));
+  if (next_dev || samp || (out && out->logits))
+    RLT_TRY(RLT_DISPATCH(m, readout_impl, m, s, next_dev, (int64_t)1, out ? out->logp : nullptr, (int64_t)1, samp, out, st));
+  return ok();
+}
+
+int32_t rlt_prefill(rlt_model* m, rlt_state* s, const int32_t* tok_dev, int32_t T, float* logp_dev, void* stream) {
+  RLT_TRY(check_state(m, s));
+  if (!tok_dev || T <= 0) return fail(RLT_E_INVAL, "need tokens and T > 0");
+  if (s->n_enc != 0 || s->n_dec != 0) return fail(RLT_E_STATE, "prefill starts from H_0");
+  if (T > s->max_len) return fail(RLT_E_CAPACITY, "T exceeds max_len");
+  cudaStream_t st = (cudaStream_t)stream;
+  RLT_TRY(RLT_DISPATCH(m, encode_prefix_impl, m, s, tok_dev, T, st));
+  for (int t = 1; t <= T; ++t) {
+    RLT_TRY(RLT_DISPATCH(m, transition_impl, m, s, st));
+    if (logp_dev && t < T)
+      RLT_TRY(RLT_DISPATCH(m, readout_impl, m, s, tok_dev + t, (int64_t)T, logp_dev + (t - 1), (int64_t)(T - 1),
+                           (const rlt_sampling*)nullptr, (const rlt_readout_out*)nullptr, st));
+  }
+  return ok();
+}
+
+int32_t rlt_replay_logprobs(rlt_model* m, const int32_t* tok_dev, int32_t B, int32_t S, float* logp_dev, void* stream) {
+  if (!m || !tok_dev || !logp_dev) return fail(RLT_E_INVAL, "null argument");
+  if (B <= 0 || S < 2) return fail(RLT_E_INVAL, "need B > 0 and S >= 2");
+  RLT_CUDA(cudaSetDevice(m->device));
+  if (m->replay && (m->replay->B != B || m->replay->max_len < S)) {
+    rlt_state_free(m->replay);
+    m->replay = nullptr;
+  }
+  if (!m->replay) RLT_TRY(make_state(m, B, S, 0, &m->replay));
+  rlt_state* st_ = m->replay;
+  cudaStream_t st = (cudaStream_t)stream;
+  RLT_TRY(RLT_DISPATCH(m, reset_state, st_, st));
+  RLT_TRY(RLT_DISPATCH(m, encode_prefix_impl, m, st_, tok_dev, S, st));
+  for (int t = 1; t <= S - 1; ++t) {
+    RLT_TRY(RLT_DISPATCH(m, transition_impl, m, st_, st));
+    RLT_TRY(RLT_DISPATCH(m, readout_impl, m, st_, tok_dev + t, (int64_t)S, logp_dev + (t - 1), (int64_t)(S - 1),
+                         (const rlt_sampling*)nullptr, (const rlt_readout_out*)nullptr, st));
+  }
+  return ok();
+}
+
+int32_t rlt_op_linear(const void* w_dev, const void* x_dev, float* y_dev, int32_t M, int32_t N, int32_t K,
+                      int32_t dtype, int32_t use_tensor_cores, void* stream) {
+  if (!w_dev || !x_dev || !y_dev || M <= 0 || N <= 0 || K <= 0) return fail(RLT_E_INVAL, "bad linear arguments");
+  cudaStream_t st = (cudaStream_t)stream;
+  const EpiParams ep = epi_out(y_dev, plain_rows(M), 0);
+  if (dtype == RLT_DTYPE_F32) {
+    if (use_tensor_cores) return fail(RLT_E_INVAL, "the tensor-core path takes bf16 operands");
+    RLT_CUDA(gemm_simt<float, float>(static_cast<const float*>(w_dev), K, static_cast<const float*>(x_dev), K, M, N, K,
+                                     EPI_STORE, ep, st));
+    return ok();
+  }
+  if (dtype != RLT_DTYPE_BF16) return fail(RLT_E_INVAL, "dtype");
+  if (!use_tensor_cores) {
+    RLT_CUDA(gemm_simt<bf16, bf16>(static_cast<const bf16*>(w_dev), K, static_cast<const bf16*>(x_dev), K, M, N, K,
+                                   EPI_STORE, ep, st));
+    return ok();
+  }
+  if (M % 128 || K % 64) return fail(RLT_E_INVAL, "tensor-core path needs M % 128 == 0 and K % 64 == 0");
+  const size_t ws = gemm_tc_workspace_floats(M, K, N);
+  float* w = nullptr;
+  if (ws) {
+    cudaError_t e = cudaMalloc(&w, ws * sizeof(float));
+    if (e != cudaSuccess) return fail(RLT_E_OOM, "split-K workspace");
+  }
+  cudaError_t e = gemm_tc(static_cast<const bf16*>(w_dev), K, static_cast<const bf16*>(x_dev), K, M, N, K, EPI_STORE,
+                          ep, w, ws, st);
+  if (w) {
+    cudaStreamSynchronize(st);
+    cudaFree(w);
+  }
+  if (e != cudaSuccess) return fail(RLT_E_CUDA, std::string("gemm_tc: ") + cudaGetErrorString(e));
+  return ok();
+}
+
+int32_t rlt_op_sample(const float* logits_dev, int32_t B, int32_t V, const rlt_sampling* samp, uint32_t t,
+                      int32_t* token_dev, float* logp_dev, float* logmu_dev, void* stream) {
+  if (!logits_dev || !samp || !token_dev || B <= 0 || V <= 0) return fail(RLT_E_INVAL, "bad sample arguments");
+  if (!(samp->temperature > 0.f) || samp->top_k < 1 || samp->top_k > 256)
+    return fail(RLT_E_INVAL, "sampler needs temperature > 0 and 1 <= top_k <= 256");
+  RLT_CUDA(sample_topk(logits_dev, B, V, samp->temperature, samp->top_k, samp->seed, t, token_dev, logp_dev, logmu_dev,
+                       (cudaStream_t)stream));
+  return ok();
+}
+
+int32_t rlt_last_error(char* buf, size_t n) {
+  if (buf && n) {
+    std::strncpy(buf, t_err.c_str(), n - 1);
+    buf[n - 1] = 0;
+  }
+  return t_err_code;
+}
+
+int32_t rlt_check_device(void) {
+  RLT_CUDA(cudaDeviceSynchronize());
+  int v = 0;
+  RLT_CUDA(cudaMemcpyFromSymbol(&v, rlt::g_device_error, sizeof(int)));
+  if (v) {
+    int z = 0;
+    RLT_CUDA(cudaMemcpyToSymbol(rlt::g_device_error, &z, sizeof(int)));
+    return fail(RLT_E_CUDA, v == 1 ? "a bounded device wait ran out" : "a token id was out of range");
+  }
+  return ok();
+}
+
+int32_t rlt_kernel_launches(int64_t* count) {
+  if (!count) return fail(RLT_E_INVAL, "null argument");
+  *count = launch_count();
+  return ok();
+}
+
+int32_t rlt_profile_enable(rlt_model* m, int32_t on) {
+  if (!m) return fail(RLT_E_INVAL, "null model");
+  m->prof.on = on != 0;
+  m->prof.used = 0;
+  m->prof.kind.clear();
+  m->prof.bytes[0] = m->prof.bytes[1] = 0;
+  m->prof.launches[0] = m->prof.launches[1] = 0;
+  return ok();
+}
+
+int32_t rlt_profile_read(rlt_model* m, int32_t kind, double* ms, int64_t* launches, double* bytes) {
+  if (!m || kind < 0 || kind > 1) return fail(RLT_E_INVAL, "bad argument");
+  RLT_CUDA(cudaSetDevice(m->device));
+  RLT_CUDA(cudaDeviceSynchronize());
+  double total = 0;
+  for (size_t i = 0; i + 1 < m->prof.used; i += 2) {
+    if (m->prof.kind[i / 2] != kind) continue;
+    float x = 0;
+    RLT_CUDA(cudaEventElapsedTime(&x, m->prof.ev[i], m->prof.ev[i + 1]));
+    total += x;
+  }
+  if (ms) *ms = total;
+  if (launches) *launches = m->prof.launches[kind];
+  if (bytes) *bytes = m->prof.bytes[kind];
+  return ok();
+}
+
+}  // extern "C"
