@@ -84,6 +84,29 @@ def step_roofline(w: dict, kind: str, peaks: dict) -> dict:
     return {"bound_ms": total * 1e3, "decoder_transitions": dec_steps}
 
 
+# ---------------------------------------------------------------- sharding
+def shard_tokens(w: dict, rank: int, world: int) -> np.ndarray:
+    """Rank `rank`'s share of the global batch: the global batch holds
+    world * B sequences drawn from the workload's seed; rank r owns rows
+    [r*B, (r+1)*B).  Sequences are independent (report §4.1), so no data
+    moves between ranks."""
+    B = w["batch"]
+    length = w["prompt"]
+    g = synth.tokens(w, batch=world * B, length=length)
+    return np.ascontiguousarray(g[rank * B:(rank + 1) * B])
+
+
+def max_over_ranks(ms: float, world: int, device=None) -> float:
+    """Step time of the job = the slowest rank's."""
+    if world <= 1:
+        return ms
+    import torch
+    import torch.distributed as dist
+    t = torch.tensor([ms], dtype=torch.float64, device=device)
+    dist.all_reduce(t, op=dist.ReduceOp.MAX)
+    return float(t.item())
+
+
 # ---------------------------------------------------------------- clocks
 class ClockSampler:
     FIELDS = ("index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
@@ -167,7 +190,7 @@ def run_gpu(args, w: dict, kind: str, peaks: dict, rank: int, world: int) -> dic
 
     if kind == "replay":
         S = w["prompt"]
-        tok_host = torch.from_numpy(synth.tokens(w, seed=w["data_seed"] + 7919 * rank)).pin_memory()
+        tok_host = torch.from_numpy(shard_tokens(w, rank, world)).pin_memory()
         tok = tok_host.cuda()
         logp = torch.empty(B, S - 1, device=dev)
         logp_host = torch.empty(B, S - 1).pin_memory()
@@ -185,7 +208,7 @@ def run_gpu(args, w: dict, kind: str, peaks: dict, rank: int, world: int) -> dic
     else:
         T, n_gen = w["prompt"], w["gen"]
         state = rlt.rlt_state_create(model, B, T + n_gen, rlt.STATE_ENCODER_CACHE)
-        tok_host = torch.from_numpy(synth.tokens(w, seed=w["data_seed"] + 7919 * rank)).pin_memory()
+        tok_host = torch.from_numpy(shard_tokens(w, rank, world)).pin_memory()
         tok = tok_host.cuda()
         ids = torch.zeros(n_gen, B, dtype=torch.int32, device=dev)
         lmu = torch.zeros(n_gen, B, device=dev)
@@ -227,11 +250,7 @@ def run_gpu(args, w: dict, kind: str, peaks: dict, rank: int, world: int) -> dic
         e1.record(stream)
         torch.cuda.synchronize()
         launches = rlt.rlt_kernel_launches() - n0
-        ms = e0.elapsed_time(e1)
-        if world > 1:
-            t = torch.tensor([ms], device=dev)
-            dist.all_reduce(t, op=dist.ReduceOp.MAX)
-            ms = t.item()
+        ms = max_over_ranks(e0.elapsed_time(e1), world, dev)
         barrier()
         return ms, launches
 

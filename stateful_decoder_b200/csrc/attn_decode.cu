@@ -105,6 +105,7 @@ __global__ void __launch_bounds__(kThreads) swa_attn_kernel(const float* __restr
                                                             KT* ring_v, int H, int t, int W,
                                                             const float* __restrict__ rope_cs, KT* out,
                                                             int64_t ld_out, float scale_log2) {
+  griddep_enter();
   constexpr int LPK = HD / 8, KPW = 32 / LPK, NKG = (kThreads / 32) * KPW, HALF = HD / 2;
   extern __shared__ float sm[];
   float* sq = sm;            // rotated, scaled query
@@ -181,6 +182,7 @@ __global__ void __launch_bounds__(kThreads) prefix_attn_kernel(const float* __re
                                                                const float* __restrict__ rope_cs, KT* out,
                                                                int64_t ld_out, float* ws, int nchunks,
                                                                float scale_log2) {
+  griddep_enter();
   constexpr int LPK = HD / 8, KPW = 32 / LPK, NKG = (kThreads / 32) * KPW, HALF = HD / 2;
   extern __shared__ float sm[];
   float* sq = sm;
@@ -237,6 +239,7 @@ __global__ void __launch_bounds__(kThreads) prefix_attn_kernel(const float* __re
 // Combines the chunk partials of one (sequence, head) in chunk order.
 template <typename KT, int HD>
 __global__ void prefix_combine_kernel(const float* __restrict__ ws, int H, int nchunks, KT* out, int64_t ld_out) {
+  griddep_enter();
   const int h = blockIdx.x, b = blockIdx.y;
   const float* p = ws + ((int64_t)b * H + h) * nchunks * (HD + 2);
   float mx = -INFINITY;
@@ -265,9 +268,11 @@ cudaError_t swa_launch(const float* qkv, int64_t ld_qkv, KT* rk, KT* rv, int B, 
     if (e != cudaSuccess) return e;
   }
   const float scale_log2 = 1.4426950408889634f / sqrtf((float)HD);
-  swa_attn_kernel<KT, HD><<<dim3(H, B), kThreads, smem, st>>>(qkv, ld_qkv, rk, rv, H, t, W, rope_cs, out, ld_out,
+  {
+    const cudaError_t e_l = launch_pdl(swa_attn_kernel<KT, HD>, dim3(dim3(H, B)), dim3(kThreads), smem, st, qkv, ld_qkv, rk, rv, H, t, W, rope_cs, out, ld_out,
                                                                scale_log2);
-  note_launch();
+    if (e_l != cudaSuccess) return e_l;
+  }
   return cudaGetLastError();
 }
 
@@ -279,13 +284,17 @@ cudaError_t prefix_launch(const float* q, int64_t ld_q, const KT* k, const KT* v
   if (nchunks > 1 && (!ws || ws_floats < (size_t)B * H * nchunks * (HD + 2))) return cudaErrorInvalidValue;
   const size_t smem = sizeof(float) * (HD + nkg_of<HD>() * HD + kPrefixChunk);
   const float scale_log2 = 1.4426950408889634f / sqrtf((float)HD);
-  prefix_attn_kernel<KT, HD><<<dim3(nchunks, H, B), kThreads, smem, st>>>(q, ld_q, k, v, ld_t, H, n, qpos, rope_cs,
+  {
+    const cudaError_t e_l = launch_pdl(prefix_attn_kernel<KT, HD>, dim3(dim3(nchunks, H, B)), dim3(kThreads), smem, st, q, ld_q, k, v, ld_t, H, n, qpos, rope_cs,
                                                                           out, ld_out, ws, nchunks, scale_log2);
-  note_launch();
+    if (e_l != cudaSuccess) return e_l;
+  }
   cudaError_t e = cudaGetLastError();
   if (e != cudaSuccess || nchunks == 1) return e;
-  prefix_combine_kernel<KT, HD><<<dim3(H, B), HD < 128 ? HD : 128, 0, st>>>(ws, H, nchunks, out, ld_out);
-  note_launch();
+  {
+    const cudaError_t e_l = launch_pdl(prefix_combine_kernel<KT, HD>, dim3(dim3(H, B)), dim3(HD < 128 ? HD : 128), 0, st, ws, H, nchunks, out, ld_out);
+    if (e_l != cudaSuccess) return e_l;
+  }
   return cudaGetLastError();
 }
 

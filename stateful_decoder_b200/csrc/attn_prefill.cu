@@ -25,6 +25,7 @@ template <typename KT, int HD>
 __global__ void __launch_bounds__(256) causal_attn_kernel(const KT* __restrict__ Q, const KT* __restrict__ K,
                                                           const KT* __restrict__ V, int64_t ld_tq, int64_t ld_tkv,
                                                           int H, int T, KT* out, int64_t ld_out, float scale_log2) {
+  griddep_enter();
   constexpr int DPT = HD / 16;
   extern __shared__ float sm[];
   float* sQt = sm;                      // [HD][PADQ]
@@ -154,8 +155,10 @@ cudaError_t launch(const KT* q, const KT* k, const KT* v, int64_t ld_tq, int64_t
   if (e != cudaSuccess) return e;
   const float scale_log2 = 1.4426950408889634f / sqrtf((float)HD);
   dim3 grid((T + BQ - 1) / BQ, H, B);
-  causal_attn_kernel<KT, HD><<<grid, 256, smem, st>>>(q, k, v, ld_tq, ld_tkv, H, T, out, ld_out, scale_log2);
-  note_launch();
+  {
+    const cudaError_t e_l = launch_pdl(causal_attn_kernel<KT, HD>, dim3(grid), dim3(256), smem, st, q, k, v, ld_tq, ld_tkv, H, T, out, ld_out, scale_log2);
+    if (e_l != cudaSuccess) return e_l;
+  }
   return cudaGetLastError();
 }
 

@@ -24,6 +24,22 @@ __device__ __forceinline__ uint64_t globaltimer_ns() {
   return t;
 }
 
+// ---------------------------------------------------------------- dependent launch
+// Every kernel of the library is launched with programmatic stream
+// serialisation, so it may start while the previous kernel of the stream is
+// still running.  It must call griddep_wait() before it reads anything the
+// previous kernels write or writes anything they read (weights and the rotary
+// table are never written during a step and may be read before).  After the
+// wait it lets its own dependents begin launching.
+__device__ __forceinline__ void griddep_wait() { asm volatile("griddepcontrol.wait;" ::: "memory"); }
+__device__ __forceinline__ void griddep_launch_dependents() {
+  asm volatile("griddepcontrol.launch_dependents;" ::: "memory");
+}
+__device__ __forceinline__ void griddep_enter() {
+  griddep_wait();
+  griddep_launch_dependents();
+}
+
 // ---------------------------------------------------------------- types
 template <typename T> struct TypeOf;
 template <> struct TypeOf<float> { static constexpr int dtype = 0; };

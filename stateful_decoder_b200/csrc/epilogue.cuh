@@ -44,37 +44,54 @@ __device__ __forceinline__ float load_bias(const EpiParams& p, int m) {
                      : reinterpret_cast<const float*>(p.bias)[m];
 }
 
-// Non-pair epilogues: one accumulator for output (n, m).
+// Does the epilogue read the aux0 rows (e_t)?
 template <int EPI>
-__device__ __forceinline__ void epi_apply(const EpiParams& p, int64_t n, int m, float acc) {
+__device__ __forceinline__ constexpr bool epi_uses_aux0() {
+  return EPI == EPI_MERGE || EPI == EPI_CONVEX;
+}
+
+// Non-pair epilogues: one accumulator for output (n, m); `orow` and `arow`
+// are the precomputed row offsets out_map.off(n) and aux0_map.off(n).
+template <int EPI>
+__device__ __forceinline__ void epi_apply_at(const EpiParams& p, int64_t n, int64_t orow, int64_t arow, int m,
+                                             float acc) {
   if constexpr (EPI == EPI_STORE) {
-    const int64_t o = p.out_map.off(n) + m;
+    const int64_t o = orow + m;
     if (p.out_bf16) reinterpret_cast<bf16*>(p.out)[o] = __float2bfloat16_rn(acc);
     else reinterpret_cast<float*>(p.out)[o] = acc;
   } else if constexpr (EPI == EPI_RESID) {
-    float* o = reinterpret_cast<float*>(p.out) + p.out_map.off(n) + m;
+    float* o = reinterpret_cast<float*>(p.out) + orow + m;
     *o = *o + acc;
   } else if constexpr (EPI == EPI_GATE) {
-    reinterpret_cast<float*>(p.out)[p.out_map.off(n) + m] = sigmoidf_(acc + load_bias(p, m));
+    reinterpret_cast<float*>(p.out)[orow + m] = sigmoidf_(acc + load_bias(p, m));
   } else if constexpr (EPI == EPI_MERGE) {
-    const float e = p.aux0[p.aux0_map.off(n) + m];
+    const float e = p.aux0[arow + m];
     const float g = p.aux1[n * p.ld_aux1 + m];
-    reinterpret_cast<float*>(p.out)[p.out_map.off(n) + m] = e + p.alpha * g * acc;
+    reinterpret_cast<float*>(p.out)[orow + m] = e + p.alpha * g * acc;
   } else if constexpr (EPI == EPI_CONVEX) {
-    const float e = p.aux0[p.aux0_map.off(n) + m];
-    float* o = reinterpret_cast<float*>(p.out) + p.out_map.off(n) + m;
+    const float e = p.aux0[arow + m];
+    float* o = reinterpret_cast<float*>(p.out) + orow + m;
     const float g = sigmoidf_(acc);
     *o = g * e + (1.0f - g) * (*o);
   }
 }
 
+template <int EPI>
+__device__ __forceinline__ void epi_apply(const EpiParams& p, int64_t n, int m, float acc) {
+  epi_apply_at<EPI>(p, n, p.out_map.off(n), epi_uses_aux0<EPI>() ? p.aux0_map.off(n) : 0, m, acc);
+}
+
 // SWIGLU pair epilogue: gate accumulator of row 2i and up accumulator of row
 // 2i+1 give hidden column i.
-__device__ __forceinline__ void epi_swiglu(const EpiParams& p, int64_t n, int i, float gate, float up) {
+__device__ __forceinline__ void epi_swiglu_at(const EpiParams& p, int64_t orow, int i, float gate, float up) {
   const float h = siluf_(gate) * up;
-  const int64_t o = p.out_map.off(n) + i;
+  const int64_t o = orow + i;
   if (p.out_bf16) reinterpret_cast<bf16*>(p.out)[o] = __float2bfloat16_rn(h);
   else reinterpret_cast<float*>(p.out)[o] = h;
+}
+
+__device__ __forceinline__ void epi_swiglu(const EpiParams& p, int64_t n, int i, float gate, float up) {
+  epi_swiglu_at(p, p.out_map.off(n), i, gate, up);
 }
 
 }  // namespace rlt

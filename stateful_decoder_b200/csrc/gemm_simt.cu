@@ -17,6 +17,7 @@ constexpr int TM = 64, TN = 64, TK = 16;
 template <typename WT, typename XT, int EPI>
 __global__ void __launch_bounds__(256) gemm_simt_kernel(const WT* __restrict__ W, int64_t ldw, const XT* __restrict__ X,
                                                         int64_t ldx, int M, int N, int K, EpiParams ep) {
+  griddep_enter();
   __shared__ float sW[TK][TM + 4];
   __shared__ float sX[TK][TN + 4];
   const int tx = threadIdx.x % 16, ty = threadIdx.x / 16;
@@ -69,8 +70,10 @@ template <typename WT, typename XT, int EPI>
 cudaError_t launch(const WT* W, int64_t ldw, const XT* X, int64_t ldx, int M, int N, int K, const EpiParams& ep,
                    cudaStream_t st) {
   dim3 grid((M + TM - 1) / TM, (N + TN - 1) / TN);
-  gemm_simt_kernel<WT, XT, EPI><<<grid, 256, 0, st>>>(W, ldw, X, ldx, M, N, K, ep);
-  note_launch();
+  {
+    const cudaError_t e_l = launch_pdl(gemm_simt_kernel<WT, XT, EPI>, dim3(grid), dim3(256), 0, st, W, ldw, X, ldx, M, N, K, ep);
+    if (e_l != cudaSuccess) return e_l;
+  }
   return cudaGetLastError();
 }
 

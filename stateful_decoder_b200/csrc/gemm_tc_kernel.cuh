@@ -1,0 +1,370 @@
+// gemm_tc_kernel.cuh -- device code of the bf16 tensor-core GEMM (sm_100a:
+// tcgen05.mma with fp32 accumulators in tensor memory, operands staged by TMA).
+//
+// C[n][m] = sum_k X[n][k] * W[m][k].  The weight rows are the 128-row A
+// operand (M = output features); the activation rows are the N operand
+// (N = sequences in a decode step, tokens in the encoder), so a decode step
+// with few sequences still fills the 128-lane MMA.  Both operands are K-major
+// bf16 in global memory, loaded by TMA with 128-byte swizzling into a
+// multi-stage ring.  One thread issues the TMA copies, one thread issues the
+// MMAs, and all four warps drain the accumulator through the fused epilogue.
+//
+// Split over K inside a thread-block cluster: the CS CTAs of one cluster own
+// the same output tile and consecutive K ranges, so every weight byte is read
+// from HBM once while all SMs stream.  Their fp32 partial tiles are exchanged
+// through distributed shared memory: CTA r adds the partials of every CTA of
+// the cluster, in rank order 0..CS-1 (a fixed order, so results never depend
+// on timing), for its 1/CS share of the tile's columns and applies the
+// epilogue there.  No global scratch and no second kernel are needed.
+//
+// No TMA multicast is used anywhere: every CTA loads its own tiles.
+#pragma once
+#include <cuda.h>
+
+#include "common.cuh"
+#include "epilogue.cuh"
+#include "internal.h"
+
+namespace rlt {
+namespace gemm_detail {
+
+constexpr int BM = 128;
+constexpr int BK = 64;
+
+template <int BN>
+struct TcCfg {
+  static constexpr int A_BYTES = BM * BK * 2;
+  static constexpr int B_BYTES = BN * BK * 2;
+  static constexpr int STAGE_BYTES = A_BYTES + B_BYTES;
+  static constexpr int STAGES = BN >= 256 ? 4 : (BN >= 128 ? 6 : 8);
+  static constexpr int PIPE_BYTES = STAGES * STAGE_BYTES;
+  static constexpr int SMEM = PIPE_BYTES + 1024 /*align*/ + 256 /*barriers*/;
+  static constexpr int TMEM_COLS = BN;  // power of two >= 32
+  static_assert(BN * BM * 4 <= PIPE_BYTES, "cluster partial tile must fit in the pipeline buffers");
+};
+
+// UMMA shared-memory matrix descriptor for a K-major tile whose rows are 128
+// bytes (64 bf16) with the 128-byte swizzle: 8-row core groups 1024 bytes
+// apart (stride byte offset), descriptor version 1, layout SWIZZLE_128B.
+__device__ __forceinline__ uint64_t sdesc_k128(uint32_t saddr) {
+  uint64_t d = 0;
+  d |= (uint64_t)((saddr & 0x3FFFFu) >> 4);
+  d |= (uint64_t)1 << 16;            // leading byte offset (unused for this layout)
+  d |= (uint64_t)(1024 >> 4) << 32;  // stride byte offset
+  d |= (uint64_t)1 << 46;            // descriptor version
+  d |= (uint64_t)2 << 61;            // SWIZZLE_128B
+  return d;
+}
+
+// Instruction descriptor: D fp32, A and B bf16, both K-major, shape 128 x BN.
+template <int BN>
+__device__ __forceinline__ constexpr uint32_t idesc_bf16() {
+  return (1u << 4) | (1u << 7) | (1u << 10) | ((uint32_t)(BN >> 3) << 17) | ((uint32_t)(BM >> 4) << 24);
+}
+
+__device__ __forceinline__ void tma_load_2d(uint32_t dst, const CUtensorMap* tm, uint32_t bar, int x, int y) {
+  asm volatile(
+      "cp.async.bulk.tensor.2d.shared::cluster.global.mbarrier::complete_tx::bytes [%0], [%1, {%3, %4}], [%2];" ::"r"(dst),
+      "l"(reinterpret_cast<uint64_t>(tm)), "r"(bar), "r"(x), "r"(y)
+      : "memory");
+}
+
+__device__ __forceinline__ void umma_bf16(uint32_t tmem_d, uint64_t a, uint64_t b, uint32_t idesc, uint32_t acc) {
+  asm volatile(
+      "{\n\t.reg .pred p;\n\t"
+      "setp.ne.b32 p, %4, 0;\n\t"
+      "tcgen05.mma.cta_group::1.kind::f16 [%0], %1, %2, %3, p;\n\t}" ::"r"(tmem_d),
+      "l"(a), "l"(b), "r"(idesc), "r"(acc));
+}
+
+__device__ __forceinline__ void umma_commit(uint32_t bar) {
+  asm volatile("tcgen05.commit.cta_group::1.mbarrier::arrive::one.shared::cluster.b64 [%0];" ::"r"(bar) : "memory");
+}
+
+__device__ __forceinline__ void tmem_ld32(uint32_t taddr, float* v) {
+  uint32_t r[32];
+  asm volatile(
+      "tcgen05.ld.sync.aligned.32x32b.x32.b32 "
+      "{%0,%1,%2,%3,%4,%5,%6,%7,%8,%9,%10,%11,%12,%13,%14,%15,"
+      "%16,%17,%18,%19,%20,%21,%22,%23,%24,%25,%26,%27,%28,%29,%30,%31}, [%32];"
+      : "=r"(r[0]), "=r"(r[1]), "=r"(r[2]), "=r"(r[3]), "=r"(r[4]), "=r"(r[5]), "=r"(r[6]), "=r"(r[7]),
+        "=r"(r[8]), "=r"(r[9]), "=r"(r[10]), "=r"(r[11]), "=r"(r[12]), "=r"(r[13]), "=r"(r[14]),
+        "=r"(r[15]), "=r"(r[16]), "=r"(r[17]), "=r"(r[18]), "=r"(r[19]), "=r"(r[20]), "=r"(r[21]),
+        "=r"(r[22]), "=r"(r[23]), "=r"(r[24]), "=r"(r[25]), "=r"(r[26]), "=r"(r[27]), "=r"(r[28]),
+        "=r"(r[29]), "=r"(r[30]), "=r"(r[31])
+      : "r"(taddr));
+  asm volatile("tcgen05.wait::ld.sync.aligned;" ::: "memory");
+#pragma unroll
+  for (int i = 0; i < 32; ++i) v[i] = __uint_as_float(r[i]);
+}
+
+__device__ __forceinline__ void cluster_sync_all() {
+  asm volatile("barrier.cluster.arrive.release.aligned;\n\tbarrier.cluster.wait.acquire.aligned;" ::: "memory");
+}
+
+__device__ __forceinline__ uint32_t dsmem_addr(uint32_t local, uint32_t rank) {
+  uint32_t r;
+  asm volatile("mapa.shared::cluster.u32 %0, %1, %2;" : "=r"(r) : "r"(local), "r"(rank));
+  return r;
+}
+
+// Remote shared-memory load; ordered after the cluster barrier that precedes
+// every use (that barrier is a volatile asm with a memory clobber).
+__device__ __forceinline__ float dsmem_ld(uint32_t addr) {
+  float v;
+  asm volatile("ld.shared::cluster.f32 %0, [%1];" : "=f"(v) : "r"(addr));
+  return v;
+}
+
+// Applies the epilogue to accumulator columns [n0, n0 + cnt) (cnt <= 32) of
+// this thread's row m.  Row offsets (which may need a division for grouped
+// rows) are computed once per column by lane j and broadcast.
+template <int EPI>
+__device__ __forceinline__ void epilogue_cols(const EpiParams& ep, int64_t n0, int cnt, int64_t N, int m, int lane,
+                                              const float* v) {
+  const int64_t my_n = n0 + lane;
+  const bool my_ok = lane < cnt && my_n < N;
+  const int64_t my_o = my_ok ? ep.out_map.off(my_n) : 0;
+  const int64_t my_a = (epi_uses_aux0<EPI>() && my_ok) ? ep.aux0_map.off(my_n) : 0;
+#pragma unroll
+  for (int j = 0; j < 32; ++j) {
+    const int64_t n = n0 + j;
+    const bool okj = j < cnt && n < N;
+    const int64_t orow = __shfl_sync(0xffffffffu, my_o, j);
+    if constexpr (EPI == EPI_SWIGLU) {
+      const float other = __shfl_xor_sync(0xffffffffu, v[j], 1);
+      if (okj && (lane & 1) == 0) epi_swiglu_at(ep, orow, m >> 1, v[j], other);
+    } else {
+      const int64_t arow = epi_uses_aux0<EPI>() ? __shfl_sync(0xffffffffu, my_a, j) : 0;
+      if (okj) epi_apply_at<EPI>(ep, n, orow, arow, m, v[j]);
+    }
+  }
+}
+
+template <int BN, int EPI, int CS>
+__global__ void __launch_bounds__(128, 1)
+    gemm_tc_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CUtensorMap tmB, int M, int N,
+                   int K, int kb_per_split, EpiParams ep) {
+  using C = TcCfg<BN>;
+  extern __shared__ uint8_t smem_raw[];
+  uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
+  uint64_t* bars = reinterpret_cast<uint64_t*>(smem + C::PIPE_BYTES);
+  uint64_t* full = bars;
+  uint64_t* empty = bars + C::STAGES;
+  uint64_t* done = bars + 2 * C::STAGES;
+  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(bars + 2 * C::STAGES + 1);
+  volatile int* abort_flag = reinterpret_cast<volatile int*>(tmem_slot + 1);
+
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  const int m_tile = blockIdx.x, n_tile = blockIdx.y, split = blockIdx.z;  // cluster spans z: rank == split
+  const int kb_total = K / BK;
+  const int kb0 = split * kb_per_split;
+  const int kb1 = min(kb_total, kb0 + kb_per_split);
+  const int nkb = kb1 > kb0 ? kb1 - kb0 : 0;
+
+  if (threadIdx.x == 0) {
+    for (int s = 0; s < C::STAGES; ++s) {
+      mbar_init(smem_u32(&full[s]), 1);
+      mbar_init(smem_u32(&empty[s]), 1);
+    }
+    mbar_init(smem_u32(done), 1);
+    *abort_flag = 0;
+    fence_mbar_init();
+    asm volatile("prefetch.tensormap [%0];" ::"l"(reinterpret_cast<uint64_t>(&tmA)) : "memory");
+    asm volatile("prefetch.tensormap [%0];" ::"l"(reinterpret_cast<uint64_t>(&tmB)) : "memory");
+  }
+  if (warp == 0) {
+    asm volatile("tcgen05.alloc.cta_group::1.sync.aligned.shared::cta.b32 [%0], %1;" ::"r"(smem_u32(tmem_slot)),
+                 "r"(C::TMEM_COLS));
+    asm volatile("tcgen05.relinquish_alloc_permit.cta_group::1.sync.aligned;");
+  }
+  asm volatile("tcgen05.fence::before_thread_sync;" ::: "memory");
+  __syncthreads();
+  asm volatile("tcgen05.fence::after_thread_sync;" ::: "memory");
+  const uint32_t tmem_base = *tmem_slot;
+
+  if (warp == 0 && lane == 0) {
+    // TMA producer.  Weights do not depend on earlier kernels of the step, so
+    // the first stages' weight tiles are requested before waiting for the
+    // previous kernel (dependent launch); activation tiles follow the wait.
+    const int pre = nkb < C::STAGES ? nkb : C::STAGES;
+    for (int i = 0; i < pre; ++i) {
+      const uint32_t a_s = smem_u32(smem + i * C::STAGE_BYTES);
+      mbar_arrive_expect_tx(smem_u32(&full[i]), C::STAGE_BYTES);
+      tma_load_2d(a_s, &tmA, smem_u32(&full[i]), (kb0 + i) * BK, m_tile * BM);
+    }
+    griddep_wait();
+    for (int i = 0; i < pre; ++i) {
+      const uint32_t b_s = smem_u32(smem + i * C::STAGE_BYTES) + C::A_BYTES;
+      tma_load_2d(b_s, &tmB, smem_u32(&full[i]), (kb0 + i) * BK, n_tile * BN);
+    }
+    int issued = pre;
+    for (int i = pre; i < nkb; ++i) {
+      const int s = i % C::STAGES;
+      const uint32_t ph = (uint32_t)(i / C::STAGES) & 1u;
+      if (!mbar_wait(smem_u32(&empty[s]), ph ^ 1u)) { *abort_flag = 1; break; }
+      if (*abort_flag) break;
+      const uint32_t a_s = smem_u32(smem + s * C::STAGE_BYTES);
+      const uint32_t b_s = a_s + C::A_BYTES;
+      mbar_arrive_expect_tx(smem_u32(&full[s]), C::STAGE_BYTES);
+      tma_load_2d(a_s, &tmA, smem_u32(&full[s]), (kb0 + i) * BK, m_tile * BM);
+      tma_load_2d(b_s, &tmB, smem_u32(&full[s]), (kb0 + i) * BK, n_tile * BN);
+      ++issued;
+    }
+    if (*abort_flag) {
+      // drain copies that may still be in flight before the CTA exits
+      const int lo = issued > C::STAGES ? issued - C::STAGES : 0;
+      for (int i = lo; i < issued; ++i)
+        mbar_wait(smem_u32(&full[i % C::STAGES]), (uint32_t)(i / C::STAGES) & 1u);
+    }
+  } else if (warp == 1 && lane == 0) {
+    // MMA issuer
+    constexpr uint32_t idesc = idesc_bf16<BN>();
+    for (int i = 0; i < nkb; ++i) {
+      const int s = i % C::STAGES;
+      const uint32_t ph = (uint32_t)(i / C::STAGES) & 1u;
+      if (!mbar_wait(smem_u32(&full[s]), ph)) { *abort_flag = 1; break; }
+      asm volatile("tcgen05.fence::after_thread_sync;" ::: "memory");
+      const uint32_t a_s = smem_u32(smem + s * C::STAGE_BYTES);
+      const uint32_t b_s = a_s + C::A_BYTES;
+#pragma unroll
+      for (int kk = 0; kk < BK / 16; ++kk) {
+        umma_bf16(tmem_base, sdesc_k128(a_s + kk * 32), sdesc_k128(b_s + kk * 32), idesc,
+                  (i > 0 || kk > 0) ? 1u : 0u);
+      }
+      umma_commit(smem_u32(&empty[s]));
+    }
+    umma_commit(smem_u32(done));
+  }
+  __syncwarp();
+
+  // Epilogue: warp w owns accumulator lanes 32w..32w+31 (output features).
+  const bool ok = mbar_wait(smem_u32(done), 0);
+  asm volatile("tcgen05.fence::after_thread_sync;" ::: "memory");
+  griddep_wait();  // epilogue reads/writes buffers of earlier kernels
+  griddep_launch_dependents();
+  const bool good = ok && !*abort_flag && nkb > 0;
+  const int row = warp * 32 + lane;
+  const int m = m_tile * BM + row;
+  const int64_t n_base = (int64_t)n_tile * BN;
+  if constexpr (CS == 1) {
+    if (good) {
+#pragma unroll 1
+      for (int c = 0; c < BN; c += 32) {
+        if (n_base + c >= N) break;
+        float v[32];
+        tmem_ld32(tmem_base + ((uint32_t)(warp * 32) << 16) + (uint32_t)c, v);
+        epilogue_cols<EPI>(ep, n_base + c, 32, N, m, lane, v);
+      }
+    }
+  } else {
+    // Partial tile to this CTA's shared memory (the pipeline buffers are idle
+    // now: every MMA that read them has completed), column-major [BN][128].
+    float* red = reinterpret_cast<float*>(smem);
+#pragma unroll 1
+    for (int c = 0; c < BN; c += 32) {
+      float v[32];
+      if (good && n_base + c < N) {
+        tmem_ld32(tmem_base + ((uint32_t)(warp * 32) << 16) + (uint32_t)c, v);
+      } else {
+#pragma unroll
+        for (int j = 0; j < 32; ++j) v[j] = 0.f;
+      }
+#pragma unroll
+      for (int j = 0; j < 32; ++j) red[(c + j) * BM + row] = v[j];
+    }
+    cluster_sync_all();
+    // This CTA reduces columns [split*COLS, (split+1)*COLS) over all ranks, in
+    // rank order.  Decode-step outputs use plain row maps (no grouped rows),
+    // so each column's row offset is a multiply, applied per element.
+    constexpr int COLS = BN / CS;
+    const uint32_t red_local = smem_u32(red);
+#pragma unroll 1
+    for (int cc = 0; cc < COLS; cc += 4) {
+      float t[4][CS];
+#pragma unroll
+      for (int j = 0; j < 4; ++j) {
+        const uint32_t off = red_local + (uint32_t)(((split * COLS + cc + j) * BM + row) * 4);
+#pragma unroll
+        for (int p = 0; p < CS; ++p) t[j][p] = (cc + j < COLS) ? dsmem_ld(dsmem_addr(off, (uint32_t)p)) : 0.f;
+      }
+#pragma unroll
+      for (int j = 0; j < 4; ++j) {
+        float acc = 0.f;
+#pragma unroll
+        for (int p = 0; p < CS; ++p) acc += t[j][p];
+        const int64_t n = n_base + split * COLS + cc + j;
+        if constexpr (EPI == EPI_SWIGLU) {
+          const float other = __shfl_xor_sync(0xffffffffu, acc, 1);
+          if (cc + j < COLS && n < N && (lane & 1) == 0) epi_swiglu(ep, n, m >> 1, acc, other);
+        } else {
+          if (cc + j < COLS && n < N) epi_apply<EPI>(ep, n, m, acc);
+        }
+      }
+    }
+    cluster_sync_all();  // peers may still read this CTA's partial until here
+  }
+  asm volatile("tcgen05.fence::before_thread_sync;" ::: "memory");
+  __syncthreads();
+  if (warp == 0) {
+    asm volatile("tcgen05.dealloc.cta_group::1.sync.aligned.b32 %0, %1;" ::"r"(tmem_base), "r"(C::TMEM_COLS));
+  }
+}
+
+template <int BN, int EPI, int CS>
+cudaError_t launch_gemm(const CUtensorMap& ta, const CUtensorMap& tb, int M, int N, int K, int kb_per_split,
+                        const EpiParams& ep, cudaStream_t st) {
+  using C = TcCfg<BN>;
+  static bool attr_set = false;
+  if (!attr_set) {
+    cudaError_t e =
+        cudaFuncSetAttribute(gemm_tc_kernel<BN, EPI, CS>, cudaFuncAttributeMaxDynamicSharedMemorySize, C::SMEM);
+    if (e != cudaSuccess) return e;
+    attr_set = true;
+  }
+  cudaLaunchConfig_t cfg = {};
+  cfg.gridDim = dim3(M / BM, (N + BN - 1) / BN, CS);
+  cfg.blockDim = dim3(128, 1, 1);
+  cfg.dynamicSmemBytes = C::SMEM;
+  cfg.stream = st;
+  cudaLaunchAttribute attr[2];
+  attr[0].id = cudaLaunchAttributeClusterDimension;
+  attr[0].val.clusterDim.x = 1;
+  attr[0].val.clusterDim.y = 1;
+  attr[0].val.clusterDim.z = CS;
+  attr[1].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+  attr[1].val.programmaticStreamSerializationAllowed = 1;
+  cfg.attrs = attr;
+  cfg.numAttrs = 2;
+  cudaError_t e = cudaLaunchKernelEx(&cfg, gemm_tc_kernel<BN, EPI, CS>, ta, tb, M, N, K, kb_per_split, ep);
+  note_launch();
+  return e != cudaSuccess ? e : cudaGetLastError();
+}
+
+template <int EPI, int CS>
+cudaError_t launch_gemm_bn(const CUtensorMap& ta, const CUtensorMap& tb, int bn, int M, int N, int K, int kb_per_split,
+                           const EpiParams& ep, cudaStream_t st) {
+  switch (bn) {
+    case 32: return launch_gemm<32, EPI, CS>(ta, tb, M, N, K, kb_per_split, ep, st);
+    case 64: return launch_gemm<64, EPI, CS>(ta, tb, M, N, K, kb_per_split, ep, st);
+    case 128: return launch_gemm<128, EPI, CS>(ta, tb, M, N, K, kb_per_split, ep, st);
+    default: return launch_gemm<256, EPI, CS>(ta, tb, M, N, K, kb_per_split, ep, st);
+  }
+}
+
+// All (BN, CS) variants of one epilogue; instantiated per epilogue in the
+// gemm_tc_epi_*.cu files so the variants compile in parallel.
+template <int EPI>
+cudaError_t launch_gemm_epi(const CUtensorMap& ta, const CUtensorMap& tb, int bn, int cs, int M, int N, int K,
+                            int kb_per_split, const EpiParams& ep, cudaStream_t st) {
+  switch (cs) {
+    case 1: return launch_gemm_bn<EPI, 1>(ta, tb, bn, M, N, K, kb_per_split, ep, st);
+    case 2: return launch_gemm_bn<EPI, 2>(ta, tb, bn, M, N, K, kb_per_split, ep, st);
+    case 4: return launch_gemm_bn<EPI, 4>(ta, tb, bn, M, N, K, kb_per_split, ep, st);
+    case 8: return launch_gemm_bn<EPI, 8>(ta, tb, bn, M, N, K, kb_per_split, ep, st);
+  }
+  return cudaErrorInvalidValue;
+}
+
+}  // namespace gemm_detail
+}  // namespace rlt

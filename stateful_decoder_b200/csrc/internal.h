@@ -16,14 +16,35 @@ constexpr int kSmCount = 148;  // B200 streaming multiprocessors
 void note_launch();
 int64_t launch_count();
 
+// Launches a kernel with programmatic stream serialisation (see
+// griddep_wait in common.cuh) and counts it.
+template <typename... KArgs, typename... Args>
+cudaError_t launch_pdl(void (*kernel)(KArgs...), dim3 grid, dim3 block, size_t smem, cudaStream_t st,
+                       Args&&... args) {
+  cudaLaunchConfig_t cfg = {};
+  cfg.gridDim = grid;
+  cfg.blockDim = block;
+  cfg.dynamicSmemBytes = smem;
+  cfg.stream = st;
+  cudaLaunchAttribute attr[1];
+  attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+  attr[0].val.programmaticStreamSerializationAllowed = 1;
+  cfg.attrs = attr;
+  cfg.numAttrs = 1;
+  const cudaError_t e = cudaLaunchKernelEx(&cfg, kernel, static_cast<Args&&>(args)...);
+  note_launch();
+  return e != cudaSuccess ? e : cudaGetLastError();
+}
+
 // ---------------------------------------------------------------- GEMMs
 // C[n][m] = sum_k X[n][k] W[m][k] with a fused epilogue (epilogue.cuh).
 // bf16 on tcgen05: M % 128 == 0, K % 64 == 0, ld* % 8 == 0, 16-byte aligned
-// bases.  `workspace` holds split-K partials (gemm_tc_workspace_floats).
+// bases.  split_mode 1 (decode steps) splits K inside a thread-block cluster
+// by a rule that depends only on M and K; split_mode 0 (token-parallel
+// encoder) never splits.  No global scratch is used.
 cudaError_t gemm_tc(const bf16* W, int64_t ldw, const bf16* X, int64_t ldx, int M, int N, int K, int epi,
-                    const EpiParams& ep, float* workspace, size_t workspace_floats, cudaStream_t st);
-size_t gemm_tc_workspace_floats(int M, int K, int N);
-int gemm_tc_splits(int M, int K, int N);
+                    const EpiParams& ep, int split_mode, cudaStream_t st);
+int gemm_tc_cluster(int M, int K, int split_mode);
 int gemm_tc_bn(int N);
 
 // CUDA-core GEMM (fp32 models; also a cross-check for the tensor-core path).

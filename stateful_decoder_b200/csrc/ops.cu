@@ -28,6 +28,7 @@ namespace {
 template <typename WT>
 __global__ void init_normal_kernel(WT* dst, int64_t rows, int64_t cols, int64_t pitch, uint32_t k0, uint32_t k1,
                                    uint32_t sid, float std) {
+  griddep_enter();
   const int64_t n = rows * cols;
   for (int64_t i = (int64_t)blockIdx.x * blockDim.x + threadIdx.x; i < n; i += (int64_t)gridDim.x * blockDim.x) {
     uint64_t sum = 0;
@@ -45,6 +46,7 @@ __global__ void init_normal_kernel(WT* dst, int64_t rows, int64_t cols, int64_t 
 
 template <typename WT>
 __global__ void init_const_kernel(WT* dst, int64_t rows, int64_t cols, int64_t pitch, float value) {
+  griddep_enter();
   const int64_t n = rows * cols;
   for (int64_t i = (int64_t)blockIdx.x * blockDim.x + threadIdx.x; i < n; i += (int64_t)gridDim.x * blockDim.x)
     dst[(i / cols) * pitch + (i % cols)] = from_f32<WT>(value);
@@ -54,6 +56,7 @@ __global__ void init_const_kernel(WT* dst, int64_t rows, int64_t cols, int64_t p
 template <typename WT>
 __global__ void embed_kernel(const int32_t* __restrict__ tok, int tok_per_seq, int64_t tok_seq_stride,
                              const WT* __restrict__ emb, int d, int vocab, float* out, RowMap out_map) {
+  griddep_enter();
   const int64_t r = blockIdx.x;
   int32_t id = tok[(r / tok_per_seq) * tok_seq_stride + (r % tok_per_seq)];
   if (id < 0 || id >= vocab) {
@@ -69,6 +72,7 @@ __global__ void embed_kernel(const int32_t* __restrict__ tok, int tok_per_seq, i
 template <typename WT, typename OT>
 __global__ void rmsnorm_kernel(const float* __restrict__ x, RowMap x_map, const WT* __restrict__ gamma, int d,
                                float eps, OT* out, int64_t ld_out) {
+  griddep_enter();
   __shared__ float red[32];
   const int64_t r = blockIdx.x;
   const float* xr = x + x_map.off(r);
@@ -85,6 +89,7 @@ __global__ void rmsnorm_kernel(const float* __restrict__ x, RowMap x_map, const 
 template <typename WT, typename OT>
 __global__ void merge_prep_kernel(const float* __restrict__ e, RowMap e_map, const float* __restrict__ s,
                                   const WT* __restrict__ gamma, int d, float eps, int kind, OT* out) {
+  griddep_enter();
   __shared__ float red[32];
   const int b = blockIdx.x;
   const float* er = e + e_map.off(b);
@@ -108,6 +113,7 @@ template <typename XT, typename KT>
 __global__ void head_scatter_kernel(const XT* __restrict__ x, int64_t ld_x, int64_t col0, int64_t rows,
                                     int rows_per_seq, int pos0, int H, int hd, int rope,
                                     const float* __restrict__ rope_cs, KT* dst, int64_t ld_t) {
+  griddep_enter();
   const int half = hd / 2;
   const int64_t n = rows * H * half;
   for (int64_t idx = (int64_t)blockIdx.x * blockDim.x + threadIdx.x; idx < n; idx += (int64_t)gridDim.x * blockDim.x) {
@@ -134,6 +140,7 @@ __global__ void head_scatter_kernel(const XT* __restrict__ x, int64_t ld_x, int6
 // ------------------------------------------------------------------ readout
 __global__ void logp_gather_kernel(const float* __restrict__ logits, int V, const int32_t* __restrict__ next,
                                    int64_t next_stride, float* logp, int64_t ld_logp) {
+  griddep_enter();
   __shared__ float red[32];
   const int b = blockIdx.x;
   const float* l = logits + (int64_t)b * V;
@@ -173,6 +180,7 @@ constexpr int kMaxTopK = 256;
 __global__ void __launch_bounds__(kSampleThreads)
     sample_kernel(const float* __restrict__ logits, int V, float temperature, int top_k, uint32_t k0, uint32_t k1,
                   uint32_t t, int32_t* token, float* logp_tok, float* logmu) {
+  griddep_enter();
   __shared__ uint32_t hist[256];
   __shared__ uint32_t s_sel[2];
   __shared__ float red[32];
@@ -296,12 +304,14 @@ __global__ void __launch_bounds__(kSampleThreads)
 
 template <typename WT>
 __global__ void broadcast_kernel(const WT* __restrict__ src, int d, float* dst, int B) {
+  griddep_enter();
   const int64_t n = (int64_t)B * d;
   for (int64_t i = (int64_t)blockIdx.x * blockDim.x + threadIdx.x; i < n; i += (int64_t)gridDim.x * blockDim.x)
     dst[i] = to_f32(src[i % d]);
 }
 
 __global__ void copy_kernel(float* dst, const float* src, int64_t n) {
+  griddep_enter();
   for (int64_t i = (int64_t)blockIdx.x * blockDim.x + threadIdx.x; i < n; i += (int64_t)gridDim.x * blockDim.x)
     dst[i] = src[i];
 }
@@ -319,24 +329,30 @@ template <typename WT>
 cudaError_t init_normal(WT* dst, int64_t rows, int64_t cols, int64_t pitch, uint64_t seed, uint32_t sid, float std,
                         cudaStream_t st) {
   const int64_t n = rows * cols;
-  init_normal_kernel<WT><<<grid_for(n, 256, 148 * 64), 256, 0, st>>>(dst, rows, cols, pitch, (uint32_t)seed,
+  {
+    const cudaError_t e_l = launch_pdl(init_normal_kernel<WT>, dim3(grid_for(n, 256, 148 * 64)), dim3(256), 0, st, dst, rows, cols, pitch, (uint32_t)seed,
                                                                      (uint32_t)(seed >> 32), sid, std);
-  note_launch();
+    if (e_l != cudaSuccess) return e_l;
+  }
   return cudaGetLastError();
 }
 
 template <typename WT>
 cudaError_t init_const(WT* dst, int64_t rows, int64_t cols, int64_t pitch, float value, cudaStream_t st) {
-  init_const_kernel<WT><<<grid_for(rows * cols, 256), 256, 0, st>>>(dst, rows, cols, pitch, value);
-  note_launch();
+  {
+    const cudaError_t e_l = launch_pdl(init_const_kernel<WT>, dim3(grid_for(rows * cols, 256)), dim3(256), 0, st, dst, rows, cols, pitch, value);
+    if (e_l != cudaSuccess) return e_l;
+  }
   return cudaGetLastError();
 }
 
 template <typename WT>
 cudaError_t embed(const int32_t* tok, int64_t n_rows, int tok_per_seq, int64_t tok_seq_stride, const WT* emb, int d,
                   int vocab, float* out, RowMap out_map, cudaStream_t st) {
-  embed_kernel<WT><<<(unsigned)n_rows, 128, 0, st>>>(tok, tok_per_seq, tok_seq_stride, emb, d, vocab, out, out_map);
-  note_launch();
+  {
+    const cudaError_t e_l = launch_pdl(embed_kernel<WT>, dim3((unsigned)n_rows), dim3(128), 0, st, tok, tok_per_seq, tok_seq_stride, emb, d, vocab, out, out_map);
+    if (e_l != cudaSuccess) return e_l;
+  }
   return cudaGetLastError();
 }
 
@@ -344,16 +360,20 @@ template <typename WT, typename OT>
 cudaError_t rmsnorm(const float* x, RowMap x_map, const WT* gamma, int64_t rows, int d, float eps, OT* out,
                     int64_t ld_out, cudaStream_t st) {
   const int threads = d >= 1024 ? 256 : 128;
-  rmsnorm_kernel<WT, OT><<<(unsigned)rows, threads, 0, st>>>(x, x_map, gamma, d, eps, out, ld_out);
-  note_launch();
+  {
+    const cudaError_t e_l = launch_pdl(rmsnorm_kernel<WT, OT>, dim3((unsigned)rows), dim3(threads), 0, st, x, x_map, gamma, d, eps, out, ld_out);
+    if (e_l != cudaSuccess) return e_l;
+  }
   return cudaGetLastError();
 }
 
 template <typename WT, typename OT>
 cudaError_t merge_prep(const float* e, RowMap e_map, const float* s, const WT* gamma, int B, int d, float eps,
                        int kind, OT* out, cudaStream_t st) {
-  merge_prep_kernel<WT, OT><<<B, d >= 1024 ? 256 : 128, 0, st>>>(e, e_map, s, gamma, d, eps, kind, out);
-  note_launch();
+  {
+    const cudaError_t e_l = launch_pdl(merge_prep_kernel<WT, OT>, dim3(B), dim3(d >= 1024 ? 256 : 128), 0, st, e, e_map, s, gamma, d, eps, kind, out);
+    if (e_l != cudaSuccess) return e_l;
+  }
   return cudaGetLastError();
 }
 
@@ -361,38 +381,48 @@ template <typename XT, typename KT>
 cudaError_t head_scatter(const XT* x, int64_t ld_x, int64_t col0, int64_t rows, int rows_per_seq, int pos0, int H,
                          int hd, int rope, const float* rope_cs, KT* dst, int64_t ld_t, cudaStream_t st) {
   const int64_t n = rows * H * (hd / 2);
-  head_scatter_kernel<XT, KT><<<grid_for(n, 256, 148 * 32), 256, 0, st>>>(x, ld_x, col0, rows, rows_per_seq, pos0, H,
+  {
+    const cudaError_t e_l = launch_pdl(head_scatter_kernel<XT, KT>, dim3(grid_for(n, 256, 148 * 32)), dim3(256), 0, st, x, ld_x, col0, rows, rows_per_seq, pos0, H,
                                                                           hd, rope, rope_cs, dst, ld_t);
-  note_launch();
+    if (e_l != cudaSuccess) return e_l;
+  }
   return cudaGetLastError();
 }
 
 cudaError_t logp_gather(const float* logits, int B, int V, const int32_t* next, int64_t next_stride, float* logp,
                         int64_t ld_logp, cudaStream_t st) {
-  logp_gather_kernel<<<B, 1024, 0, st>>>(logits, V, next, next_stride, logp, ld_logp);
-  note_launch();
+  {
+    const cudaError_t e_l = launch_pdl(logp_gather_kernel, dim3(B), dim3(1024), 0, st, logits, V, next, next_stride, logp, ld_logp);
+    if (e_l != cudaSuccess) return e_l;
+  }
   return cudaGetLastError();
 }
 
 cudaError_t sample_topk(const float* logits, int B, int V, float temperature, int top_k, uint64_t seed, uint32_t t,
                         int32_t* token, float* logp_tok, float* logmu, cudaStream_t st) {
   if (top_k < 1 || top_k > kMaxTopK || !(temperature > 0.f)) return cudaErrorInvalidValue;
-  sample_kernel<<<B, kSampleThreads, 0, st>>>(logits, V, temperature, top_k, (uint32_t)seed, (uint32_t)(seed >> 32), t,
+  {
+    const cudaError_t e_l = launch_pdl(sample_kernel, dim3(B), dim3(kSampleThreads), 0, st, logits, V, temperature, top_k, (uint32_t)seed, (uint32_t)(seed >> 32), t,
                                              token, logp_tok, logmu);
-  note_launch();
+    if (e_l != cudaSuccess) return e_l;
+  }
   return cudaGetLastError();
 }
 
 template <typename WT>
 cudaError_t broadcast_row(const WT* src, int d, float* dst, int B, cudaStream_t st) {
-  broadcast_kernel<WT><<<grid_for((int64_t)B * d, 256), 256, 0, st>>>(src, d, dst, B);
-  note_launch();
+  {
+    const cudaError_t e_l = launch_pdl(broadcast_kernel<WT>, dim3(grid_for((int64_t)B * d, 256)), dim3(256), 0, st, src, d, dst, B);
+    if (e_l != cudaSuccess) return e_l;
+  }
   return cudaGetLastError();
 }
 
 cudaError_t copy_f32(float* dst, const float* src, int64_t n, cudaStream_t st) {
-  copy_kernel<<<grid_for(n, 256), 256, 0, st>>>(dst, src, n);
-  note_launch();
+  {
+    const cudaError_t e_l = launch_pdl(copy_kernel, dim3(grid_for(n, 256)), dim3(256), 0, st, dst, src, n);
+    if (e_l != cudaSuccess) return e_l;
+  }
   return cudaGetLastError();
 }
 

@@ -117,14 +117,12 @@ struct rlt_state {
   void* hbuf = nullptr;        // [B][F]
   float* gate = nullptr;       // [B][d]
   float* logits = nullptr;     // [B][V]
-  float* gemm_ws = nullptr; size_t gemm_ws_floats = 0;
   float* attn_ws = nullptr; size_t attn_ws_floats = 0;
   // encoder-prefill workspace, rows = sequences x tokens of one chunk
   int64_t pf_rows = 0;
   void* pf_x = nullptr; void* pf_big = nullptr; void* pf_q = nullptr; void* pf_k = nullptr; void* pf_v = nullptr;
   void* pf_attn = nullptr;
   int64_t pf_big_cols = 0;
-  float* pf_ws = nullptr; size_t pf_ws_floats = 0;
 };
 
 namespace {
@@ -287,21 +285,26 @@ int32_t init_views(rlt_model* m, uint64_t seed) {
 }
 
 // ------------------------------------------------------------------ GEMM dispatch
+// Decode-step contractions pass the state's split workspace and may split K;
+// token-parallel (encoder prefill) contractions pass no workspace and never
+// split, so that no reduction order depends on how many rows share a GEMM.
+// Decode-step contractions (split = true) may split K inside a cluster;
+// token-parallel encoder contractions never split.
 template <typename T>
 int32_t gemm(rlt_state* S, const void* W, int64_t ldw, const void* X, int64_t ldx, int M, int N, int K, int epi,
-             const EpiParams& ep, float* ws, size_t ws_floats, cudaStream_t st);
+             const EpiParams& ep, bool split, cudaStream_t st);
 
 template <>
 int32_t gemm<bf16>(rlt_state*, const void* W, int64_t ldw, const void* X, int64_t ldx, int M, int N, int K, int epi,
-                   const EpiParams& ep, float* ws, size_t ws_floats, cudaStream_t st) {
-  RLT_CUDA(gemm_tc(static_cast<const bf16*>(W), ldw, static_cast<const bf16*>(X), ldx, M, N, K, epi, ep, ws, ws_floats,
-                   st));
+                   const EpiParams& ep, bool split, cudaStream_t st) {
+  RLT_CUDA(gemm_tc(static_cast<const bf16*>(W), ldw, static_cast<const bf16*>(X), ldx, M, N, K, epi, ep,
+                   split ? 1 : 0, st));
   return RLT_OK;
 }
 
 template <>
 int32_t gemm<float>(rlt_state*, const void* W, int64_t ldw, const void* X, int64_t ldx, int M, int N, int K, int epi,
-                    const EpiParams& ep, float*, size_t, cudaStream_t st) {
+                    const EpiParams& ep, bool, cudaStream_t st) {
   RLT_CUDA(gemm_simt<float, float>(static_cast<const float*>(W), ldw, static_cast<const float*>(X), ldx, M, N, K, epi,
                                    ep, st));
   return RLT_OK;
@@ -381,16 +384,6 @@ int32_t make_state(rlt_model* m, int32_t B, int32_t max_len, int32_t flags, rlt_
   S->gate = static_cast<float*>(p);
   if ((r = A(&p, (int64_t)B * V * 4))) goto fail_;
   S->logits = static_cast<float*>(p);
-  if (c.dtype == RLT_DTYPE_BF16) {
-    size_t w = 0;
-    const int Ms[] = {(int)(3 * d), (int)d, (int)(2 * F), (int)(2 * d * G), (int)V};
-    const int Ks[] = {(int)d, (int)F, (int)(2 * d)};
-    for (int M : Ms)
-      for (int K : Ks) w = std::max(w, gemm_tc_workspace_floats(M, K, B));
-    S->gemm_ws_floats = w;
-    if ((r = A(&p, (int64_t)w * 4))) goto fail_;
-    S->gemm_ws = static_cast<float*>(p);
-  }
   S->attn_ws_floats = prefix_attn_workspace_floats(B, c.n_heads, (int)(d / c.n_heads), max_len);
   if ((r = A(&p, (int64_t)S->attn_ws_floats * 4))) goto fail_;
   S->attn_ws = static_cast<float*>(p);
@@ -423,14 +416,13 @@ int32_t ensure_prefill_ws(rlt_state* S, int T) {
   int64_t seqs = std::max<int64_t>(1, std::min<int64_t>(S->B, budget / (per_row * T)));
   const int64_t rows = seqs * T;
   if (rows <= S->pf_rows && S->pf_big_cols == big_cols) return RLT_OK;
-  for (void* p : {S->pf_x, S->pf_big, S->pf_q, S->pf_k, S->pf_v, S->pf_attn, (void*)S->pf_ws}) {
+  for (void* p : {S->pf_x, S->pf_big, S->pf_q, S->pf_k, S->pf_v, S->pf_attn}) {
     if (!p) continue;
     cudaFree(p);
     for (auto it = S->allocs.begin(); it != S->allocs.end(); ++it)
       if (*it == p) { S->allocs.erase(it); break; }
   }
   S->pf_x = S->pf_big = S->pf_q = S->pf_k = S->pf_v = S->pf_attn = nullptr;
-  S->pf_ws = nullptr;
   S->pf_rows = 0;
   auto A = [&](void** p, int64_t bytes) { return dev_alloc(S->allocs, p, (size_t)bytes); };
   RLT_TRY(A(&S->pf_x, rows * d * (int64_t)es));
@@ -440,15 +432,6 @@ int32_t ensure_prefill_ws(rlt_state* S, int T) {
   if (!cache) {
     RLT_TRY(A(&S->pf_k, rows * d * (int64_t)es));
     RLT_TRY(A(&S->pf_v, rows * d * (int64_t)es));
-  }
-  if (c.dtype == RLT_DTYPE_BF16) {
-    size_t w = 0;
-    for (int M : {(int)(3 * d), (int)d, (int)(2 * F), (int)(2 * d * G)})
-      for (int K : {(int)d, (int)F}) w = std::max(w, gemm_tc_workspace_floats(M, K, (int)rows));
-    S->pf_ws_floats = w;
-    void* p = nullptr;
-    RLT_TRY(A(&p, (int64_t)w * 4));
-    S->pf_ws = static_cast<float*>(p);
   }
   S->pf_rows = rows;
   S->pf_big_cols = big_cols;
@@ -484,7 +467,7 @@ int32_t encode_prefix_impl(rlt_model* m, rlt_state* S, const int32_t* tok, int32
       const LayerW& w = m->layers[l];
       RLT_CUDA(rmsnorm<T, T>(e0, emap, static_cast<const T*>(w.g_ea), rows, d, c.rms_eps, static_cast<T*>(S->pf_x), d, st));
       RLT_TRY(gemm<T>(S, w.qkv, d, S->pf_x, d, 3 * d, (int)rows, d, EPI_STORE, epi_out(S->pf_big, plain_rows(3 * d), is_bf16),
-                      S->pf_ws, S->pf_ws_floats, st));
+                      false, st));
       T* kdst;
       T* vdst;
       int64_t ld_tk;
@@ -504,18 +487,16 @@ int32_t encode_prefix_impl(rlt_model* m, rlt_state* S, const int32_t* tok, int32
       RLT_CUDA((head_scatter<T, T>(qkv, 3 * d, 2 * d, rows, Tn, 0, H, hd, 0, m->rope_cs, vdst, ld_tk, st)));
       RLT_CUDA(causal_attn<T>(static_cast<const T*>(S->pf_q), kdst, vdst, Tn, ld_tk, Bc, H, hd, Tn,
                               static_cast<T*>(S->pf_attn), d, st));
-      RLT_TRY(gemm<T>(S, w.wo, d, S->pf_attn, d, d, (int)rows, d, EPI_RESID, epi_out(e0, emap, 0), S->pf_ws,
-                      S->pf_ws_floats, st));
+      RLT_TRY(gemm<T>(S, w.wo, d, S->pf_attn, d, d, (int)rows, d, EPI_RESID, epi_out(e0, emap, 0), false, st));
       RLT_CUDA(rmsnorm<T, T>(e0, emap, static_cast<const T*>(w.g_ef), rows, d, c.rms_eps, static_cast<T*>(S->pf_x), d, st));
       RLT_TRY(gemm<T>(S, w.w13, d, S->pf_x, d, 2 * F, (int)rows, d, EPI_SWIGLU, epi_out(S->pf_big, plain_rows(F), is_bf16),
-                      S->pf_ws, S->pf_ws_floats, st));
-      RLT_TRY(gemm<T>(S, w.w2, F, S->pf_big, F, d, (int)rows, F, EPI_RESID, epi_out(e0, emap, 0), S->pf_ws,
-                      S->pf_ws_floats, st));
+                      false, st));
+      RLT_TRY(gemm<T>(S, w.w2, F, S->pf_big, F, d, (int)rows, F, EPI_RESID, epi_out(e0, emap, 0), false, st));
     }
     // memory projection (eq. 2.2): n = RMSNorm_E(e); k^g = RoPE(W_K^g n), v^g = W_V^g n
     RLT_CUDA(rmsnorm<T, T>(e0, emap, static_cast<const T*>(m->g_mem), rows, d, c.rms_eps, static_cast<T*>(S->pf_x), d, st));
     RLT_TRY(gemm<T>(S, m->w_kvm, d, S->pf_x, d, 2 * d * G, (int)rows, d, EPI_STORE,
-                    epi_out(S->pf_big, plain_rows(2 * d * G), is_bf16), S->pf_ws, S->pf_ws_floats, st));
+                    epi_out(S->pf_big, plain_rows(2 * d * G), is_bf16), false, st));
     for (int g = 0; g < G; ++g) {
       const int64_t grp = ((int64_t)g * S->B + b0) * H * S->max_len * hd;
       const T* kv = static_cast<const T*>(S->pf_big);
@@ -545,23 +526,21 @@ int32_t encode_step_impl(rlt_model* m, rlt_state* S, const int32_t* tok, cudaStr
     T* ck = static_cast<T*>(S->ce_k) + lay;
     T* cv = static_cast<T*>(S->ce_v) + lay;
     RLT_CUDA(rmsnorm<T, T>(et, emap, static_cast<const T*>(w.g_ea), B, d, c.rms_eps, static_cast<T*>(S->xb), d, st));
-    RLT_TRY(gemm<T>(S, w.qkv, d, S->xb, d, 3 * d, B, d, EPI_STORE, epi_out(S->qkv, plain_rows(S->ld_qkv), 0), S->gemm_ws,
-                    S->gemm_ws_floats, st));
+    RLT_TRY(gemm<T>(S, w.qkv, d, S->xb, d, 3 * d, B, d, EPI_STORE, epi_out(S->qkv, plain_rows(S->ld_qkv), 0), true, st));
     RLT_CUDA((head_scatter<float, T>(S->qkv, S->ld_qkv, d, B, 1, t - 1, H, hd, 1, m->rope_cs, ck, S->max_len, st)));
     RLT_CUDA((head_scatter<float, T>(S->qkv, S->ld_qkv, 2 * d, B, 1, t - 1, H, hd, 0, m->rope_cs, cv, S->max_len, st)));
     prof_begin(m, st);
     RLT_CUDA(prefix_attn<T>(S->qkv, S->ld_qkv, ck, cv, S->max_len, B, H, hd, t, t - 1, m->rope_cs,
                             static_cast<T*>(S->attn), d, S->attn_ws, S->attn_ws_floats, st));
     prof_end(m, st, 0, (double)B * H * t * hd * 2 * m->esz);
-    RLT_TRY(gemm<T>(S, w.wo, d, S->attn, d, d, B, d, EPI_RESID, epi_out(et, emap, 0), S->gemm_ws, S->gemm_ws_floats, st));
+    RLT_TRY(gemm<T>(S, w.wo, d, S->attn, d, d, B, d, EPI_RESID, epi_out(et, emap, 0), true, st));
     RLT_CUDA(rmsnorm<T, T>(et, emap, static_cast<const T*>(w.g_ef), B, d, c.rms_eps, static_cast<T*>(S->xb), d, st));
-    RLT_TRY(gemm<T>(S, w.w13, d, S->xb, d, 2 * F, B, d, EPI_SWIGLU, epi_out(S->hbuf, plain_rows(F), is_bf16), S->gemm_ws,
-                    S->gemm_ws_floats, st));
-    RLT_TRY(gemm<T>(S, w.w2, F, S->hbuf, F, d, B, F, EPI_RESID, epi_out(et, emap, 0), S->gemm_ws, S->gemm_ws_floats, st));
+    RLT_TRY(gemm<T>(S, w.w13, d, S->xb, d, 2 * F, B, d, EPI_SWIGLU, epi_out(S->hbuf, plain_rows(F), is_bf16), true, st));
+    RLT_TRY(gemm<T>(S, w.w2, F, S->hbuf, F, d, B, F, EPI_RESID, epi_out(et, emap, 0), true, st));
   }
   RLT_CUDA(rmsnorm<T, T>(et, emap, static_cast<const T*>(m->g_mem), B, d, c.rms_eps, static_cast<T*>(S->xb), d, st));
   RLT_TRY(gemm<T>(S, m->w_kvm, d, S->xb, d, 2 * d * G, B, d, EPI_STORE, epi_out(S->qkv, plain_rows(S->ld_qkv), 0),
-                  S->gemm_ws, S->gemm_ws_floats, st));
+                  true, st));
   for (int g = 0; g < G; ++g) {
     const int64_t grp = (int64_t)g * B * H * S->max_len * hd;
     RLT_CUDA((head_scatter<float, T>(S->qkv, S->ld_qkv, (int64_t)2 * d * g, B, 1, t - 1, H, hd, 1, m->rope_cs,
@@ -592,20 +571,19 @@ int32_t transition_impl(rlt_model* m, rlt_state* S, cudaStream_t st) {
     EpiParams g = epi_out(S->gate, srow, 0);
     g.bias = m->b_gate;
     g.bias_bf16 = is_bf16;
-    RLT_TRY(gemm<T>(S, m->w_gate, 2 * d, S->xb, 2 * d, d, B, 2 * d, EPI_GATE, g, S->gemm_ws, S->gemm_ws_floats, st));
+    RLT_TRY(gemm<T>(S, m->w_gate, 2 * d, S->xb, 2 * d, d, B, 2 * d, EPI_GATE, g, true, st));
     EpiParams u = epi_out(S->s, srow, 0);
     u.aux0 = et;
     u.aux0_map = emap;
     u.aux1 = S->gate;
     u.ld_aux1 = d;
     u.alpha = c.alpha;
-    RLT_TRY(gemm<T>(S, m->w_state, d, off(S->xb, d, m->esz), 2 * d, d, B, d, EPI_MERGE, u, S->gemm_ws,
-                    S->gemm_ws_floats, st));
+    RLT_TRY(gemm<T>(S, m->w_state, d, off(S->xb, d, m->esz), 2 * d, d, B, d, EPI_MERGE, u, true, st));
   } else {
     EpiParams u = epi_out(S->s, srow, 0);
     u.aux0 = et;
     u.aux0_map = emap;
-    RLT_TRY(gemm<T>(S, m->w_gate, 2 * d, S->xb, 2 * d, d, B, 2 * d, EPI_CONVEX, u, S->gemm_ws, S->gemm_ws_floats, st));
+    RLT_TRY(gemm<T>(S, m->w_gate, 2 * d, S->xb, 2 * d, d, B, 2 * d, EPI_CONVEX, u, true, st));
   }
   const int n_ring = std::min(t - 1, W - 1);
   for (int l = 0; l < L; ++l) {
@@ -613,32 +591,29 @@ int32_t transition_impl(rlt_model* m, rlt_state* S, cudaStream_t st) {
     const int grp = c.groups == 1 ? 0 : l;
     // SWA sublayer (eqs. 2.12-2.14)
     RLT_CUDA(rmsnorm<T, T>(S->s, srow, static_cast<const T*>(w.g_dsa), B, d, c.rms_eps, static_cast<T*>(S->xb), d, st));
-    RLT_TRY(gemm<T>(S, w.dqkv, d, S->xb, d, 3 * d, B, d, EPI_STORE, epi_out(S->qkv, plain_rows(3 * d), 0), S->gemm_ws,
-                    S->gemm_ws_floats, st));
+    RLT_TRY(gemm<T>(S, w.dqkv, d, S->xb, d, 3 * d, B, d, EPI_STORE, epi_out(S->qkv, plain_rows(3 * d), 0), true, st));
     const int64_t rlay = (int64_t)l * B * H * (W > 1 ? W - 1 : 0) * hd;
     T* rk = W > 1 ? static_cast<T*>(S->ring_k) + rlay : nullptr;
     T* rv = W > 1 ? static_cast<T*>(S->ring_v) + rlay : nullptr;
     prof_begin(m, st);
     RLT_CUDA(swa_attn<T>(S->qkv, 3 * d, rk, rv, B, H, hd, t, W, m->rope_cs, static_cast<T*>(S->attn), d, st));
     prof_end(m, st, 1, (double)B * H * hd * m->esz * (2.0 * n_ring + (W > 1 ? 2.0 : 0.0)));
-    RLT_TRY(gemm<T>(S, w.dwo, d, S->attn, d, d, B, d, EPI_RESID, epi_out(S->s, srow, 0), S->gemm_ws, S->gemm_ws_floats, st));
+    RLT_TRY(gemm<T>(S, w.dwo, d, S->attn, d, d, B, d, EPI_RESID, epi_out(S->s, srow, 0), true, st));
     // cross-attention to M^{g(l)}_{<=t} (eq. 2.15)
     RLT_CUDA(rmsnorm<T, T>(S->s, srow, static_cast<const T*>(w.g_dmem), B, d, c.rms_eps, static_cast<T*>(S->xb), d, st));
-    RLT_TRY(gemm<T>(S, w.wq_mem, d, S->xb, d, d, B, d, EPI_STORE, epi_out(S->qkv, plain_rows(d), 0), S->gemm_ws,
-                    S->gemm_ws_floats, st));
+    RLT_TRY(gemm<T>(S, w.wq_mem, d, S->xb, d, d, B, d, EPI_STORE, epi_out(S->qkv, plain_rows(d), 0), true, st));
     const int64_t mg = (int64_t)grp * B * H * S->max_len * hd;
     prof_begin(m, st);
     RLT_CUDA(prefix_attn<T>(S->qkv, d, static_cast<const T*>(S->mem_k) + mg, static_cast<const T*>(S->mem_v) + mg,
                             S->max_len, B, H, hd, t, t - 1, m->rope_cs, static_cast<T*>(S->attn), d, S->attn_ws,
                             S->attn_ws_floats, st));
     prof_end(m, st, 0, (double)B * H * t * hd * 2 * m->esz);
-    RLT_TRY(gemm<T>(S, w.wo_mem, d, S->attn, d, d, B, d, EPI_RESID, epi_out(S->s, srow, 0), S->gemm_ws,
-                    S->gemm_ws_floats, st));
+    RLT_TRY(gemm<T>(S, w.wo_mem, d, S->attn, d, d, B, d, EPI_RESID, epi_out(S->s, srow, 0), true, st));
     // FFN (eq. 2.16)
     RLT_CUDA(rmsnorm<T, T>(S->s, srow, static_cast<const T*>(w.g_dffn), B, d, c.rms_eps, static_cast<T*>(S->xb), d, st));
     RLT_TRY(gemm<T>(S, w.dw13, d, S->xb, d, 2 * F, B, d, EPI_SWIGLU, epi_out(S->hbuf, plain_rows(F), is_bf16),
-                    S->gemm_ws, S->gemm_ws_floats, st));
-    RLT_TRY(gemm<T>(S, w.dw2, F, S->hbuf, F, d, B, F, EPI_RESID, epi_out(S->s, srow, 0), S->gemm_ws, S->gemm_ws_floats, st));
+                    true, st));
+    RLT_TRY(gemm<T>(S, w.dw2, F, S->hbuf, F, d, B, F, EPI_RESID, epi_out(S->s, srow, 0), true, st));
   }
   S->n_dec = t;
   return RLT_OK;
@@ -652,8 +627,7 @@ int32_t readout_impl(rlt_model* m, rlt_state* S, const int32_t* next, int64_t ne
   const rlt_config& c = m->cfg;
   const int d = c.d_model, V = c.vocab, B = S->B;
   RLT_CUDA(rmsnorm<T, T>(S->s, plain_rows(d), static_cast<const T*>(m->g_out), B, d, c.rms_eps, static_cast<T*>(S->xb), d, st));
-  RLT_TRY(gemm<T>(S, m->w_out, d, S->xb, d, V, B, d, EPI_STORE, epi_out(S->logits, plain_rows(V), 0), S->gemm_ws,
-                  S->gemm_ws_floats, st));
+  RLT_TRY(gemm<T>(S, m->w_out, d, S->xb, d, V, B, d, EPI_STORE, epi_out(S->logits, plain_rows(V), 0), true, st));
   if (next && logp) RLT_CUDA(logp_gather(S->logits, B, V, next, next_stride, logp, ld_logp, st));
   if (samp)
     RLT_CUDA(sample_topk(S->logits, B, V, samp->temperature, samp->top_k, samp->seed, (uint32_t)S->n_dec,
@@ -879,7 +853,7 @@ int32_t rlt_prefill(rlt_model* m, rlt_state* s, const int32_t* tok_dev, int32_t 
     RLT_TRY(RLT_DISPATCH(m, transition_impl, m, s, st));
     if (logp_dev && t < T)
       RLT_TRY(RLT_DISPATCH(m, readout_impl, m, s, tok_dev + t, (int64_t)T, logp_dev + (t - 1), (int64_t)(T - 1),
-                           (const rlt_sampling*)nullptr, (const rlt_readout_out*)nullptr, st));
+                           (const rlt_sampling*)nullptr, (const rlt_readout_out*)false, st));
   }
   return ok();
 }
@@ -900,7 +874,7 @@ int32_t rlt_replay_logprobs(rlt_model* m, const int32_t* tok_dev, int32_t B, int
   for (int t = 1; t <= S - 1; ++t) {
     RLT_TRY(RLT_DISPATCH(m, transition_impl, m, st_, st));
     RLT_TRY(RLT_DISPATCH(m, readout_impl, m, st_, tok_dev + t, (int64_t)S, logp_dev + (t - 1), (int64_t)(S - 1),
-                         (const rlt_sampling*)nullptr, (const rlt_readout_out*)nullptr, st));
+                         (const rlt_sampling*)nullptr, (const rlt_readout_out*)false, st));
   }
   return ok();
 }
@@ -923,18 +897,8 @@ int32_t rlt_op_linear(const void* w_dev, const void* x_dev, float* y_dev, int32_
     return ok();
   }
   if (M % 128 || K % 64) return fail(RLT_E_INVAL, "tensor-core path needs M % 128 == 0 and K % 64 == 0");
-  const size_t ws = gemm_tc_workspace_floats(M, K, N);
-  float* w = nullptr;
-  if (ws) {
-    cudaError_t e = cudaMalloc(&w, ws * sizeof(float));
-    if (e != cudaSuccess) return fail(RLT_E_OOM, "split-K workspace");
-  }
   cudaError_t e = gemm_tc(static_cast<const bf16*>(w_dev), K, static_cast<const bf16*>(x_dev), K, M, N, K, EPI_STORE,
-                          ep, w, ws, st);
-  if (w) {
-    cudaStreamSynchronize(st);
-    cudaFree(w);
-  }
+                          ep, 1, st);
   if (e != cudaSuccess) return fail(RLT_E_CUDA, std::string("gemm_tc: ") + cudaGetErrorString(e));
   return ok();
 }
