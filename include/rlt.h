@@ -228,6 +228,22 @@ int32_t rlt_replay_logprobs(rlt_model* m, const int32_t* tok_dev, int32_t B, int
 int32_t rlt_op_linear(const void* w_dev, const void* x_dev, float* y_dev, int32_t M, int32_t N, int32_t K,
                       int32_t dtype, int32_t use_tensor_cores, void* stream);
 
+/* Kernel-level check of the decode attention of eq. 2.15 / eq. 2.8: for
+ * every sequence b and head h, softmax over keys j < n of
+ * (q_b,h . k_b,h,j) / sqrt(hd), weighting v_b,h,j.  q_dev [B][H*hd] fp32 (a
+ * query row per sequence, heads concatenated); k_dev, v_dev [B][H][ld_t][hd]
+ * in `dtype` (rows 0..n-1 are read); out_dev [B][H*hd] in `dtype`.  When
+ * rope_cs_dev is not NULL the query is first rotated at position qpos with
+ * the rotate-half map, using the table rope_cs_dev[p][i][0..1] =
+ * (cos, sin)(p * base^(-2i/hd)) (fp32, rows 0..qpos).  Keys are taken as
+ * given.  n > 256 splits the keys into 256-key chunks whose partial results
+ * need scratch of B*H*ceil(n/256)*(hd+2) floats, allocated and freed inside
+ * the call (the call synchronises the stream in that case).
+ * Errors: RLT_E_INVAL (shape/dtype), RLT_E_OOM, RLT_E_CUDA. */
+int32_t rlt_op_prefix_attention(const float* q_dev, const void* k_dev, const void* v_dev, int64_t ld_t, int32_t B,
+                                int32_t H, int32_t hd, int32_t n, int32_t dtype, const float* rope_cs_dev,
+                                int32_t qpos, void* out_dev, void* stream);
+
 /* Behaviour sampler (see rlt_sampling) on caller-given logits_dev [B][V]
  * fp32, as position t: writes token_dev [B] int32, logp_dev [B] (raw
  * log-softmax of the token, may be NULL) and logmu_dev [B] (tempered and

@@ -43,7 +43,7 @@ EXPORTED = (
     "rlt_state_create", "rlt_state_free", "rlt_state_reset", "rlt_state_info_get", "rlt_state_read",
     "rlt_encode_prefix", "rlt_readout", "rlt_decoder_step", "rlt_prefill", "rlt_replay_logprobs",
     "rlt_last_error", "rlt_check_device", "rlt_profile_enable", "rlt_profile_read", "rlt_op_linear",
-    "rlt_op_sample", "rlt_kernel_launches",
+    "rlt_op_sample", "rlt_kernel_launches", "rlt_op_prefix_attention",
 )
 
 
@@ -98,6 +98,7 @@ _sig = {
     "rlt_prefill": [_vp, _vp, _vp, _i32, _vp, _vp],
     "rlt_replay_logprobs": [_vp, _vp, _i32, _i32, _vp, _vp],
     "rlt_op_linear": [_vp, _vp, _vp, _i32, _i32, _i32, _i32, _i32, _vp],
+    "rlt_op_prefix_attention": [_vp, _vp, _vp, ctypes.c_int64, _i32, _i32, _i32, _i32, _i32, _vp, _i32, _vp, _vp],
     "rlt_op_sample": [_vp, _i32, _i32, ctypes.POINTER(Sampling), ctypes.c_uint32, _vp, _vp, _vp, _vp],
     "rlt_last_error": [ctypes.c_char_p, ctypes.c_size_t],
     "rlt_check_device": [],
@@ -295,6 +296,19 @@ def rlt_op_linear(w, x, y, use_tensor_cores: bool = True, stream=None) -> None:
     dt = DTYPE_BF16 if str(w.dtype) == "torch.bfloat16" else DTYPE_F32
     _check(_lib.rlt_op_linear(_dev(w), _dev(x), _dev(y, "torch.float32"), M, N, K, dt, int(use_tensor_cores),
                               _stream(stream)))
+
+
+def _prefix_attention_args(q, k, v, n, out, rope_cs, qpos, stream):
+    B, H, ld_t, hd = k.shape
+    dt = DTYPE_BF16 if str(k.dtype) == "torch.bfloat16" else DTYPE_F32
+    return (_dev(q, "torch.float32"), _dev(k), _dev(v), ld_t, B, H, hd, n, dt, _dev(rope_cs, "torch.float32"),
+            qpos, _dev(out), _stream(stream))
+
+
+def rlt_op_prefix_attention(q, k, v, n: int, out, rope_cs=None, qpos: int = 0, stream=None) -> None:
+    """out [B, H*hd] = attention of q [B, H*hd] (fp32) over rows 0..n-1 of
+    k, v [B, H, ld_t, hd] (bf16 or fp32); rope_cs [pos, hd/2, 2] rotates q at qpos."""
+    _check(_lib.rlt_op_prefix_attention(*_prefix_attention_args(q, k, v, n, out, rope_cs, qpos, stream)))
 
 
 def rlt_op_sample(logits, sampling: dict, t: int, token, logp=None, logmu=None, stream=None) -> None:

@@ -192,12 +192,16 @@ __global__ void __launch_bounds__(kThreads) prefix_attn_kernel(const float* __re
   const int c = blockIdx.x, h = blockIdx.y, b = blockIdx.z;
   const int j0 = c * kPrefixChunk, j1 = min(n, j0 + kPrefixChunk);
   const float* qrow = q + (int64_t)b * ld_q + h * HD;
-  const float* cs = rope_cs + (int64_t)qpos * HALF * 2;
-  for (int i = threadIdx.x; i < HALF; i += kThreads) {
-    float a, bb;
-    rope_pair(qrow[i], qrow[i + HALF], cs + 2 * i, a, bb);
-    sq[i] = a * scale_log2;
-    sq[i + HALF] = bb * scale_log2;
+  if (rope_cs != nullptr) {
+    const float* cs = rope_cs + (int64_t)qpos * HALF * 2;
+    for (int i = threadIdx.x; i < HALF; i += kThreads) {
+      float a, bb;
+      rope_pair(qrow[i], qrow[i + HALF], cs + 2 * i, a, bb);
+      sq[i] = a * scale_log2;
+      sq[i + HALF] = bb * scale_log2;
+    }
+  } else {
+    for (int i = threadIdx.x; i < HD; i += kThreads) sq[i] = qrow[i] * scale_log2;
   }
   __syncthreads();
   const int64_t base = ((int64_t)b * H + h) * ld_t * HD;

@@ -61,7 +61,9 @@ cudaError_t swa_attn(const float* qkv, int64_t ld_qkv, KT* ring_k, KT* ring_v, i
 
 // Decode attention of one query per (sequence, head) over key/value rows
 // 0..n-1 of a [B][H][ld_t][hd] cache; the query is rotated at position
-// qpos (0-based) first.  Split over fixed chunks of keys when n is large.
+// qpos (0-based) first unless rope_cs is null.  Split over fixed chunks of
+// keys when n is large; the chunk partials go to `ws`
+// (prefix_attn_workspace_floats).
 template <typename KT>
 cudaError_t prefix_attn(const float* q, int64_t ld_q, const KT* k, const KT* v, int64_t ld_t, int B, int H, int hd,
                         int n, int qpos, const float* rope_cs, KT* out, int64_t ld_out, float* ws, size_t ws_floats,

@@ -903,6 +903,36 @@ int32_t rlt_op_linear(const void* w_dev, const void* x_dev, float* y_dev, int32_
   return ok();
 }
 
+int32_t rlt_op_prefix_attention(const float* q_dev, const void* k_dev, const void* v_dev, int64_t ld_t, int32_t B,
+                                int32_t H, int32_t hd, int32_t n, int32_t dtype, const float* rope_cs_dev,
+                                int32_t qpos, void* out_dev, void* stream) {
+  if (!q_dev || !k_dev || !v_dev || !out_dev || B <= 0 || H <= 0 || n <= 0 || ld_t < n || qpos < 0)
+    return fail(RLT_E_INVAL, "bad prefix attention arguments");
+  if (!(hd == 16 || hd == 32 || hd == 64 || hd == 128 || hd == 256)) return fail(RLT_E_INVAL, "head size");
+  if (dtype != RLT_DTYPE_F32 && dtype != RLT_DTYPE_BF16) return fail(RLT_E_INVAL, "dtype");
+  cudaStream_t st = (cudaStream_t)stream;
+  const size_t wsf = prefix_attn_workspace_floats(B, H, hd, n);
+  float* ws = nullptr;
+  if (wsf && cudaMalloc(&ws, wsf * sizeof(float)) != cudaSuccess) {
+    cudaGetLastError();
+    return fail(RLT_E_OOM, "prefix attention scratch");
+  }
+  cudaError_t e;
+  if (dtype == RLT_DTYPE_BF16)
+    e = prefix_attn<bf16>(q_dev, (int64_t)H * hd, static_cast<const bf16*>(k_dev), static_cast<const bf16*>(v_dev), ld_t,
+                          B, H, hd, n, qpos, rope_cs_dev, static_cast<bf16*>(out_dev), (int64_t)H * hd, ws, wsf, st);
+  else
+    e = prefix_attn<float>(q_dev, (int64_t)H * hd, static_cast<const float*>(k_dev), static_cast<const float*>(v_dev),
+                           ld_t, B, H, hd, n, qpos, rope_cs_dev, static_cast<float*>(out_dev), (int64_t)H * hd, ws, wsf,
+                           st);
+  if (ws) {
+    cudaStreamSynchronize(st);
+    cudaFree(ws);
+  }
+  if (e != cudaSuccess) return fail(RLT_E_CUDA, std::string("prefix attention: ") + cudaGetErrorString(e));
+  return ok();
+}
+
 int32_t rlt_op_sample(const float* logits_dev, int32_t B, int32_t V, const rlt_sampling* samp, uint32_t t,
                       int32_t* token_dev, float* logp_dev, float* logmu_dev, void* stream) {
   if (!logits_dev || !samp || !token_dev || B <= 0 || V <= 0) return fail(RLT_E_INVAL, "bad sample arguments");
