@@ -244,6 +244,28 @@ int32_t rlt_op_prefix_attention(const float* q_dev, const void* k_dev, const voi
                                 int32_t H, int32_t hd, int32_t n, int32_t dtype, const float* rope_cs_dev,
                                 int32_t qpos, void* out_dev, void* stream);
 
+/* The same attention as rlt_op_prefix_attention, for callers that cannot
+ * allocate device memory: serving engines that reserve all of the GPU's
+ * memory for their own pool up front, and latency-critical paths that cannot
+ * afford the device-wide synchronisation that cudaMalloc/cudaFree imply.  It
+ * calls no allocating routine.  The chunk partials of the split-key attention
+ * go to a scratch array of at most 16 MiB (4,194,304 floats) that the library
+ * places in device memory as a static array; every GPU that loads the library
+ * holds it until the process exits.  A call needs B*H*ceil(n/256)*(hd+2)
+ * floats of it (none when n <= 256); larger calls are rejected with
+ * RLT_E_CAPACITY and nothing is launched.  The first call on a device looks
+ * up the array's device address (once per device, with that device current);
+ * make that first call before any stream capture.  All calls share the one
+ * array and it keeps the last call's contents; nothing in it needs to start
+ * at zero, since every partial a call reads is written earlier in that call.
+ * Calls that overlap on the GPU (other streams, other threads) race on the
+ * array: order them.  The report has no counterpart to this entry point; it
+ * exists for the callers above.
+ * Errors: RLT_E_INVAL, RLT_E_CAPACITY, RLT_E_CUDA. */
+int32_t rlt_op_prefix_attention_noalloc(const float* q_dev, const void* k_dev, const void* v_dev, int64_t ld_t,
+                                        int32_t B, int32_t H, int32_t hd, int32_t n, int32_t dtype,
+                                        const float* rope_cs_dev, int32_t qpos, void* out_dev, void* stream);
+
 /* Behaviour sampler (see rlt_sampling) on caller-given logits_dev [B][V]
  * fp32, as position t: writes token_dev [B] int32, logp_dev [B] (raw
  * log-softmax of the token, may be NULL) and logmu_dev [B] (tempered and

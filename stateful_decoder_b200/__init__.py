@@ -43,7 +43,7 @@ EXPORTED = (
     "rlt_state_create", "rlt_state_free", "rlt_state_reset", "rlt_state_info_get", "rlt_state_read",
     "rlt_encode_prefix", "rlt_readout", "rlt_decoder_step", "rlt_prefill", "rlt_replay_logprobs",
     "rlt_last_error", "rlt_check_device", "rlt_profile_enable", "rlt_profile_read", "rlt_op_linear",
-    "rlt_op_sample", "rlt_kernel_launches", "rlt_op_prefix_attention",
+    "rlt_op_sample", "rlt_kernel_launches", "rlt_op_prefix_attention", "rlt_op_prefix_attention_noalloc",
 )
 
 
@@ -99,6 +99,8 @@ _sig = {
     "rlt_replay_logprobs": [_vp, _vp, _i32, _i32, _vp, _vp],
     "rlt_op_linear": [_vp, _vp, _vp, _i32, _i32, _i32, _i32, _i32, _vp],
     "rlt_op_prefix_attention": [_vp, _vp, _vp, ctypes.c_int64, _i32, _i32, _i32, _i32, _i32, _vp, _i32, _vp, _vp],
+    "rlt_op_prefix_attention_noalloc": [_vp, _vp, _vp, ctypes.c_int64, _i32, _i32, _i32, _i32, _i32, _vp, _i32, _vp,
+                                        _vp],
     "rlt_op_sample": [_vp, _i32, _i32, ctypes.POINTER(Sampling), ctypes.c_uint32, _vp, _vp, _vp, _vp],
     "rlt_last_error": [ctypes.c_char_p, ctypes.c_size_t],
     "rlt_check_device": [],
@@ -309,6 +311,13 @@ def rlt_op_prefix_attention(q, k, v, n: int, out, rope_cs=None, qpos: int = 0, s
     """out [B, H*hd] = attention of q [B, H*hd] (fp32) over rows 0..n-1 of
     k, v [B, H, ld_t, hd] (bf16 or fp32); rope_cs [pos, hd/2, 2] rotates q at qpos."""
     _check(_lib.rlt_op_prefix_attention(*_prefix_attention_args(q, k, v, n, out, rope_cs, qpos, stream)))
+
+
+def rlt_op_prefix_attention_noalloc(q, k, v, n: int, out, rope_cs=None, qpos: int = 0, stream=None) -> None:
+    """Same as rlt_op_prefix_attention, but its scratch is the library's static
+    16 MiB device array instead of a per-call allocation (for callers that
+    cannot allocate device memory); calls that overlap on the GPU race on it."""
+    _check(_lib.rlt_op_prefix_attention_noalloc(*_prefix_attention_args(q, k, v, n, out, rope_cs, qpos, stream)))
 
 
 def rlt_op_sample(logits, sampling: dict, t: int, token, logp=None, logmu=None, stream=None) -> None:

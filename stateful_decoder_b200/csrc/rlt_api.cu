@@ -21,6 +21,7 @@
 #include <cstdio>
 #include <cstring>
 #include <map>
+#include <mutex>
 #include <string>
 #include <vector>
 
@@ -997,3 +998,61 @@ int32_t rlt_profile_read(rlt_model* m, int32_t kind, double* ms, int64_t* launch
 }
 
 }  // extern "C"
+
+// ====================================================================== no-alloc variant
+// rlt_op_prefix_attention_noalloc: the split-key attention with its chunk
+// partials in a static device array instead of memory allocated per call (for
+// callers that own all device memory or cannot take an allocation's implicit
+// synchronisation).  The array is 16 MiB; host code must not use its name as
+// a device pointer (in host code it is only a stand-in), so the device
+// address is looked up per device with cudaGetSymbolAddress.
+namespace {
+constexpr size_t kNoallocScratchFloats = (size_t)4 << 20;  // 16 MiB
+static __device__ __align__(256) float g_noalloc_scratch[kNoallocScratchFloats];
+
+std::mutex g_noalloc_mu;
+std::map<int, float*> g_noalloc_ptr;  // device ordinal -> device address of the array
+
+int32_t noalloc_scratch(float** out) {
+  int dev = 0;
+  RLT_CUDA(cudaGetDevice(&dev));
+  std::lock_guard<std::mutex> g(g_noalloc_mu);
+  auto it = g_noalloc_ptr.find(dev);
+  if (it == g_noalloc_ptr.end()) {
+    void* p = nullptr;
+    RLT_CUDA(cudaGetSymbolAddress(&p, g_noalloc_scratch));
+    it = g_noalloc_ptr.emplace(dev, static_cast<float*>(p)).first;
+  }
+  *out = it->second;
+  return RLT_OK;
+}
+}  // namespace
+
+extern "C" int32_t rlt_op_prefix_attention_noalloc(const float* q_dev, const void* k_dev, const void* v_dev,
+                                                   int64_t ld_t, int32_t B, int32_t H, int32_t hd, int32_t n,
+                                                   int32_t dtype, const float* rope_cs_dev, int32_t qpos,
+                                                   void* out_dev, void* stream) {
+  if (!q_dev || !k_dev || !v_dev || !out_dev || B <= 0 || H <= 0 || n <= 0 || ld_t < n || qpos < 0)
+    return fail(RLT_E_INVAL, "bad prefix attention arguments");
+  if (!(hd == 16 || hd == 32 || hd == 64 || hd == 128 || hd == 256)) return fail(RLT_E_INVAL, "head size");
+  if (dtype != RLT_DTYPE_F32 && dtype != RLT_DTYPE_BF16) return fail(RLT_E_INVAL, "dtype");
+  const size_t need = prefix_attn_workspace_floats(B, H, hd, n);
+  if (need > kNoallocScratchFloats)
+    return fail(RLT_E_CAPACITY, "prefix attention needs " + std::to_string(need) +
+                                    " floats of scratch; the static scratch array holds " +
+                                    std::to_string(kNoallocScratchFloats));
+  float* ws = nullptr;
+  if (need) RLT_TRY(noalloc_scratch(&ws));
+  cudaStream_t st = (cudaStream_t)stream;
+  cudaError_t e;
+  if (dtype == RLT_DTYPE_BF16)
+    e = prefix_attn<bf16>(q_dev, (int64_t)H * hd, static_cast<const bf16*>(k_dev), static_cast<const bf16*>(v_dev), ld_t,
+                          B, H, hd, n, qpos, rope_cs_dev, static_cast<bf16*>(out_dev), (int64_t)H * hd, ws,
+                          kNoallocScratchFloats, st);
+  else
+    e = prefix_attn<float>(q_dev, (int64_t)H * hd, static_cast<const float*>(k_dev), static_cast<const float*>(v_dev),
+                           ld_t, B, H, hd, n, qpos, rope_cs_dev, static_cast<float*>(out_dev), (int64_t)H * hd, ws,
+                           kNoallocScratchFloats, st);
+  if (e != cudaSuccess) return fail(RLT_E_CUDA, std::string("prefix attention: ") + cudaGetErrorString(e));
+  return ok();
+}
