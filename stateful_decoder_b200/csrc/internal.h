@@ -77,6 +77,11 @@ template <typename KT>
 cudaError_t causal_attn(const KT* q, const KT* k, const KT* v, int64_t ld_tq, int64_t ld_tkv, int B, int H, int hd,
                         int T, KT* out, int64_t ld_out, cudaStream_t st);
 
+// The same on the tensor cores (bf16, hd 64 or 128): two-pass softmax with
+// S and O in tensor memory.
+cudaError_t causal_attn_tc(const bf16* q, const bf16* k, const bf16* v, int64_t ld_tq, int64_t ld_tkv, int B, int H,
+                           int hd, int T, bf16* out, int64_t ld_out, cudaStream_t st);
+
 // ---------------------------------------------------------------- elementwise
 // Generator fill of a [rows][cols] view (rows `pitch` elements apart).
 template <typename WT>

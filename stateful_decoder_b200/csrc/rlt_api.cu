@@ -18,6 +18,7 @@
 #include <cuda_runtime.h>
 
 #include <cmath>
+#include <type_traits>
 #include <cstdio>
 #include <cstring>
 #include <map>
@@ -486,8 +487,17 @@ int32_t encode_prefix_impl(rlt_model* m, rlt_state* S, const int32_t* tok, int32
       RLT_CUDA((head_scatter<T, T>(qkv, 3 * d, 0, rows, Tn, 0, H, hd, 1, m->rope_cs, static_cast<T*>(S->pf_q), Tn, st)));
       RLT_CUDA((head_scatter<T, T>(qkv, 3 * d, d, rows, Tn, 0, H, hd, 1, m->rope_cs, kdst, ld_tk, st)));
       RLT_CUDA((head_scatter<T, T>(qkv, 3 * d, 2 * d, rows, Tn, 0, H, hd, 0, m->rope_cs, vdst, ld_tk, st)));
-      RLT_CUDA(causal_attn<T>(static_cast<const T*>(S->pf_q), kdst, vdst, Tn, ld_tk, Bc, H, hd, Tn,
-                              static_cast<T*>(S->pf_attn), d, st));
+      if constexpr (std::is_same<T, bf16>::value) {
+        if (hd == 64 || hd == 128)
+          RLT_CUDA(causal_attn_tc(static_cast<const bf16*>(S->pf_q), kdst, vdst, Tn, ld_tk, Bc, H, hd, Tn,
+                                  static_cast<bf16*>(S->pf_attn), d, st));
+        else
+          RLT_CUDA(causal_attn<T>(static_cast<const T*>(S->pf_q), kdst, vdst, Tn, ld_tk, Bc, H, hd, Tn,
+                                  static_cast<T*>(S->pf_attn), d, st));
+      } else {
+        RLT_CUDA(causal_attn<T>(static_cast<const T*>(S->pf_q), kdst, vdst, Tn, ld_tk, Bc, H, hd, Tn,
+                                static_cast<T*>(S->pf_attn), d, st));
+      }
       RLT_TRY(gemm<T>(S, w.wo, d, S->pf_attn, d, d, (int)rows, d, EPI_RESID, epi_out(e0, emap, 0), false, st));
       RLT_CUDA(rmsnorm<T, T>(e0, emap, static_cast<const T*>(w.g_ef), rows, d, c.rms_eps, static_cast<T*>(S->pf_x), d, st));
       RLT_TRY(gemm<T>(S, w.w13, d, S->pf_x, d, 2 * F, (int)rows, d, EPI_SWIGLU, epi_out(S->pf_big, plain_rows(F), is_bf16),
