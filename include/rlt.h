@@ -285,8 +285,11 @@ int32_t rlt_last_error(char* buf, size_t n);
 int32_t rlt_check_device(void);
 
 /* Kernel timing hook for measurement: when enabled, the library records CUDA
- * events on the launching stream around every launch of the decode-attention
- * kernels.  Enabling (or disabling) clears the record.  rlt_profile_read
+ * events on the launching stream around the decode-attention launches of
+ * every 4th position (t = 0 mod 4), and wraps the token-parallel encoder and
+ * the transitions with t = 64 (mod 128) in an NVTX range "rlt_sample" (a
+ * stratified sample a kernel profiler can select).  Enabling (or disabling)
+ * clears the record.  rlt_profile_read
  * synchronises the device and, for kind 0 (prefix attention: cross-attention
  * to the memory and the encoder step) or kind 1 (SWA attention), returns the
  * summed event intervals in milliseconds, the launch count and the

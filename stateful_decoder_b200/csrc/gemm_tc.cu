@@ -123,37 +123,55 @@ int max_active_clusters(int cs) {
   return cache[cs];
 }
 
-// Cluster (K-split) size of a decode-step GEMM: the power of two <= 8 that
-// minimises waves x (K blocks per CTA + a fixed per-CTA cost of about four K
-// blocks), with waves counted against the clusters the device can hold at
-// once.  It depends on M and K only (never on N), so a sequence's result does
-// not depend on the batch it shares a step with.  Encoder (token-parallel)
-// GEMMs have many activation tiles and never split.
-int gemm_tc_cluster(int M, int K, int split_mode) {
-  if (!split_mode) return 1;
+// Decode-step plan (activation tile width and K-split cluster size) for an
+// M x K weight, worked out once for the design batch of 256 rows: prefer an
+// unsplit grid of 128- or 256-wide tiles that gives 80..148 CTAs (one wave,
+// no reduction); otherwise the cluster split with the most CTAs that still
+// fit in one wave (cluster occupancy included), wider tiles first.  The
+// cluster size therefore depends on M and K only -- never on the actual
+// batch -- so a sequence's result does not depend on the batch it shares a
+// step with; only the tile width follows the batch (which does not change
+// the accumulation order).
+struct DecodePlan {
+  int bn, cs;
+};
+
+DecodePlan decode_plan(int M, int K) {
   const int tiles = M / BM, kb = K / BK;
-  int best = 1;
-  long best_cost = -1;
-  for (int cs = 1; cs <= 8; cs *= 2) {
-    if (cs > 1 && kb < 2 * cs) break;
-    const int slots = cs == 1 ? kSmCount : max_active_clusters(cs);
-    const long waves = (tiles + slots - 1) / slots;
-    const long cost = waves * ((kb + cs - 1) / cs + 4);
-    if (best_cost < 0 || cost < best_cost) {
-      best = cs;
-      best_cost = cost;
+  for (int bn : {256, 128}) {
+    const int ctas = tiles * (256 / bn);
+    if (ctas >= 80 && ctas <= kSmCount) return {bn, 1};
+  }
+  if (tiles >= 80) return {256, 1};
+  DecodePlan best{256, 1};
+  int best_ctas = tiles;
+  for (int cs = 2; cs <= 8; cs *= 2) {
+    if (kb < 2 * cs) break;
+    for (int bn : {256, 128}) {
+      const int clusters = tiles * (256 / bn), ctas = clusters * cs;
+      if (ctas > kSmCount || clusters > max_active_clusters(cs)) continue;
+      if (ctas > best_ctas || (ctas == best_ctas && bn > best.bn)) {
+        best = {bn, cs};
+        best_ctas = ctas;
+      }
     }
   }
   return best;
 }
 
-// Activation tile width: the smallest of 32/64/128/256 that covers N.
-int gemm_tc_bn(int N) { return N <= 32 ? 32 : N <= 64 ? 64 : N <= 128 ? 128 : 256; }
+int gemm_tc_cluster(int M, int K, int split_mode) { return split_mode ? decode_plan(M, K).cs : 1; }
+
+// Activation tile width: the smallest of 32/64/128/256 that covers N, except
+// that decode steps with more than 128 rows use the planned width.
+int gemm_tc_bn(int M, int N, int K, int split_mode) {
+  if (split_mode && N > 128) return decode_plan(M, K).bn;
+  return N <= 32 ? 32 : N <= 64 ? 64 : N <= 128 ? 128 : 256;
+}
 
 cudaError_t gemm_tc(const bf16* W, int64_t ldw, const bf16* X, int64_t ldx, int M, int N, int K, int epi,
                     const EpiParams& ep, int split_mode, cudaStream_t st) {
   if (M % BM || K % BK || N <= 0) return cudaErrorInvalidValue;
-  const int bn = gemm_tc_bn(N);
+  const int bn = gemm_tc_bn(M, N, K, split_mode);
   const int cs = gemm_tc_cluster(M, K, split_mode);
   const int kb = K / BK;
   const int per = (kb + cs - 1) / cs;

@@ -45,7 +45,7 @@ cudaError_t launch_pdl(void (*kernel)(KArgs...), dim3 grid, dim3 block, size_t s
 cudaError_t gemm_tc(const bf16* W, int64_t ldw, const bf16* X, int64_t ldx, int M, int N, int K, int epi,
                     const EpiParams& ep, int split_mode, cudaStream_t st);
 int gemm_tc_cluster(int M, int K, int split_mode);
-int gemm_tc_bn(int N);
+int gemm_tc_bn(int M, int N, int K, int split_mode);
 
 // CUDA-core GEMM (fp32 models; also a cross-check for the tensor-core path).
 template <typename WT, typename XT>
