@@ -34,6 +34,24 @@ struct EpiParams {
   const void* bias;     // GATE: b_g [M], model storage type
   int bias_bf16;
   float alpha;          // MERGE: feedback scale
+  // RMSNorm of the next sublayer folded into the epilogues.  A producer
+  // (RESID/MERGE/CONVEX with zb != null) also writes zb[n][m] =
+  // bf16(gamma_next[m] * z) and, per 128-row weight tile mt, the partial sum
+  // ss_out[mt][n] of z^2 over that tile's rows.  A consumer (STORE/SWIGLU
+  // with ss_in != null) reads such a zb as its activation operand and scales
+  // each accumulator of row n by 1/sqrt(norm_scale * sum_mt ss_in[mt][n] +
+  // norm_eps): gamma * z / rms(z) times a weight row equals 1/rms(z) times
+  // the weight row applied to gamma * z.
+  bf16* zb;
+  int64_t ld_zb;
+  const void* gamma_next;
+  int gamma_bf16;
+  float* ss_out;
+  const float* ss_in;
+  int n_ss;
+  int64_t ss_ld;
+  float norm_scale;
+  float norm_eps;
 };
 
 __device__ __forceinline__ float sigmoidf_(float x) { return 1.0f / (1.0f + __expf(-x)); }
@@ -79,6 +97,70 @@ __device__ __forceinline__ void epi_apply_at(const EpiParams& p, int64_t n, int6
 template <int EPI>
 __device__ __forceinline__ void epi_apply(const EpiParams& p, int64_t n, int m, float acc) {
   epi_apply_at<EPI>(p, n, p.out_map.off(n), epi_uses_aux0<EPI>() ? p.aux0_map.off(n) : 0, m, acc);
+}
+
+// Two-phase form of the same epilogues, so that a thread can issue the loads
+// of many outputs before any store (read-modify-write epilogues would
+// otherwise wait on one load per output): epi_load fetches what the
+// epilogue reads (old residual, e_t, gate), epi_store finishes it.
+struct EpiPre {
+  float a, b;
+};
+
+template <int EPI>
+__device__ __forceinline__ EpiPre epi_load(const EpiParams& p, int64_t n, int64_t orow, int64_t arow, int m) {
+  EpiPre r{0.f, 0.f};
+  if constexpr (EPI == EPI_RESID) {
+    r.a = reinterpret_cast<const float*>(p.out)[orow + m];
+  } else if constexpr (EPI == EPI_MERGE) {
+    r.a = p.aux0[arow + m];
+    r.b = p.aux1[n * p.ld_aux1 + m];
+  } else if constexpr (EPI == EPI_CONVEX) {
+    r.a = p.aux0[arow + m];
+    r.b = reinterpret_cast<const float*>(p.out)[orow + m];
+  } else if constexpr (EPI == EPI_GATE) {
+    r.a = load_bias(p, m);
+  }
+  return r;
+}
+
+// Does the epilogue produce a residual-stream value z (and so may feed the
+// next sublayer's folded RMSNorm)?
+template <int EPI>
+__device__ __forceinline__ constexpr bool epi_produces_z() {
+  return EPI == EPI_RESID || EPI == EPI_MERGE || EPI == EPI_CONVEX;
+}
+
+__device__ __forceinline__ float load_gamma(const EpiParams& p, int m) {
+  return p.gamma_bf16 ? __bfloat162float(reinterpret_cast<const bf16*>(p.gamma_next)[m])
+                      : reinterpret_cast<const float*>(p.gamma_next)[m];
+}
+
+// Finishes the epilogue of output (n, m); returns z for producers (0 else).
+template <int EPI>
+__device__ __forceinline__ float epi_store(const EpiParams& p, int64_t n, int64_t orow, int m, float acc, EpiPre pre) {
+  float z = 0.f;
+  if constexpr (EPI == EPI_STORE) {
+    const int64_t o = orow + m;
+    if (p.out_bf16) reinterpret_cast<bf16*>(p.out)[o] = __float2bfloat16_rn(acc);
+    else reinterpret_cast<float*>(p.out)[o] = acc;
+  } else if constexpr (EPI == EPI_RESID) {
+    z = pre.a + acc;
+    reinterpret_cast<float*>(p.out)[orow + m] = z;
+  } else if constexpr (EPI == EPI_GATE) {
+    reinterpret_cast<float*>(p.out)[orow + m] = sigmoidf_(acc + pre.a);
+  } else if constexpr (EPI == EPI_MERGE) {
+    z = pre.a + p.alpha * pre.b * acc;
+    reinterpret_cast<float*>(p.out)[orow + m] = z;
+  } else if constexpr (EPI == EPI_CONVEX) {
+    const float g = sigmoidf_(acc);
+    z = g * pre.a + (1.0f - g) * pre.b;
+    reinterpret_cast<float*>(p.out)[orow + m] = z;
+  }
+  if constexpr (epi_produces_z<EPI>()) {
+    if (p.zb != nullptr) p.zb[n * p.ld_zb + m] = __float2bfloat16_rn(load_gamma(p, m) * z);
+  }
+  return z;
 }
 
 // SWIGLU pair epilogue: gate accumulator of row 2i and up accumulator of row

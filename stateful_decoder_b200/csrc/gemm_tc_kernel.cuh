@@ -38,7 +38,9 @@ struct TcCfg {
   static constexpr int STAGE_BYTES = A_BYTES + B_BYTES;
   static constexpr int STAGES = BN >= 256 ? 4 : (BN >= 128 ? 6 : 8);
   static constexpr int PIPE_BYTES = STAGES * STAGE_BYTES;
-  static constexpr int SMEM = PIPE_BYTES + 1024 /*align*/ + 256 /*barriers*/;
+  static constexpr int EXTRA_OFF = PIPE_BYTES + 256;  // after the barriers
+  static constexpr int SMEM = PIPE_BYTES + 1024 /*align*/ + 256 /*barriers*/ + 1024 /*1/rms per column*/ +
+                              512 /*per-warp column sums*/;
   static constexpr int TMEM_COLS = BN;  // power of two >= 32
   static_assert(BN * BM * 4 <= PIPE_BYTES, "cluster partial tile must fit in the pipeline buffers");
 };
@@ -116,27 +118,73 @@ __device__ __forceinline__ float dsmem_ld(uint32_t addr) {
   return v;
 }
 
-// Applies the epilogue to accumulator columns [n0, n0 + cnt) (cnt <= 32) of
-// this thread's row m.  Row offsets (which may need a division for grouped
-// rows) are computed once per column by lane j and broadcast.
+// Butterfly transpose-reduction over the 32 lanes of a warp: on entry zv[j]
+// is this lane's value for column j; on exit zv[0] of lane j is the sum over
+// all lanes of column j (31 shuffles, fixed order).
+__device__ __forceinline__ void warp_column_sums(float* zv, int lane) {
+#pragma unroll
+  for (int off = 16; off >= 1; off >>= 1) {
+    const bool upper = (lane & off) != 0;
+#pragma unroll
+    for (int i = 0; i < off; ++i) {
+      const float send = upper ? zv[i] : zv[i + off];
+      const float keep = upper ? zv[i + off] : zv[i];
+      zv[i] = keep + __shfl_xor_sync(0xffffffffu, send, off);
+    }
+  }
+}
+
+// Finishes accumulator columns [n0, n0 + cnt) (cnt <= 32) of this thread's
+// row m (row `row` of weight tile m_tile): folded RMSNorm scale (consumers),
+// the epilogue (loads of each 16-column group issued before its stores), and
+// for producers the tile's per-column sums of z^2.  Called by all 128
+// threads together (it contains block barriers).  Row offsets, which may
+// need a division for grouped rows, are computed once per column by lane j.
 template <int EPI>
-__device__ __forceinline__ void epilogue_cols(const EpiParams& ep, int64_t n0, int cnt, int64_t N, int m, int lane,
-                                              const float* v) {
+__device__ __forceinline__ void finish_chunk(const EpiParams& ep, int64_t n0, int cnt, int64_t N, int m, int m_tile,
+                                             int warp, int lane, float* v, const float* rinv, float* red) {
+  if (ep.ss_in != nullptr) {
+#pragma unroll
+    for (int j = 0; j < 32; ++j) v[j] *= rinv[j];
+  }
   const int64_t my_n = n0 + lane;
   const bool my_ok = lane < cnt && my_n < N;
   const int64_t my_o = my_ok ? ep.out_map.off(my_n) : 0;
   const int64_t my_a = (epi_uses_aux0<EPI>() && my_ok) ? ep.aux0_map.off(my_n) : 0;
+  if constexpr (EPI == EPI_SWIGLU) {
 #pragma unroll
-  for (int j = 0; j < 32; ++j) {
-    const int64_t n = n0 + j;
-    const bool okj = j < cnt && n < N;
-    const int64_t orow = __shfl_sync(0xffffffffu, my_o, j);
-    if constexpr (EPI == EPI_SWIGLU) {
+    for (int j = 0; j < 32; ++j) {
+      const int64_t orow = __shfl_sync(0xffffffffu, my_o, j);
       const float other = __shfl_xor_sync(0xffffffffu, v[j], 1);
-      if (okj && (lane & 1) == 0) epi_swiglu_at(ep, orow, m >> 1, v[j], other);
-    } else {
-      const int64_t arow = epi_uses_aux0<EPI>() ? __shfl_sync(0xffffffffu, my_a, j) : 0;
-      if (okj) epi_apply_at<EPI>(ep, n, orow, arow, m, v[j]);
+      if (j < cnt && n0 + j < N && (lane & 1) == 0) epi_swiglu_at(ep, orow, m >> 1, v[j], other);
+    }
+  } else {
+#pragma unroll
+    for (int h = 0; h < 32; h += 16) {
+      int64_t orow[16];
+      EpiPre pre[16];
+#pragma unroll
+      for (int j = 0; j < 16; ++j) {
+        orow[j] = __shfl_sync(0xffffffffu, my_o, h + j);
+        const int64_t arow = epi_uses_aux0<EPI>() ? __shfl_sync(0xffffffffu, my_a, h + j) : 0;
+        pre[j] = (h + j < cnt && n0 + h + j < N) ? epi_load<EPI>(ep, n0 + h + j, orow[j], arow, m) : EpiPre{0.f, 0.f};
+      }
+#pragma unroll
+      for (int j = 0; j < 16; ++j) {
+        const bool okj = h + j < cnt && n0 + h + j < N;
+        const float z = okj ? epi_store<EPI>(ep, n0 + h + j, orow[j], m, v[h + j], pre[j]) : 0.f;
+        v[h + j] = z * z;  // v is free now: reuse it for z^2
+      }
+    }
+    if constexpr (epi_produces_z<EPI>()) {
+      if (ep.ss_out != nullptr) {
+        warp_column_sums(v, lane);
+        red[warp * 32 + lane] = v[0];
+        __syncthreads();
+        if (warp == 0 && lane < cnt && n0 + lane < N)
+          ep.ss_out[(int64_t)m_tile * ep.ss_ld + n0 + lane] = red[lane] + red[32 + lane] + red[64 + lane] + red[96 + lane];
+        __syncthreads();
+      }
     }
   }
 }
@@ -247,20 +295,35 @@ __global__ void __launch_bounds__(128, 1)
   const int row = warp * 32 + lane;
   const int m = m_tile * BM + row;
   const int64_t n_base = (int64_t)n_tile * BN;
+  float* rinv = reinterpret_cast<float*>(smem + C::EXTRA_OFF);  // [BN] folded RMSNorm scale per column
+  float* red = rinv + 256;                                        // [4][32] per-warp column sums
+  if (ep.ss_in != nullptr) {
+    for (int i = threadIdx.x; i < BN; i += 128) {
+      const int64_t n = n_base + i;
+      float ss = 0.f;
+      if (n < N)
+        for (int mt = 0; mt < ep.n_ss; ++mt) ss += ep.ss_in[(int64_t)mt * ep.ss_ld + n];
+      rinv[i] = rsqrtf(ss * ep.norm_scale + ep.norm_eps);
+    }
+  }
+  __syncthreads();
   if constexpr (CS == 1) {
-    if (good) {
 #pragma unroll 1
-      for (int c = 0; c < BN; c += 32) {
-        if (n_base + c >= N) break;
-        float v[32];
+    for (int c = 0; c < BN; c += 32) {
+      if (n_base + c >= N) break;
+      float v[32];
+      if (good) {
         tmem_ld32(tmem_base + ((uint32_t)(warp * 32) << 16) + (uint32_t)c, v);
-        epilogue_cols<EPI>(ep, n_base + c, 32, N, m, lane, v);
+      } else {
+#pragma unroll
+        for (int j = 0; j < 32; ++j) v[j] = 0.f;
       }
+      finish_chunk<EPI>(ep, n_base + c, 32, N, m, m_tile, warp, lane, v, rinv + c, red);
     }
   } else {
     // Partial tile to this CTA's shared memory (the pipeline buffers are idle
     // now: every MMA that read them has completed), column-major [BN][128].
-    float* red = reinterpret_cast<float*>(smem);
+    float* part = reinterpret_cast<float*>(smem);
 #pragma unroll 1
     for (int c = 0; c < BN; c += 32) {
       float v[32];
@@ -271,36 +334,37 @@ __global__ void __launch_bounds__(128, 1)
         for (int j = 0; j < 32; ++j) v[j] = 0.f;
       }
 #pragma unroll
-      for (int j = 0; j < 32; ++j) red[(c + j) * BM + row] = v[j];
+      for (int j = 0; j < 32; ++j) part[(c + j) * BM + row] = v[j];
     }
     cluster_sync_all();
     // This CTA reduces columns [split*COLS, (split+1)*COLS) over all ranks, in
-    // rank order.  Decode-step outputs use plain row maps (no grouped rows),
-    // so each column's row offset is a multiply, applied per element.
+    // rank order, 32 columns at a time.
     constexpr int COLS = BN / CS;
-    const uint32_t red_local = smem_u32(red);
+    const uint32_t part_local = smem_u32(part);
 #pragma unroll 1
-    for (int cc = 0; cc < COLS; cc += 4) {
-      float t[4][CS];
+    for (int cc = 0; cc < COLS; cc += 32) {
+      const int c0 = split * COLS + cc;
+      const int cnt = COLS - cc < 32 ? COLS - cc : 32;
+      if (n_base + c0 >= N) break;
+      float v[32];
 #pragma unroll
-      for (int j = 0; j < 4; ++j) {
-        const uint32_t off = red_local + (uint32_t)(((split * COLS + cc + j) * BM + row) * 4);
+      for (int g = 0; g < 32; g += 8) {
+        float t[8][CS];
 #pragma unroll
-        for (int p = 0; p < CS; ++p) t[j][p] = (cc + j < COLS) ? dsmem_ld(dsmem_addr(off, (uint32_t)p)) : 0.f;
-      }
+        for (int j = 0; j < 8; ++j) {
+          const uint32_t off = part_local + (uint32_t)(((c0 + g + j) * BM + row) * 4);
 #pragma unroll
-      for (int j = 0; j < 4; ++j) {
-        float acc = 0.f;
+          for (int p = 0; p < CS; ++p) t[j][p] = (g + j < cnt) ? dsmem_ld(dsmem_addr(off, (uint32_t)p)) : 0.f;
+        }
 #pragma unroll
-        for (int p = 0; p < CS; ++p) acc += t[j][p];
-        const int64_t n = n_base + split * COLS + cc + j;
-        if constexpr (EPI == EPI_SWIGLU) {
-          const float other = __shfl_xor_sync(0xffffffffu, acc, 1);
-          if (cc + j < COLS && n < N && (lane & 1) == 0) epi_swiglu(ep, n, m >> 1, acc, other);
-        } else {
-          if (cc + j < COLS && n < N) epi_apply<EPI>(ep, n, m, acc);
+        for (int j = 0; j < 8; ++j) {
+          float acc = 0.f;
+#pragma unroll
+          for (int p = 0; p < CS; ++p) acc += t[j][p];
+          v[g + j] = acc;
         }
       }
+      finish_chunk<EPI>(ep, n_base + c0, cnt, N, m, m_tile, warp, lane, v, rinv + c0, red);
     }
     cluster_sync_all();  // peers may still read this CTA's partial until here
   }

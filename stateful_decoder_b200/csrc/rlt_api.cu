@@ -16,6 +16,7 @@
 //   wk_mem.g/wv_mem.g    -> rows [2dg, 2dg+d) and [2dg+d, 2d(g+1)) of [2dG][d]
 // The named tensors of rlt.h are views into these blocks.
 #include <cuda_runtime.h>
+#include <nvtx3/nvToolsExt.h>
 
 #include <cmath>
 #include <type_traits>
@@ -76,6 +77,7 @@ struct LayerW {
 
 struct ProfileRec {
   bool on = false;
+  bool sample_now = false;  // current transition is one of the sampled ones
   std::vector<cudaEvent_t> ev;
   size_t used = 0;
   double bytes[2] = {0, 0};
@@ -113,6 +115,8 @@ struct rlt_state {
   void* ring_k = nullptr; void* ring_v = nullptr;  // [L][B][H][W-1][hd]
   float* s = nullptr;          // [B][d]
   void* xb = nullptr;          // [B][2d] GEMM operand (model dtype)
+  void* zb = nullptr;          // [B][d] bf16 gamma*z operand of the folded RMSNorm (bf16 models)
+  float* ss = nullptr;         // [d/128][B] partial sums of z^2 for the folded RMSNorm
   float* qkv = nullptr;        // [B][max(3d, 2dG)]
   int64_t ld_qkv = 0;
   void* attn = nullptr;        // [B][d]
@@ -321,12 +325,34 @@ EpiParams epi_out(void* out, RowMap map, int out_bf16) {
   return p;
 }
 
+// Folded RMSNorm (bf16 models): a producer epilogue writes gamma_next * z as
+// the next GEMM's bf16 operand plus per-weight-tile sums of z^2; the
+// consumer GEMM scales its accumulators by 1/rms(z).  The layer norms of the
+// decoder therefore need no kernel of their own.
+EpiParams norm_out(EpiParams p, rlt_state* S, const void* gamma) {
+  p.zb = static_cast<bf16*>(S->zb);
+  p.ld_zb = S->m->cfg.d_model;
+  p.gamma_next = gamma;
+  p.gamma_bf16 = 1;
+  p.ss_out = S->ss;
+  p.ss_ld = S->B;
+  return p;
+}
+EpiParams norm_in(EpiParams p, rlt_state* S) {
+  p.ss_in = S->ss;
+  p.n_ss = S->m->cfg.d_model / 128;
+  p.ss_ld = S->B;
+  p.norm_scale = 1.0f / (float)S->m->cfg.d_model;
+  p.norm_eps = S->m->cfg.rms_eps;
+  return p;
+}
+
 // ------------------------------------------------------------------ profiling
 // Records an event before (prof_begin) and after (prof_end) one kernel launch
 // on the launching stream; kind 0 = prefix attention, 1 = SWA attention.
 void prof_begin(rlt_model* m, cudaStream_t st) {
   ProfileRec& p = m->prof;
-  if (!p.on) return;
+  if (!p.on || !p.sample_now) return;
   if (p.used + 2 > p.ev.size()) {
     for (int i = 0; i < 1024; ++i) {
       cudaEvent_t e;
@@ -338,7 +364,7 @@ void prof_begin(rlt_model* m, cudaStream_t st) {
 }
 void prof_end(rlt_model* m, cudaStream_t st, int kind, double bytes) {
   ProfileRec& p = m->prof;
-  if (!p.on || p.used + 2 > p.ev.size()) return;
+  if (!p.on || !p.sample_now || p.used + 2 > p.ev.size()) return;
   cudaEventRecord(p.ev[p.used + 1], st);
   p.kind.push_back(kind);
   p.bytes[kind] += bytes;
@@ -377,6 +403,11 @@ int32_t make_state(rlt_model* m, int32_t B, int32_t max_len, int32_t flags, rlt_
   if ((r = A(&p, (int64_t)B * d * 4))) goto fail_;
   S->s = static_cast<float*>(p);
   if ((r = A(&S->xb, (int64_t)B * 2 * d * es))) goto fail_;
+  if (c.dtype == RLT_DTYPE_BF16) {
+    if ((r = A(&S->zb, (int64_t)B * d * 2))) goto fail_;
+    if ((r = A(&p, (int64_t)(d / 128) * B * 4))) goto fail_;
+    S->ss = static_cast<float*>(p);
+  }
   S->ld_qkv = std::max<int64_t>(3 * d, 2 * d * G);
   if ((r = A(&p, (int64_t)B * S->ld_qkv * 4))) goto fail_;
   S->qkv = static_cast<float*>(p);
@@ -453,6 +484,11 @@ int32_t check_state(rlt_model* m, rlt_state* S) {
 // memory projection of eq. 2.2, chunked over sequences.
 template <typename T>
 int32_t encode_prefix_impl(rlt_model* m, rlt_state* S, const int32_t* tok, int32_t Tn, cudaStream_t st) {
+  struct Range {
+    bool on;
+    explicit Range(bool o) : on(o) { if (on) nvtxRangePushA("rlt_sample"); }
+    ~Range() { if (on) nvtxRangePop(); }
+  } range(m->prof.on);
   const rlt_config& c = m->cfg;
   const int d = c.d_model, H = c.n_heads, hd = m->hd, F = c.ffn, G = c.groups, L = c.n_layers;
   const int is_bf16 = c.dtype == RLT_DTYPE_BF16;
@@ -528,6 +564,7 @@ int32_t encode_step_impl(rlt_model* m, rlt_state* S, const int32_t* tok, cudaStr
   const int d = c.d_model, H = c.n_heads, hd = m->hd, F = c.ffn, G = c.groups, L = c.n_layers, B = S->B;
   const int is_bf16 = c.dtype == RLT_DTYPE_BF16;
   const int t = S->n_enc + 1;
+  m->prof.sample_now = (t % 4) == 0;
   float* et = S->e + (int64_t)(t - 1) * d;
   const RowMap emap = plain_rows((int64_t)S->max_len * d);
   RLT_CUDA(embed<T>(tok, B, 1, 1, static_cast<const T*>(m->emb), d, c.vocab, et, emap, st));
@@ -566,15 +603,35 @@ int32_t encode_step_impl(rlt_model* m, rlt_state* S, const int32_t* tok, cudaStr
 // One decoder transition H_t = D_phi(Merge(e_t, s_{t-1}); M_<=t, C^D_{t-1}, t)
 // (eqs. 2.4-2.5, 2.9-2.16) for t = n_dec + 1.  s is updated in place: it
 // holds u_t after the merge, then z^l after every block, and s_t at the end.
+// While profiling is on, every 4th transition records kernel events
+// (prof_begin/prof_end), and each position with t = 64 (mod 128) -- its
+// encoder step, transition and readout -- is wrapped in an NVTX range named
+// "rlt_sample", so a kernel profiler can capture a stratified sample of a
+// long schedule instead of every launch.
+struct StepRange {
+  bool nvtx = false;
+  StepRange(rlt_model* m, int t) {
+    if (m->prof.on && (t % 128) == 64) {
+      nvtxRangePushA("rlt_sample");
+      nvtx = true;
+    }
+  }
+  ~StepRange() {
+    if (nvtx) nvtxRangePop();
+  }
+};
+
 template <typename T>
 int32_t transition_impl(rlt_model* m, rlt_state* S, cudaStream_t st) {
   const rlt_config& c = m->cfg;
   const int d = c.d_model, H = c.n_heads, hd = m->hd, F = c.ffn, L = c.n_layers, B = S->B, W = c.window;
   const int is_bf16 = c.dtype == RLT_DTYPE_BF16;
   const int t = S->n_dec + 1;
+  m->prof.sample_now = (t % 4) == 0;
   const float* et = S->e + (int64_t)(t - 1) * d;
   const RowMap emap = plain_rows((int64_t)S->max_len * d);
   const RowMap srow = plain_rows(d);
+  constexpr bool fused = std::is_same<T, bf16>::value;  // folded RMSNorm on the tensor-core path
   // merge
   RLT_CUDA((merge_prep<T, T>(et, emap, S->s, static_cast<const T*>(m->g_merge), B, d, c.rms_eps, c.merge_kind,
                              static_cast<T*>(S->xb), st)));
@@ -589,42 +646,55 @@ int32_t transition_impl(rlt_model* m, rlt_state* S, cudaStream_t st) {
     u.aux1 = S->gate;
     u.ld_aux1 = d;
     u.alpha = c.alpha;
+    if (fused) u = norm_out(u, S, m->layers[0].g_dsa);
     RLT_TRY(gemm<T>(S, m->w_state, d, off(S->xb, d, m->esz), 2 * d, d, B, d, EPI_MERGE, u, true, st));
   } else {
     EpiParams u = epi_out(S->s, srow, 0);
     u.aux0 = et;
     u.aux0_map = emap;
+    if (fused) u = norm_out(u, S, m->layers[0].g_dsa);
     RLT_TRY(gemm<T>(S, m->w_gate, 2 * d, S->xb, 2 * d, d, B, 2 * d, EPI_CONVEX, u, true, st));
   }
+  // operand of a normalised sublayer: gamma*z from the previous epilogue
+  // (fused), or a separate RMSNorm of the residual stream
+  auto normed = [&](const void* gamma) -> int32_t {
+    if (fused) return RLT_OK;
+    RLT_CUDA(rmsnorm<T, T>(S->s, srow, static_cast<const T*>(gamma), B, d, c.rms_eps, static_cast<T*>(S->xb), d, st));
+    return RLT_OK;
+  };
+  const void* xin = fused ? S->zb : S->xb;
+  auto cin = [&](EpiParams p) { return fused ? norm_in(p, S) : p; };
+  auto cout_ = [&](EpiParams p, const void* gamma_next) { return fused ? norm_out(p, S, gamma_next) : p; };
   const int n_ring = std::min(t - 1, W - 1);
   for (int l = 0; l < L; ++l) {
     const LayerW& w = m->layers[l];
     const int grp = c.groups == 1 ? 0 : l;
+    const void* g_next = l + 1 < L ? m->layers[l + 1].g_dsa : m->g_out;
     // SWA sublayer (eqs. 2.12-2.14)
-    RLT_CUDA(rmsnorm<T, T>(S->s, srow, static_cast<const T*>(w.g_dsa), B, d, c.rms_eps, static_cast<T*>(S->xb), d, st));
-    RLT_TRY(gemm<T>(S, w.dqkv, d, S->xb, d, 3 * d, B, d, EPI_STORE, epi_out(S->qkv, plain_rows(3 * d), 0), true, st));
+    RLT_TRY(normed(w.g_dsa));
+    RLT_TRY(gemm<T>(S, w.dqkv, d, xin, d, 3 * d, B, d, EPI_STORE, cin(epi_out(S->qkv, plain_rows(3 * d), 0)), true, st));
     const int64_t rlay = (int64_t)l * B * H * (W > 1 ? W - 1 : 0) * hd;
     T* rk = W > 1 ? static_cast<T*>(S->ring_k) + rlay : nullptr;
     T* rv = W > 1 ? static_cast<T*>(S->ring_v) + rlay : nullptr;
     prof_begin(m, st);
     RLT_CUDA(swa_attn<T>(S->qkv, 3 * d, rk, rv, B, H, hd, t, W, m->rope_cs, static_cast<T*>(S->attn), d, st));
     prof_end(m, st, 1, (double)B * H * hd * m->esz * (2.0 * n_ring + (W > 1 ? 2.0 : 0.0)));
-    RLT_TRY(gemm<T>(S, w.dwo, d, S->attn, d, d, B, d, EPI_RESID, epi_out(S->s, srow, 0), true, st));
+    RLT_TRY(gemm<T>(S, w.dwo, d, S->attn, d, d, B, d, EPI_RESID, cout_(epi_out(S->s, srow, 0), w.g_dmem), true, st));
     // cross-attention to M^{g(l)}_{<=t} (eq. 2.15)
-    RLT_CUDA(rmsnorm<T, T>(S->s, srow, static_cast<const T*>(w.g_dmem), B, d, c.rms_eps, static_cast<T*>(S->xb), d, st));
-    RLT_TRY(gemm<T>(S, w.wq_mem, d, S->xb, d, d, B, d, EPI_STORE, epi_out(S->qkv, plain_rows(d), 0), true, st));
+    RLT_TRY(normed(w.g_dmem));
+    RLT_TRY(gemm<T>(S, w.wq_mem, d, xin, d, d, B, d, EPI_STORE, cin(epi_out(S->qkv, plain_rows(d), 0)), true, st));
     const int64_t mg = (int64_t)grp * B * H * S->max_len * hd;
     prof_begin(m, st);
     RLT_CUDA(prefix_attn<T>(S->qkv, d, static_cast<const T*>(S->mem_k) + mg, static_cast<const T*>(S->mem_v) + mg,
                             S->max_len, B, H, hd, t, t - 1, m->rope_cs, static_cast<T*>(S->attn), d, S->attn_ws,
                             S->attn_ws_floats, st));
     prof_end(m, st, 0, (double)B * H * t * hd * 2 * m->esz);
-    RLT_TRY(gemm<T>(S, w.wo_mem, d, S->attn, d, d, B, d, EPI_RESID, epi_out(S->s, srow, 0), true, st));
+    RLT_TRY(gemm<T>(S, w.wo_mem, d, S->attn, d, d, B, d, EPI_RESID, cout_(epi_out(S->s, srow, 0), w.g_dffn), true, st));
     // FFN (eq. 2.16)
-    RLT_CUDA(rmsnorm<T, T>(S->s, srow, static_cast<const T*>(w.g_dffn), B, d, c.rms_eps, static_cast<T*>(S->xb), d, st));
-    RLT_TRY(gemm<T>(S, w.dw13, d, S->xb, d, 2 * F, B, d, EPI_SWIGLU, epi_out(S->hbuf, plain_rows(F), is_bf16),
-                    true, st));
-    RLT_TRY(gemm<T>(S, w.dw2, F, S->hbuf, F, d, B, F, EPI_RESID, epi_out(S->s, srow, 0), true, st));
+    RLT_TRY(normed(w.g_dffn));
+    RLT_TRY(gemm<T>(S, w.dw13, d, xin, d, 2 * F, B, d, EPI_SWIGLU, cin(epi_out(S->hbuf, plain_rows(F), is_bf16)), true,
+                    st));
+    RLT_TRY(gemm<T>(S, w.dw2, F, S->hbuf, F, d, B, F, EPI_RESID, cout_(epi_out(S->s, srow, 0), g_next), true, st));
   }
   S->n_dec = t;
   return RLT_OK;
@@ -637,8 +707,15 @@ int32_t readout_impl(rlt_model* m, rlt_state* S, const int32_t* next, int64_t ne
                      const rlt_sampling* samp, const rlt_readout_out* out, cudaStream_t st) {
   const rlt_config& c = m->cfg;
   const int d = c.d_model, V = c.vocab, B = S->B;
-  RLT_CUDA(rmsnorm<T, T>(S->s, plain_rows(d), static_cast<const T*>(m->g_out), B, d, c.rms_eps, static_cast<T*>(S->xb), d, st));
-  RLT_TRY(gemm<T>(S, m->w_out, d, S->xb, d, V, B, d, EPI_STORE, epi_out(S->logits, plain_rows(V), 0), true, st));
+  if constexpr (std::is_same<T, bf16>::value) {
+    // the last transition's final epilogue left gamma_o * s_t and its sums of squares
+    RLT_TRY(gemm<T>(S, m->w_out, d, S->zb, d, V, B, d, EPI_STORE, norm_in(epi_out(S->logits, plain_rows(V), 0), S),
+                    true, st));
+  } else {
+    RLT_CUDA(rmsnorm<T, T>(S->s, plain_rows(d), static_cast<const T*>(m->g_out), B, d, c.rms_eps,
+                           static_cast<T*>(S->xb), d, st));
+    RLT_TRY(gemm<T>(S, m->w_out, d, S->xb, d, V, B, d, EPI_STORE, epi_out(S->logits, plain_rows(V), 0), true, st));
+  }
   if (next && logp) RLT_CUDA(logp_gather(S->logits, B, V, next, next_stride, logp, ld_logp, st));
   if (samp)
     RLT_CUDA(sample_topk(S->logits, B, V, samp->temperature, samp->top_k, samp->seed, (uint32_t)S->n_dec,
@@ -842,6 +919,7 @@ int32_t rlt_decoder_step(rlt_model* m, rlt_state* s, const int32_t* tok_dev, con
   const int t = s->n_dec + 1;
   if (t > s->max_len) return fail(RLT_E_CAPACITY, "position would pass max_len");
   cudaStream_t st = (cudaStream_t)stream;
+  StepRange range(m, t);
   if (s->n_enc < t) {
     if (!(s->flags & RLT_STATE_ENCODER_CACHE)) return fail(RLT_E_STATE, "x_t not encoded and the state has no encoder cache");
     if (!tok_dev) return fail(RLT_E_INVAL, "x_t must be given when it is not yet encoded");
@@ -861,6 +939,7 @@ int32_t rlt_prefill(rlt_model* m, rlt_state* s, const int32_t* tok_dev, int32_t 
   cudaStream_t st = (cudaStream_t)stream;
   RLT_TRY(RLT_DISPATCH(m, encode_prefix_impl, m, s, tok_dev, T, st));
   for (int t = 1; t <= T; ++t) {
+    StepRange range(m, t);
     RLT_TRY(RLT_DISPATCH(m, transition_impl, m, s, st));
     if (logp_dev && t < T)
       RLT_TRY(RLT_DISPATCH(m, readout_impl, m, s, tok_dev + t, (int64_t)T, logp_dev + (t - 1), (int64_t)(T - 1),
@@ -883,6 +962,7 @@ int32_t rlt_replay_logprobs(rlt_model* m, const int32_t* tok_dev, int32_t B, int
   RLT_TRY(RLT_DISPATCH(m, reset_state, st_, st));
   RLT_TRY(RLT_DISPATCH(m, encode_prefix_impl, m, st_, tok_dev, S, st));
   for (int t = 1; t <= S - 1; ++t) {
+    StepRange range(m, t);
     RLT_TRY(RLT_DISPATCH(m, transition_impl, m, st_, st));
     RLT_TRY(RLT_DISPATCH(m, readout_impl, m, st_, tok_dev + t, (int64_t)S, logp_dev + (t - 1), (int64_t)(S - 1),
                          (const rlt_sampling*)nullptr, (const rlt_readout_out*)false, st));
