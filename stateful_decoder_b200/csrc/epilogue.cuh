@@ -102,27 +102,19 @@ __device__ __forceinline__ void epi_apply(const EpiParams& p, int64_t n, int m, 
 // Two-phase form of the same epilogues, so that a thread can issue the loads
 // of many outputs before any store (read-modify-write epilogues would
 // otherwise wait on one load per output): epi_load fetches what the
-// epilogue reads (old residual, e_t, gate), epi_store finishes it.
+// epilogue reads (old residual, e_t, gate), epi_store finishes it.  What
+// depends on the output feature m alone (bias, next gain) is loaded once per
+// thread into EpiRowConst; the output type (OBF: bf16) and the folded-norm
+// operand (ZB) are template parameters, so a run of outputs compiles to
+// straight-line code.
 struct EpiPre {
   float a, b;
 };
 
-template <int EPI>
-__device__ __forceinline__ EpiPre epi_load(const EpiParams& p, int64_t n, int64_t orow, int64_t arow, int m) {
-  EpiPre r{0.f, 0.f};
-  if constexpr (EPI == EPI_RESID) {
-    r.a = reinterpret_cast<const float*>(p.out)[orow + m];
-  } else if constexpr (EPI == EPI_MERGE) {
-    r.a = p.aux0[arow + m];
-    r.b = p.aux1[n * p.ld_aux1 + m];
-  } else if constexpr (EPI == EPI_CONVEX) {
-    r.a = p.aux0[arow + m];
-    r.b = reinterpret_cast<const float*>(p.out)[orow + m];
-  } else if constexpr (EPI == EPI_GATE) {
-    r.a = load_bias(p, m);
-  }
-  return r;
-}
+struct EpiRowConst {
+  float bias;   // GATE: b_g[m]
+  float gamma;  // producers with zb: gamma_next[m]
+};
 
 // Does the epilogue produce a residual-stream value z (and so may feed the
 // next sublayer's folded RMSNorm)?
@@ -136,19 +128,44 @@ __device__ __forceinline__ float load_gamma(const EpiParams& p, int m) {
                       : reinterpret_cast<const float*>(p.gamma_next)[m];
 }
 
-// Finishes the epilogue of output (n, m); returns z for producers (0 else).
 template <int EPI>
-__device__ __forceinline__ float epi_store(const EpiParams& p, int64_t n, int64_t orow, int m, float acc, EpiPre pre) {
+__device__ __forceinline__ EpiRowConst epi_row_const(const EpiParams& p, int m) {
+  EpiRowConst r{0.f, 0.f};
+  if constexpr (EPI == EPI_GATE) r.bias = load_bias(p, m);
+  if constexpr (epi_produces_z<EPI>()) {
+    if (p.zb != nullptr) r.gamma = load_gamma(p, m);
+  }
+  return r;
+}
+
+template <int EPI>
+__device__ __forceinline__ EpiPre epi_load(const EpiParams& p, int64_t n, int64_t orow, int64_t arow, int m) {
+  EpiPre r{0.f, 0.f};
+  if constexpr (EPI == EPI_RESID) {
+    r.a = reinterpret_cast<const float*>(p.out)[orow + m];
+  } else if constexpr (EPI == EPI_MERGE) {
+    r.a = p.aux0[arow + m];
+    r.b = p.aux1[n * p.ld_aux1 + m];
+  } else if constexpr (EPI == EPI_CONVEX) {
+    r.a = p.aux0[arow + m];
+    r.b = reinterpret_cast<const float*>(p.out)[orow + m];
+  }
+  return r;
+}
+
+// Finishes the epilogue of output (n, m); returns z for producers (0 else).
+template <int EPI, bool OBF, bool ZB>
+__device__ __forceinline__ float epi_store(const EpiParams& p, const EpiRowConst& rc, int64_t n, int64_t orow, int m,
+                                           float acc, EpiPre pre) {
   float z = 0.f;
   if constexpr (EPI == EPI_STORE) {
-    const int64_t o = orow + m;
-    if (p.out_bf16) reinterpret_cast<bf16*>(p.out)[o] = __float2bfloat16_rn(acc);
-    else reinterpret_cast<float*>(p.out)[o] = acc;
+    if constexpr (OBF) reinterpret_cast<bf16*>(p.out)[orow + m] = __float2bfloat16_rn(acc);
+    else reinterpret_cast<float*>(p.out)[orow + m] = acc;
   } else if constexpr (EPI == EPI_RESID) {
     z = pre.a + acc;
     reinterpret_cast<float*>(p.out)[orow + m] = z;
   } else if constexpr (EPI == EPI_GATE) {
-    reinterpret_cast<float*>(p.out)[orow + m] = sigmoidf_(acc + pre.a);
+    reinterpret_cast<float*>(p.out)[orow + m] = sigmoidf_(acc + rc.bias);
   } else if constexpr (EPI == EPI_MERGE) {
     z = pre.a + p.alpha * pre.b * acc;
     reinterpret_cast<float*>(p.out)[orow + m] = z;
@@ -157,9 +174,7 @@ __device__ __forceinline__ float epi_store(const EpiParams& p, int64_t n, int64_
     z = g * pre.a + (1.0f - g) * pre.b;
     reinterpret_cast<float*>(p.out)[orow + m] = z;
   }
-  if constexpr (epi_produces_z<EPI>()) {
-    if (p.zb != nullptr) p.zb[n * p.ld_zb + m] = __float2bfloat16_rn(load_gamma(p, m) * z);
-  }
+  if constexpr (ZB && epi_produces_z<EPI>()) p.zb[n * p.ld_zb + m] = __float2bfloat16_rn(rc.gamma * z);
   return z;
 }
 
@@ -170,6 +185,13 @@ __device__ __forceinline__ void epi_swiglu_at(const EpiParams& p, int64_t orow, 
   const int64_t o = orow + i;
   if (p.out_bf16) reinterpret_cast<bf16*>(p.out)[o] = __float2bfloat16_rn(h);
   else reinterpret_cast<float*>(p.out)[o] = h;
+}
+
+template <bool OBF>
+__device__ __forceinline__ void epi_swiglu_store(const EpiParams& p, int64_t orow, int i, float gate, float up) {
+  const float h = siluf_(gate) * up;
+  if constexpr (OBF) reinterpret_cast<bf16*>(p.out)[orow + i] = __float2bfloat16_rn(h);
+  else reinterpret_cast<float*>(p.out)[orow + i] = h;
 }
 
 __device__ __forceinline__ void epi_swiglu(const EpiParams& p, int64_t n, int i, float gate, float up) {

@@ -134,58 +134,98 @@ __device__ __forceinline__ void warp_column_sums(float* zv, int lane) {
   }
 }
 
-// Finishes accumulator columns [n0, n0 + cnt) (cnt <= 32) of this thread's
-// row m (row `row` of weight tile m_tile): folded RMSNorm scale (consumers),
-// the epilogue (loads of each 16-column group issued before its stores), and
-// for producers the tile's per-column sums of z^2.  Called by all 128
-// threads together (it contains block barriers).  Row offsets, which may
-// need a division for grouped rows, are computed once per column by lane j.
-template <int EPI>
-__device__ __forceinline__ void finish_chunk(const EpiParams& ep, int64_t n0, int cnt, int64_t N, int m, int m_tile,
-                                             int warp, int lane, float* v, const float* rinv, float* red) {
+// Epilogue of CNT accumulator columns n0.. of this thread's row m: loads of
+// each run of up to 16 outputs are issued before their stores.  `full` (all
+// CNT columns exist) selects straight-line code; the ragged tail of N checks
+// every column.  On return v[j] holds z^2 of producers (0 otherwise).
+template <int EPI, int CNT, bool OBF, bool ZB>
+__device__ __forceinline__ void epi_columns(const EpiParams& ep, const EpiRowConst& rc, int64_t n0, int64_t N,
+                                            bool full, int m, int64_t my_o, int64_t my_a, float* v) {
+  constexpr int RUN = CNT < 16 ? CNT : 16;
+#pragma unroll
+  for (int h = 0; h < CNT; h += RUN) {
+    int64_t orow[RUN], arow[RUN];
+    EpiPre pre[RUN];
+#pragma unroll
+    for (int j = 0; j < RUN; ++j) {
+      orow[j] = __shfl_sync(0xffffffffu, my_o, h + j);
+      arow[j] = epi_uses_aux0<EPI>() ? __shfl_sync(0xffffffffu, my_a, h + j) : 0;
+    }
+    if (full) {
+#pragma unroll
+      for (int j = 0; j < RUN; ++j) pre[j] = epi_load<EPI>(ep, n0 + h + j, orow[j], arow[j], m);
+#pragma unroll
+      for (int j = 0; j < RUN; ++j) {
+        const float z = epi_store<EPI, OBF, ZB>(ep, rc, n0 + h + j, orow[j], m, v[h + j], pre[j]);
+        v[h + j] = z * z;
+      }
+    } else {
+#pragma unroll
+      for (int j = 0; j < RUN; ++j)
+        pre[j] = n0 + h + j < N ? epi_load<EPI>(ep, n0 + h + j, orow[j], arow[j], m) : EpiPre{0.f, 0.f};
+#pragma unroll
+      for (int j = 0; j < RUN; ++j) {
+        const float z = n0 + h + j < N ? epi_store<EPI, OBF, ZB>(ep, rc, n0 + h + j, orow[j], m, v[h + j], pre[j]) : 0.f;
+        v[h + j] = z * z;
+      }
+    }
+  }
+}
+
+template <int CNT, bool OBF>
+__device__ __forceinline__ void swiglu_columns(const EpiParams& ep, int64_t n0, int64_t N, bool full, int m,
+                                               int lane, int64_t my_o, const float* v) {
+#pragma unroll
+  for (int j = 0; j < CNT; ++j) {
+    const int64_t orow = __shfl_sync(0xffffffffu, my_o, j);
+    const float other = __shfl_xor_sync(0xffffffffu, v[j], 1);
+    if ((lane & 1) == 0 && (full || n0 + j < N)) epi_swiglu_store<OBF>(ep, orow, m >> 1, v[j], other);
+  }
+}
+
+// Finishes accumulator columns [n0, n0 + CNT) of this thread's row m (row
+// `row` of weight tile m_tile): folded RMSNorm scale (consumers), the
+// epilogue, and for producers the tile's per-column sums of z^2.  Called by
+// all 128 threads together (it contains block barriers).  Row offsets, which
+// may need a division for grouped rows, are computed once per column by
+// lane j and broadcast.
+template <int EPI, int CNT>
+__device__ __forceinline__ void finish_chunk(const EpiParams& ep, const EpiRowConst& rc, int64_t n0, int64_t N, int m,
+                                             int m_tile, int warp, int lane, float* v, const float* rinv,
+                                             float* red) {
   if (ep.ss_in != nullptr) {
 #pragma unroll
-    for (int j = 0; j < 32; ++j) v[j] *= rinv[j];
+    for (int j = 0; j < CNT; ++j) v[j] *= rinv[j];
   }
   const int64_t my_n = n0 + lane;
-  const bool my_ok = lane < cnt && my_n < N;
+  const bool my_ok = lane < CNT && my_n < N;
   const int64_t my_o = my_ok ? ep.out_map.off(my_n) : 0;
   const int64_t my_a = (epi_uses_aux0<EPI>() && my_ok) ? ep.aux0_map.off(my_n) : 0;
+  const bool full = n0 + CNT <= N;
   if constexpr (EPI == EPI_SWIGLU) {
-#pragma unroll
-    for (int j = 0; j < 32; ++j) {
-      const int64_t orow = __shfl_sync(0xffffffffu, my_o, j);
-      const float other = __shfl_xor_sync(0xffffffffu, v[j], 1);
-      if (j < cnt && n0 + j < N && (lane & 1) == 0) epi_swiglu_at(ep, orow, m >> 1, v[j], other);
-    }
-  } else {
-#pragma unroll
-    for (int h = 0; h < 32; h += 16) {
-      int64_t orow[16];
-      EpiPre pre[16];
-#pragma unroll
-      for (int j = 0; j < 16; ++j) {
-        orow[j] = __shfl_sync(0xffffffffu, my_o, h + j);
-        const int64_t arow = epi_uses_aux0<EPI>() ? __shfl_sync(0xffffffffu, my_a, h + j) : 0;
-        pre[j] = (h + j < cnt && n0 + h + j < N) ? epi_load<EPI>(ep, n0 + h + j, orow[j], arow, m) : EpiPre{0.f, 0.f};
-      }
-#pragma unroll
-      for (int j = 0; j < 16; ++j) {
-        const bool okj = h + j < cnt && n0 + h + j < N;
-        const float z = okj ? epi_store<EPI>(ep, n0 + h + j, orow[j], m, v[h + j], pre[j]) : 0.f;
-        v[h + j] = z * z;  // v is free now: reuse it for z^2
-      }
-    }
-    if constexpr (epi_produces_z<EPI>()) {
+    if (ep.out_bf16) swiglu_columns<CNT, true>(ep, n0, N, full, m, lane, my_o, v);
+    else swiglu_columns<CNT, false>(ep, n0, N, full, m, lane, my_o, v);
+  } else if constexpr (EPI == EPI_STORE) {
+    if (ep.out_bf16) epi_columns<EPI, CNT, true, false>(ep, rc, n0, N, full, m, my_o, my_a, v);
+    else epi_columns<EPI, CNT, false, false>(ep, rc, n0, N, full, m, my_o, my_a, v);
+  } else if constexpr (epi_produces_z<EPI>()) {
+    if (ep.zb != nullptr) {
+      epi_columns<EPI, CNT, false, true>(ep, rc, n0, N, full, m, my_o, my_a, v);
       if (ep.ss_out != nullptr) {
+#pragma unroll
+        for (int j = CNT; j < 32; ++j) v[j] = 0.f;
         warp_column_sums(v, lane);
         red[warp * 32 + lane] = v[0];
         __syncthreads();
-        if (warp == 0 && lane < cnt && n0 + lane < N)
+        if (warp == 0 && lane < CNT && n0 + lane < N)
           ep.ss_out[(int64_t)m_tile * ep.ss_ld + n0 + lane] = red[lane] + red[32 + lane] + red[64 + lane] + red[96 + lane];
         __syncthreads();
       }
+    } else {
+      epi_columns<EPI, CNT, false, false>(ep, rc, n0, N, full, m, my_o, my_a, v);
     }
+  } else {
+    epi_columns<EPI, CNT, false, false>(ep, rc, n0, N, full, m, my_o, my_a, v);
   }
 }
 
@@ -294,6 +334,7 @@ __global__ void __launch_bounds__(128, 1)
   const bool good = ok && !*abort_flag && nkb > 0;
   const int row = warp * 32 + lane;
   const int m = m_tile * BM + row;
+  const EpiRowConst rc = epi_row_const<EPI>(ep, m);
   const int64_t n_base = (int64_t)n_tile * BN;
   float* rinv = reinterpret_cast<float*>(smem + C::EXTRA_OFF);  // [BN] folded RMSNorm scale per column
   float* red = rinv + 256;                                        // [4][32] per-warp column sums
@@ -318,7 +359,7 @@ __global__ void __launch_bounds__(128, 1)
 #pragma unroll
         for (int j = 0; j < 32; ++j) v[j] = 0.f;
       }
-      finish_chunk<EPI>(ep, n_base + c, 32, N, m, m_tile, warp, lane, v, rinv + c, red);
+      finish_chunk<EPI, 32>(ep, rc, n_base + c, N, m, m_tile, warp, lane, v, rinv + c, red);
     }
   } else {
     // Partial tile to this CTA's shared memory (the pipeline buffers are idle
@@ -340,31 +381,34 @@ __global__ void __launch_bounds__(128, 1)
     // This CTA reduces columns [split*COLS, (split+1)*COLS) over all ranks, in
     // rank order, 32 columns at a time.
     constexpr int COLS = BN / CS;
+    constexpr int CNT = COLS < 32 ? COLS : 32;
+    constexpr int GRP = CNT < 8 ? CNT : 8;
     const uint32_t part_local = smem_u32(part);
 #pragma unroll 1
-    for (int cc = 0; cc < COLS; cc += 32) {
+    for (int cc = 0; cc < COLS; cc += CNT) {
       const int c0 = split * COLS + cc;
-      const int cnt = COLS - cc < 32 ? COLS - cc : 32;
       if (n_base + c0 >= N) break;
       float v[32];
 #pragma unroll
-      for (int g = 0; g < 32; g += 8) {
-        float t[8][CS];
+      for (int g = 0; g < CNT; g += GRP) {
+        float t[GRP][CS];
 #pragma unroll
-        for (int j = 0; j < 8; ++j) {
+        for (int j = 0; j < GRP; ++j) {
           const uint32_t off = part_local + (uint32_t)(((c0 + g + j) * BM + row) * 4);
 #pragma unroll
-          for (int p = 0; p < CS; ++p) t[j][p] = (g + j < cnt) ? dsmem_ld(dsmem_addr(off, (uint32_t)p)) : 0.f;
+          for (int p = 0; p < CS; ++p) t[j][p] = dsmem_ld(dsmem_addr(off, (uint32_t)p));
         }
 #pragma unroll
-        for (int j = 0; j < 8; ++j) {
+        for (int j = 0; j < GRP; ++j) {
           float acc = 0.f;
 #pragma unroll
           for (int p = 0; p < CS; ++p) acc += t[j][p];
           v[g + j] = acc;
         }
       }
-      finish_chunk<EPI>(ep, n_base + c0, cnt, N, m, m_tile, warp, lane, v, rinv + c0, red);
+#pragma unroll
+      for (int j = CNT; j < 32; ++j) v[j] = 0.f;
+      finish_chunk<EPI, CNT>(ep, rc, n_base + c0, N, m, m_tile, warp, lane, v, rinv + c0, red);
     }
     cluster_sync_all();  // peers may still read this CTA's partial until here
   }
