@@ -12,7 +12,7 @@ namespace rlt {
 namespace gemm_detail {
 template <int EPI>
 cudaError_t launch_gemm_epi(const CUtensorMap& ta, const CUtensorMap& tb, int bn, int cs, int M, int N, int K,
-                            int kb_per_split, const EpiParams& ep, cudaStream_t st);
+                            int kb_per_split, float* split_ws, const EpiParams& ep, cudaStream_t st);
 }
 
 namespace {
@@ -168,11 +168,22 @@ int gemm_tc_bn(int M, int N, int K, int split_mode) {
   return N <= 32 ? 32 : N <= 64 ? 64 : N <= 128 ? 128 : 256;
 }
 
+size_t gemm_tc_workspace_floats(int M, int N, int K, int split_mode) {
+  if (M % BM || K % BK || N <= 0) return 0;
+  const int cs = gemm_tc_cluster(M, K, split_mode);
+  if (cs == 1) return 0;
+  const int bn = gemm_tc_bn(M, N, K, split_mode);
+  // every CTA of the grid owns cs slots of (bn / cs) x 128 floats
+  return (size_t)(M / BM) * (size_t)((N + bn - 1) / bn) * cs * (size_t)bn * BM;
+}
+
 cudaError_t gemm_tc(const bf16* W, int64_t ldw, const bf16* X, int64_t ldx, int M, int N, int K, int epi,
-                    const EpiParams& ep, int split_mode, cudaStream_t st) {
+                    const EpiParams& ep, int split_mode, float* ws, size_t ws_floats, cudaStream_t st) {
   if (M % BM || K % BK || N <= 0) return cudaErrorInvalidValue;
   const int bn = gemm_tc_bn(M, N, K, split_mode);
   const int cs = gemm_tc_cluster(M, K, split_mode);
+  if (cs > 1 && (ws == nullptr || ws_floats < gemm_tc_workspace_floats(M, N, K, split_mode)))
+    return cudaErrorInvalidValue;
   const int kb = K / BK;
   const int per = (kb + cs - 1) / cs;
   CUtensorMap ta, tb;
@@ -180,12 +191,12 @@ cudaError_t gemm_tc(const bf16* W, int64_t ldw, const bf16* X, int64_t ldx, int 
   if (!make_tmap(&tb, X, N, K, ldx, bn)) return cudaErrorInvalidValue;
   using namespace gemm_detail;
   switch (epi) {
-    case EPI_STORE: return launch_gemm_epi<EPI_STORE>(ta, tb, bn, cs, M, N, K, per, ep, st);
-    case EPI_RESID: return launch_gemm_epi<EPI_RESID>(ta, tb, bn, cs, M, N, K, per, ep, st);
-    case EPI_SWIGLU: return launch_gemm_epi<EPI_SWIGLU>(ta, tb, bn, cs, M, N, K, per, ep, st);
-    case EPI_GATE: return launch_gemm_epi<EPI_GATE>(ta, tb, bn, cs, M, N, K, per, ep, st);
-    case EPI_MERGE: return launch_gemm_epi<EPI_MERGE>(ta, tb, bn, cs, M, N, K, per, ep, st);
-    case EPI_CONVEX: return launch_gemm_epi<EPI_CONVEX>(ta, tb, bn, cs, M, N, K, per, ep, st);
+    case EPI_STORE: return launch_gemm_epi<EPI_STORE>(ta, tb, bn, cs, M, N, K, per, ws, ep, st);
+    case EPI_RESID: return launch_gemm_epi<EPI_RESID>(ta, tb, bn, cs, M, N, K, per, ws, ep, st);
+    case EPI_SWIGLU: return launch_gemm_epi<EPI_SWIGLU>(ta, tb, bn, cs, M, N, K, per, ws, ep, st);
+    case EPI_GATE: return launch_gemm_epi<EPI_GATE>(ta, tb, bn, cs, M, N, K, per, ws, ep, st);
+    case EPI_MERGE: return launch_gemm_epi<EPI_MERGE>(ta, tb, bn, cs, M, N, K, per, ws, ep, st);
+    case EPI_CONVEX: return launch_gemm_epi<EPI_CONVEX>(ta, tb, bn, cs, M, N, K, per, ws, ep, st);
   }
   return cudaErrorInvalidValue;
 }

@@ -4,9 +4,9 @@
 
 namespace rlt {
 namespace gemm_detail {
-template cudaError_t launch_gemm_epi<EPI_STORE>(const CUtensorMap&, const CUtensorMap&, int, int, int, int, int, int,
+template cudaError_t launch_gemm_epi<EPI_STORE>(const CUtensorMap&, const CUtensorMap&, int, int, int, int, int, int, float*,
                                              const EpiParams&, cudaStream_t);
-template cudaError_t launch_gemm_epi<EPI_RESID>(const CUtensorMap&, const CUtensorMap&, int, int, int, int, int, int,
+template cudaError_t launch_gemm_epi<EPI_RESID>(const CUtensorMap&, const CUtensorMap&, int, int, int, int, int, int, float*,
                                              const EpiParams&, cudaStream_t);
 }  // namespace gemm_detail
 }  // namespace rlt

@@ -11,11 +11,13 @@
 //
 // Split over K inside a thread-block cluster: the CS CTAs of one cluster own
 // the same output tile and consecutive K ranges, so every weight byte is read
-// from HBM once while all SMs stream.  Their fp32 partial tiles are exchanged
-// through distributed shared memory: CTA r adds the partials of every CTA of
-// the cluster, in rank order 0..CS-1 (a fixed order, so results never depend
-// on timing), for its 1/CS share of the tile's columns and applies the
-// epilogue there.  No global scratch and no second kernel are needed.
+// from HBM once while all SMs stream.  CTA r finishes columns
+// [r*BN/CS, (r+1)*BN/CS) of the tile: every CTA writes the other CTAs'
+// shares of its fp32 partial to a global (L2-resident) exchange area, the
+// cluster barrier publishes them, and each owner adds the CS partials of its
+// columns in rank order 0..CS-1 (a fixed order, so results never depend on
+// timing) before applying the epilogue.  Distributed shared memory was
+// measured slower for this exchange than a round trip through L2.
 //
 // No TMA multicast is used anywhere: every CTA loads its own tiles.
 #pragma once
@@ -42,7 +44,7 @@ struct TcCfg {
   static constexpr int SMEM = PIPE_BYTES + 1024 /*align*/ + 256 /*barriers*/ + 1024 /*1/rms per column*/ +
                               512 /*per-warp column sums*/;
   static constexpr int TMEM_COLS = BN;  // power of two >= 32
-  static_assert(BN * BM * 4 <= PIPE_BYTES, "cluster partial tile must fit in the pipeline buffers");
+
 };
 
 // UMMA shared-memory matrix descriptor for a K-major tile whose rows are 128
@@ -100,23 +102,47 @@ __device__ __forceinline__ void tmem_ld32(uint32_t taddr, float* v) {
   for (int i = 0; i < 32; ++i) v[i] = __uint_as_float(r[i]);
 }
 
+// Loads CNT (4, 8, 16 or 32) consecutive accumulator columns of this warp's 32
+// lanes.
+template <int CNT>
+__device__ __forceinline__ void tmem_ld_cols(uint32_t taddr, float* v) {
+  if constexpr (CNT == 32) {
+    tmem_ld32(taddr, v);
+  } else if constexpr (CNT == 16) {
+    uint32_t r[16];
+    asm volatile(
+        "tcgen05.ld.sync.aligned.32x32b.x16.b32 "
+        "{%0,%1,%2,%3,%4,%5,%6,%7,%8,%9,%10,%11,%12,%13,%14,%15}, [%16];"
+        : "=r"(r[0]), "=r"(r[1]), "=r"(r[2]), "=r"(r[3]), "=r"(r[4]), "=r"(r[5]), "=r"(r[6]), "=r"(r[7]),
+          "=r"(r[8]), "=r"(r[9]), "=r"(r[10]), "=r"(r[11]), "=r"(r[12]), "=r"(r[13]), "=r"(r[14]), "=r"(r[15])
+        : "r"(taddr));
+    asm volatile("tcgen05.wait::ld.sync.aligned;" ::: "memory");
+#pragma unroll
+    for (int i = 0; i < 16; ++i) v[i] = __uint_as_float(r[i]);
+  } else if constexpr (CNT == 4) {
+    uint32_t r[4];
+    asm volatile("tcgen05.ld.sync.aligned.32x32b.x4.b32 {%0,%1,%2,%3}, [%4];"
+                 : "=r"(r[0]), "=r"(r[1]), "=r"(r[2]), "=r"(r[3])
+                 : "r"(taddr));
+    asm volatile("tcgen05.wait::ld.sync.aligned;" ::: "memory");
+#pragma unroll
+    for (int i = 0; i < 4; ++i) v[i] = __uint_as_float(r[i]);
+  } else {
+    static_assert(CNT == 8, "column count");
+    uint32_t r[8];
+    asm volatile("tcgen05.ld.sync.aligned.32x32b.x8.b32 {%0,%1,%2,%3,%4,%5,%6,%7}, [%8];"
+                 : "=r"(r[0]), "=r"(r[1]), "=r"(r[2]), "=r"(r[3]), "=r"(r[4]), "=r"(r[5]), "=r"(r[6]), "=r"(r[7])
+                 : "r"(taddr));
+    asm volatile("tcgen05.wait::ld.sync.aligned;" ::: "memory");
+#pragma unroll
+    for (int i = 0; i < CNT; ++i) v[i] = __uint_as_float(r[i]);
+  }
+}
+
 __device__ __forceinline__ void cluster_sync_all() {
   asm volatile("barrier.cluster.arrive.release.aligned;\n\tbarrier.cluster.wait.acquire.aligned;" ::: "memory");
 }
 
-__device__ __forceinline__ uint32_t dsmem_addr(uint32_t local, uint32_t rank) {
-  uint32_t r;
-  asm volatile("mapa.shared::cluster.u32 %0, %1, %2;" : "=r"(r) : "r"(local), "r"(rank));
-  return r;
-}
-
-// Remote shared-memory load; ordered after the cluster barrier that precedes
-// every use (that barrier is a volatile asm with a memory clobber).
-__device__ __forceinline__ float dsmem_ld(uint32_t addr) {
-  float v;
-  asm volatile("ld.shared::cluster.f32 %0, [%1];" : "=f"(v) : "r"(addr));
-  return v;
-}
 
 // Butterfly transpose-reduction over the 32 lanes of a warp: on entry zv[j]
 // is this lane's value for column j; on exit zv[0] of lane j is the sum over
@@ -232,7 +258,7 @@ __device__ __forceinline__ void finish_chunk(const EpiParams& ep, const EpiRowCo
 template <int BN, int EPI, int CS>
 __global__ void __launch_bounds__(128, 1)
     gemm_tc_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CUtensorMap tmB, int M, int N,
-                   int K, int kb_per_split, EpiParams ep) {
+                   int K, int kb_per_split, float* split_ws, EpiParams ep) {
   using C = TcCfg<BN>;
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
@@ -362,55 +388,57 @@ __global__ void __launch_bounds__(128, 1)
       finish_chunk<EPI, 32>(ep, rc, n_base + c, N, m, m_tile, warp, lane, v, rinv + c, red);
     }
   } else {
-    // Partial tile to this CTA's shared memory (the pipeline buffers are idle
-    // now: every MMA that read them has completed), column-major [BN][128].
-    float* part = reinterpret_cast<float*>(smem);
-#pragma unroll 1
-    for (int c = 0; c < BN; c += 32) {
-      float v[32];
-      if (good && n_base + c < N) {
-        tmem_ld32(tmem_base + ((uint32_t)(warp * 32) << 16) + (uint32_t)c, v);
-      } else {
-#pragma unroll
-        for (int j = 0; j < 32; ++j) v[j] = 0.f;
-      }
-#pragma unroll
-      for (int j = 0; j < 32; ++j) part[(c + j) * BM + row] = v[j];
-    }
-    cluster_sync_all();
-    // This CTA reduces columns [split*COLS, (split+1)*COLS) over all ranks, in
-    // rank order, 32 columns at a time.
+    // Cluster split-K through L2: this CTA's exchange area holds CS slots of
+    // COLS x 128 floats, slot o for owner o (its own slot stays unused).
     constexpr int COLS = BN / CS;
     constexpr int CNT = COLS < 32 ? COLS : 32;
-    constexpr int GRP = CNT < 8 ? CNT : 8;
-    const uint32_t part_local = smem_u32(part);
+    constexpr int64_t SLICE = (int64_t)COLS * BM;  // floats of one share, column-major [COLS][128]
+    const int rank = split;
+    const int64_t col_cta = blockIdx.x + (int64_t)gridDim.x * blockIdx.y;  // same for every rank of the cluster
+    const int64_t lin_stride = (int64_t)gridDim.x * gridDim.y;             // linear CTA id = col_cta + z * lin_stride
+    float* mine = split_ws + (col_cta + rank * lin_stride) * CS * SLICE;
+#pragma unroll 1
+    for (int o = 0; o < CS; ++o) {
+      if (o == rank) continue;
+#pragma unroll 1
+      for (int c = 0; c < COLS; c += CNT) {
+        float v[32];
+        if (good && n_base + o * COLS + c < N) {
+          tmem_ld_cols<CNT>(tmem_base + ((uint32_t)(warp * 32) << 16) + (uint32_t)(o * COLS + c), v);
+        } else {
+#pragma unroll
+          for (int j = 0; j < CNT; ++j) v[j] = 0.f;
+        }
+#pragma unroll
+        for (int j = 0; j < CNT; ++j) __stcg(mine + o * SLICE + (int64_t)(c + j) * BM + row, v[j]);
+      }
+    }
+    cluster_sync_all();  // release/acquire at cluster scope: the shares are visible to their owners
 #pragma unroll 1
     for (int cc = 0; cc < COLS; cc += CNT) {
-      const int c0 = split * COLS + cc;
+      const int c0 = rank * COLS + cc;
       if (n_base + c0 >= N) break;
-      float v[32];
+      float own[32], v[32];
+      if (good) {
+        tmem_ld_cols<CNT>(tmem_base + ((uint32_t)(warp * 32) << 16) + (uint32_t)c0, own);
+      } else {
 #pragma unroll
-      for (int g = 0; g < CNT; g += GRP) {
-        float t[GRP][CS];
+        for (int j = 0; j < CNT; ++j) own[j] = 0.f;
+      }
 #pragma unroll
-        for (int j = 0; j < GRP; ++j) {
-          const uint32_t off = part_local + (uint32_t)(((c0 + g + j) * BM + row) * 4);
+      for (int j = 0; j < CNT; ++j) {
+        float acc = 0.f;
 #pragma unroll
-          for (int p = 0; p < CS; ++p) t[j][p] = dsmem_ld(dsmem_addr(off, (uint32_t)p));
+        for (int p = 0; p < CS; ++p) {
+          const float* src = split_ws + ((col_cta + p * lin_stride) * CS + rank) * SLICE + (int64_t)(cc + j) * BM + row;
+          acc += p == rank ? own[j] : __ldcg(src);
         }
-#pragma unroll
-        for (int j = 0; j < GRP; ++j) {
-          float acc = 0.f;
-#pragma unroll
-          for (int p = 0; p < CS; ++p) acc += t[j][p];
-          v[g + j] = acc;
-        }
+        v[j] = acc;
       }
 #pragma unroll
       for (int j = CNT; j < 32; ++j) v[j] = 0.f;
       finish_chunk<EPI, CNT>(ep, rc, n_base + c0, N, m, m_tile, warp, lane, v, rinv + c0, red);
     }
-    cluster_sync_all();  // peers may still read this CTA's partial until here
   }
   asm volatile("tcgen05.fence::before_thread_sync;" ::: "memory");
   __syncthreads();
@@ -420,7 +448,7 @@ __global__ void __launch_bounds__(128, 1)
 }
 
 template <int BN, int EPI, int CS>
-cudaError_t launch_gemm(const CUtensorMap& ta, const CUtensorMap& tb, int M, int N, int K, int kb_per_split,
+cudaError_t launch_gemm(const CUtensorMap& ta, const CUtensorMap& tb, int M, int N, int K, int kb_per_split, float* split_ws,
                         const EpiParams& ep, cudaStream_t st) {
   using C = TcCfg<BN>;
   static bool attr_set = false;
@@ -444,19 +472,20 @@ cudaError_t launch_gemm(const CUtensorMap& ta, const CUtensorMap& tb, int M, int
   attr[1].val.programmaticStreamSerializationAllowed = 1;
   cfg.attrs = attr;
   cfg.numAttrs = 2;
-  cudaError_t e = cudaLaunchKernelEx(&cfg, gemm_tc_kernel<BN, EPI, CS>, ta, tb, M, N, K, kb_per_split, ep);
+  cudaError_t e = cudaLaunchKernelEx(&cfg, gemm_tc_kernel<BN, EPI, CS>, ta, tb, M, N, K, kb_per_split, split_ws, ep);
   note_launch();
   return e != cudaSuccess ? e : cudaGetLastError();
 }
 
 template <int EPI, int CS>
-cudaError_t launch_gemm_bn(const CUtensorMap& ta, const CUtensorMap& tb, int bn, int M, int N, int K, int kb_per_split,
+cudaError_t launch_gemm_bn(const CUtensorMap& ta, const CUtensorMap& tb, int bn, int M, int N, int K, int kb_per_split, float* split_ws,
                            const EpiParams& ep, cudaStream_t st) {
   switch (bn) {
-    case 32: return launch_gemm<32, EPI, CS>(ta, tb, M, N, K, kb_per_split, ep, st);
-    case 64: return launch_gemm<64, EPI, CS>(ta, tb, M, N, K, kb_per_split, ep, st);
-    case 128: return launch_gemm<128, EPI, CS>(ta, tb, M, N, K, kb_per_split, ep, st);
-    default: return launch_gemm<256, EPI, CS>(ta, tb, M, N, K, kb_per_split, ep, st);
+    case 32: return launch_gemm<32, EPI, CS>(ta, tb, M, N, K, kb_per_split, split_ws, ep, st);
+    case 64: return launch_gemm<64, EPI, CS>(ta, tb, M, N, K, kb_per_split, split_ws, ep, st);
+    case 128: return launch_gemm<128, EPI, CS>(ta, tb, M, N, K, kb_per_split, split_ws, ep, st);
+    default:
+      return launch_gemm<256, EPI, CS>(ta, tb, M, N, K, kb_per_split, split_ws, ep, st);
   }
 }
 
@@ -464,12 +493,12 @@ cudaError_t launch_gemm_bn(const CUtensorMap& ta, const CUtensorMap& tb, int bn,
 // gemm_tc_epi_*.cu files so the variants compile in parallel.
 template <int EPI>
 cudaError_t launch_gemm_epi(const CUtensorMap& ta, const CUtensorMap& tb, int bn, int cs, int M, int N, int K,
-                            int kb_per_split, const EpiParams& ep, cudaStream_t st) {
+                            int kb_per_split, float* split_ws, const EpiParams& ep, cudaStream_t st) {
   switch (cs) {
-    case 1: return launch_gemm_bn<EPI, 1>(ta, tb, bn, M, N, K, kb_per_split, ep, st);
-    case 2: return launch_gemm_bn<EPI, 2>(ta, tb, bn, M, N, K, kb_per_split, ep, st);
-    case 4: return launch_gemm_bn<EPI, 4>(ta, tb, bn, M, N, K, kb_per_split, ep, st);
-    case 8: return launch_gemm_bn<EPI, 8>(ta, tb, bn, M, N, K, kb_per_split, ep, st);
+    case 1: return launch_gemm_bn<EPI, 1>(ta, tb, bn, M, N, K, kb_per_split, split_ws, ep, st);
+    case 2: return launch_gemm_bn<EPI, 2>(ta, tb, bn, M, N, K, kb_per_split, split_ws, ep, st);
+    case 4: return launch_gemm_bn<EPI, 4>(ta, tb, bn, M, N, K, kb_per_split, split_ws, ep, st);
+    case 8: return launch_gemm_bn<EPI, 8>(ta, tb, bn, M, N, K, kb_per_split, split_ws, ep, st);
   }
   return cudaErrorInvalidValue;
 }

@@ -40,10 +40,14 @@ cudaError_t launch_pdl(void (*kernel)(KArgs...), dim3 grid, dim3 block, size_t s
 // C[n][m] = sum_k X[n][k] W[m][k] with a fused epilogue (epilogue.cuh).
 // bf16 on tcgen05: M % 128 == 0, K % 64 == 0, ld* % 8 == 0, 16-byte aligned
 // bases.  split_mode 1 (decode steps) splits K inside a thread-block cluster
-// by a rule that depends only on M and K; split_mode 0 (token-parallel
-// encoder) never splits.  No global scratch is used.
+// by a rule that depends only on M and K, exchanging the fp32 partials
+// through `ws` (gemm_tc_workspace_floats; the caller keeps it private to the
+// stream); split_mode 0 (token-parallel encoder) never splits and needs none.
 cudaError_t gemm_tc(const bf16* W, int64_t ldw, const bf16* X, int64_t ldx, int M, int N, int K, int epi,
-                    const EpiParams& ep, int split_mode, cudaStream_t st);
+                    const EpiParams& ep, int split_mode, float* ws, size_t ws_floats, cudaStream_t st);
+// Exchange area (floats) a split_mode launch of this shape needs (0 when it
+// is not split over a cluster).
+size_t gemm_tc_workspace_floats(int M, int N, int K, int split_mode);
 int gemm_tc_cluster(int M, int K, int split_mode);
 int gemm_tc_bn(int M, int N, int K, int split_mode);
 

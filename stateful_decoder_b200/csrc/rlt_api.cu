@@ -124,6 +124,7 @@ struct rlt_state {
   float* gate = nullptr;       // [B][d]
   float* logits = nullptr;     // [B][V]
   float* attn_ws = nullptr; size_t attn_ws_floats = 0;
+  float* gemm_ws = nullptr; size_t gemm_ws_floats = 0;  // split-K exchange of the decode GEMMs (bf16)
   // encoder-prefill workspace, rows = sequences x tokens of one chunk
   int64_t pf_rows = 0;
   void* pf_x = nullptr; void* pf_big = nullptr; void* pf_q = nullptr; void* pf_k = nullptr; void* pf_v = nullptr;
@@ -291,20 +292,19 @@ int32_t init_views(rlt_model* m, uint64_t seed) {
 }
 
 // ------------------------------------------------------------------ GEMM dispatch
-// Decode-step contractions pass the state's split workspace and may split K;
-// token-parallel (encoder prefill) contractions pass no workspace and never
-// split, so that no reduction order depends on how many rows share a GEMM.
-// Decode-step contractions (split = true) may split K inside a cluster;
-// token-parallel encoder contractions never split.
+// Decode-step contractions (split = true) may split K inside a cluster and
+// exchange partials through the state's exchange area; token-parallel
+// encoder contractions never split.  The split depends on the weight shape
+// only, so no reduction order depends on how many rows share a GEMM.
 template <typename T>
 int32_t gemm(rlt_state* S, const void* W, int64_t ldw, const void* X, int64_t ldx, int M, int N, int K, int epi,
              const EpiParams& ep, bool split, cudaStream_t st);
 
 template <>
-int32_t gemm<bf16>(rlt_state*, const void* W, int64_t ldw, const void* X, int64_t ldx, int M, int N, int K, int epi,
+int32_t gemm<bf16>(rlt_state* S, const void* W, int64_t ldw, const void* X, int64_t ldx, int M, int N, int K, int epi,
                    const EpiParams& ep, bool split, cudaStream_t st) {
   RLT_CUDA(gemm_tc(static_cast<const bf16*>(W), ldw, static_cast<const bf16*>(X), ldx, M, N, K, epi, ep,
-                   split ? 1 : 0, st));
+                   split ? 1 : 0, split ? S->gemm_ws : nullptr, split ? S->gemm_ws_floats : 0, st));
   return RLT_OK;
 }
 
@@ -420,6 +420,14 @@ int32_t make_state(rlt_model* m, int32_t B, int32_t max_len, int32_t flags, rlt_
   S->attn_ws_floats = prefix_attn_workspace_floats(B, c.n_heads, (int)(d / c.n_heads), max_len);
   if ((r = A(&p, (int64_t)S->attn_ws_floats * 4))) goto fail_;
   S->attn_ws = static_cast<float*>(p);
+  if (c.dtype == RLT_DTYPE_BF16) {
+    // every weight shape a step contracts with B rows
+    const int64_t shapes[][2] = {{d, 2 * d}, {d, d}, {3 * d, d}, {2 * (int64_t)F, d}, {d, F}, {V, d}, {2 * d * G, d}};
+    for (const auto& mk : shapes)
+      S->gemm_ws_floats = std::max(S->gemm_ws_floats, gemm_tc_workspace_floats((int)mk[0], B, (int)mk[1], 1));
+    if ((r = A(&p, (int64_t)S->gemm_ws_floats * 4))) goto fail_;
+    S->gemm_ws = static_cast<float*>(p);
+  }
   *out = S;
   return RLT_OK;
 fail_:
@@ -988,8 +996,14 @@ int32_t rlt_op_linear(const void* w_dev, const void* x_dev, float* y_dev, int32_
     return ok();
   }
   if (M % 128 || K % 64) return fail(RLT_E_INVAL, "tensor-core path needs M % 128 == 0 and K % 64 == 0");
+  const size_t ws_floats = gemm_tc_workspace_floats(M, N, K, 1);
+  float* ws = nullptr;
+  if (ws_floats > 0) {
+    RLT_CUDA(cudaMallocAsync(reinterpret_cast<void**>(&ws), ws_floats * 4, st));
+  }
   cudaError_t e = gemm_tc(static_cast<const bf16*>(w_dev), K, static_cast<const bf16*>(x_dev), K, M, N, K, EPI_STORE,
-                          ep, 1, st);
+                          ep, 1, ws, ws_floats, st);
+  if (ws) cudaFreeAsync(ws, st);
   if (e != cudaSuccess) return fail(RLT_E_CUDA, std::string("gemm_tc: ") + cudaGetErrorString(e));
   return ok();
 }
