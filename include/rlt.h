@@ -112,6 +112,7 @@ typedef struct rlt_state_info {
   int32_t ring_head;    /* slot the next transition writes: n_dec mod (W-1), 0 if W = 1 */
   int32_t has_encoder_cache;
   uint64_t model_version;
+  int32_t has_pending;  /* a sampled x_{t+1} awaits its transition (App. A, pending token) */
 } rlt_state_info;
 
 #define RLT_STATE_ENCODER_CACHE 1   /* keep C^E (needed for incremental encoding, eq. 2.8) */
@@ -177,18 +178,52 @@ int32_t rlt_state_info_get(const rlt_state* s, rlt_state_info* out);
 /* Copies one state component to host memory (synchronous); layouts above. */
 int32_t rlt_state_read(const rlt_state* s, int32_t what, int32_t index, void* host, size_t bytes);
 
+/* Exact prefix snapshot (report §6, "Multi-turn Serving and Cache
+ * Semantics"): writes to host memory everything the continuation depends on
+ * -- the encoder cache C^E (when the state keeps it) and the memory M for
+ * positions 1..n_enc, the encoder outputs e_1..e_n_enc, the decoder state
+ * H_t = (s_t, C^D_t) with the whole SWA ring, the positions n_enc and n_dec,
+ * the pending sampled token (App. A) if any, the model configuration
+ * (window convention included) and the identity of the weights (generator
+ * seed and model version).  bf16 models also store the readout operand the
+ * last transition left (gamma_o * s_t in bf16 and its sums of squares), so
+ * that a restored state reads out bit-identically.  Layout: a 120-byte
+ * little-endian header ("RLTSNAP1") followed by the sections in that order.
+ * *used receives the size; with host == NULL nothing is copied and the call
+ * only reports the size.  Ordered on `stream`, and synchronises it.
+ * Errors: RLT_E_CAPACITY (cap < size), RLT_E_INVAL. */
+int32_t rlt_state_export(const rlt_state* s, void* host, size_t cap, size_t* used, void* stream);
+
+/* Restores a snapshot into a state of the same batch size created under the
+ * same model configuration, replacing its contents; max_len may differ as
+ * long as it covers the snapshot's positions.  A state without the encoder
+ * cache drops the snapshot's cache (it can then decode up to n_enc but not
+ * encode further); a state with the cache needs a snapshot that has one.
+ * Weight updates invalidate snapshots (report §6): the model's generator
+ * seed and version must equal the snapshot's, else RLT_E_STALE.
+ * Synchronises `stream` (host may be freed on return).
+ * Errors: RLT_E_INVAL (format, configuration, batch, size), RLT_E_STALE,
+ * RLT_E_CAPACITY (positions > max_len), RLT_E_STATE (cache missing). */
+int32_t rlt_state_import(rlt_state* s, const void* host, size_t bytes, void* stream);
+
 /* ---------------------------------------------------------------- schedules */
 
 /* Token-parallel causal encoder (eq. 2.1) and memory projection (eq. 2.2) for
  * T tokens per sequence, tok_dev [B][T] int32 (row-major), placed at positions
- * n_enc+1..n_enc+T.  Only an empty encoder (n_enc == 0) is supported by this
- * schedule; later tokens are encoded by rlt_decoder_step.  Does not advance
- * the decoder.  Errors: RLT_E_CAPACITY (n_enc+T > max_len), RLT_E_STATE
- * (n_enc != 0), RLT_E_STALE, RLT_E_INVAL. */
+ * n_enc+1..n_enc+T.  With n_enc > 0 the tokens attend to the encoded prefix
+ * through the encoder cache: the chunked schedule of App. A.2 (an appended
+ * span -- a user turn or a tool result -- is encoded in one pass; every
+ * token still receives its decoder transition through rlt_decoder_step).
+ * Does not advance the decoder.  Errors: RLT_E_CAPACITY (n_enc+T >
+ * max_len), RLT_E_STATE (n_enc > 0 without the encoder cache), RLT_E_STALE,
+ * RLT_E_INVAL. */
 int32_t rlt_encode_prefix(rlt_model* m, rlt_state* s, const int32_t* tok_dev, int32_t T, void* stream);
 
 /* Readout of the current s_t (eq. 2.6): log p of next_dev [B] (may be NULL),
- * and/or a sample from the behaviour sampler (samp may be NULL).  Requires
+ * and/or a sample from the behaviour sampler (samp may be NULL).  A sample
+ * is also recorded in the state as the pending token x_{t+1} (App. A): the
+ * state represents the consumed prefix only, and the next rlt_decoder_step
+ * consumes the pending token when it is given no tokens.  Requires
  * n_dec >= 1. */
 int32_t rlt_readout(rlt_model* m, rlt_state* s, const int32_t* next_dev, const rlt_sampling* samp,
                     const rlt_readout_out* out, void* stream);
@@ -198,9 +233,11 @@ int32_t rlt_readout(rlt_model* m, rlt_state* s, const int32_t* next_dev, const r
  * cache) and the memory append; then the merge and the L_D decoder blocks
  * (eqs. 2.4, 2.5, 2.12-2.16) with one SWA insert per layer; then the readout
  * as rlt_readout does (skipped when next_dev, samp and out are all NULL).
- * tok_dev [B] int32 is read only when the token is encoded here.
+ * tok_dev [B] int32 is read only when the token is encoded here; NULL takes
+ * the pending sampled token.  Every transition clears the pending record.
  * Errors: RLT_E_CAPACITY (t > max_len), RLT_E_STATE (no encoder cache and x_t
- * not encoded), RLT_E_STALE, RLT_E_INVAL. */
+ * not encoded, or no token given and none pending), RLT_E_STALE,
+ * RLT_E_INVAL. */
 int32_t rlt_decoder_step(rlt_model* m, rlt_state* s, const int32_t* tok_dev, const int32_t* next_dev,
                          const rlt_sampling* samp, const rlt_readout_out* out, void* stream);
 

@@ -44,6 +44,7 @@ EXPORTED = (
     "rlt_encode_prefix", "rlt_readout", "rlt_decoder_step", "rlt_prefill", "rlt_replay_logprobs",
     "rlt_last_error", "rlt_check_device", "rlt_profile_enable", "rlt_profile_read", "rlt_op_linear",
     "rlt_op_sample", "rlt_kernel_launches", "rlt_op_prefix_attention", "rlt_op_prefix_attention_noalloc",
+    "rlt_state_export", "rlt_state_import",
 )
 
 
@@ -75,7 +76,8 @@ class ReadoutOut(ctypes.Structure):
 class StateInfo(ctypes.Structure):
     _fields_ = [("batch", ctypes.c_int32), ("max_len", ctypes.c_int32), ("n_enc", ctypes.c_int32),
                 ("n_dec", ctypes.c_int32), ("ring_valid", ctypes.c_int32), ("ring_head", ctypes.c_int32),
-                ("has_encoder_cache", ctypes.c_int32), ("model_version", ctypes.c_uint64)]
+                ("has_encoder_cache", ctypes.c_int32), ("model_version", ctypes.c_uint64),
+                ("has_pending", ctypes.c_int32)]
 
 
 _vp = ctypes.c_void_p
@@ -92,6 +94,8 @@ _sig = {
     "rlt_state_reset": [_vp, _vp],
     "rlt_state_info_get": [_vp, ctypes.POINTER(StateInfo)],
     "rlt_state_read": [_vp, _i32, _i32, _vp, ctypes.c_size_t],
+    "rlt_state_export": [_vp, _vp, ctypes.c_size_t, ctypes.POINTER(ctypes.c_size_t), _vp],
+    "rlt_state_import": [_vp, _vp, ctypes.c_size_t, _vp],
     "rlt_encode_prefix": [_vp, _vp, _vp, _i32, _vp],
     "rlt_readout": [_vp, _vp, _vp, ctypes.POINTER(Sampling), ctypes.POINTER(ReadoutOut), _vp],
     "rlt_decoder_step": [_vp, _vp, _vp, _vp, ctypes.POINTER(Sampling), ctypes.POINTER(ReadoutOut), _vp],
@@ -248,8 +252,22 @@ def rlt_state_reset(state: State, stream=None) -> None:
     _check(_lib.rlt_state_reset(state.h, _stream(stream)))
 
 
+def rlt_state_export(state: State, stream=None) -> np.ndarray:
+    """Exact prefix snapshot of the state as a uint8 array (host memory)."""
+    n = ctypes.c_size_t()
+    _check(_lib.rlt_state_export(state.h, None, 0, ctypes.byref(n), _stream(stream)))
+    buf = np.zeros(n.value, np.uint8)
+    _check(_lib.rlt_state_export(state.h, buf.ctypes.data, buf.nbytes, ctypes.byref(n), _stream(stream)))
+    return buf
+
+
+def rlt_state_import(state: State, snapshot: np.ndarray, stream=None) -> None:
+    snap = np.ascontiguousarray(snapshot, dtype=np.uint8)
+    _check(_lib.rlt_state_import(state.h, snap.ctypes.data, snap.nbytes, _stream(stream)))
+
+
 def rlt_encode_prefix(model: Model, state: State, tokens, stream=None) -> None:
-    """tokens: int32 CUDA tensor [B, T]."""
+    """tokens: int32 CUDA tensor [B, T], placed at positions n_enc+1..n_enc+T."""
     _check(_lib.rlt_encode_prefix(model.h, state.h, _dev(tokens, "torch.int32"), tokens.shape[1], _stream(stream)))
 
 

@@ -3,7 +3,9 @@
 // processed together under a causal mask).
 //
 // Flash-style tiling on CUDA cores: a block owns 64 queries of one (sequence,
-// head) and streams 64-key tiles up to the diagonal.  S = Q K^T is formed as a
+// head) and streams 64-key tiles up to the diagonal.  The queries may start
+// at position q_off > 0 (a chunk appended to an encoded prefix, whose keys
+// and values are rows 0..q_off-1 of the cache).  S = Q K^T is formed as a
 // 4x4 register tile per thread from transposed shared-memory copies of Q and
 // K, the online softmax keeps a running max and sum per query row, and
 // O += P V accumulates 4 rows x (hd/16) columns per thread.
@@ -24,7 +26,8 @@ constexpr size_t causal_smem_floats() {
 template <typename KT, int HD>
 __global__ void __launch_bounds__(256) causal_attn_kernel(const KT* __restrict__ Q, const KT* __restrict__ K,
                                                           const KT* __restrict__ V, int64_t ld_tq, int64_t ld_tkv,
-                                                          int H, int T, KT* out, int64_t ld_out, float scale_log2) {
+                                                          int H, int T, int q_off, KT* out, int64_t ld_out,
+                                                          float scale_log2) {
   griddep_enter();
   constexpr int DPT = HD / 16;
   extern __shared__ float sm[];
@@ -57,12 +60,14 @@ __global__ void __launch_bounds__(256) causal_attn_kernel(const KT* __restrict__
 #pragma unroll
     for (int j = 0; j < DPT; ++j) o[i][j] = 0.f;
 
-  const int kv_end = min(T, q0 + BQ);
+  // queries are positions q_off + 0..T-1; keys 0..q_off+T-1
+  const int Tk = q_off + T;
+  const int kv_end = min(Tk, q_off + q0 + BQ);
   for (int k0 = 0; k0 < kv_end; k0 += BKV) {
     __syncthreads();
     for (int i = tid; i < BKV * HD; i += 256) {
       const int r = i / HD, c = i % HD;
-      const bool ok = k0 + r < T;
+      const bool ok = k0 + r < Tk;
       sKt[c * PADK + r] = ok ? to_f32(Kb[(int64_t)(k0 + r) * HD + c]) : 0.f;
       sV[r * (HD + 4) + c] = ok ? to_f32(Vb[(int64_t)(k0 + r) * HD + c]) : 0.f;
     }
@@ -86,8 +91,8 @@ __global__ void __launch_bounds__(256) causal_attn_kernel(const KT* __restrict__
     for (int i = 0; i < 4; ++i)
 #pragma unroll
       for (int j = 0; j < 4; ++j) {
-        const int qi = q0 + ty * 4 + i, kj = k0 + tx * 4 + j;
-        sP[(tx * 4 + j) * PADQ + ty * 4 + i] = (kj <= qi && kj < T) ? s[i][j] : -INFINITY;
+        const int qpos = q_off + q0 + ty * 4 + i, kj = k0 + tx * 4 + j;
+        sP[(tx * 4 + j) * PADQ + ty * 4 + i] = (kj <= qpos && kj < Tk) ? s[i][j] : -INFINITY;
       }
     __syncthreads();
     {
@@ -148,15 +153,15 @@ __global__ void __launch_bounds__(256) causal_attn_kernel(const KT* __restrict__
 }
 
 template <typename KT, int HD>
-cudaError_t launch(const KT* q, const KT* k, const KT* v, int64_t ld_tq, int64_t ld_tkv, int B, int H, int T, KT* out,
-                   int64_t ld_out, cudaStream_t st) {
+cudaError_t launch(const KT* q, const KT* k, const KT* v, int64_t ld_tq, int64_t ld_tkv, int B, int H, int T, int q_off,
+                   KT* out, int64_t ld_out, cudaStream_t st) {
   const size_t smem = causal_smem_floats<HD>() * sizeof(float);
   cudaError_t e = cudaFuncSetAttribute(causal_attn_kernel<KT, HD>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
   if (e != cudaSuccess) return e;
   const float scale_log2 = 1.4426950408889634f / sqrtf((float)HD);
   dim3 grid((T + BQ - 1) / BQ, H, B);
   {
-    const cudaError_t e_l = launch_pdl(causal_attn_kernel<KT, HD>, dim3(grid), dim3(256), smem, st, q, k, v, ld_tq, ld_tkv, H, T, out, ld_out, scale_log2);
+    const cudaError_t e_l = launch_pdl(causal_attn_kernel<KT, HD>, dim3(grid), dim3(256), smem, st, q, k, v, ld_tq, ld_tkv, H, T, q_off, out, ld_out, scale_log2);
     if (e_l != cudaSuccess) return e_l;
   }
   return cudaGetLastError();
@@ -166,20 +171,20 @@ cudaError_t launch(const KT* q, const KT* k, const KT* v, int64_t ld_tq, int64_t
 
 template <typename KT>
 cudaError_t causal_attn(const KT* q, const KT* k, const KT* v, int64_t ld_tq, int64_t ld_tkv, int B, int H, int hd,
-                        int T, KT* out, int64_t ld_out, cudaStream_t st) {
-  if (T <= 0 || B <= 0) return cudaErrorInvalidValue;
+                        int T, int q_off, KT* out, int64_t ld_out, cudaStream_t st) {
+  if (T <= 0 || B <= 0 || q_off < 0) return cudaErrorInvalidValue;
   switch (hd) {
-    case 16: return launch<KT, 16>(q, k, v, ld_tq, ld_tkv, B, H, T, out, ld_out, st);
-    case 32: return launch<KT, 32>(q, k, v, ld_tq, ld_tkv, B, H, T, out, ld_out, st);
-    case 64: return launch<KT, 64>(q, k, v, ld_tq, ld_tkv, B, H, T, out, ld_out, st);
-    case 128: return launch<KT, 128>(q, k, v, ld_tq, ld_tkv, B, H, T, out, ld_out, st);
+    case 16: return launch<KT, 16>(q, k, v, ld_tq, ld_tkv, B, H, T, q_off, out, ld_out, st);
+    case 32: return launch<KT, 32>(q, k, v, ld_tq, ld_tkv, B, H, T, q_off, out, ld_out, st);
+    case 64: return launch<KT, 64>(q, k, v, ld_tq, ld_tkv, B, H, T, q_off, out, ld_out, st);
+    case 128: return launch<KT, 128>(q, k, v, ld_tq, ld_tkv, B, H, T, q_off, out, ld_out, st);
   }
   return cudaErrorInvalidValue;
 }
 
 template cudaError_t causal_attn<float>(const float*, const float*, const float*, int64_t, int64_t, int, int, int, int,
-                                        float*, int64_t, cudaStream_t);
+                                        int, float*, int64_t, cudaStream_t);
 template cudaError_t causal_attn<bf16>(const bf16*, const bf16*, const bf16*, int64_t, int64_t, int, int, int, int,
-                                       bf16*, int64_t, cudaStream_t);
+                                       int, bf16*, int64_t, cudaStream_t);
 
 }  // namespace rlt

@@ -102,7 +102,7 @@ template <int HD>
 __global__ void __launch_bounds__(128, 2)
     causal_attn_tc_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUtensorMap tmK,
                           const __grid_constant__ CUtensorMap tmV, int64_t ld_tq, int64_t ld_tkv, int H, int T,
-                          bf16* out, int64_t ld_out, float scale_log2) {
+                          int q_off, bf16* out, int64_t ld_out, float scale_log2) {
   using C = FaCfg<HD>;
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
@@ -118,8 +118,11 @@ __global__ void __launch_bounds__(128, 2)
   const int q0 = blockIdx.x * FQ, h = blockIdx.y, b = blockIdx.z;
   const int qrow0 = (int)(((int64_t)b * H + h) * ld_tq + q0);
   const int krow0 = (int)(((int64_t)b * H + h) * ld_tkv);
-  const int n_tiles = (min(T, q0 + FQ) + FKV - 1) / FKV;
+  // queries: chunk rows q0 + row at positions q_off + q0 + row; keys 0..Tk-1
+  const int Tk = q_off + T;
+  const int n_tiles = (min(Tk, q_off + q0 + FQ) + FKV - 1) / FKV;
   const int qi = q0 + row;
+  const int qpos = q_off + qi;
 
   griddep_enter();
   if (threadIdx.x == 0) {
@@ -184,7 +187,7 @@ __global__ void __launch_bounds__(128, 2)
 #pragma unroll
       for (int i = 0; i < 32; ++i) {
         const int kj = j * FKV + c + i;
-        if (kj <= qi && kj < T) mrow = fmaxf(mrow, v[i] * scale_log2);
+        if (kj <= qpos && kj < Tk) mrow = fmaxf(mrow, v[i] * scale_log2);
       }
     }
     asm volatile("tcgen05.fence::before_thread_sync;" ::: "memory");
@@ -205,7 +208,7 @@ __global__ void __launch_bounds__(128, 2)
     // Value rows past the sequence end (rows of another head, or cache rows
     // never written) get probability 0, but 0 * NaN would still poison O:
     // zero them.
-    if (j * FKV + row >= T) {
+    if (j * FKV + row >= Tk) {
 #pragma unroll
       for (int s = 0; s < HD / 64; ++s) {
         const uint32_t vrow = sV + (uint32_t)(s * 16384 + (row >> 3) * 1024 + (row & 7) * 128);
@@ -228,8 +231,8 @@ __global__ void __launch_bounds__(128, 2)
 #pragma unroll
       for (int i = 0; i < 32; i += 2) {
         const int kj = j * FKV + c + i;
-        const float p0 = (kj <= qi && kj < T) ? exp2f(v[i] * scale_log2 - mrow) : 0.f;
-        const float p1 = (kj + 1 <= qi && kj + 1 < T) ? exp2f(v[i + 1] * scale_log2 - mrow) : 0.f;
+        const float p0 = (kj <= qpos && kj < Tk) ? exp2f(v[i] * scale_log2 - mrow) : 0.f;
+        const float p1 = (kj + 1 <= qpos && kj + 1 < Tk) ? exp2f(v[i + 1] * scale_log2 - mrow) : 0.f;
         lrow += p0 + p1;
         __nv_bfloat162 h2 = __floats2bfloat162_rn(p0, p1);
         pk[i / 2] = *reinterpret_cast<uint32_t*>(&h2);
@@ -318,7 +321,7 @@ bool fa_tmap(CUtensorMap* tm, const void* base, int64_t rows, int hd) {
 
 template <int HD>
 cudaError_t launch_fa(const bf16* q, const bf16* k, const bf16* v, int64_t ld_tq, int64_t ld_tkv, int B, int H, int T,
-                      bf16* out, int64_t ld_out, cudaStream_t st) {
+                      int q_off, bf16* out, int64_t ld_out, cudaStream_t st) {
   using C = FaCfg<HD>;
   CUtensorMap tq, tk, tv;
   if (!fa_tmap(&tq, q, (int64_t)B * H * ld_tq, HD) || !fa_tmap(&tk, k, (int64_t)B * H * ld_tkv, HD) ||
@@ -333,18 +336,18 @@ cudaError_t launch_fa(const bf16* q, const bf16* k, const bf16* v, int64_t ld_tq
   }
   const float scale_log2 = 1.4426950408889634f / sqrtf((float)HD);
   return launch_pdl(causal_attn_tc_kernel<HD>, dim3((T + FQ - 1) / FQ, H, B), dim3(128), (size_t)C::SMEM, st, tq, tk,
-                    tv, ld_tq, ld_tkv, H, T, out, ld_out, scale_log2);
+                    tv, ld_tq, ld_tkv, H, T, q_off, out, ld_out, scale_log2);
 }
 
 }  // namespace
 
 cudaError_t causal_attn_tc(const bf16* q, const bf16* k, const bf16* v, int64_t ld_tq, int64_t ld_tkv, int B, int H,
-                           int hd, int T, bf16* out, int64_t ld_out, cudaStream_t st) {
-  if (T <= 0 || B <= 0) return cudaErrorInvalidValue;
+                           int hd, int T, int q_off, bf16* out, int64_t ld_out, cudaStream_t st) {
+  if (T <= 0 || B <= 0 || q_off < 0) return cudaErrorInvalidValue;
   if ((int64_t)B * H * (ld_tq > ld_tkv ? ld_tq : ld_tkv) >= ((int64_t)1 << 31)) return cudaErrorInvalidValue;
   switch (hd) {
-    case 64: return launch_fa<64>(q, k, v, ld_tq, ld_tkv, B, H, T, out, ld_out, st);
-    case 128: return launch_fa<128>(q, k, v, ld_tq, ld_tkv, B, H, T, out, ld_out, st);
+    case 64: return launch_fa<64>(q, k, v, ld_tq, ld_tkv, B, H, T, q_off, out, ld_out, st);
+    case 128: return launch_fa<128>(q, k, v, ld_tq, ld_tkv, B, H, T, q_off, out, ld_out, st);
   }
   return cudaErrorInvalidValue;
 }

@@ -75,16 +75,18 @@ cudaError_t prefix_attn(const float* q, int64_t ld_q, const KT* k, const KT* v, 
 size_t prefix_attn_workspace_floats(int B, int H, int hd, int n);
 constexpr int kPrefixChunk = 256;
 
-// Token-parallel causal attention for the encoder (eq. 2.1): Q, K, V are
-// [B][H][ld_t][hd] (rows 0..T-1 used); out row b*T+i, columns h*hd.
+// Token-parallel causal attention for the encoder (eq. 2.1): query rows
+// 0..T-1 of Q ([B][H][ld_tq][hd]) are positions q_off..q_off+T-1 and attend
+// to key/value rows 0..q_off+i of K, V ([B][H][ld_tkv][hd]); out row b*T+i,
+// columns h*hd.  q_off > 0 continues an encoded prefix held in the cache.
 template <typename KT>
 cudaError_t causal_attn(const KT* q, const KT* k, const KT* v, int64_t ld_tq, int64_t ld_tkv, int B, int H, int hd,
-                        int T, KT* out, int64_t ld_out, cudaStream_t st);
+                        int T, int q_off, KT* out, int64_t ld_out, cudaStream_t st);
 
 // The same on the tensor cores (bf16, hd 64 or 128): two-pass softmax with
 // S and O in tensor memory.
 cudaError_t causal_attn_tc(const bf16* q, const bf16* k, const bf16* v, int64_t ld_tq, int64_t ld_tkv, int B, int H,
-                           int hd, int T, bf16* out, int64_t ld_out, cudaStream_t st);
+                           int hd, int T, int q_off, bf16* out, int64_t ld_out, cudaStream_t st);
 
 // ---------------------------------------------------------------- elementwise
 // Generator fill of a [rows][cols] view (rows `pitch` elements apart).
@@ -109,11 +111,13 @@ template <typename WT, typename OT>
 cudaError_t merge_prep(const float* e, RowMap e_map, const float* s, const WT* gamma, int B, int d, float eps,
                        int kind, OT* out, cudaStream_t st);
 
-// Scatter head-split rows into a [B][H][ld_t][hd] store at positions
-// pos0 + (r % rows_per_seq), rotating (rope != 0) at that position.
+// Scatter head-split rows into a [B][H][ld_t][hd] store: row i = r %
+// rows_per_seq of a sequence goes to store row dst_row0 + i, rotated (rope
+// != 0) at position pos0 + i.
 template <typename XT, typename KT>
-cudaError_t head_scatter(const XT* x, int64_t ld_x, int64_t col0, int64_t rows, int rows_per_seq, int pos0, int H,
-                         int hd, int rope, const float* rope_cs, KT* dst, int64_t ld_t, cudaStream_t st);
+cudaError_t head_scatter(const XT* x, int64_t ld_x, int64_t col0, int64_t rows, int rows_per_seq, int pos0,
+                         int dst_row0, int H, int hd, int rope, const float* rope_cs, KT* dst, int64_t ld_t,
+                         cudaStream_t st);
 
 // logp[b*ld_logp] = logits[b][next[b*next_stride]] - logsumexp(logits[b])
 cudaError_t logp_gather(const float* logits, int B, int V, const int32_t* next, int64_t next_stride, float* logp,

@@ -111,7 +111,7 @@ __global__ void merge_prep_kernel(const float* __restrict__ e, RowMap e_map, con
 // (i, i+hd/2) by pos * base^(-2i/hd) when rope != 0.
 template <typename XT, typename KT>
 __global__ void head_scatter_kernel(const XT* __restrict__ x, int64_t ld_x, int64_t col0, int64_t rows,
-                                    int rows_per_seq, int pos0, int H, int hd, int rope,
+                                    int rows_per_seq, int pos0, int dst_row0, int H, int hd, int rope,
                                     const float* __restrict__ rope_cs, KT* dst, int64_t ld_t) {
   griddep_enter();
   const int half = hd / 2;
@@ -121,7 +121,8 @@ __global__ void head_scatter_kernel(const XT* __restrict__ x, int64_t ld_x, int6
     const int h = (int)((idx / half) % H);
     const int64_t r = idx / ((int64_t)half * H);
     const int64_t b = r / rows_per_seq;
-    const int pos = pos0 + (int)(r % rows_per_seq);
+    const int i_seq = (int)(r % rows_per_seq);
+    const int pos = pos0 + i_seq;
     const XT* xr = x + r * ld_x + col0 + (int64_t)h * hd;
     float a = to_f32(xr[i]), c = to_f32(xr[i + half]);
     if (rope) {
@@ -131,7 +132,7 @@ __global__ void head_scatter_kernel(const XT* __restrict__ x, int64_t ld_x, int6
       a = ra;
       c = rc;
     }
-    KT* o = dst + ((b * H + h) * ld_t + pos) * hd;
+    KT* o = dst + ((b * H + h) * ld_t + dst_row0 + i_seq) * hd;
     o[i] = from_f32<KT>(a);
     o[i + half] = from_f32<KT>(c);
   }
@@ -378,11 +379,11 @@ cudaError_t merge_prep(const float* e, RowMap e_map, const float* s, const WT* g
 }
 
 template <typename XT, typename KT>
-cudaError_t head_scatter(const XT* x, int64_t ld_x, int64_t col0, int64_t rows, int rows_per_seq, int pos0, int H,
+cudaError_t head_scatter(const XT* x, int64_t ld_x, int64_t col0, int64_t rows, int rows_per_seq, int pos0, int dst_row0, int H,
                          int hd, int rope, const float* rope_cs, KT* dst, int64_t ld_t, cudaStream_t st) {
   const int64_t n = rows * H * (hd / 2);
   {
-    const cudaError_t e_l = launch_pdl(head_scatter_kernel<XT, KT>, dim3(grid_for(n, 256, 148 * 32)), dim3(256), 0, st, x, ld_x, col0, rows, rows_per_seq, pos0, H,
+    const cudaError_t e_l = launch_pdl(head_scatter_kernel<XT, KT>, dim3(grid_for(n, 256, 148 * 32)), dim3(256), 0, st, x, ld_x, col0, rows, rows_per_seq, pos0, dst_row0, H,
                                                                           hd, rope, rope_cs, dst, ld_t);
     if (e_l != cudaSuccess) return e_l;
   }
@@ -435,13 +436,13 @@ cudaError_t copy_f32(float* dst, const float* src, int64_t n, cudaStream_t st) {
                                        cudaStream_t);                                                             \
   template cudaError_t merge_prep<WT, WT>(const float*, RowMap, const float*, const WT*, int, int, float, int,    \
                                           WT*, cudaStream_t);                                                     \
-  template cudaError_t head_scatter<float, WT>(const float*, int64_t, int64_t, int64_t, int, int, int, int, int,   \
+  template cudaError_t head_scatter<float, WT>(const float*, int64_t, int64_t, int64_t, int, int, int, int, int, int,   \
                                                const float*, WT*, int64_t, cudaStream_t);                         \
   template cudaError_t broadcast_row<WT>(const WT*, int, float*, int, cudaStream_t);
 
 RLT_INST_W(float)
 RLT_INST_W(bf16)
-template cudaError_t head_scatter<bf16, bf16>(const bf16*, int64_t, int64_t, int64_t, int, int, int, int, int,
+template cudaError_t head_scatter<bf16, bf16>(const bf16*, int64_t, int64_t, int64_t, int, int, int, int, int, int,
                                               const float*, bf16*, int64_t, cudaStream_t);
 
 }  // namespace rlt

@@ -87,6 +87,7 @@ struct ProfileRec {
 
 struct rlt_model {
   rlt_config cfg;
+  uint64_t seed = 0;  // generator seed of rlt_init_weights (part of the weights' identity)
   int hd = 0;
   size_t esz = 0;
   int device = 0;
@@ -125,6 +126,8 @@ struct rlt_state {
   float* logits = nullptr;     // [B][V]
   float* attn_ws = nullptr; size_t attn_ws_floats = 0;
   float* gemm_ws = nullptr; size_t gemm_ws_floats = 0;  // split-K exchange of the decode GEMMs (bf16)
+  int32_t* pending = nullptr;  // [B] last sampled x_{t+1}, not yet consumed (report App. A, pending token)
+  bool has_pending = false;
   // encoder-prefill workspace, rows = sequences x tokens of one chunk
   int64_t pf_rows = 0;
   void* pf_x = nullptr; void* pf_big = nullptr; void* pf_q = nullptr; void* pf_k = nullptr; void* pf_v = nullptr;
@@ -420,6 +423,8 @@ int32_t make_state(rlt_model* m, int32_t B, int32_t max_len, int32_t flags, rlt_
   S->attn_ws_floats = prefix_attn_workspace_floats(B, c.n_heads, (int)(d / c.n_heads), max_len);
   if ((r = A(&p, (int64_t)S->attn_ws_floats * 4))) goto fail_;
   S->attn_ws = static_cast<float*>(p);
+  if ((r = A(&p, (int64_t)B * 4))) goto fail_;
+  S->pending = static_cast<int32_t*>(p);
   if (c.dtype == RLT_DTYPE_BF16) {
     // every weight shape a step contracts with B rows
     const int64_t shapes[][2] = {{d, 2 * d}, {d, d}, {3 * d, d}, {2 * (int64_t)F, d}, {d, F}, {V, d}, {2 * d * G, d}};
@@ -441,6 +446,7 @@ int32_t reset_state(rlt_state* S, cudaStream_t st) {
   RLT_CUDA(broadcast_row<T>(static_cast<const T*>(S->m->s_star), S->m->cfg.d_model, S->s, S->B, st));
   S->n_enc = 0;
   S->n_dec = 0;
+  S->has_pending = false;
   S->version = S->m->version;
   return RLT_OK;
 }
@@ -489,7 +495,10 @@ int32_t check_state(rlt_model* m, rlt_state* S) {
 
 // ------------------------------------------------------------------ schedules
 // Token-parallel encoder over T tokens of every sequence (eq. 2.1) and the
-// memory projection of eq. 2.2, chunked over sequences.
+// memory projection of eq. 2.2, chunked over sequences.  With an encoded
+// prefix (n_enc > 0, keys and values in the encoder cache) the tokens are
+// positions n_enc+1..n_enc+T and attend to the cached prefix too: the
+// chunked schedule of the same causal computation (App. A.2).
 template <typename T>
 int32_t encode_prefix_impl(rlt_model* m, rlt_state* S, const int32_t* tok, int32_t Tn, cudaStream_t st) {
   struct Range {
@@ -502,11 +511,12 @@ int32_t encode_prefix_impl(rlt_model* m, rlt_state* S, const int32_t* tok, int32
   const int is_bf16 = c.dtype == RLT_DTYPE_BF16;
   const bool cache = (S->flags & RLT_STATE_ENCODER_CACHE) != 0;
   RLT_TRY(ensure_prefill_ws(S, Tn));
+  const int p0 = S->n_enc;  // positions p0+1..p0+Tn; p0 > 0 continues an encoded prefix (keys in the cache)
   const int64_t seqs_per_chunk = S->pf_rows / Tn;
   for (int64_t b0 = 0; b0 < S->B; b0 += seqs_per_chunk) {
     const int Bc = (int)std::min<int64_t>(seqs_per_chunk, S->B - b0);
     const int64_t rows = (int64_t)Bc * Tn;
-    float* e0 = S->e + b0 * S->max_len * d;
+    float* e0 = S->e + b0 * S->max_len * d + (int64_t)p0 * d;
     const RowMap emap{d, Tn, (int64_t)S->max_len * d};
     RLT_CUDA(embed<T>(tok + b0 * Tn, rows, Tn, Tn, static_cast<const T*>(m->emb), d, c.vocab, e0, emap, st));
     for (int l = 0; l < L; ++l) {
@@ -528,18 +538,20 @@ int32_t encode_prefix_impl(rlt_model* m, rlt_state* S, const int32_t* tok, int32
         ld_tk = Tn;
       }
       const T* qkv = static_cast<const T*>(S->pf_big);
-      RLT_CUDA((head_scatter<T, T>(qkv, 3 * d, 0, rows, Tn, 0, H, hd, 1, m->rope_cs, static_cast<T*>(S->pf_q), Tn, st)));
-      RLT_CUDA((head_scatter<T, T>(qkv, 3 * d, d, rows, Tn, 0, H, hd, 1, m->rope_cs, kdst, ld_tk, st)));
-      RLT_CUDA((head_scatter<T, T>(qkv, 3 * d, 2 * d, rows, Tn, 0, H, hd, 0, m->rope_cs, vdst, ld_tk, st)));
+      const int kv_row0 = cache ? p0 : 0;
+      RLT_CUDA((head_scatter<T, T>(qkv, 3 * d, 0, rows, Tn, p0, 0, H, hd, 1, m->rope_cs, static_cast<T*>(S->pf_q), Tn,
+                                   st)));
+      RLT_CUDA((head_scatter<T, T>(qkv, 3 * d, d, rows, Tn, p0, kv_row0, H, hd, 1, m->rope_cs, kdst, ld_tk, st)));
+      RLT_CUDA((head_scatter<T, T>(qkv, 3 * d, 2 * d, rows, Tn, p0, kv_row0, H, hd, 0, m->rope_cs, vdst, ld_tk, st)));
       if constexpr (std::is_same<T, bf16>::value) {
         if (hd == 64 || hd == 128)
-          RLT_CUDA(causal_attn_tc(static_cast<const bf16*>(S->pf_q), kdst, vdst, Tn, ld_tk, Bc, H, hd, Tn,
+          RLT_CUDA(causal_attn_tc(static_cast<const bf16*>(S->pf_q), kdst, vdst, Tn, ld_tk, Bc, H, hd, Tn, p0,
                                   static_cast<bf16*>(S->pf_attn), d, st));
         else
-          RLT_CUDA(causal_attn<T>(static_cast<const T*>(S->pf_q), kdst, vdst, Tn, ld_tk, Bc, H, hd, Tn,
+          RLT_CUDA(causal_attn<T>(static_cast<const T*>(S->pf_q), kdst, vdst, Tn, ld_tk, Bc, H, hd, Tn, p0,
                                   static_cast<T*>(S->pf_attn), d, st));
       } else {
-        RLT_CUDA(causal_attn<T>(static_cast<const T*>(S->pf_q), kdst, vdst, Tn, ld_tk, Bc, H, hd, Tn,
+        RLT_CUDA(causal_attn<T>(static_cast<const T*>(S->pf_q), kdst, vdst, Tn, ld_tk, Bc, H, hd, Tn, p0,
                                 static_cast<T*>(S->pf_attn), d, st));
       }
       RLT_TRY(gemm<T>(S, w.wo, d, S->pf_attn, d, d, (int)rows, d, EPI_RESID, epi_out(e0, emap, 0), false, st));
@@ -555,13 +567,13 @@ int32_t encode_prefix_impl(rlt_model* m, rlt_state* S, const int32_t* tok, int32
     for (int g = 0; g < G; ++g) {
       const int64_t grp = ((int64_t)g * S->B + b0) * H * S->max_len * hd;
       const T* kv = static_cast<const T*>(S->pf_big);
-      RLT_CUDA((head_scatter<T, T>(kv, 2 * d * G, (int64_t)2 * d * g, rows, Tn, 0, H, hd, 1, m->rope_cs,
+      RLT_CUDA((head_scatter<T, T>(kv, 2 * d * G, (int64_t)2 * d * g, rows, Tn, p0, p0, H, hd, 1, m->rope_cs,
                                    static_cast<T*>(S->mem_k) + grp, S->max_len, st)));
-      RLT_CUDA((head_scatter<T, T>(kv, 2 * d * G, (int64_t)2 * d * g + d, rows, Tn, 0, H, hd, 0, m->rope_cs,
+      RLT_CUDA((head_scatter<T, T>(kv, 2 * d * G, (int64_t)2 * d * g + d, rows, Tn, p0, p0, H, hd, 0, m->rope_cs,
                                    static_cast<T*>(S->mem_v) + grp, S->max_len, st)));
     }
   }
-  S->n_enc = Tn;
+  S->n_enc = p0 + Tn;
   return RLT_OK;
 }
 
@@ -583,8 +595,8 @@ int32_t encode_step_impl(rlt_model* m, rlt_state* S, const int32_t* tok, cudaStr
     T* cv = static_cast<T*>(S->ce_v) + lay;
     RLT_CUDA(rmsnorm<T, T>(et, emap, static_cast<const T*>(w.g_ea), B, d, c.rms_eps, static_cast<T*>(S->xb), d, st));
     RLT_TRY(gemm<T>(S, w.qkv, d, S->xb, d, 3 * d, B, d, EPI_STORE, epi_out(S->qkv, plain_rows(S->ld_qkv), 0), true, st));
-    RLT_CUDA((head_scatter<float, T>(S->qkv, S->ld_qkv, d, B, 1, t - 1, H, hd, 1, m->rope_cs, ck, S->max_len, st)));
-    RLT_CUDA((head_scatter<float, T>(S->qkv, S->ld_qkv, 2 * d, B, 1, t - 1, H, hd, 0, m->rope_cs, cv, S->max_len, st)));
+    RLT_CUDA((head_scatter<float, T>(S->qkv, S->ld_qkv, d, B, 1, t - 1, t - 1, H, hd, 1, m->rope_cs, ck, S->max_len, st)));
+    RLT_CUDA((head_scatter<float, T>(S->qkv, S->ld_qkv, 2 * d, B, 1, t - 1, t - 1, H, hd, 0, m->rope_cs, cv, S->max_len, st)));
     prof_begin(m, st);
     RLT_CUDA(prefix_attn<T>(S->qkv, S->ld_qkv, ck, cv, S->max_len, B, H, hd, t, t - 1, m->rope_cs,
                             static_cast<T*>(S->attn), d, S->attn_ws, S->attn_ws_floats, st));
@@ -599,9 +611,9 @@ int32_t encode_step_impl(rlt_model* m, rlt_state* S, const int32_t* tok, cudaStr
                   true, st));
   for (int g = 0; g < G; ++g) {
     const int64_t grp = (int64_t)g * B * H * S->max_len * hd;
-    RLT_CUDA((head_scatter<float, T>(S->qkv, S->ld_qkv, (int64_t)2 * d * g, B, 1, t - 1, H, hd, 1, m->rope_cs,
+    RLT_CUDA((head_scatter<float, T>(S->qkv, S->ld_qkv, (int64_t)2 * d * g, B, 1, t - 1, t - 1, H, hd, 1, m->rope_cs,
                                      static_cast<T*>(S->mem_k) + grp, S->max_len, st)));
-    RLT_CUDA((head_scatter<float, T>(S->qkv, S->ld_qkv, (int64_t)2 * d * g + d, B, 1, t - 1, H, hd, 0, m->rope_cs,
+    RLT_CUDA((head_scatter<float, T>(S->qkv, S->ld_qkv, (int64_t)2 * d * g + d, B, 1, t - 1, t - 1, H, hd, 0, m->rope_cs,
                                      static_cast<T*>(S->mem_v) + grp, S->max_len, st)));
   }
   S->n_enc = t;
@@ -725,9 +737,14 @@ int32_t readout_impl(rlt_model* m, rlt_state* S, const int32_t* next, int64_t ne
     RLT_TRY(gemm<T>(S, m->w_out, d, S->xb, d, V, B, d, EPI_STORE, epi_out(S->logits, plain_rows(V), 0), true, st));
   }
   if (next && logp) RLT_CUDA(logp_gather(S->logits, B, V, next, next_stride, logp, ld_logp, st));
-  if (samp)
-    RLT_CUDA(sample_topk(S->logits, B, V, samp->temperature, samp->top_k, samp->seed, (uint32_t)S->n_dec,
-                         out ? out->sampled : nullptr, out ? out->logp_sampled : nullptr, out ? out->logmu : nullptr, st));
+  if (samp) {
+    int32_t* tok_out = out && out->sampled ? out->sampled : S->pending;
+    RLT_CUDA(sample_topk(S->logits, B, V, samp->temperature, samp->top_k, samp->seed, (uint32_t)S->n_dec, tok_out,
+                         out ? out->logp_sampled : nullptr, out ? out->logmu : nullptr, st));
+    if (tok_out != S->pending)
+      RLT_CUDA(cudaMemcpyAsync(S->pending, tok_out, (size_t)B * 4, cudaMemcpyDeviceToDevice, st));
+    S->has_pending = true;  // the sampled token is owed to the next transition
+  }
   if (out && out->logits) RLT_CUDA(copy_f32(out->logits, S->logits, (int64_t)B * V, st));
   return RLT_OK;
 }
@@ -754,6 +771,7 @@ int32_t rlt_init_weights(const rlt_config* cfg, uint64_t seed, rlt_model** out) 
   RLT_TRY(validate(cfg));
   rlt_model* m = new rlt_model();
   m->cfg = *cfg;
+  m->seed = seed;
   m->hd = cfg->d_model / cfg->n_heads;
   m->esz = cfg->dtype == RLT_DTYPE_BF16 ? 2 : 4;
   cudaGetDevice(&m->device);
@@ -862,8 +880,76 @@ int32_t rlt_state_info_get(const rlt_state* s, rlt_state_info* out) {
   out->ring_head = Wm1 > 0 ? s->n_dec % Wm1 : 0;
   out->has_encoder_cache = (s->flags & RLT_STATE_ENCODER_CACHE) ? 1 : 0;
   out->model_version = s->version;
+  out->has_pending = s->has_pending ? 1 : 0;
   return ok();
 }
+
+// ------------------------------------------------------------------ snapshots
+namespace {
+
+// Exact prefix snapshot (report §6): encoder cache, memory M_<=t, H_t =
+// (s_t, C^D_t), positions, window and model identity.  Little-endian; the
+// payload follows the header in the order of snapshot_sections().
+struct SnapHeader {
+  char magic[8];  // "RLTSNAP1"
+  uint32_t header_bytes, flags;
+  int32_t d_model, n_heads, n_layers, window, groups, ffn, vocab, tied, merge_kind, dtype, bos_id, batch;
+  float alpha, rms_eps, rope_base, reserved_f;
+  int32_t n_enc, n_dec, reserved0, reserved1;
+  uint64_t weight_seed, model_version, payload_bytes;
+};
+constexpr uint32_t kSnapCache = 1, kSnapPending = 2, kSnapFold = 4;
+
+struct SnapSection {
+  void* dev;      // first byte on the device
+  size_t width;   // bytes per row in the snapshot
+  size_t pitch;   // bytes between rows on the device
+  size_t rows;
+};
+
+std::vector<SnapSection> snapshot_sections(rlt_state* S, int n_enc, uint32_t flags) {
+  const rlt_model* m = S->m;
+  const rlt_config& c = m->cfg;
+  const size_t es = m->esz, d = c.d_model, hd = m->hd, B = S->B, H = c.n_heads, L = c.n_layers, G = c.groups;
+  const size_t ml = S->max_len, Wm1 = c.window - 1;
+  std::vector<SnapSection> v;
+  v.push_back({S->s, B * d * 4, B * d * 4, 1});
+  if (n_enc > 0) {
+    v.push_back({S->e, (size_t)n_enc * d * 4, ml * d * 4, B});
+    v.push_back({S->mem_k, (size_t)n_enc * hd * es, ml * hd * es, G * B * H});
+    v.push_back({S->mem_v, (size_t)n_enc * hd * es, ml * hd * es, G * B * H});
+    if (flags & kSnapCache) {
+      v.push_back({S->ce_k, (size_t)n_enc * hd * es, ml * hd * es, L * B * H});
+      v.push_back({S->ce_v, (size_t)n_enc * hd * es, ml * hd * es, L * B * H});
+    }
+  }
+  if (Wm1 > 0) {
+    v.push_back({S->ring_k, L * B * H * Wm1 * hd * es, L * B * H * Wm1 * hd * es, 1});
+    v.push_back({S->ring_v, L * B * H * Wm1 * hd * es, L * B * H * Wm1 * hd * es, 1});
+  }
+  if (flags & kSnapPending) v.push_back({S->pending, B * 4, B * 4, 1});
+  if (flags & kSnapFold) {
+    v.push_back({S->zb, B * d * 2, B * d * 2, 1});
+    v.push_back({S->ss, (d / 128) * B * 4, (d / 128) * B * 4, 1});
+  }
+  return v;
+}
+
+size_t payload_bytes(const std::vector<SnapSection>& v) {
+  size_t n = 0;
+  for (const auto& x : v) n += x.width * x.rows;
+  return n;
+}
+
+uint32_t snapshot_flags(const rlt_state* S) {
+  uint32_t f = 0;
+  if ((S->flags & RLT_STATE_ENCODER_CACHE) && S->n_enc > 0) f |= kSnapCache;
+  if (S->has_pending) f |= kSnapPending;
+  if (S->m->cfg.dtype == RLT_DTYPE_BF16 && S->n_dec > 0) f |= kSnapFold;
+  return f;
+}
+
+}  // namespace
 
 int32_t rlt_state_read(const rlt_state* s, int32_t what, int32_t index, void* host, size_t bytes) {
   if (!s || !host) return fail(RLT_E_INVAL, "null argument");
@@ -903,11 +989,91 @@ int32_t rlt_state_read(const rlt_state* s, int32_t what, int32_t index, void* ho
   return ok();
 }
 
+int32_t rlt_state_export(const rlt_state* s_const, void* host, size_t cap, size_t* used, void* stream) {
+  if (!s_const || !used) return fail(RLT_E_INVAL, "null argument");
+  rlt_state* S = const_cast<rlt_state*>(s_const);
+  const rlt_model* m = S->m;
+  const uint32_t flags = snapshot_flags(S);
+  const std::vector<SnapSection> secs = snapshot_sections(S, S->n_enc, flags);
+  const size_t total = sizeof(SnapHeader) + payload_bytes(secs);
+  *used = total;
+  if (!host) return ok();
+  if (cap < total) return fail(RLT_E_CAPACITY, "snapshot needs " + std::to_string(total) + " bytes");
+  const rlt_config& c = m->cfg;
+  SnapHeader h{};
+  std::memcpy(h.magic, "RLTSNAP1", 8);
+  h.header_bytes = sizeof(SnapHeader);
+  h.flags = flags;
+  h.d_model = c.d_model; h.n_heads = c.n_heads; h.n_layers = c.n_layers; h.window = c.window; h.groups = c.groups;
+  h.ffn = c.ffn; h.vocab = c.vocab; h.tied = c.tied; h.merge_kind = c.merge_kind; h.dtype = c.dtype;
+  h.bos_id = c.bos_id; h.batch = S->B;
+  h.alpha = c.alpha; h.rms_eps = c.rms_eps; h.rope_base = c.rope_base;
+  h.n_enc = S->n_enc; h.n_dec = S->n_dec;
+  h.weight_seed = m->seed; h.model_version = S->version;
+  h.payload_bytes = total - sizeof(SnapHeader);
+  std::memcpy(host, &h, sizeof h);
+  RLT_CUDA(cudaSetDevice(m->device));
+  cudaStream_t st = (cudaStream_t)stream;
+  uint8_t* dst = static_cast<uint8_t*>(host) + sizeof h;
+  for (const auto& x : secs) {
+    RLT_CUDA(cudaMemcpy2DAsync(dst, x.width, x.dev, x.pitch, x.width, x.rows, cudaMemcpyDeviceToHost, st));
+    dst += x.width * x.rows;
+  }
+  RLT_CUDA(cudaStreamSynchronize(st));
+  return ok();
+}
+
+int32_t rlt_state_import(rlt_state* S, const void* host, size_t bytes, void* stream) {
+  if (!S || !host) return fail(RLT_E_INVAL, "null argument");
+  if (bytes < sizeof(SnapHeader)) return fail(RLT_E_INVAL, "not a snapshot (too short)");
+  SnapHeader h;
+  std::memcpy(&h, host, sizeof h);
+  if (std::memcmp(h.magic, "RLTSNAP1", 8) != 0 || h.header_bytes != sizeof(SnapHeader))
+    return fail(RLT_E_INVAL, "not a snapshot of this format");
+  rlt_model* m = S->m;
+  const rlt_config& c = m->cfg;
+  if (h.d_model != c.d_model || h.n_heads != c.n_heads || h.n_layers != c.n_layers || h.window != c.window ||
+      h.groups != c.groups || h.ffn != c.ffn || h.vocab != c.vocab || h.tied != c.tied ||
+      h.merge_kind != c.merge_kind || h.dtype != c.dtype || h.bos_id != c.bos_id || h.alpha != c.alpha ||
+      h.rms_eps != c.rms_eps || h.rope_base != c.rope_base)
+    return fail(RLT_E_INVAL, "snapshot of a model with another configuration");
+  if (h.weight_seed != m->seed || h.model_version != m->version)
+    return fail(RLT_E_STALE, "snapshot was taken under other weights");
+  if (h.batch != S->B) return fail(RLT_E_INVAL, "snapshot batch differs from the state's");
+  if (h.n_enc < 0 || h.n_dec < 0 || h.n_dec > h.n_enc) return fail(RLT_E_INVAL, "bad positions in snapshot");
+  if (h.n_enc > S->max_len) return fail(RLT_E_CAPACITY, "snapshot positions exceed the state's max_len");
+  const bool want_cache = (S->flags & RLT_STATE_ENCODER_CACHE) && h.n_enc > 0;
+  if (want_cache && !(h.flags & kSnapCache))
+    return fail(RLT_E_STATE, "the state keeps an encoder cache but the snapshot has none");
+  if (c.dtype == RLT_DTYPE_BF16 && h.n_dec > 0 && !(h.flags & kSnapFold))
+    return fail(RLT_E_INVAL, "snapshot lacks the readout operand");
+  const std::vector<SnapSection> secs = snapshot_sections(S, h.n_enc, h.flags);
+  if (h.payload_bytes != payload_bytes(secs) || bytes < sizeof(SnapHeader) + h.payload_bytes)
+    return fail(RLT_E_INVAL, "snapshot payload size mismatch");
+  RLT_CUDA(cudaSetDevice(m->device));
+  cudaStream_t st = (cudaStream_t)stream;
+  const uint8_t* src = static_cast<const uint8_t*>(host) + sizeof h;
+  const bool has_cache_here = (S->flags & RLT_STATE_ENCODER_CACHE) != 0;
+  for (const auto& x : secs) {
+    const bool cache_sec = x.dev == S->ce_k || x.dev == S->ce_v;
+    if (!(cache_sec && !has_cache_here))  // a state without the cache drops those sections
+      RLT_CUDA(cudaMemcpy2DAsync(x.dev, x.pitch, src, x.width, x.width, x.rows, cudaMemcpyHostToDevice, st));
+    src += x.width * x.rows;
+  }
+  RLT_CUDA(cudaStreamSynchronize(st));
+  S->n_enc = h.n_enc;
+  S->n_dec = h.n_dec;
+  S->has_pending = (h.flags & kSnapPending) != 0;
+  S->version = m->version;
+  return ok();
+}
+
 int32_t rlt_encode_prefix(rlt_model* m, rlt_state* s, const int32_t* tok_dev, int32_t T, void* stream) {
   RLT_TRY(check_state(m, s));
   if (!tok_dev || T <= 0) return fail(RLT_E_INVAL, "need tokens and T > 0");
-  if (s->n_enc != 0) return fail(RLT_E_STATE, "token-parallel encoding starts from an empty encoder");
-  if (T > s->max_len) return fail(RLT_E_CAPACITY, "T exceeds max_len");
+  if (s->n_enc != 0 && !(s->flags & RLT_STATE_ENCODER_CACHE))
+    return fail(RLT_E_STATE, "continuing an encoded prefix needs the encoder cache");
+  if ((int64_t)s->n_enc + T > s->max_len) return fail(RLT_E_CAPACITY, "n_enc + T exceeds max_len");
   return RLT_DISPATCH(m, encode_prefix_impl, m, s, tok_dev, T, (cudaStream_t)stream);
 }
 
@@ -930,10 +1096,12 @@ int32_t rlt_decoder_step(rlt_model* m, rlt_state* s, const int32_t* tok_dev, con
   StepRange range(m, t);
   if (s->n_enc < t) {
     if (!(s->flags & RLT_STATE_ENCODER_CACHE)) return fail(RLT_E_STATE, "x_t not encoded and the state has no encoder cache");
-    if (!tok_dev) return fail(RLT_E_INVAL, "x_t must be given when it is not yet encoded");
-    RLT_TRY(RLT_DISPATCH(m, encode_step_impl, m, s, tok_dev, st));
+    if (!tok_dev && !s->has_pending)
+      return fail(RLT_E_STATE, "x_t must be given: it is not yet encoded and no sampled token is pending");
+    RLT_TRY(RLT_DISPATCH(m, encode_step_impl, m, s, tok_dev ? tok_dev : s->pending, st));
   }
   RLT_TRY(RLT_DISPATCH(m, transition_impl, m, s, st));
+  s->has_pending = false;
   if (next_dev || samp || (out && out->logits))
     RLT_TRY(RLT_DISPATCH(m, readout_impl, m, s, next_dev, (int64_t)1, out ? out->logp : nullptr, (int64_t)1, samp, out, st));
   return ok();
