@@ -254,6 +254,24 @@ int32_t rlt_prefill(rlt_model* m, rlt_state* s, const int32_t* tok_dev, int32_t 
 int32_t rlt_replay_logprobs(rlt_model* m, const int32_t* tok_dev, int32_t B, int32_t S, float* logp_dev,
                             void* stream);
 
+/* RL replay with importance ratios (report §5.3, eq. 5.5, and App. A.4):
+ * rlt_replay_logprobs under the current weights, then for every scored
+ * token t = 1..S-1 (row-major [B][S-1], the same indexing as logp_dev)
+ *   ratio_dev[b][t]      = exp(logp - logmu_dev)  where action_mask_dev != 0,
+ *                        = 1                      elsewhere (user/tool/prompt
+ *                          tokens get no action factor, report §6),
+ *   seq_logratio_dev[b]  = sum over action tokens of (logp - logmu_dev), the
+ *                          log of the trajectory ratio prod_i r_i,
+ * summed in double in a fixed order.  logmu_dev holds the behaviour
+ * log-probabilities the sampler recorded (temperature, truncation and
+ * renormalisation included, as rlt_readout's logmu); action_mask_dev is
+ * uint8.  logp_dev [B][S-1] receives the current-policy log-probs.  Either
+ * ratio output may be NULL (not both).  Errors: as rlt_replay_logprobs,
+ * RLT_E_INVAL. */
+int32_t rlt_replay_ratios(rlt_model* m, const int32_t* tok_dev, int32_t B, int32_t S, const float* logmu_dev,
+                          const uint8_t* action_mask_dev, float* logp_dev, float* ratio_dev,
+                          float* seq_logratio_dev, void* stream);
+
 /* ---------------------------------------------------------------- ops */
 
 /* Kernel-level check of the step's contraction: y_dev [N][M] fp32 =

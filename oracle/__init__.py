@@ -87,6 +87,8 @@ def lib():
                                  ctypes.c_uint64, ctypes.c_uint32, ctypes.c_uint32, _c_int32_p, _c_double_p,
                                  _c_double_p, _c_double_p]
         L.orc_replay_logprobs.argtypes = [ctypes.c_void_p, _c_int32_p, ctypes.c_int32, ctypes.c_int32, _c_double_p]
+        L.orc_replay_ratios.argtypes = [ctypes.c_void_p, _c_int32_p, ctypes.c_int32, _c_double_p,
+                                        ctypes.POINTER(ctypes.c_uint8), _c_double_p, _c_double_p, _c_double_p]
         L.orc_generate.argtypes = [ctypes.c_void_p, _c_int32_p, ctypes.c_int32, ctypes.c_int32, ctypes.c_float,
                                    ctypes.c_int32, ctypes.c_uint64, ctypes.c_uint32, _c_int32_p, _c_double_p,
                                    _c_double_p, _c_double_p]
@@ -239,6 +241,19 @@ class Model:
         if lib().orc_replay_logprobs(self.h, _ip(tok), tok.size, schedule, _dp(out)):
             raise ValueError("orc_replay_logprobs failed")
         return out
+
+    def replay_ratios(self, tokens, logmu, mask) -> dict:
+        tok = np.ascontiguousarray(tokens, dtype=np.int32)
+        lmu = np.ascontiguousarray(logmu, dtype=np.float64)
+        msk = np.ascontiguousarray(mask, dtype=np.uint8)
+        if lmu.size != tok.size - 1 or msk.size != tok.size - 1:
+            raise ValueError("logmu and mask need S-1 entries")
+        lp, r, tot = np.zeros(tok.size - 1), np.zeros(tok.size - 1), ctypes.c_double()
+        if lib().orc_replay_ratios(self.h, _ip(tok), tok.size, _dp(lmu),
+                                   msk.ctypes.data_as(ctypes.POINTER(ctypes.c_uint8)), _dp(lp), _dp(r),
+                                   ctypes.byref(tot)):
+            raise ValueError("orc_replay_ratios failed")
+        return {"logp": lp, "ratio": r, "seq_logratio": tot.value}
 
     def generate(self, prompt, n_new: int, temperature: float, top_k: int, seed: int, b: int) -> dict:
         p = np.ascontiguousarray(prompt, dtype=np.int32)

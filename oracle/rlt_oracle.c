@@ -20,7 +20,8 @@
  *   report §2.5  eqs. 2.9-2.11 gated merge; eqs. 2.12-2.16 decoder block;
  *                cache retention max(1,t-W+2)..t
  *   report §2.6  tied configuration
- *   report §5.3  behaviour log-probabilities under the actual sampler
+ *   report §5.3  behaviour log-probabilities under the actual sampler;
+ *                eq. 5.5 replay ratios
  *   report App. A.1/A.2/A.4 execution schedules (prefill, generation, replay)
  *   project page, "The complete state matters" (clean forms of 2.3/2.5/2.6)
  *
@@ -780,6 +781,25 @@ int orc_replay_logprobs(const orc_model *m, const int32_t *tok, int32_t S, int32
   free(lg); free(lp);
   orc_seq_free(q);
   return rc;
+}
+
+/* RL replay with importance ratios (report §5.3, eq. 5.5; App. A.4): the
+ * current-policy replay of one rollout, then per scored token
+ * r = exp(log p - log mu) for sampled actions (mask != 0) and no factor (1)
+ * for external tokens (report §6), and the log of the trajectory ratio, the
+ * sum of log r over the actions. */
+int orc_replay_ratios(const orc_model *m, const int32_t *tok, int32_t S, const double *logmu, const uint8_t *mask,
+                      double *out_logp, double *out_ratio, double *out_seq_logratio) {
+  const int rc = orc_replay_logprobs(m, tok, S, 0, out_logp);
+  if (rc) return rc;
+  double sum = 0.0;
+  for (int32_t i = 0; i < S - 1; ++i) {
+    const double lr = out_logp[i] - logmu[i];
+    out_ratio[i] = mask[i] ? exp(lr) : 1.0;
+    if (mask[i]) sum += lr;
+  }
+  *out_seq_logratio = sum;
+  return 0;
 }
 
 /* Prompt prefill (App. A.1) then sampled generation (App. A.2) for one

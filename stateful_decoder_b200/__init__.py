@@ -44,7 +44,7 @@ EXPORTED = (
     "rlt_encode_prefix", "rlt_readout", "rlt_decoder_step", "rlt_prefill", "rlt_replay_logprobs",
     "rlt_last_error", "rlt_check_device", "rlt_profile_enable", "rlt_profile_read", "rlt_op_linear",
     "rlt_op_sample", "rlt_kernel_launches", "rlt_op_prefix_attention", "rlt_op_prefix_attention_noalloc",
-    "rlt_state_export", "rlt_state_import",
+    "rlt_state_export", "rlt_state_import", "rlt_replay_ratios",
 )
 
 
@@ -101,6 +101,7 @@ _sig = {
     "rlt_decoder_step": [_vp, _vp, _vp, _vp, ctypes.POINTER(Sampling), ctypes.POINTER(ReadoutOut), _vp],
     "rlt_prefill": [_vp, _vp, _vp, _i32, _vp, _vp],
     "rlt_replay_logprobs": [_vp, _vp, _i32, _i32, _vp, _vp],
+    "rlt_replay_ratios": [_vp, _vp, _i32, _i32, _vp, _vp, _vp, _vp, _vp, _vp],
     "rlt_op_linear": [_vp, _vp, _vp, _i32, _i32, _i32, _i32, _i32, _vp],
     "rlt_op_prefix_attention": [_vp, _vp, _vp, ctypes.c_int64, _i32, _i32, _i32, _i32, _i32, _vp, _i32, _vp, _vp],
     "rlt_op_prefix_attention_noalloc": [_vp, _vp, _vp, ctypes.c_int64, _i32, _i32, _i32, _i32, _i32, _vp, _i32, _vp,
@@ -307,6 +308,17 @@ def rlt_replay_logprobs(model: Model, tokens, logp, stream=None) -> None:
     B, S = tokens.shape
     _check(_lib.rlt_replay_logprobs(model.h, _dev(tokens, "torch.int32"), B, S, _dev(logp, "torch.float32"),
                                     _stream(stream)))
+
+
+def rlt_replay_ratios(model: Model, tokens, logmu, action_mask, logp, ratio=None, seq_logratio=None,
+                      stream=None) -> None:
+    """tokens int32 [B, S]; logmu float32 and action_mask uint8 [B, S-1]; outputs
+    logp and ratio float32 [B, S-1], seq_logratio float32 [B] (CUDA tensors)."""
+    B, S = tokens.shape
+    _check(_lib.rlt_replay_ratios(model.h, _dev(tokens, "torch.int32"), B, S, _dev(logmu, "torch.float32"),
+                                  _dev(action_mask, "torch.uint8"), _dev(logp, "torch.float32"),
+                                  _dev(ratio, "torch.float32"), _dev(seq_logratio, "torch.float32"),
+                                  _stream(stream)))
 
 
 def rlt_op_linear(w, x, y, use_tensor_cores: bool = True, stream=None) -> None:

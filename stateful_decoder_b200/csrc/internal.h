@@ -111,6 +111,12 @@ template <typename WT, typename OT>
 cudaError_t merge_prep(const float* e, RowMap e_map, const float* s, const WT* gamma, int B, int d, float eps,
                        int kind, OT* out, cudaStream_t st);
 
+// RL replay ratios over [B][n] log-probs: ratio = exp(logp - logmu) where
+// mask != 0, else 1; seq_logratio[b] = sum over masked tokens of
+// (logp - logmu).  Either output may be null.
+cudaError_t replay_ratios(const float* logp, const float* logmu, const uint8_t* mask, int B, int n, float* ratio,
+                          float* seq_logratio, cudaStream_t st);
+
 // Scatter head-split rows into a [B][H][ld_t][hd] store: row i = r %
 // rows_per_seq of a sequence goes to store row dst_row0 + i, rotated (rope
 // != 0) at position pos0 + i.

@@ -161,6 +161,33 @@ __global__ void logp_gather_kernel(const float* __restrict__ logits, int V, cons
   }
 }
 
+// RL replay ratios (eq. 5.5): per token r = exp(log p - log mu) where the
+// token is a sampled action, 1 (no action factor) elsewhere; per sequence
+// the log of the product of the action ratios.  One block per sequence; the
+// sum runs in double in a fixed order (thread-strided partials, then a fixed
+// tree), so it does not depend on timing.
+__global__ void replay_ratio_kernel(const float* __restrict__ logp, const float* __restrict__ logmu,
+                                    const uint8_t* __restrict__ mask, int n, float* ratio, float* seq_logratio) {
+  griddep_enter();
+  __shared__ double part[256];
+  const int b = blockIdx.x;
+  const int64_t base = (int64_t)b * n;
+  double acc = 0.0;
+  for (int i = threadIdx.x; i < n; i += 256) {
+    const bool act = mask[base + i] != 0;
+    const float dl = logp[base + i] - logmu[base + i];
+    if (ratio) ratio[base + i] = act ? expf(dl) : 1.0f;
+    if (act) acc += (double)dl;
+  }
+  part[threadIdx.x] = acc;
+  __syncthreads();
+  for (int w = 128; w > 0; w >>= 1) {
+    if (threadIdx.x < w) part[threadIdx.x] += part[threadIdx.x + w];
+    __syncthreads();
+  }
+  if (threadIdx.x == 0 && seq_logratio) seq_logratio[b] = (float)part[0];
+}
+
 // order-preserving key of a float (larger float -> larger key); -0 and +0
 // share a key so equal values compare equal as floats do
 __device__ __forceinline__ uint32_t fkey(float f) {
@@ -394,6 +421,16 @@ cudaError_t logp_gather(const float* logits, int B, int V, const int32_t* next, 
                         int64_t ld_logp, cudaStream_t st) {
   {
     const cudaError_t e_l = launch_pdl(logp_gather_kernel, dim3(B), dim3(1024), 0, st, logits, V, next, next_stride, logp, ld_logp);
+    if (e_l != cudaSuccess) return e_l;
+  }
+  return cudaGetLastError();
+}
+
+cudaError_t replay_ratios(const float* logp, const float* logmu, const uint8_t* mask, int B, int n, float* ratio,
+                          float* seq_logratio, cudaStream_t st) {
+  {
+    const cudaError_t e_l = launch_pdl(replay_ratio_kernel, dim3(B), dim3(256), 0, st, logp, logmu, mask, n, ratio,
+                                       seq_logratio);
     if (e_l != cudaSuccess) return e_l;
   }
   return cudaGetLastError();

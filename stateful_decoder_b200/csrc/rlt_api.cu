@@ -1141,8 +1141,19 @@ int32_t rlt_replay_logprobs(rlt_model* m, const int32_t* tok_dev, int32_t B, int
     StepRange range(m, t);
     RLT_TRY(RLT_DISPATCH(m, transition_impl, m, st_, st));
     RLT_TRY(RLT_DISPATCH(m, readout_impl, m, st_, tok_dev + t, (int64_t)S, logp_dev + (t - 1), (int64_t)(S - 1),
-                         (const rlt_sampling*)nullptr, (const rlt_readout_out*)false, st));
+                         (const rlt_sampling*)nullptr, (const rlt_readout_out*)nullptr, st));
   }
+  return ok();
+}
+
+int32_t rlt_replay_ratios(rlt_model* m, const int32_t* tok_dev, int32_t B, int32_t S, const float* logmu_dev,
+                          const uint8_t* action_mask_dev, float* logp_dev, float* ratio_dev, float* seq_logratio_dev,
+                          void* stream) {
+  if (!logmu_dev || !action_mask_dev) return fail(RLT_E_INVAL, "null behaviour log-probs or action mask");
+  if (!ratio_dev && !seq_logratio_dev) return fail(RLT_E_INVAL, "no ratio output requested");
+  RLT_TRY(rlt_replay_logprobs(m, tok_dev, B, S, logp_dev, stream));
+  RLT_CUDA(replay_ratios(logp_dev, logmu_dev, action_mask_dev, B, S - 1, ratio_dev, seq_logratio_dev,
+                         (cudaStream_t)stream));
   return ok();
 }
 

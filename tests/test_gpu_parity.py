@@ -6,6 +6,8 @@ token ids of the sampler on identical fp32 logits, cache positions and ring
 indices.  Inputs come from the seeded generator in ``synth``; the oracle
 never sees a value produced by the CUDA path.
 """
+import math
+
 import numpy as np
 import pytest
 
@@ -337,3 +339,41 @@ def test_batched_equals_single_wide_tiles(rlt, torch_mod):
     for b in (0, 131, 255):
         one, _ = _gpu_replay(rlt, torch_mod, cfg, tok[b:b + 1].copy(), model=m)
         assert np.array_equal(one[0], full[b]), (b, np.max(np.abs(one[0] - full[b])))
+
+
+# ------------------------------------------------------------------ RL replay ratios
+def test_replay_ratios_match_oracle(rlt, torch_mod, oracle_lib):
+    """Eq. 5.5 through rlt_replay_ratios: current-policy log-probs as
+    rlt_replay_logprobs gives them, ratios exp(log p - log mu) on the action
+    tokens and 1 elsewhere, and the trajectory log-ratio; against the
+    oracle's replay on the same rollout, recorded log mu and action mask."""
+    torch = torch_mod
+    for (w, cfg), tol in ((_tiny(), TOL_F32), (_bf16_small(prompt=120), TOL_BF16)):
+        tok = synth.tokens(w)
+        B, S = tok.shape
+        rng = np.random.default_rng(5150)
+        logmu = rng.normal(-4.0, 1.0, (B, S - 1)).astype(np.float32)
+        mask = (rng.random((B, S - 1)) < 0.6).astype(np.uint8)
+        m = rlt.rlt_init_weights(cfg, synth.WEIGHT_SEED)
+        tdev = torch.from_numpy(tok).cuda()
+        lp = torch.zeros(B, S - 1, device="cuda")
+        ratio = torch.zeros(B, S - 1, device="cuda")
+        seq = torch.zeros(B, device="cuda")
+        rlt.rlt_replay_ratios(m, tdev, torch.from_numpy(logmu).cuda(), torch.from_numpy(mask).cuda(), lp, ratio, seq)
+        ref = torch.zeros(B, S - 1, device="cuda")
+        rlt.rlt_replay_logprobs(m, tdev, ref)
+        torch.cuda.synchronize()
+        rlt.rlt_check_device()
+        lp, ratio, seq, ref = (x.cpu().numpy().astype(np.float64) for x in (lp, ratio, seq, ref))
+        assert np.array_equal(lp, ref)
+        assert np.all(ratio[mask == 0] == 1.0)
+        # the kernel's arithmetic on its own log-probs (fp32 exp, fp64 sum)
+        mine = np.where(mask == 1, np.exp(lp - logmu), 1.0)
+        assert np.allclose(ratio, mine, rtol=1e-6, atol=0)
+        assert np.allclose(seq, ((lp - logmu) * mask).sum(1), rtol=1e-6, atol=1e-4)
+        om = oracle_lib.Model(cfg, seed=synth.WEIGHT_SEED)
+        for b in range(B):
+            o = om.replay_ratios(tok[b], logmu[b], mask[b])
+            assert np.max(np.abs(lp[b] - o["logp"])) <= tol
+            assert np.all(np.abs(ratio[b] - o["ratio"]) <= o["ratio"] * math.expm1(tol) + 1e-6)
+            assert abs(seq[b] - o["seq_logratio"]) <= tol * int(mask[b].sum()) + 1e-4

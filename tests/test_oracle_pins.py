@@ -301,3 +301,38 @@ def test_sampler_distribution_chi2(oracle_lib):
             assert math.isclose(lp, sps.log_softmax(lg.astype(np.float64))[tok], rel_tol=1e-9)
     chi2 = ((counts - n * p) ** 2 / (n * p)).sum()
     assert chi2 < st.chi2.ppf(0.999, k - 1)
+
+
+def test_replay_ratios_pins(oracle_lib):
+    """Eq. 5.5 replay ratios.  Pinned by: (a) an untempered, untruncated
+    sampler (tau = 1, top_k = V) records log mu equal to the raw model log-prob,
+    so the replay of its own rollout gives ratio 1 at every action (this ties
+    the sampler's generation schedule to the replay schedule, Prop. 3.1);
+    (b) tokens outside the action mask get no factor; (c) the trajectory
+    log-ratio is the log of the product of the action ratios; (d) shifting
+    log mu by c on k actions shifts the trajectory log-ratio by -k c."""
+    w = synth.workload("tiny")
+    cfg = synth.model_config(w)
+    m = oracle_lib.Model(cfg, seed=42)
+    prompt = synth.tokens(w)[0, :10]
+    V = cfg["vocab"]
+    g = m.generate(prompt, 8, 1.0, V, 11, 0)
+    hist = np.concatenate([prompt, g["tokens"]])
+    n = hist.size - 1
+    logmu = np.zeros(n)
+    mask = np.zeros(n, np.uint8)
+    logmu[prompt.size - 1:] = g["logmu"]
+    mask[prompt.size - 1:] = 1  # the sampled response tokens are the actions
+    r = m.replay_ratios(hist, logmu, mask)
+    assert np.allclose(r["ratio"][mask == 1], 1.0, atol=1e-6)
+    assert abs(r["seq_logratio"]) <= 1e-5
+    assert np.all(r["ratio"][mask == 0] == 1.0)
+    assert np.allclose(r["logp"], m.replay_logprobs(hist), atol=0, rtol=0)
+    rng = np.random.default_rng(3)
+    lmu2 = r["logp"] + rng.normal(0, 0.3, n)
+    mask2 = (rng.random(n) < 0.5).astype(np.uint8)
+    r2 = m.replay_ratios(hist, lmu2, mask2)
+    assert np.all(r2["ratio"][mask2 == 0] == 1.0)
+    assert math.isclose(np.prod(r2["ratio"]), math.exp(r2["seq_logratio"]), rel_tol=1e-12)
+    r3 = m.replay_ratios(hist, lmu2 + 0.25 * mask2, mask2)
+    assert math.isclose(r3["seq_logratio"], r2["seq_logratio"] - 0.25 * int(mask2.sum()), abs_tol=1e-12)
