@@ -54,8 +54,12 @@ struct EpiParams {
   float norm_eps;
 };
 
-__device__ __forceinline__ float sigmoidf_(float x) { return 1.0f / (1.0f + __expf(-x)); }
-__device__ __forceinline__ float siluf_(float x) { return x / (1.0f + __expf(-x)); }
+// The fast division (__fdividef) keeps the epilogue free of the IEEE division
+// subroutine and its branches; 1 + exp(-x) lies in [1, inf), where it is
+// accurate to a few ulp and returns 0 for an infinite divisor (the correct
+// limits sigmoid -> 0, silu -> -0).
+__device__ __forceinline__ float sigmoidf_(float x) { return __fdividef(1.0f, 1.0f + __expf(-x)); }
+__device__ __forceinline__ float siluf_(float x) { return __fdividef(x, 1.0f + __expf(-x)); }
 
 __device__ __forceinline__ float load_bias(const EpiParams& p, int m) {
   return p.bias_bf16 ? __bfloat162float(reinterpret_cast<const bf16*>(p.bias)[m])
