@@ -101,7 +101,7 @@ __device__ __forceinline__ float2 softmax_inplace(float* sc, int n, float* red) 
 
 // ------------------------------------------------------------------ SWA
 template <typename KT, int HD>
-__global__ void __launch_bounds__(kThreads) swa_attn_kernel(const float* __restrict__ qkv, int64_t ld_qkv, KT* ring_k,
+__global__ void __launch_bounds__(kThreads, 9) swa_attn_kernel(const float* __restrict__ qkv, int64_t ld_qkv, KT* ring_k,
                                                             KT* ring_v, int H, int t, int W,
                                                             const float* __restrict__ rope_cs, KT* out,
                                                             int64_t ld_out, float scale_log2) {

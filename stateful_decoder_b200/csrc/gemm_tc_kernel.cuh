@@ -353,26 +353,41 @@ __global__ void __launch_bounds__(128, 1)
   __syncwarp();
 
   // Epilogue: warp w owns accumulator lanes 32w..32w+31 (output features).
+  const int row = warp * 32 + lane;
+  const int m = m_tile * BM + row;
+  const EpiRowConst rc = epi_row_const<EPI>(ep, m);  // weights only: no wait needed
+  const int64_t n_base = (int64_t)n_tile * BN;
+  float* rinv = reinterpret_cast<float*>(smem + C::EXTRA_OFF);  // [BN] folded RMSNorm scale per column
+  float* red = rinv + 256;                                        // [4][32] per-warp column sums
+  if (warp >= 2) {
+    // Warps 2 and 3 have no main-loop role: while the MMAs run they wait for
+    // the previous kernel and turn its sums of squares into the per-column
+    // 1/rms of the folded RMSNorm (16-load batches keep the summation order).
+    griddep_wait();
+    if (ep.ss_in != nullptr) {
+      for (int i = threadIdx.x - 64; i < BN; i += 64) {
+        const int64_t n = n_base + i;
+        float ss = 0.f;
+        if (n < N) {
+          int mt = 0;
+          for (; mt + 8 <= ep.n_ss; mt += 8) {
+            float t8[8];
+#pragma unroll
+            for (int j = 0; j < 8; ++j) t8[j] = ep.ss_in[(int64_t)(mt + j) * ep.ss_ld + n];
+#pragma unroll
+            for (int j = 0; j < 8; ++j) ss += t8[j];
+          }
+          for (; mt < ep.n_ss; ++mt) ss += ep.ss_in[(int64_t)mt * ep.ss_ld + n];
+        }
+        rinv[i] = rsqrtf(ss * ep.norm_scale + ep.norm_eps);
+      }
+    }
+  }
   const bool ok = mbar_wait(smem_u32(done), 0);
   asm volatile("tcgen05.fence::after_thread_sync;" ::: "memory");
   griddep_wait();  // epilogue reads/writes buffers of earlier kernels
   griddep_launch_dependents();
   const bool good = ok && !*abort_flag && nkb > 0;
-  const int row = warp * 32 + lane;
-  const int m = m_tile * BM + row;
-  const EpiRowConst rc = epi_row_const<EPI>(ep, m);
-  const int64_t n_base = (int64_t)n_tile * BN;
-  float* rinv = reinterpret_cast<float*>(smem + C::EXTRA_OFF);  // [BN] folded RMSNorm scale per column
-  float* red = rinv + 256;                                        // [4][32] per-warp column sums
-  if (ep.ss_in != nullptr) {
-    for (int i = threadIdx.x; i < BN; i += 128) {
-      const int64_t n = n_base + i;
-      float ss = 0.f;
-      if (n < N)
-        for (int mt = 0; mt < ep.n_ss; ++mt) ss += ep.ss_in[(int64_t)mt * ep.ss_ld + n];
-      rinv[i] = rsqrtf(ss * ep.norm_scale + ep.norm_eps);
-    }
-  }
   __syncthreads();
   if constexpr (CS == 1) {
 #pragma unroll 1
