@@ -105,7 +105,10 @@ __global__ void __launch_bounds__(kThreads, 9) swa_attn_kernel(const float* __re
                                                             KT* ring_v, int H, int t, int W,
                                                             const float* __restrict__ rope_cs, KT* out,
                                                             int64_t ld_out, float scale_log2) {
-  griddep_enter();
+  // Dependents (the next GEMM) are released only once this block has issued
+  // all its ring loads: released at the start, their CTAs would take SMs
+  // (shared memory, registers) from the blocks of this HBM-bound kernel.
+  griddep_wait();
   constexpr int LPK = HD / 8, KPW = 32 / LPK, NKG = (kThreads / 32) * KPW, HALF = HD / 2;
   extern __shared__ float sm[];
   float* sq = sm;            // rotated, scaled query
@@ -154,6 +157,7 @@ __global__ void __launch_bounds__(kThreads, 9) swa_attn_kernel(const float* __re
 
   float o[8] = {0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f};
   accumulate_values<KT, HD>(vb, 0, n_ring, sc, o, kg, NKG, sub);
+  griddep_launch_dependents();
 #pragma unroll
   for (int i = 0; i < 8; ++i) red_o[kg * HD + sub * 8 + i] = o[i];
   __syncthreads();
@@ -182,7 +186,7 @@ __global__ void __launch_bounds__(kThreads) prefix_attn_kernel(const float* __re
                                                                const float* __restrict__ rope_cs, KT* out,
                                                                int64_t ld_out, float* ws, int nchunks,
                                                                float scale_log2) {
-  griddep_enter();
+  griddep_wait();  // dependents are released after the last K/V load, as in swa_attn_kernel
   constexpr int LPK = HD / 8, KPW = 32 / LPK, NKG = (kThreads / 32) * KPW, HALF = HD / 2;
   extern __shared__ float sm[];
   float* sq = sm;
@@ -215,6 +219,7 @@ __global__ void __launch_bounds__(kThreads) prefix_attn_kernel(const float* __re
   const float2 ml = softmax_inplace(sc, j1 - j0, red);
   float o[8] = {0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f};
   accumulate_values<KT, HD>(vc + base, j0, j1, sc, o, kg, NKG, sub);
+  griddep_launch_dependents();
 #pragma unroll
   for (int i = 0; i < 8; ++i) red_o[kg * HD + sub * 8 + i] = o[i];
   __syncthreads();

@@ -191,13 +191,6 @@ __device__ __forceinline__ void epi_swiglu_at(const EpiParams& p, int64_t orow, 
   else reinterpret_cast<float*>(p.out)[o] = h;
 }
 
-template <bool OBF>
-__device__ __forceinline__ void epi_swiglu_store(const EpiParams& p, int64_t orow, int i, float gate, float up) {
-  const float h = siluf_(gate) * up;
-  if constexpr (OBF) reinterpret_cast<bf16*>(p.out)[orow + i] = __float2bfloat16_rn(h);
-  else reinterpret_cast<float*>(p.out)[orow + i] = h;
-}
-
 __device__ __forceinline__ void epi_swiglu(const EpiParams& p, int64_t n, int i, float gate, float up) {
   epi_swiglu_at(p, p.out_map.off(n), i, gate, up);
 }

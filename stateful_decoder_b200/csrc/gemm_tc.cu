@@ -102,7 +102,7 @@ int max_active_clusters(int cs) {
   if (cache[cs] == 0) {
     cudaLaunchConfig_t cfg = {};
     cfg.gridDim = dim3(1, 1, cs);
-    cfg.blockDim = dim3(128, 1, 1);
+    cfg.blockDim = dim3(256, 1, 1);
     cfg.dynamicSmemBytes = gemm_detail::TcCfg<256>::SMEM;
     cudaLaunchAttribute attr[1];
     attr[0].id = cudaLaunchAttributeClusterDimension;

@@ -7,7 +7,9 @@
 // with few sequences still fills the 128-lane MMA.  Both operands are K-major
 // bf16 in global memory, loaded by TMA with 128-byte swizzling into a
 // multi-stage ring.  One thread issues the TMA copies, one thread issues the
-// MMAs, and all four warps drain the accumulator through the fused epilogue.
+// MMAs, and eight warps (two groups of four) drain the accumulator through
+// the fused epilogue; the four warps without a main-loop role prepare the
+// folded RMSNorm scales while the MMAs run.
 //
 // Split over K inside a thread-block cluster: the CS CTAs of one cluster own
 // the same output tile and consecutive K ranges, so every weight byte is read
@@ -42,7 +44,7 @@ struct TcCfg {
   static constexpr int PIPE_BYTES = STAGES * STAGE_BYTES;
   static constexpr int EXTRA_OFF = PIPE_BYTES + 256;  // after the barriers
   static constexpr int SMEM = PIPE_BYTES + 1024 /*align*/ + 256 /*barriers*/ + 1024 /*1/rms per column*/ +
-                              512 /*per-warp column sums*/;
+                              1024 /*per-warp column sums, two groups*/;
   static constexpr int TMEM_COLS = BN;  // power of two >= 32
 
 };
@@ -144,6 +146,12 @@ __device__ __forceinline__ void cluster_sync_all() {
 }
 
 
+// Barrier of one 128-thread epilogue group (named barrier 1 or 2; the block
+// barrier 0 is __syncthreads).
+__device__ __forceinline__ void group_sync(int g) {
+  asm volatile("bar.sync %0, 128;" ::"r"(1 + g) : "memory");
+}
+
 // Butterfly transpose-reduction over the 32 lanes of a warp: on entry zv[j]
 // is this lane's value for column j; on exit zv[0] of lane j is the sum over
 // all lanes of column j (31 shuffles, fixed order).
@@ -201,23 +209,45 @@ __device__ __forceinline__ void epi_columns(const EpiParams& ep, const EpiRowCon
 template <int CNT, bool OBF>
 __device__ __forceinline__ void swiglu_columns(const EpiParams& ep, int64_t n0, int64_t N, bool full, int m,
                                                int lane, int64_t my_o, const float* v) {
+  // Lanes 2k and 2k+1 hold the gate and up rows of hidden unit k.  For each
+  // pair of columns (j, j+1) they swap one value, so that the even lane
+  // finishes unit k of column j and the odd lane unit k of column j+1: every
+  // lane evaluates one silu per column pair, with no branch, and stores one
+  // output.
+  static_assert(CNT % 2 == 0, "column pairs");
+  const bool odd = (lane & 1) != 0;
+  float hv[CNT / 2];
 #pragma unroll
-  for (int j = 0; j < CNT; ++j) {
-    const int64_t orow = __shfl_sync(0xffffffffu, my_o, j);
-    const float other = __shfl_xor_sync(0xffffffffu, v[j], 1);
-    if ((lane & 1) == 0 && (full || n0 + j < N)) epi_swiglu_store<OBF>(ep, orow, m >> 1, v[j], other);
+  for (int j = 0; j < CNT; j += 2) {
+    const float send = odd ? v[j] : v[j + 1];  // up of column j / gate of column j+1
+    const float recv = __shfl_xor_sync(0xffffffffu, send, 1);
+    const float gate = odd ? recv : v[j];
+    const float up = odd ? v[j + 1] : recv;
+    hv[j / 2] = siluf_(gate) * up;
+  }
+#pragma unroll
+  for (int j = 0; j < CNT; j += 2) {
+    const int64_t orow_e = __shfl_sync(0xffffffffu, my_o, j);
+    const int64_t orow_o = __shfl_sync(0xffffffffu, my_o, j + 1);
+    const int jj = odd ? j + 1 : j;
+    const int64_t orow = odd ? orow_o : orow_e;
+    if (full || n0 + jj < N) {
+      if constexpr (OBF) reinterpret_cast<bf16*>(ep.out)[orow + (m >> 1)] = __float2bfloat16_rn(hv[j / 2]);
+      else reinterpret_cast<float*>(ep.out)[orow + (m >> 1)] = hv[j / 2];
+    }
   }
 }
 
 // Finishes accumulator columns [n0, n0 + CNT) of this thread's row m (row
 // `row` of weight tile m_tile): folded RMSNorm scale (consumers), the
 // epilogue, and for producers the tile's per-column sums of z^2.  Called by
-// all 128 threads together (it contains block barriers).  Row offsets, which
-// may need a division for grouped rows, are computed once per column by
-// lane j and broadcast.
+// the four warps of one epilogue group together (g: group, q: the warp's
+// quarter of the 128 accumulator rows; it contains group barriers).  Row
+// offsets, which may need a division for grouped rows, are computed once per
+// column by lane j and broadcast.
 template <int EPI, int CNT>
 __device__ __forceinline__ void finish_chunk(const EpiParams& ep, const EpiRowConst& rc, int64_t n0, int64_t N, int m,
-                                             int m_tile, int warp, int lane, float* v, const float* rinv,
+                                             int m_tile, int g, int q, int lane, float* v, const float* rinv,
                                              float* red) {
   if (ep.ss_in != nullptr) {
 #pragma unroll
@@ -241,11 +271,12 @@ __device__ __forceinline__ void finish_chunk(const EpiParams& ep, const EpiRowCo
 #pragma unroll
         for (int j = CNT; j < 32; ++j) v[j] = 0.f;
         warp_column_sums(v, lane);
-        red[warp * 32 + lane] = v[0];
-        __syncthreads();
-        if (warp == 0 && lane < CNT && n0 + lane < N)
-          ep.ss_out[(int64_t)m_tile * ep.ss_ld + n0 + lane] = red[lane] + red[32 + lane] + red[64 + lane] + red[96 + lane];
-        __syncthreads();
+        float* rg = red + g * 128;
+        rg[q * 32 + lane] = v[0];
+        group_sync(g);
+        if (q == 0 && lane < CNT && n0 + lane < N)
+          ep.ss_out[(int64_t)m_tile * ep.ss_ld + n0 + lane] = rg[lane] + rg[32 + lane] + rg[64 + lane] + rg[96 + lane];
+        group_sync(g);
       }
     } else {
       epi_columns<EPI, CNT, false, false>(ep, rc, n0, N, full, m, my_o, my_a, v);
@@ -256,7 +287,7 @@ __device__ __forceinline__ void finish_chunk(const EpiParams& ep, const EpiRowCo
 }
 
 template <int BN, int EPI, int CS>
-__global__ void __launch_bounds__(128, 1)
+__global__ void __launch_bounds__(256, 1)
     gemm_tc_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CUtensorMap tmB, int M, int N,
                    int K, int kb_per_split, float* split_ws, EpiParams ep) {
   using C = TcCfg<BN>;
@@ -352,20 +383,24 @@ __global__ void __launch_bounds__(128, 1)
   }
   __syncwarp();
 
-  // Epilogue: warp w owns accumulator lanes 32w..32w+31 (output features).
-  const int row = warp * 32 + lane;
+  // Epilogue: eight warps in two groups of four.  Warp w reads accumulator
+  // lanes 32(w%4)..+31 (the tensor-memory quarter its SM sub-partition may
+  // access) and its group g = w/4 takes every other column chunk, so two
+  // warps per scheduler overlap their epilogue work.
+  const int g = warp >> 2, q = warp & 3;
+  const int row = q * 32 + lane;
   const int m = m_tile * BM + row;
   const EpiRowConst rc = epi_row_const<EPI>(ep, m);  // weights only: no wait needed
   const int64_t n_base = (int64_t)n_tile * BN;
   float* rinv = reinterpret_cast<float*>(smem + C::EXTRA_OFF);  // [BN] folded RMSNorm scale per column
-  float* red = rinv + 256;                                        // [4][32] per-warp column sums
-  if (warp >= 2) {
-    // Warps 2 and 3 have no main-loop role: while the MMAs run they wait for
+  float* red = rinv + 256;                                        // [2][4][32] per-warp column sums
+  if (warp >= 4) {
+    // Warps 4..7 have no main-loop role: while the MMAs run they wait for
     // the previous kernel and turn its sums of squares into the per-column
-    // 1/rms of the folded RMSNorm (16-load batches keep the summation order).
+    // 1/rms of the folded RMSNorm (8-load batches keep the summation order).
     griddep_wait();
     if (ep.ss_in != nullptr) {
-      for (int i = threadIdx.x - 64; i < BN; i += 64) {
+      for (int i = threadIdx.x - 128; i < BN; i += 128) {
         const int64_t n = n_base + i;
         float ss = 0.f;
         if (n < N) {
@@ -391,35 +426,39 @@ __global__ void __launch_bounds__(128, 1)
   __syncthreads();
   if constexpr (CS == 1) {
 #pragma unroll 1
-    for (int c = 0; c < BN; c += 32) {
+    for (int c = 32 * g; c < BN; c += 64) {
       if (n_base + c >= N) break;
       float v[32];
       if (good) {
-        tmem_ld32(tmem_base + ((uint32_t)(warp * 32) << 16) + (uint32_t)c, v);
+        tmem_ld32(tmem_base + ((uint32_t)(q * 32) << 16) + (uint32_t)c, v);
       } else {
 #pragma unroll
         for (int j = 0; j < 32; ++j) v[j] = 0.f;
       }
-      finish_chunk<EPI, 32>(ep, rc, n_base + c, N, m, m_tile, warp, lane, v, rinv + c, red);
+      finish_chunk<EPI, 32>(ep, rc, n_base + c, N, m, m_tile, g, q, lane, v, rinv + c, red);
     }
   } else {
     // Cluster split-K through L2: this CTA's exchange area holds CS slots of
     // COLS x 128 floats, slot o for owner o (its own slot stays unused).
     constexpr int COLS = BN / CS;
-    constexpr int CNT = COLS < 32 ? COLS : 32;
+    // chunk width: two or more chunks per share where possible, so that both
+    // epilogue groups have work
+    constexpr int CNT = COLS >= 64 ? 32 : (COLS >= 8 ? COLS / 2 : COLS);
     constexpr int64_t SLICE = (int64_t)COLS * BM;  // floats of one share, column-major [COLS][128]
     const int rank = split;
     const int64_t col_cta = blockIdx.x + (int64_t)gridDim.x * blockIdx.y;  // same for every rank of the cluster
     const int64_t lin_stride = (int64_t)gridDim.x * gridDim.y;             // linear CTA id = col_cta + z * lin_stride
     float* mine = split_ws + (col_cta + rank * lin_stride) * CS * SLICE;
+    int e = 0;  // chunk counter: group g takes the chunks with e % 2 == g
 #pragma unroll 1
     for (int o = 0; o < CS; ++o) {
       if (o == rank) continue;
 #pragma unroll 1
-      for (int c = 0; c < COLS; c += CNT) {
+      for (int c = 0; c < COLS; c += CNT, ++e) {
+        if ((e & 1) != g) continue;
         float v[32];
         if (good && n_base + o * COLS + c < N) {
-          tmem_ld_cols<CNT>(tmem_base + ((uint32_t)(warp * 32) << 16) + (uint32_t)(o * COLS + c), v);
+          tmem_ld_cols<CNT>(tmem_base + ((uint32_t)(q * 32) << 16) + (uint32_t)(o * COLS + c), v);
         } else {
 #pragma unroll
           for (int j = 0; j < CNT; ++j) v[j] = 0.f;
@@ -430,12 +469,12 @@ __global__ void __launch_bounds__(128, 1)
     }
     cluster_sync_all();  // release/acquire at cluster scope: the shares are visible to their owners
 #pragma unroll 1
-    for (int cc = 0; cc < COLS; cc += CNT) {
+    for (int cc = CNT * g; cc < COLS; cc += 2 * CNT) {
       const int c0 = rank * COLS + cc;
       if (n_base + c0 >= N) break;
       float own[32], v[32];
       if (good) {
-        tmem_ld_cols<CNT>(tmem_base + ((uint32_t)(warp * 32) << 16) + (uint32_t)c0, own);
+        tmem_ld_cols<CNT>(tmem_base + ((uint32_t)(q * 32) << 16) + (uint32_t)c0, own);
       } else {
 #pragma unroll
         for (int j = 0; j < CNT; ++j) own[j] = 0.f;
@@ -452,7 +491,7 @@ __global__ void __launch_bounds__(128, 1)
       }
 #pragma unroll
       for (int j = CNT; j < 32; ++j) v[j] = 0.f;
-      finish_chunk<EPI, CNT>(ep, rc, n_base + c0, N, m, m_tile, warp, lane, v, rinv + c0, red);
+      finish_chunk<EPI, CNT>(ep, rc, n_base + c0, N, m, m_tile, g, q, lane, v, rinv + c0, red);
     }
   }
   asm volatile("tcgen05.fence::before_thread_sync;" ::: "memory");
@@ -475,7 +514,7 @@ cudaError_t launch_gemm(const CUtensorMap& ta, const CUtensorMap& tb, int M, int
   }
   cudaLaunchConfig_t cfg = {};
   cfg.gridDim = dim3(M / BM, (N + BN - 1) / BN, CS);
-  cfg.blockDim = dim3(128, 1, 1);
+  cfg.blockDim = dim3(256, 1, 1);
   cfg.dynamicSmemBytes = C::SMEM;
   cfg.stream = st;
   cudaLaunchAttribute attr[2];

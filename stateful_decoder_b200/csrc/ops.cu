@@ -145,11 +145,29 @@ __global__ void logp_gather_kernel(const float* __restrict__ logits, int V, cons
   __shared__ float red[32];
   const int b = blockIdx.x;
   const float* l = logits + (int64_t)b * V;
+  // 16-byte loads when every row starts 16-byte aligned (V % 4 == 0); the
+  // second pass finds the row in L1/L2
+  const bool vec = (V & 3) == 0;
+  const float4* l4 = reinterpret_cast<const float4*>(l);
   float mx = -INFINITY;
-  for (int i = threadIdx.x; i < V; i += blockDim.x) mx = fmaxf(mx, l[i]);
+  if (vec) {
+    for (int i = threadIdx.x; i < V / 4; i += blockDim.x) {
+      const float4 x = l4[i];
+      mx = fmaxf(mx, fmaxf(fmaxf(x.x, x.y), fmaxf(x.z, x.w)));
+    }
+  } else {
+    for (int i = threadIdx.x; i < V; i += blockDim.x) mx = fmaxf(mx, l[i]);
+  }
   mx = block_max(mx, red);
   float s = 0.f;
-  for (int i = threadIdx.x; i < V; i += blockDim.x) s += __expf(l[i] - mx);
+  if (vec) {
+    for (int i = threadIdx.x; i < V / 4; i += blockDim.x) {
+      const float4 x = l4[i];
+      s += __expf(x.x - mx) + __expf(x.y - mx) + __expf(x.z - mx) + __expf(x.w - mx);
+    }
+  } else {
+    for (int i = threadIdx.x; i < V; i += blockDim.x) s += __expf(l[i] - mx);
+  }
   s = block_sum(s, red);
   if (threadIdx.x == 0) {
     int32_t id = next[(int64_t)b * next_stride];
@@ -420,7 +438,7 @@ cudaError_t head_scatter(const XT* x, int64_t ld_x, int64_t col0, int64_t rows, 
 cudaError_t logp_gather(const float* logits, int B, int V, const int32_t* next, int64_t next_stride, float* logp,
                         int64_t ld_logp, cudaStream_t st) {
   {
-    const cudaError_t e_l = launch_pdl(logp_gather_kernel, dim3(B), dim3(1024), 0, st, logits, V, next, next_stride, logp, ld_logp);
+    const cudaError_t e_l = launch_pdl(logp_gather_kernel, dim3(B), dim3(256), 0, st, logits, V, next, next_stride, logp, ld_logp);
     if (e_l != cudaSuccess) return e_l;
   }
   return cudaGetLastError();
