@@ -63,7 +63,7 @@ extern "C" {
 
 typedef struct rlt_config {
   int32_t d_model;     /* residual width d */
-  int32_t n_heads;     /* heads; head size d/n_heads must be even */
+  int32_t n_heads;     /* heads; head size d/n_heads is 16, 32, 64 or 128 */
   int32_t n_layers;    /* L_E = L_D = L */
   int32_t window;      /* SWA window W >= 1, includes the current token */
   int32_t groups;      /* memory groups G: 1 (shared) or n_layers (per layer) */

@@ -5,6 +5,8 @@
 
 #include <atomic>
 
+#include <type_traits>
+
 #include "common.cuh"
 #include "internal.h"
 
@@ -84,6 +86,51 @@ __global__ void rmsnorm_kernel(const float* __restrict__ x, RowMap x_map, const 
   for (int i = threadIdx.x; i < d; i += blockDim.x) o[i] = from_f32<OT>(to_f32(gamma[i]) * xr[i] * inv);
 }
 
+// The same, one warp per row for d = 128 * NV: the row stays in registers
+// (NV float4 per lane), the sum of squares is a warp butterfly, and the
+// output is written with 16-byte stores.  Used for the token-parallel
+// encoder's many rows.
+template <typename WT, typename OT, int NV>
+__global__ void __launch_bounds__(256) rmsnorm_warp_kernel(const float* __restrict__ x, RowMap x_map, int64_t rows,
+                                                           const WT* __restrict__ gamma, float eps, OT* out,
+                                                           int64_t ld_out) {
+  griddep_enter();
+  constexpr int d = 128 * NV;
+  const int lane = threadIdx.x & 31;
+  const int64_t r = (int64_t)blockIdx.x * 8 + (threadIdx.x >> 5);
+  if (r >= rows) return;
+  const float4* xr = reinterpret_cast<const float4*>(x + x_map.off(r));
+  float4 v[NV];
+  float ss = 0.f;
+#pragma unroll
+  for (int k = 0; k < NV; ++k) {
+    v[k] = xr[k * 32 + lane];
+    ss = fmaf(v[k].x, v[k].x, ss);
+    ss = fmaf(v[k].y, v[k].y, ss);
+    ss = fmaf(v[k].z, v[k].z, ss);
+    ss = fmaf(v[k].w, v[k].w, ss);
+  }
+  ss = warp_sum(ss);
+  const float inv = rsqrtf(ss / (float)d + eps);
+  OT* o = out + r * ld_out;
+#pragma unroll
+  for (int k = 0; k < NV; ++k) {
+    const int i = 4 * (k * 32 + lane);  // this lane's float4 of chunk k
+    const float y0 = to_f32(gamma[i]) * v[k].x * inv, y1 = to_f32(gamma[i + 1]) * v[k].y * inv;
+    const float y2 = to_f32(gamma[i + 2]) * v[k].z * inv, y3 = to_f32(gamma[i + 3]) * v[k].w * inv;
+    if constexpr (std::is_same<OT, bf16>::value) {
+      __nv_bfloat162 p0 = __floats2bfloat162_rn(y0, y1);
+      __nv_bfloat162 p1 = __floats2bfloat162_rn(y2, y3);
+      uint2 w;
+      w.x = *reinterpret_cast<uint32_t*>(&p0);
+      w.y = *reinterpret_cast<uint32_t*>(&p1);
+      *reinterpret_cast<uint2*>(o + i) = w;
+    } else {
+      *reinterpret_cast<float4*>(o + i) = make_float4(y0, y1, y2, y3);
+    }
+  }
+}
+
 // Merge operand (eqs. 2.9-2.10): row b = [e_t ; RMSNorm_s(s_{t-1})] for the
 // report's merge, [e_t ; s_{t-1}] for the convex gate.
 template <typename WT, typename OT>
@@ -106,35 +153,44 @@ __global__ void merge_prep_kernel(const float* __restrict__ e, RowMap e_map, con
 }
 
 // ------------------------------------------------------------------ scatter
-// Row r of x (columns col0 + h*hd + i) goes to dst[b][h][pos][i] with
-// b = r / rows_per_seq, pos = pos0 + r % rows_per_seq, rotating the pair
-// (i, i+hd/2) by pos * base^(-2i/hd) when rope != 0.
+// Row r of x (columns col0 + h*hd + i) goes to dst[b][h][dst_row0 + i_seq][i]
+// with b = r / rows_per_seq, i_seq = r % rows_per_seq, rotating the pair
+// (i, i+hd/2) by (pos0 + i_seq) * base^(-2i/hd) when rope != 0.  A thread
+// moves eight consecutive pairs with 16-byte accesses (hd % 16 == 0).
 template <typename XT, typename KT>
 __global__ void head_scatter_kernel(const XT* __restrict__ x, int64_t ld_x, int64_t col0, int64_t rows,
                                     int rows_per_seq, int pos0, int dst_row0, int H, int hd, int rope,
                                     const float* __restrict__ rope_cs, KT* dst, int64_t ld_t) {
   griddep_enter();
-  const int half = hd / 2;
-  const int64_t n = rows * H * half;
+  const int half = hd / 2, oct = half / 8;
+  const int64_t n = rows * H * oct;
   for (int64_t idx = (int64_t)blockIdx.x * blockDim.x + threadIdx.x; idx < n; idx += (int64_t)gridDim.x * blockDim.x) {
-    const int i = (int)(idx % half);
-    const int h = (int)((idx / half) % H);
-    const int64_t r = idx / ((int64_t)half * H);
+    const int i = (int)(idx % oct) * 8;
+    const int h = (int)((idx / oct) % H);
+    const int64_t r = idx / ((int64_t)oct * H);
     const int64_t b = r / rows_per_seq;
     const int i_seq = (int)(r % rows_per_seq);
     const int pos = pos0 + i_seq;
     const XT* xr = x + r * ld_x + col0 + (int64_t)h * hd;
-    float a = to_f32(xr[i]), c = to_f32(xr[i + half]);
+    float a[8], c[8];
+    load8(xr + i, a);
+    load8(xr + i + half, c);
     if (rope) {
-      const float* cs = rope_cs + ((int64_t)pos * half + i) * 2;
-      const float ra = a * cs[0] - c * cs[1];
-      const float rc = a * cs[1] + c * cs[0];
-      a = ra;
-      c = rc;
+      const float4* cs = reinterpret_cast<const float4*>(rope_cs + ((int64_t)pos * half + i) * 2);
+#pragma unroll
+      for (int u = 0; u < 4; ++u) {
+        const float4 t = cs[u];  // (cos, sin) of pairs i+2u and i+2u+1
+        const float a0 = a[2 * u] * t.x - c[2 * u] * t.y, c0 = a[2 * u] * t.y + c[2 * u] * t.x;
+        const float a1 = a[2 * u + 1] * t.z - c[2 * u + 1] * t.w, c1 = a[2 * u + 1] * t.w + c[2 * u + 1] * t.z;
+        a[2 * u] = a0;
+        c[2 * u] = c0;
+        a[2 * u + 1] = a1;
+        c[2 * u + 1] = c1;
+      }
     }
     KT* o = dst + ((b * H + h) * ld_t + dst_row0 + i_seq) * hd;
-    o[i] = from_f32<KT>(a);
-    o[i + half] = from_f32<KT>(c);
+    store8(o + i, a);
+    store8(o + i + half, c);
   }
 }
 
@@ -405,6 +461,17 @@ cudaError_t embed(const int32_t* tok, int64_t n_rows, int tok_per_seq, int64_t t
 template <typename WT, typename OT>
 cudaError_t rmsnorm(const float* x, RowMap x_map, const WT* gamma, int64_t rows, int d, float eps, OT* out,
                     int64_t ld_out, cudaStream_t st) {
+  if (rows >= 4096 && ld_out % 4 == 0 && (d == 256 || d == 512 || d == 1024 || d == 2048)) {
+    const dim3 grid((unsigned)((rows + 7) / 8));
+    cudaError_t e_l;
+    switch (d) {
+      case 256: e_l = launch_pdl(rmsnorm_warp_kernel<WT, OT, 2>, grid, dim3(256), 0, st, x, x_map, rows, gamma, eps, out, ld_out); break;
+      case 512: e_l = launch_pdl(rmsnorm_warp_kernel<WT, OT, 4>, grid, dim3(256), 0, st, x, x_map, rows, gamma, eps, out, ld_out); break;
+      case 1024: e_l = launch_pdl(rmsnorm_warp_kernel<WT, OT, 8>, grid, dim3(256), 0, st, x, x_map, rows, gamma, eps, out, ld_out); break;
+      default: e_l = launch_pdl(rmsnorm_warp_kernel<WT, OT, 16>, grid, dim3(256), 0, st, x, x_map, rows, gamma, eps, out, ld_out); break;
+    }
+    return e_l != cudaSuccess ? e_l : cudaGetLastError();
+  }
   const int threads = d >= 1024 ? 256 : 128;
   {
     const cudaError_t e_l = launch_pdl(rmsnorm_kernel<WT, OT>, dim3((unsigned)rows), dim3(threads), 0, st, x, x_map, gamma, d, eps, out, ld_out);
@@ -426,7 +493,8 @@ cudaError_t merge_prep(const float* e, RowMap e_map, const float* s, const WT* g
 template <typename XT, typename KT>
 cudaError_t head_scatter(const XT* x, int64_t ld_x, int64_t col0, int64_t rows, int rows_per_seq, int pos0, int dst_row0, int H,
                          int hd, int rope, const float* rope_cs, KT* dst, int64_t ld_t, cudaStream_t st) {
-  const int64_t n = rows * H * (hd / 2);
+  if (hd % 16) return cudaErrorInvalidValue;
+  const int64_t n = rows * H * (hd / 16);
   {
     const cudaError_t e_l = launch_pdl(head_scatter_kernel<XT, KT>, dim3(grid_for(n, 256, 148 * 32)), dim3(256), 0, st, x, ld_x, col0, rows, rows_per_seq, pos0, dst_row0, H,
                                                                           hd, rope, rope_cs, dst, ld_t);
