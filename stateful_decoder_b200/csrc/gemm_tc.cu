@@ -140,7 +140,14 @@ DecodePlan decode_plan(int M, int K) {
   const int tiles = M / BM, kb = K / BK;
   for (int bn : {256, 128}) {
     const int ctas = tiles * (256 / bn);
-    if (ctas >= 80 && ctas <= kSmCount) return {bn, 1};
+    if (ctas >= 80 && ctas <= kSmCount) {
+      // A long K split in two over 256-wide tiles keeps the same CTA count
+      // with half the k-blocks each: the main loop (about 0.5 us per
+      // 256-wide k-block against 0.35 us at 128) then ends sooner.
+      if (bn == 128 && kb >= 32 && 2 * tiles <= kSmCount && tiles <= max_active_clusters(2))
+        return {256, 2};
+      return {bn, 1};
+    }
   }
   if (tiles >= 80) return {256, 1};
   DecodePlan best{256, 1};

@@ -123,6 +123,20 @@ def test_replay_parity_bf16(rlt, torch_mod, oracle_lib, kw):
     assert err <= TOL_BF16, err
 
 
+def test_replay_parity_bf16_many_rows(rlt, torch_mod, oracle_lib):
+    """A token-parallel encoder pass with more than 4096 rows (16 x 300) takes
+    the warp-per-row RMSNorm; the GPU replays all 16 sequences and the oracle
+    checks three of them, including the last."""
+    w, cfg = _bf16_small(batch=16, data_seed=1202)
+    tok = synth.tokens(w)
+    assert tok.shape[0] * tok.shape[1] >= 4096
+    got, _ = _gpu_replay(rlt, torch_mod, cfg, tok)
+    pick = [0, 7, 15]
+    want, _ = _oracle_replay(oracle_lib, cfg, tok[pick])
+    err = np.max(np.abs(got[pick] - want))
+    assert err <= TOL_BF16, err
+
+
 def test_generation_path_teacher_forced(rlt, torch_mod, oracle_lib):
     """Prompt prefill then incremental encoder steps (eq. 2.8) and decoder
     transitions, scored on teacher tokens, equal the oracle's replay
