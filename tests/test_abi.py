@@ -61,3 +61,20 @@ def test_op_arguments_validated_on_host():
     s = rlt.Sampling(temperature=0.8, top_k=257, seed=1)
     assert lib.rlt_op_sample(ctypes.c_void_p(16), 1, 10, ctypes.byref(s), 0, ctypes.c_void_p(16), None, None,
                              None) == rlt.RLT_E_INVAL
+
+
+def test_state_and_replay_arguments_validated_on_host():
+    """Snapshot, replay and step entry points reject missing handles and
+    buffers before touching a device."""
+    import stateful_decoder_b200 as rlt
+    lib = rlt._lib
+    used = ctypes.c_size_t(0)
+    assert lib.rlt_state_export(None, None, 0, ctypes.byref(used), None) == rlt.RLT_E_INVAL
+    assert lib.rlt_state_import(None, None, 0, None) == rlt.RLT_E_INVAL
+    assert lib.rlt_replay_logprobs(None, None, 1, 2, None, None) == rlt.RLT_E_INVAL
+    assert lib.rlt_replay_ratios(None, None, 1, 2, None, None, None, None, None, None) == rlt.RLT_E_INVAL
+    assert lib.rlt_decoder_step(None, None, None, None, None, None, None) == rlt.RLT_E_INVAL
+    assert lib.rlt_encode_prefix(None, None, None, 0, None) == rlt.RLT_E_INVAL
+    buf = ctypes.create_string_buffer(256)
+    assert lib.rlt_last_error(buf, 256) == rlt.RLT_E_INVAL
+    assert buf.value  # the last failure's text
