@@ -1,7 +1,8 @@
 """Profiling helpers for librlt, used to make the ncu summaries in profiles/.
 
-  python -m stateful_decoder_b200.profile_case step --workload replay --batch 64 --len 640 --t 601
-      Builds the workload's model (random weights), encodes `len` tokens of
+  python -m stateful_decoder_b200.profile_case step --workload replay --batch 64 --len 640 --t 601 [--layers 2]
+      Builds the workload's model (random weights; --layers keeps every
+      kernel shape but holds fewer layers' state), encodes `len` tokens of
       `batch` sequences, applies t-1 decoder transitions, then runs
       transition t between cudaProfilerStart/Stop, so that
       `ncu --profile-from-start off -k <kernel> -c 1` captures one launch of a
@@ -33,7 +34,10 @@ def step(args) -> None:
 
     import stateful_decoder_b200 as rlt
     import synth
-    w = synth.workload(args.workload, batch=args.batch, prompt=args.len)
+    over = dict(batch=args.batch, prompt=args.len)
+    if args.layers:
+        over["n_layers"] = args.layers  # same kernel shapes, fewer layers' state on the device
+    w = synth.workload(args.workload, **over)
     m = rlt.rlt_init_weights(synth.model_config(w), synth.WEIGHT_SEED)
     tok = torch.from_numpy(synth.tokens(w)).cuda()
     st = rlt.rlt_state_create(m, args.batch, args.len, 0)
@@ -86,6 +90,7 @@ def main() -> None:
     a.add_argument("--batch", type=int, default=64)
     a.add_argument("--len", type=int, default=640)
     a.add_argument("--t", type=int, default=601)
+    a.add_argument("--layers", type=int, default=0, help="override the workload's layer count (0: keep)")
     b = sub.add_parser("summarize")
     b.add_argument("csv")
     b.add_argument("S", type=int, nargs="?", default=1024)
