@@ -164,7 +164,11 @@ int32_t rlt_model_free(rlt_model* m);
  * at H_0 = (s_*, empty) with empty encoder caches (eq. 2.3).  Device memory:
  * encoder outputs [B][max_len][d] fp32, memory 2*G*B*max_len*d elements, SWA
  * ring 2*L*B*(W-1)*d elements, plus (flag RLT_STATE_ENCODER_CACHE) the encoder
- * cache 2*L*B*max_len*d elements, plus step workspace.
+ * cache 2*L*B*max_len*d elements, plus step workspace: the GEMM operands and
+ * bf16 folded-norm operand of one step, the split-K exchange area of the
+ * decode GEMMs (at most a few tens of MB), the attention chunk partials, the
+ * logits [B][V] fp32 and the pending-token record.  The token-parallel
+ * encoder adds its own workspace on first use (at most 4 GB).
  * Errors: RLT_E_INVAL, RLT_E_OOM. */
 int32_t rlt_state_create(rlt_model* m, int32_t batch, int32_t max_len, int32_t flags, rlt_state** out);
 int32_t rlt_state_free(rlt_state* s);
