@@ -18,7 +18,7 @@ _HERE = os.path.dirname(os.path.abspath(__file__))
 LIB_PATH = os.path.join(_HERE, "librlt.so")
 
 if not os.path.exists(LIB_PATH):
-    raise ImportError(f"{LIB_PATH} is missing: build it with `python -m stateful_decoder_b200.build`")
+    raise ImportError(f"{LIB_PATH} is missing: build it with `python stateful_decoder_b200/build.py`")
 
 _lib = ctypes.CDLL(LIB_PATH)
 
