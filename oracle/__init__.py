@@ -11,8 +11,11 @@ of each matrix-vector product).  This module is a ctypes binding to it: it
 marshals arguments and nothing else.  The module header of the C file lists
 which passage of "Recurrent Looped Transformer" each function follows.
 
+``bptt.py`` adds the full-BPTT gradient of the replay loss (plain PyTorch
+fp64 with autograd, no code shared with the C file or the library).
+
 Functions that no test pins to anything but themselves: none.  The pins are in
-``tests/test_oracle_pins.py``.
+``tests/test_oracle_pins.py`` and ``tests/test_oracle_bptt.py``.
 """
 from __future__ import annotations
 
