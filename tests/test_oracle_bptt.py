@@ -14,6 +14,12 @@ The gradient oracle is tied to things other than itself:
   gradients differ from the finite differences far beyond the tolerance,
   which also shows that the finite-difference pin would catch a dropped
   path.
+
+A hand-derived reverse-time schedule (``tests/manual_backward.py``: segment
+recompute from checkpoints, SWA adjoints owed across segment boundaries,
+deferred memory-key/value adjoints, one weight product per segment) gives
+the autograd gradient to 1e-11.  This holds for segment lengths from 1 to the
+whole sequence.
 """
 import numpy as np
 import pytest
@@ -191,3 +197,37 @@ def test_objective_weights_and_masked_targets(oracle_lib):
     later = set(tok[4:].tolist()) - set(tok[:4].tolist())
     for v in later:
         assert np.all(g3["emb"][v] == 0.0)
+
+
+# --------------------------------------------------------------------------
+# the hand-derived, segment-checkpointed reverse-time schedule
+# --------------------------------------------------------------------------
+
+@pytest.mark.parametrize("kw,seg", [(dict(), 1), (dict(), 3), (dict(window=1), 4),
+                                    (dict(tied=0, merge_kind=1, groups=2, window=3), 2),
+                                    (dict(window=32, alpha=0.5), 5), (dict(dtype=1, window=5), 31)],
+                         ids=["seg1", "seg3", "W1_seg4", "untied_convex_GL_seg2", "fullwin_seg5", "bf16_oneseg"])
+def test_manual_reverse_time_schedule_equals_autograd(oracle_lib, kw, seg):
+    """The reverse-time schedule (segment recompute from checkpoints,
+    deferred memory adjoints, per-segment weight products) gives the
+    autograd gradient of full BPTT; checkpointing changes no value (§4.3,
+    §5.4, App. C)."""
+    from oracle import bptt
+    from tests.manual_backward import ManualBPTT
+    w = synth.workload("tiny", **kw)
+    cfg = synth.model_config(w)
+    m = oracle_lib.Model(cfg, seed=42)
+    rng = np.random.default_rng(4)
+    for name, shp in bptt.tensor_shapes(cfg).items():
+        if cfg["dtype"] == 0 and (name.startswith("g_") or name == "b_gate"):
+            m.set(name, 1.0 * (name != "b_gate") + 0.2 * rng.standard_normal(shp))
+    tok = synth.tokens(w, batch=1)[0]
+    wts = rng.uniform(-1.0, 1.0, tok.size - 1)
+    loss, g_auto = bptt.loss_and_grads(m, tok, wts)
+    P = {k: v.detach().numpy() for k, v in bptt.parameters(m).items()}
+    mloss, mlogp, g_man = ManualBPTT(P, cfg).loss_and_grads(tok, wts, seg)
+    assert np.max(np.abs(mlogp - m.replay_logprobs(tok))) < 1e-11
+    assert abs(mloss - loss) < 1e-11
+    for k in g_auto:
+        scale = max(1.0, np.max(np.abs(g_auto[k])))
+        assert np.max(np.abs(g_man[k] - g_auto[k])) < 1e-11 * scale, k
