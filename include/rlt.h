@@ -36,6 +36,10 @@
  *    (report §5.4 and App. C: caches built under other weights are invalid).
  *  - All sequences of one state advance in lock step (report §4.1 batching of
  *    ready transitions): they share positions n_enc and n_dec.
+ *  - A model and its states are used from one host thread at a time: calls
+ *    on one model, or on its states, must not overlap across threads (the
+ *    model holds the state of rlt_replay_logprobs and the profiling record).
+ *    Different models may be used from different threads.
  */
 #ifndef RLT_H_
 #define RLT_H_
@@ -156,6 +160,9 @@ int32_t rlt_get_weights(const rlt_model* m, const char* name, void* host, size_t
  * wv_mem.g 17+2g, layer slot k of layer l 1024+32l+k in the order listed. */
 int32_t rlt_tensor_info(const rlt_model* m, const char* name, int64_t* rows, int64_t* cols, int32_t* stream_id);
 
+/* Frees the model's device memory, after a device synchronisation.  Every
+ * state made by rlt_state_create on it must be freed first; otherwise the
+ * call frees nothing and returns RLT_E_STATE. */
 int32_t rlt_model_free(rlt_model* m);
 
 /* ---------------------------------------------------------------- state */

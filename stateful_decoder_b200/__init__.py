@@ -170,10 +170,15 @@ class Model:
     def __del__(self):
         self.free()
 
-    def free(self):
+    def free(self) -> int:
+        """Frees the model; returns RLT_E_STATE (and keeps the model) while
+        states made on it are alive."""
         if getattr(self, "h", None):
-            _lib.rlt_model_free(self.h)
+            code = _lib.rlt_model_free(self.h)
+            if code != RLT_OK:
+                return code
             self.h = None
+        return RLT_OK
 
     @property
     def storage_dtype(self):

@@ -100,7 +100,8 @@ struct rlt_model {
   std::map<std::string, View> views;
   float* rope_cs = nullptr;
   int rope_len = 0;
-  rlt_state* replay = nullptr;
+  rlt_state* replay = nullptr;  // model-owned state of rlt_replay_logprobs
+  int64_t live_states = 0;      // states made by rlt_state_create and not yet freed
   ProfileRec prof;
 };
 
@@ -824,6 +825,8 @@ int32_t rlt_state_free(rlt_state* s);
 
 int32_t rlt_model_free(rlt_model* m) {
   if (!m) return ok();
+  if (m->live_states > 0)
+    return fail(RLT_E_STATE, std::to_string(m->live_states) + " state(s) of this model are still alive; free them first");
   cudaSetDevice(m->device);
   cudaDeviceSynchronize();
   if (m->replay) rlt_state_free(m->replay);
@@ -850,12 +853,14 @@ int32_t rlt_state_create(rlt_model* m, int32_t batch, int32_t max_len, int32_t f
     delete S;
     return r;
   }
+  m->live_states += 1;
   *out = S;
   return ok();
 }
 
 int32_t rlt_state_free(rlt_state* s) {
   if (!s) return ok();
+  if (s != s->m->replay) s->m->live_states -= 1;
   cudaSetDevice(s->m->device);
   cudaDeviceSynchronize();
   free_all(s->allocs);
@@ -1119,7 +1124,7 @@ int32_t rlt_prefill(rlt_model* m, rlt_state* s, const int32_t* tok_dev, int32_t 
     RLT_TRY(RLT_DISPATCH(m, transition_impl, m, s, st));
     if (logp_dev && t < T)
       RLT_TRY(RLT_DISPATCH(m, readout_impl, m, s, tok_dev + t, (int64_t)T, logp_dev + (t - 1), (int64_t)(T - 1),
-                           (const rlt_sampling*)nullptr, (const rlt_readout_out*)false, st));
+                           (const rlt_sampling*)nullptr, (const rlt_readout_out*)nullptr, st));
   }
   return ok();
 }

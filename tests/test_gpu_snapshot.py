@@ -263,3 +263,21 @@ def test_snapshot_errors(rlt, torch_mod):
         == rlt.RLT_E_STALE
     torch.cuda.synchronize()
     rlt.rlt_check_device()
+
+
+def test_model_free_refuses_live_states(rlt, torch_mod):
+    """A model is not freed under a live state (its handle stays valid); once
+    the state is gone it frees normally.  The model-owned replay state does
+    not count."""
+    w, cfg = _tiny()
+    m = rlt.rlt_init_weights(cfg, synth.WEIGHT_SEED)
+    tok = torch_mod.from_numpy(synth.tokens(w)[:, :6].copy()).cuda()
+    lp = torch_mod.zeros((tok.shape[0], 5), dtype=torch_mod.float32, device="cuda")
+    rlt.rlt_replay_logprobs(m, tok, lp)
+    st = rlt.rlt_state_create(m, 2, 8)
+    assert m.free() == rlt.RLT_E_STATE
+    assert rlt.rlt_last_error()[0] == rlt.RLT_E_STATE
+    rlt.rlt_prefill(m, st, tok)  # the model still works
+    st.free()
+    assert m.free() == rlt.RLT_OK
+    assert m.free() == rlt.RLT_OK  # idempotent
