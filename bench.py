@@ -297,17 +297,27 @@ def run_gpu(args, w: dict, kind: str, peaks: dict, rank: int, world: int) -> dic
     }
 
 
-def read_traffic_ratio() -> float | None:
+def read_traffic_ratio() -> tuple[float | None, str]:
     """DRAM bytes per algorithmic byte of the prefix-attention kernel from the
-    committed ncu summary (None until one exists for the current kernel)."""
+    committed ncu summary, with a note.  The summary records the SHA-1 of the
+    kernel's source file at capture time; if the source has changed since,
+    the counters no longer describe the kernel and the ratio is None."""
+    import hashlib
     p = os.path.join(ROOT, "profiles", "prefix_attn_replay.md")
     if not os.path.exists(p):
-        return None
+        return None, "no ncu summary"
+    ratio, sha = None, None
     for line in open(p):
         if line.startswith("traffic_per_algorithmic_byte:"):
             v = line.split(":", 1)[1].strip()
-            return None if v in ("", "null") else float(v)
-    return None
+            ratio = None if v in ("", "null") else float(v)
+        elif line.startswith("kernel_source_sha1:"):
+            sha = line.split(":", 1)[1].strip()
+    src = os.path.join(ROOT, "stateful_decoder_b200", "csrc", "attn_decode.cu")
+    now = hashlib.sha1(open(src, "rb").read()).hexdigest()
+    if sha != now:
+        return None, "kernel source changed since the ncu capture in profiles/prefix_attn_replay.md"
+    return ratio, "from profiles/prefix_attn_replay.md, scaled to the mean timed launch"
 
 
 def main():
@@ -378,7 +388,7 @@ def main():
         dist.destroy_process_group()
     if rank != 0:
         return
-    ratio = read_traffic_ratio()
+    ratio, traffic_note = read_traffic_ratio()
     a = r["attn"]
     traffic = ratio * (a["bytes"] / a["n"]) if (ratio is not None and a["n"]) else None
     line = {
@@ -389,6 +399,7 @@ def main():
         "roofline": {"bound": "hbm", "kernel": "prefix_attn (cross-attention over M_<=t)",
                      "achieved": a["gbs"], "peak": peaks["hbm_gbs"], "unit": "GB/s",
                      "frac": (a["gbs"] / peaks["hbm_gbs"]) if a["gbs"] else None, "traffic": traffic,
+                     "traffic_note": traffic_note,
                      "peak_source": peaks["source"] + " (copy bandwidth)",
                      "timed_launches": a["n"], "sampling": "launches at every 4th position, CUDA events",
                      "share_of_step": a["ms_all"] / (r["ms_per_step"] * args.steps) if a["ms_all"] else None},

@@ -3,7 +3,8 @@ workload: the mean bytes one decoder transition must move are the weights
 (about 3.03 GB at bf16) plus the ring, the cross-attention memory reads and
 the ring insert (about 37.1 GB averaged over t = 1..1023), which at the
 measured copy bandwidth is about 6.1 ms per transition.  Also checks that the
-bound scales with the work it counts."""
+bound scales with the work it counts, and that the reported DRAM traffic is
+taken from an ncu summary only while the kernel source is the one captured."""
 import bench
 import synth
 
@@ -35,3 +36,23 @@ def test_bound_grows_with_work():
     assert bench.step_roofline(dict(base, prompt=512), "replay", PEAKS)["bound_ms"] > 2 * b0
     g = synth.workload("small")
     assert bench.step_roofline(g, "generate", PEAKS)["decoder_transitions"] == g["prompt"] + g["gen"] - 1
+
+
+def test_traffic_ratio_only_for_the_captured_source(tmp_path, monkeypatch):
+    """roofline.traffic comes from the committed ncu summary only while the
+    kernel source still has the SHA-1 recorded at capture time."""
+    import hashlib
+
+    import bench
+    (tmp_path / "profiles").mkdir()
+    src = tmp_path / "stateful_decoder_b200" / "csrc"
+    src.mkdir(parents=True)
+    (src / "attn_decode.cu").write_bytes(b"// kernel v1\n")
+    sha = hashlib.sha1(b"// kernel v1\n").hexdigest()
+    (tmp_path / "profiles" / "prefix_attn_replay.md").write_text(
+        f"x\ntraffic_per_algorithmic_byte: 1.015\nkernel_source_sha1: {sha}\n")
+    monkeypatch.setattr(bench, "ROOT", str(tmp_path))
+    assert bench.read_traffic_ratio()[0] == 1.015
+    (src / "attn_decode.cu").write_bytes(b"// kernel v2\n")
+    ratio, note = bench.read_traffic_ratio()
+    assert ratio is None and "changed" in note
