@@ -283,6 +283,41 @@ int32_t rlt_replay_ratios(rlt_model* m, const int32_t* tok_dev, int32_t B, int32
                           const uint8_t* action_mask_dev, float* logp_dev, float* ratio_dev,
                           float* seq_logratio_dev, void* stream);
 
+/* ---------------------------------------------------------------- gradients */
+
+/* Full back-propagation through time of the replay (report §5.1-§5.4 and
+ * App. C): for tok_dev [B][S] int32 and target weights w_dev [B][S-1] fp32,
+ *   L_w = - sum_{b,t} w[b][t] log p(x_{b,t+1} | x_{b,1..t}),
+ * and its gradient with respect to every stored tensor.  The gradient runs
+ * through the causal encoder, the memory projections, the merge, every
+ * decoder SWA key/value and the recurrent output over all positions.
+ * Nothing is detached: evicting an entry from the SWA window is not a
+ * stop-gradient.  The objectives of report §5 are choices of w: eq. 5.1
+ * (1/(S-1) on every target), eq. 5.2 (the assistant mask over its count),
+ * eq. 5.4 (R - b on the response targets, 0 on the prompt).
+ * The decoder is reversed one step at a time in segments of `segment`
+ * steps.  Each segment is recomputed from the recurrent output at its
+ * start, with the same parameters (activation checkpointing, §4.3).  The
+ * arithmetic is fp32 on fp32 copies of the weights.  Gradients are
+ * accumulated into fp32 buffers the model owns, one per stored tensor, read
+ * with rlt_grad_read and cleared with rlt_grad_zero.  logp_dev [B][S-1]
+ * (may be NULL) receives the log-probs the pass computed.  Device memory
+ * is allocated inside the call and freed before it returns: about
+ * 4 * B * S * (L * (13d + 3F) + 4 G d + 14d) bytes, plus the fp32 weight
+ * copies.  The stream is synchronised.  Head size at most 128.
+ * Errors: RLT_E_INVAL, RLT_E_OOM, RLT_E_CUDA. */
+int32_t rlt_replay_backward(rlt_model* m, const int32_t* tok_dev, int32_t B, int32_t S, const float* w_dev,
+                            int32_t segment, float* logp_dev, void* stream);
+
+/* Copies the accumulated fp32 gradient of a stored tensor (rlt_tensor_info
+ * names and shapes, [rows][cols] row-major) to host.  Before any
+ * rlt_replay_backward the gradient is zero.  Errors: RLT_E_INVAL (name or
+ * size). */
+int32_t rlt_grad_read(const rlt_model* m, const char* name, float* host, size_t bytes);
+
+/* Sets every accumulated gradient of the model to zero. */
+int32_t rlt_grad_zero(rlt_model* m, void* stream);
+
 /* ---------------------------------------------------------------- ops */
 
 /* Kernel-level check of the step's contraction: y_dev [N][M] fp32 =

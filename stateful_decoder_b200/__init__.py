@@ -44,7 +44,8 @@ EXPORTED = (
     "rlt_encode_prefix", "rlt_readout", "rlt_decoder_step", "rlt_prefill", "rlt_replay_logprobs",
     "rlt_last_error", "rlt_check_device", "rlt_profile_enable", "rlt_profile_read", "rlt_op_linear",
     "rlt_op_sample", "rlt_kernel_launches", "rlt_op_prefix_attention", "rlt_op_prefix_attention_noalloc",
-    "rlt_state_export", "rlt_state_import", "rlt_replay_ratios",
+    "rlt_state_export", "rlt_state_import", "rlt_replay_ratios", "rlt_replay_backward", "rlt_grad_read",
+    "rlt_grad_zero",
 )
 
 
@@ -102,6 +103,9 @@ _sig = {
     "rlt_prefill": [_vp, _vp, _vp, _i32, _vp, _vp],
     "rlt_replay_logprobs": [_vp, _vp, _i32, _i32, _vp, _vp],
     "rlt_replay_ratios": [_vp, _vp, _i32, _i32, _vp, _vp, _vp, _vp, _vp, _vp],
+    "rlt_replay_backward": [_vp, _vp, _i32, _i32, _vp, _i32, _vp, _vp],
+    "rlt_grad_read": [_vp, ctypes.c_char_p, _vp, ctypes.c_size_t],
+    "rlt_grad_zero": [_vp, _vp],
     "rlt_op_linear": [_vp, _vp, _vp, _i32, _i32, _i32, _i32, _i32, _vp],
     "rlt_op_prefix_attention": [_vp, _vp, _vp, ctypes.c_int64, _i32, _i32, _i32, _i32, _i32, _vp, _i32, _vp, _vp],
     "rlt_op_prefix_attention_noalloc": [_vp, _vp, _vp, ctypes.c_int64, _i32, _i32, _i32, _i32, _i32, _vp, _i32, _vp,
@@ -197,6 +201,13 @@ class Model:
         r, c, _ = self.tensor_info(name)
         out = np.zeros((r, c), dtype=self.storage_dtype)
         _check(_lib.rlt_get_weights(self.h, name.encode(), out.ctypes.data, out.nbytes))
+        return out
+
+    def grad(self, name: str) -> np.ndarray:
+        """Accumulated fp32 gradient of a stored tensor (rlt_replay_backward)."""
+        r, c, _ = self.tensor_info(name)
+        out = np.zeros((r, c), dtype=np.float32)
+        _check(_lib.rlt_grad_read(self.h, name.encode(), out.ctypes.data, out.nbytes))
         return out
 
 
@@ -324,6 +335,19 @@ def rlt_replay_ratios(model: Model, tokens, logmu, action_mask, logp, ratio=None
                                   _dev(action_mask, "torch.uint8"), _dev(logp, "torch.float32"),
                                   _dev(ratio, "torch.float32"), _dev(seq_logratio, "torch.float32"),
                                   _stream(stream)))
+
+
+def rlt_replay_backward(model: Model, tokens, weights, segment: int = 32, logp=None, stream=None) -> None:
+    """Full-BPTT gradient of -sum w[b][t] log p(x_{t+1} | x_1..t): tokens int32
+    [B, S], weights float32 [B, S-1], optional logp float32 [B, S-1] (CUDA
+    tensors).  Gradients accumulate in the model (Model.grad, rlt_grad_zero)."""
+    B, S = tokens.shape
+    _check(_lib.rlt_replay_backward(model.h, _dev(tokens, "torch.int32"), B, S, _dev(weights, "torch.float32"),
+                                    segment, _dev(logp, "torch.float32"), _stream(stream)))
+
+
+def rlt_grad_zero(model: Model, stream=None) -> None:
+    _check(_lib.rlt_grad_zero(model.h, _stream(stream)))
 
 
 def rlt_op_linear(w, x, y, use_tensor_cores: bool = True, stream=None) -> None:

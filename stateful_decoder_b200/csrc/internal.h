@@ -4,6 +4,7 @@
 #include <cuda_runtime.h>
 #include <stdint.h>
 
+#include "bptt_core.h"
 #include "common.cuh"
 #include "epilogue.cuh"
 
@@ -138,5 +139,17 @@ cudaError_t copy_f32(float* dst, const float* src, int64_t n, cudaStream_t st);
 // dst[b][:] = src[:] (fp32) for b < B
 template <typename WT>
 cudaError_t broadcast_row(const WT* src, int d, float* dst, int B, cudaStream_t st);
+
+// ---------------------------------------------------------------- gradients
+namespace bptt {
+// dst [rows][cols] fp32 = src (dtype 0 fp32, 1 bf16; rows `pitch` elements apart)
+cudaError_t widen_to_f32(const void* src, int dtype, int64_t rows, int64_t cols, int64_t pitch, float* dst,
+                         cudaStream_t st);
+// Full-BPTT gradient of the weighted replay loss (bptt_core.h) on fp32
+// weights W32 into G32 (per catalogue index; null where a tensor is absent).
+// Drains the stream before it returns.
+cudaError_t replay_backward_f32(const Dims& D, const float* const* W32, float* const* G32, const int32_t* tok,
+                                const float* wts, int seg, float* logp, cudaStream_t st);
+}  // namespace bptt
 
 }  // namespace rlt

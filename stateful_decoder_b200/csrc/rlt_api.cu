@@ -102,6 +102,7 @@ struct rlt_model {
   int rope_len = 0;
   rlt_state* replay = nullptr;  // model-owned state of rlt_replay_logprobs
   int64_t live_states = 0;      // states made by rlt_state_create and not yet freed
+  std::vector<float*> grad;     // fp32 gradient per catalogue index of bptt_core.h (rlt_replay_backward)
   ProfileRec prof;
 };
 
@@ -1229,6 +1230,117 @@ int32_t rlt_op_sample(const float* logits_dev, int32_t B, int32_t V, const rlt_s
     return fail(RLT_E_INVAL, "sampler needs temperature > 0 and 1 <= top_k <= 256");
   RLT_CUDA(sample_topk(logits_dev, B, V, samp->temperature, samp->top_k, samp->seed, t, token_dev, logp_dev, logmu_dev,
                        (cudaStream_t)stream));
+  return ok();
+}
+
+// ------------------------------------------------------------------ gradients
+}  // extern "C"
+
+namespace {
+
+bptt::Dims bptt_dims(const rlt_model* m, int B, int S) {
+  const rlt_config& c = m->cfg;
+  bptt::Dims D{};
+  D.B = B; D.S = S; D.d = c.d_model; D.H = c.n_heads; D.L = c.n_layers; D.W = c.window; D.G = c.groups;
+  D.F = c.ffn; D.V = c.vocab; D.tied = c.tied; D.merge_kind = c.merge_kind;
+  D.alpha = c.alpha; D.eps = c.rms_eps; D.rope_base = c.rope_base;
+  return D;
+}
+
+// The model's view of catalogue index i (null when the model does not store it).
+const View* bptt_view(const rlt_model* m, const bptt::Dims& D, int i) {
+  if (!bptt::tensor_exists(D, i)) return nullptr;
+  auto it = m->views.find(bptt::tensor_name(D, i));
+  return it == m->views.end() ? nullptr : &it->second;
+}
+
+int32_t ensure_grads(rlt_model* m, const bptt::Dims& D) {
+  if (!m->grad.empty()) return RLT_OK;
+  const int n = bptt::n_tensors(D);
+  std::vector<float*> g(n, nullptr);
+  for (int i = 0; i < n; ++i) {
+    const View* v = bptt_view(m, D, i);
+    if (!v) continue;
+    void* p = nullptr;
+    RLT_TRY(dev_alloc(m->allocs, &p, (size_t)(v->rows * v->cols) * 4));
+    RLT_CUDA(cudaMemset(p, 0, (size_t)(v->rows * v->cols) * 4));
+    g[i] = static_cast<float*>(p);
+  }
+  m->grad = g;
+  return RLT_OK;
+}
+
+}  // namespace
+
+extern "C" {
+
+int32_t rlt_replay_backward(rlt_model* m, const int32_t* tok_dev, int32_t B, int32_t S, const float* w_dev,
+                            int32_t segment, float* logp_dev, void* stream) {
+  if (!m || !tok_dev || !w_dev) return fail(RLT_E_INVAL, "null argument");
+  if (B <= 0 || S < 2) return fail(RLT_E_INVAL, "need B > 0 and S >= 2");
+  if (segment < 1) return fail(RLT_E_INVAL, "segment must be at least 1");
+  if (m->hd > bptt::kMaxHead) return fail(RLT_E_INVAL, "the backward pass takes head sizes up to 128");
+  RLT_CUDA(cudaSetDevice(m->device));
+  cudaStream_t st = (cudaStream_t)stream;
+  const bptt::Dims D = bptt_dims(m, B, S);
+  RLT_TRY(ensure_grads(m, D));
+  // fp32 copies of the current weights, freed before returning
+  const int n = bptt::n_tensors(D);
+  std::vector<float*> w32(n, nullptr);
+  std::vector<void*> tmp;
+  int32_t r = RLT_OK;
+  for (int i = 0; i < n && r == RLT_OK; ++i) {
+    const View* v = bptt_view(m, D, i);
+    if (!v) continue;
+    void* p = nullptr;
+    r = dev_alloc(tmp, &p, (size_t)(v->rows * v->cols) * 4);
+    if (r != RLT_OK) break;
+    w32[i] = static_cast<float*>(p);
+    const cudaError_t e = bptt::widen_to_f32(v->base, m->cfg.dtype, v->rows, v->cols, v->pitch, w32[i], st);
+    if (e != cudaSuccess) r = fail(RLT_E_CUDA, std::string("widen: ") + cudaGetErrorString(e));
+  }
+  if (r == RLT_OK) {
+    const cudaError_t e = bptt::replay_backward_f32(D, w32.data(), m->grad.data(), tok_dev, w_dev, segment, logp_dev, st);
+    if (e == cudaErrorMemoryAllocation) r = fail(RLT_E_OOM, "backward buffers: out of device memory");
+    else if (e != cudaSuccess) r = fail(RLT_E_CUDA, std::string("backward: ") + cudaGetErrorString(e));
+  }
+  cudaStreamSynchronize(st);
+  free_all(tmp);
+  return r;
+}
+
+int32_t rlt_grad_read(const rlt_model* m, const char* name, float* host, size_t bytes) {
+  if (!m || !name || !host) return fail(RLT_E_INVAL, "null argument");
+  auto it = m->views.find(name);
+  if (it == m->views.end()) return fail(RLT_E_INVAL, std::string("unknown tensor ") + name);
+  const View& v = it->second;
+  const size_t need = (size_t)(v.rows * v.cols) * 4;
+  if (bytes != need) return fail(RLT_E_INVAL, "size mismatch: need " + std::to_string(need));
+  if (m->grad.empty()) {
+    std::memset(host, 0, bytes);
+    return ok();
+  }
+  const bptt::Dims D = bptt_dims(m, 1, 2);
+  for (int i = 0; i < bptt::n_tensors(D); ++i) {
+    if (!bptt::tensor_exists(D, i) || bptt::tensor_name(D, i) != name) continue;
+    RLT_CUDA(cudaSetDevice(m->device));
+    RLT_CUDA(cudaDeviceSynchronize());
+    RLT_CUDA(cudaMemcpy(host, m->grad[i], bytes, cudaMemcpyDeviceToHost));
+    return ok();
+  }
+  return fail(RLT_E_INVAL, std::string("no gradient for ") + name);
+}
+
+int32_t rlt_grad_zero(rlt_model* m, void* stream) {
+  if (!m) return fail(RLT_E_INVAL, "null model");
+  if (m->grad.empty()) return ok();
+  RLT_CUDA(cudaSetDevice(m->device));
+  const bptt::Dims D = bptt_dims(m, 1, 2);
+  for (int i = 0; i < bptt::n_tensors(D); ++i) {
+    const View* v = bptt_view(m, D, i);
+    if (v && m->grad[i])
+      RLT_CUDA(cudaMemsetAsync(m->grad[i], 0, (size_t)(v->rows * v->cols) * 4, (cudaStream_t)stream));
+  }
   return ok();
 }
 

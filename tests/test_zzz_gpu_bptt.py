@@ -1,0 +1,78 @@
+"""Full-BPTT backward on the GPU through the C ABI (rlt_replay_backward),
+against the gradient oracle (``oracle.bptt``: autograd over the fp64
+forward, itself pinned by finite differences).
+
+The engine differentiates fp32 copies of the stored weights, so the bar is
+fp32 accumulation error.  Per tensor, the largest deviation must stay within
+1e-4 of the tensor's largest gradient entry, plus 1e-6.  The host build of
+the same engine meets the oracle to 1e-10 in fp64 (``test_bptt_host.py``).
+"""
+import numpy as np
+import pytest
+
+import synth
+
+pytestmark = pytest.mark.gpu
+
+
+@pytest.fixture(scope="module")
+def rlt():
+    import torch
+    torch.cuda.init()
+    import stateful_decoder_b200 as m
+    return m
+
+
+VARIANTS = [
+    (dict(d=32, n_heads=4, ffn=48, vocab=40, prompt=12), 4),
+    (dict(d=32, n_heads=4, ffn=48, vocab=40, prompt=12, tied=0, merge_kind=1, groups=2, window=3), 3),
+    (dict(d=128, n_heads=2, ffn=192, vocab=256, prompt=10, dtype=1, window=3), 9),
+]
+
+
+@pytest.mark.parametrize("kw,seg", VARIANTS, ids=["f32_tied", "f32_untied_convex_GL", "bf16_hd64"])
+def test_backward_matches_gradient_oracle(rlt, oracle_lib, kw, seg):
+    import torch
+
+    from oracle import bptt
+    w = synth.workload("tiny", **kw)
+    cfg = synth.model_config(w)
+    m = rlt.rlt_init_weights(cfg, synth.WEIGHT_SEED)
+    om = oracle_lib.Model(cfg, seed=synth.WEIGHT_SEED)
+    tok = synth.tokens(w, batch=2)
+    B, S = tok.shape
+    wts = np.random.default_rng(7).uniform(-1.0, 1.0, (B, S - 1)).astype(np.float32)
+    lp = torch.zeros((B, S - 1), dtype=torch.float32, device="cuda")
+    rlt.rlt_replay_backward(m, torch.from_numpy(tok).cuda(), torch.from_numpy(wts).cuda(), segment=seg, logp=lp)
+    want = None
+    for b in range(B):
+        assert np.max(np.abs(lp[b].cpu().numpy() - om.replay_logprobs(tok[b]))) < 1e-4
+        _, g = bptt.loss_and_grads(om, tok[b], wts[b].astype(np.float64))
+        want = g if want is None else {k: want[k] + g[k] for k in want}
+    for name, ref in want.items():
+        got = m.grad(name)
+        scale = float(np.max(np.abs(ref)))
+        assert np.max(np.abs(got - ref)) <= 1e-4 * scale + 1e-6, name
+    rlt.rlt_check_device()
+
+
+def test_backward_accumulates_and_zeroes(rlt):
+    import torch
+    w = synth.workload("tiny", d=32, n_heads=4, ffn=48, vocab=40, prompt=8)
+    cfg = synth.model_config(w)
+    m = rlt.rlt_init_weights(cfg, synth.WEIGHT_SEED)
+    tok = torch.from_numpy(synth.tokens(w, batch=2)).cuda()
+    wts = torch.full((2, 7), 1.0 / 7, dtype=torch.float32, device="cuda")
+    assert not np.any(m.grad("w_out"))
+    rlt.rlt_replay_backward(m, tok, wts, segment=2)
+    one = {n: m.grad(n) for n in ("emb", "s_star", "w_gate", "wq.0", "g_dffn.1")}
+    rlt.rlt_replay_backward(m, tok, wts, segment=7)  # a different segment length gives the same gradient
+    for n, g in one.items():
+        assert np.allclose(m.grad(n), 2 * g, rtol=1e-5, atol=1e-7), n
+    rlt.rlt_grad_zero(m)
+    torch.cuda.synchronize()
+    assert not np.any(m.grad("emb"))
+    with pytest.raises(rlt.RltError) as e:
+        rlt.rlt_replay_backward(m, tok, wts, segment=0)
+    assert e.value.code == rlt.RLT_E_INVAL
+    rlt.rlt_check_device()
