@@ -24,8 +24,8 @@ def rlt():
 
 
 VARIANTS = [
-    (dict(d=32, n_heads=4, ffn=48, vocab=40, prompt=12), 4),
-    (dict(d=32, n_heads=4, ffn=48, vocab=40, prompt=12, tied=0, merge_kind=1, groups=2, window=3), 3),
+    (dict(d=32, n_heads=2, ffn=48, vocab=40, prompt=12), 4),
+    (dict(d=32, n_heads=2, ffn=48, vocab=40, prompt=12, tied=0, merge_kind=1, groups=2, window=3), 3),
     (dict(d=128, n_heads=2, ffn=192, vocab=256, prompt=10, dtype=1, window=3), 9),
 ]
 
@@ -58,7 +58,7 @@ def test_backward_matches_gradient_oracle(rlt, oracle_lib, kw, seg):
 
 def test_backward_accumulates_and_zeroes(rlt):
     import torch
-    w = synth.workload("tiny", d=32, n_heads=4, ffn=48, vocab=40, prompt=8)
+    w = synth.workload("tiny", d=32, n_heads=2, ffn=48, vocab=40, prompt=8)
     cfg = synth.model_config(w)
     m = rlt.rlt_init_weights(cfg, synth.WEIGHT_SEED)
     tok = torch.from_numpy(synth.tokens(w, batch=2)).cuda()
