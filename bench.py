@@ -39,7 +39,11 @@ BENCH_WORKLOADS = {
     "small": ("small", {}, "generate"),
     "refdepth-b64": ("refdepth", {"batch": 64}, "generate"),
     "refdepth-b128-t3072": ("refdepth", {"gen": 1024}, "generate"),
+    # full-BPTT forward + backward (rlt_replay_backward) of the small model
+    "bptt-small": ("small", {"prompt": 256, "gen": 0}, "backward"),
 }
+BPTT_METRIC = "RLT full-BPTT tokens/s (replay forward + backward through the whole history) on 1 B200"
+BPTT_SEGMENT = 32
 
 METRIC = "RLT decoder tokens/s (B seqs, 48+48 tied) on 1 B200; % of step roofline"
 
@@ -166,6 +170,22 @@ def oracle_sample(w: dict, n_tokens: int, seed_seq: int = 0) -> tuple[float, int
     om.replay_logprobs(tok)
     dt = time.perf_counter() - t0
     return (n_tokens - 1) / dt, oracle.num_threads(), f"1 sequence x {n_tokens} tokens (teacher-forced replay), fp64"
+
+
+def oracle_bptt_sample(w: dict, n_tokens: int, seed_seq: int = 0) -> tuple[float, int, str]:
+    """Times the gradient oracle (fp64 autograd, full BPTT) on one sequence
+    truncated to n_tokens.  Returns (scored tokens/s, threads, description)."""
+    import torch
+
+    import oracle
+    from oracle import bptt
+    om = oracle.Model(synth.model_config(w), seed=synth.WEIGHT_SEED)
+    tok = synth.tokens(w, batch=1, length=n_tokens, seed=w["data_seed"] + seed_seq)[0]
+    t0 = time.perf_counter()
+    bptt.loss_and_grads(om, tok, bptt.target_weights("pretrain", n_tokens))
+    dt = time.perf_counter() - t0
+    return ((n_tokens - 1) / dt, torch.get_num_threads(),
+            f"1 sequence x {n_tokens} tokens, forward + full-BPTT backward, fp64 autograd")
 
 
 def oracle_tokens_for(w: dict) -> int:
@@ -297,6 +317,45 @@ def run_gpu(args, w: dict, kind: str, peaks: dict, rank: int, world: int) -> dic
     }
 
 
+def run_backward(args, w: dict, rank: int, world: int) -> dict:
+    """Times rlt_replay_backward (eq. 5.1 weights) over the workload's token
+    ids, already resident on the device: K calls after W warm-up calls."""
+    import torch
+    import stateful_decoder_b200 as rlt
+
+    dev = torch.device("cuda", int(os.environ.get("LOCAL_RANK", 0)))
+    torch.cuda.set_device(dev)
+    model = rlt.rlt_init_weights(synth.model_config(w), synth.WEIGHT_SEED)
+    tok = torch.from_numpy(shard_tokens(w, rank, world)).cuda()
+    B, S = tok.shape
+    wts = torch.full((B, S - 1), 1.0 / (B * (S - 1)), dtype=torch.float32, device=dev)
+    stream = torch.cuda.current_stream()
+    for _ in range(args.warmup):
+        rlt.rlt_replay_backward(model, tok, wts, segment=BPTT_SEGMENT)
+    torch.cuda.synchronize()
+    rlt.rlt_check_device()
+    clocks = ClockSampler(dev.index)
+    clocks.start()
+    if world > 1:
+        import torch.distributed as dist
+        dist.barrier()
+    torch.cuda.synchronize()
+    n0 = rlt.rlt_kernel_launches()
+    e0 = torch.cuda.Event(enable_timing=True)
+    e1 = torch.cuda.Event(enable_timing=True)
+    e0.record(stream)
+    for _ in range(args.steps):
+        rlt.rlt_replay_backward(model, tok, wts, segment=BPTT_SEGMENT)
+    e1.record(stream)
+    torch.cuda.synchronize()
+    launches = rlt.rlt_kernel_launches() - n0
+    ms = max_over_ranks(e0.elapsed_time(e1), world, dev)
+    clk = clocks.stop()
+    rlt.rlt_check_device()
+    return {"value": world * B * (S - 1) * args.steps / (ms / 1e3), "ms_per_step": ms / args.steps,
+            "launches": launches, "clocks": clk, "B": B, "S": S}
+
+
 def read_traffic_ratio() -> tuple[float | None, str]:
     """DRAM bytes per algorithmic byte of the prefix-attention kernel from the
     committed ncu summary, with a note.  The summary records the SHA-1 of the
@@ -348,17 +407,20 @@ def main():
         if rank != 0:
             return
         n_tok = oracle_tokens_for(w)
+        sample = oracle_sample
+        if kind == "backward":
+            n_tok, sample = min(n_tok, 16), oracle_bptt_sample
         for _ in range(args.warmup):
-            oracle_sample(w, n_tok)
+            sample(w, n_tok)
         vals = []
         t0 = time.perf_counter()
         for i in range(args.steps):
-            v, cores, desc = oracle_sample(w, n_tok, seed_seq=i)
+            v, cores, desc = sample(w, n_tok, seed_seq=i)
             vals.append(v)
         dt = time.perf_counter() - t0
         value = statistics.mean(vals)
         print(json.dumps({
-            "impl": "reference", "metric": METRIC, "value": value, "unit": "tokens/s", "n_gpus": args.gpus,
+            "impl": "reference", "metric": BPTT_METRIC if kind == "backward" else METRIC, "value": value, "unit": "tokens/s", "n_gpus": args.gpus,
             "steps": args.steps, "warmup": args.warmup, "ms_per_step": dt * 1e3 / args.steps,
             "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "f64", "data": "synthetic",
             "config": cfg_desc,
@@ -373,6 +435,24 @@ def main():
         from datetime import timedelta
         torch.cuda.set_device(int(os.environ.get("LOCAL_RANK", 0)))
         dist.init_process_group("nccl", timeout=timedelta(seconds=600))
+
+    if kind == "backward":
+        r = run_backward(args, w, rank, world)
+        if world > 1:
+            import torch.distributed as dist
+            dist.barrier()
+            dist.destroy_process_group()
+        if rank == 0:
+            print(json.dumps({
+                "metric": BPTT_METRIC, "value": r["value"], "unit": "tokens/s", "n_gpus": world,
+                "steps": args.steps, "warmup": args.warmup, "ms_per_step": r["ms_per_step"],
+                "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "f32",
+                "data": "synthetic (seeded Zipf(1.1) token ids, random-init weights)",
+                "config": dict(cfg_desc, tokens=r["S"], schedule=f"full BPTT, segments of {BPTT_SEGMENT}",
+                               objective="eq. 5.1 weights"),
+                "roofline": None, "note": "first backward engine (CUDA-core functor kernels), not yet characterised",
+                "gpu_launches": r["launches"], "clocks": r["clocks"]}), flush=True)
+        return
 
     r = run_gpu(args, w, kind, peaks, rank, world)
 
