@@ -304,8 +304,10 @@ int32_t rlt_replay_ratios(rlt_model* m, const int32_t* tok_dev, int32_t B, int32
  * (may be NULL) receives the log-probs the pass computed.  Device memory
  * is allocated inside the call and freed before it returns: about
  * 4 * B * S * (L * (13d + 3F) + 4 G d + 14d) bytes, plus the fp32 weight
- * copies.  The stream is synchronised.  Head size at most 128.
- * Errors: RLT_E_INVAL, RLT_E_OOM, RLT_E_CUDA. */
+ * copies.  The stream is synchronised.  Head size at most 128.  The token
+ * ids are copied to the host and checked against the vocabulary before any
+ * work is enqueued.  Errors: RLT_E_INVAL (arguments, a token id out of
+ * range), RLT_E_OOM, RLT_E_CUDA. */
 int32_t rlt_replay_backward(rlt_model* m, const int32_t* tok_dev, int32_t B, int32_t S, const float* w_dev,
                             int32_t segment, float* logp_dev, void* stream);
 

@@ -1282,6 +1282,13 @@ int32_t rlt_replay_backward(rlt_model* m, const int32_t* tok_dev, int32_t B, int
   if (m->hd > bptt::kMaxHead) return fail(RLT_E_INVAL, "the backward pass takes head sizes up to 128");
   RLT_CUDA(cudaSetDevice(m->device));
   cudaStream_t st = (cudaStream_t)stream;
+  {  // the engine indexes the embedding and the targets by these ids: check them first
+    std::vector<int32_t> ids((size_t)B * S);
+    RLT_CUDA(cudaMemcpyAsync(ids.data(), tok_dev, ids.size() * 4, cudaMemcpyDeviceToHost, st));
+    RLT_CUDA(cudaStreamSynchronize(st));
+    for (int32_t v : ids)
+      if (v < 0 || v >= m->cfg.vocab) return fail(RLT_E_INVAL, "token id " + std::to_string(v) + " out of range");
+  }
   const bptt::Dims D = bptt_dims(m, B, S);
   RLT_TRY(ensure_grads(m, D));
   // fp32 copies of the current weights, freed before returning

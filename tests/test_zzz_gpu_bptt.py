@@ -75,4 +75,9 @@ def test_backward_accumulates_and_zeroes(rlt):
     with pytest.raises(rlt.RltError) as e:
         rlt.rlt_replay_backward(m, tok, wts, segment=0)
     assert e.value.code == rlt.RLT_E_INVAL
+    bad = tok.clone()
+    bad[1, 3] = cfg["vocab"]  # rejected on the host before any launch
+    with pytest.raises(rlt.RltError) as e:
+        rlt.rlt_replay_backward(m, bad, wts, segment=2)
+    assert e.value.code == rlt.RLT_E_INVAL and "out of range" in str(e.value)
     rlt.rlt_check_device()
