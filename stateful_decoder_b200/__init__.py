@@ -145,10 +145,14 @@ def _stream(stream):
     return ctypes.c_void_p(stream.cuda_stream)
 
 
-def _dev(t, dtype_name: str | None = None):
-    """Device pointer of a contiguous CUDA tensor (or None)."""
+def _dev(t, dtype_name: str | None = None, numel: int | None = None):
+    """Device pointer of a contiguous CUDA tensor (or None).  The library
+    reads or writes `numel` elements through it: a smaller tensor is refused
+    here, since the C ABI receives a bare pointer and cannot check."""
     if t is None:
         return None
+    if numel is not None and t.numel() < numel:
+        raise ValueError(f"tensor of {t.numel()} elements where {numel} are needed")
     if not t.is_cuda or not t.is_contiguous():
         raise ValueError("expected a contiguous CUDA tensor")
     if dtype_name is not None and str(t.dtype) != dtype_name:
@@ -283,15 +287,23 @@ def rlt_state_import(state: State, snapshot: np.ndarray, stream=None) -> None:
     _check(_lib.rlt_state_import(state.h, snap.ctypes.data, snap.nbytes, _stream(stream)))
 
 
+def _rows(tokens, batch: int) -> int:
+    """T of a [batch, T] token tensor."""
+    if tokens.dim() != 2 or tokens.shape[0] != batch:
+        raise ValueError(f"expected tokens of shape [{batch}, T], got {tuple(tokens.shape)}")
+    return tokens.shape[1]
+
+
 def rlt_encode_prefix(model: Model, state: State, tokens, stream=None) -> None:
     """tokens: int32 CUDA tensor [B, T], placed at positions n_enc+1..n_enc+T."""
-    _check(_lib.rlt_encode_prefix(model.h, state.h, _dev(tokens, "torch.int32"), tokens.shape[1], _stream(stream)))
+    T = _rows(tokens, state.batch)
+    _check(_lib.rlt_encode_prefix(model.h, state.h, _dev(tokens, "torch.int32"), T, _stream(stream)))
 
 
-def _readout_out(logp=None, sampled=None, logp_sampled=None, logmu=None, logits=None):
-    return ReadoutOut(logp=_dev(logp, "torch.float32"), sampled=_dev(sampled, "torch.int32"),
-                      logp_sampled=_dev(logp_sampled, "torch.float32"), logmu=_dev(logmu, "torch.float32"),
-                      logits=_dev(logits, "torch.float32"))
+def _readout_out(B: int, V: int, logp=None, sampled=None, logp_sampled=None, logmu=None, logits=None):
+    return ReadoutOut(logp=_dev(logp, "torch.float32", B), sampled=_dev(sampled, "torch.int32", B),
+                      logp_sampled=_dev(logp_sampled, "torch.float32", B), logmu=_dev(logmu, "torch.float32", B),
+                      logits=_dev(logits, "torch.float32", B * V))
 
 
 def _sampling(sampling):
@@ -302,28 +314,31 @@ def _sampling(sampling):
 
 def rlt_readout(model: Model, state: State, next_tokens=None, sampling: dict | None = None, stream=None,
                 **outs) -> None:
-    o = _readout_out(**outs)
-    _check(_lib.rlt_readout(model.h, state.h, _dev(next_tokens, "torch.int32"), _sampling(sampling),
+    o = _readout_out(state.batch, model.cfg["vocab"], **outs)
+    _check(_lib.rlt_readout(model.h, state.h, _dev(next_tokens, "torch.int32", state.batch), _sampling(sampling),
                             ctypes.byref(o), _stream(stream)))
 
 
 def rlt_decoder_step(model: Model, state: State, tokens=None, next_tokens=None, sampling: dict | None = None,
                      stream=None, **outs) -> None:
-    o = _readout_out(**outs)
-    _check(_lib.rlt_decoder_step(model.h, state.h, _dev(tokens, "torch.int32"), _dev(next_tokens, "torch.int32"),
-                                 _sampling(sampling), ctypes.byref(o), _stream(stream)))
+    o = _readout_out(state.batch, model.cfg["vocab"], **outs)
+    _check(_lib.rlt_decoder_step(model.h, state.h, _dev(tokens, "torch.int32", state.batch),
+                                 _dev(next_tokens, "torch.int32", state.batch), _sampling(sampling), ctypes.byref(o),
+                                 _stream(stream)))
 
 
 def rlt_prefill(model: Model, state: State, tokens, logp=None, stream=None) -> None:
-    _check(_lib.rlt_prefill(model.h, state.h, _dev(tokens, "torch.int32"), tokens.shape[1],
-                            _dev(logp, "torch.float32"), _stream(stream)))
+    """tokens int32 [B, T]; logp (optional) float32 [B, T-1] (CUDA tensors)."""
+    T = _rows(tokens, state.batch)
+    _check(_lib.rlt_prefill(model.h, state.h, _dev(tokens, "torch.int32"), T,
+                            _dev(logp, "torch.float32", state.batch * (T - 1)), _stream(stream)))
 
 
 def rlt_replay_logprobs(model: Model, tokens, logp, stream=None) -> None:
     """tokens int32 [B, S] and logp float32 [B, S-1], both CUDA tensors."""
     B, S = tokens.shape
-    _check(_lib.rlt_replay_logprobs(model.h, _dev(tokens, "torch.int32"), B, S, _dev(logp, "torch.float32"),
-                                    _stream(stream)))
+    _check(_lib.rlt_replay_logprobs(model.h, _dev(tokens, "torch.int32"), B, S,
+                                    _dev(logp, "torch.float32", B * (S - 1)), _stream(stream)))
 
 
 def rlt_replay_ratios(model: Model, tokens, logmu, action_mask, logp, ratio=None, seq_logratio=None,
@@ -331,9 +346,10 @@ def rlt_replay_ratios(model: Model, tokens, logmu, action_mask, logp, ratio=None
     """tokens int32 [B, S]; logmu float32 and action_mask uint8 [B, S-1]; outputs
     logp and ratio float32 [B, S-1], seq_logratio float32 [B] (CUDA tensors)."""
     B, S = tokens.shape
-    _check(_lib.rlt_replay_ratios(model.h, _dev(tokens, "torch.int32"), B, S, _dev(logmu, "torch.float32"),
-                                  _dev(action_mask, "torch.uint8"), _dev(logp, "torch.float32"),
-                                  _dev(ratio, "torch.float32"), _dev(seq_logratio, "torch.float32"),
+    n = B * (S - 1)
+    _check(_lib.rlt_replay_ratios(model.h, _dev(tokens, "torch.int32"), B, S, _dev(logmu, "torch.float32", n),
+                                  _dev(action_mask, "torch.uint8", n), _dev(logp, "torch.float32", n),
+                                  _dev(ratio, "torch.float32", n), _dev(seq_logratio, "torch.float32", B),
                                   _stream(stream)))
 
 
@@ -342,8 +358,9 @@ def rlt_replay_backward(model: Model, tokens, weights, segment: int = 32, logp=N
     [B, S], weights float32 [B, S-1], optional logp float32 [B, S-1] (CUDA
     tensors).  Gradients accumulate in the model (Model.grad, rlt_grad_zero)."""
     B, S = tokens.shape
-    _check(_lib.rlt_replay_backward(model.h, _dev(tokens, "torch.int32"), B, S, _dev(weights, "torch.float32"),
-                                    segment, _dev(logp, "torch.float32"), _stream(stream)))
+    _check(_lib.rlt_replay_backward(model.h, _dev(tokens, "torch.int32"), B, S,
+                                    _dev(weights, "torch.float32", B * (S - 1)), segment,
+                                    _dev(logp, "torch.float32", B * (S - 1)), _stream(stream)))
 
 
 def rlt_grad_zero(model: Model, stream=None) -> None:
@@ -354,16 +371,20 @@ def rlt_op_linear(w, x, y, use_tensor_cores: bool = True, stream=None) -> None:
     """y [N, M] fp32 = x [N, K] @ w [M, K]^T (CUDA tensors, bf16 or fp32)."""
     M, K = w.shape
     N = x.shape[0]
+    if x.dim() != 2 or x.shape[1] != K or x.dtype != w.dtype:
+        raise ValueError("x must be [N, K] in the dtype of w")
     dt = DTYPE_BF16 if str(w.dtype) == "torch.bfloat16" else DTYPE_F32
-    _check(_lib.rlt_op_linear(_dev(w), _dev(x), _dev(y, "torch.float32"), M, N, K, dt, int(use_tensor_cores),
+    _check(_lib.rlt_op_linear(_dev(w), _dev(x), _dev(y, "torch.float32", N * M), M, N, K, dt, int(use_tensor_cores),
                               _stream(stream)))
 
 
 def _prefix_attention_args(q, k, v, n, out, rope_cs, qpos, stream):
     B, H, ld_t, hd = k.shape
+    if tuple(v.shape) != tuple(k.shape) or v.dtype != k.dtype or out.dtype != k.dtype:
+        raise ValueError("v and out must match k's shape and dtype")
     dt = DTYPE_BF16 if str(k.dtype) == "torch.bfloat16" else DTYPE_F32
-    return (_dev(q, "torch.float32"), _dev(k), _dev(v), ld_t, B, H, hd, n, dt, _dev(rope_cs, "torch.float32"),
-            qpos, _dev(out), _stream(stream))
+    return (_dev(q, "torch.float32", B * H * hd), _dev(k), _dev(v), ld_t, B, H, hd, n, dt,
+            _dev(rope_cs, "torch.float32", (qpos + 1) * hd), qpos, _dev(out, None, B * H * hd), _stream(stream))
 
 
 def rlt_op_prefix_attention(q, k, v, n: int, out, rope_cs=None, qpos: int = 0, stream=None) -> None:
@@ -382,8 +403,9 @@ def rlt_op_prefix_attention_noalloc(q, k, v, n: int, out, rope_cs=None, qpos: in
 def rlt_op_sample(logits, sampling: dict, t: int, token, logp=None, logmu=None, stream=None) -> None:
     """Sample from fp32 logits [B, V] (CUDA) as position t."""
     B, V = logits.shape
-    _check(_lib.rlt_op_sample(_dev(logits, "torch.float32"), B, V, _sampling(sampling), t, _dev(token, "torch.int32"),
-                              _dev(logp, "torch.float32"), _dev(logmu, "torch.float32"), _stream(stream)))
+    _check(_lib.rlt_op_sample(_dev(logits, "torch.float32"), B, V, _sampling(sampling), t,
+                              _dev(token, "torch.int32", B), _dev(logp, "torch.float32", B),
+                              _dev(logmu, "torch.float32", B), _stream(stream)))
 
 
 def rlt_check_device() -> None:

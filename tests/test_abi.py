@@ -78,3 +78,84 @@ def test_state_and_replay_arguments_validated_on_host():
     buf = ctypes.create_string_buffer(256)
     assert lib.rlt_last_error(buf, 256) == rlt.RLT_E_INVAL
     assert buf.value  # the last failure's text
+
+
+def test_backward_arguments_validated_on_host():
+    """The backward entry points reject missing handles and buffers, and
+    a gradient of an unknown tensor, before touching a device."""
+    import stateful_decoder_b200 as rlt
+    lib = rlt._lib
+    assert lib.rlt_replay_backward(None, None, 1, 2, None, 4, None, None) == rlt.RLT_E_INVAL
+    assert lib.rlt_grad_zero(None, None) == rlt.RLT_E_INVAL
+    buf = (ctypes.c_float * 4)()
+    assert lib.rlt_grad_read(None, b"emb", buf, 16) == rlt.RLT_E_INVAL
+
+
+class _FakeCuda:
+    """A CPU tensor that passes the binding's device checks and hands the
+    library a null pointer, so that only the binding's size checks can
+    refuse a call (and a call that got through would be rejected by the
+    library's own null checks, never reach a device)."""
+
+    def __init__(self, t):
+        self.t = t
+        self.is_cuda = True
+        self.shape = t.shape
+        self.dtype = t.dtype
+
+    def numel(self):
+        return self.t.numel()
+
+    def dim(self):
+        return self.t.dim()
+
+    def is_contiguous(self):
+        return True
+
+    def data_ptr(self):
+        return 0
+
+
+def test_binding_refuses_short_buffers():
+    """The C ABI receives bare pointers, so the binding checks every buffer
+    the library writes or reads against the size the call implies."""
+    import types
+
+    import torch
+
+    import stateful_decoder_b200 as rlt
+
+    def z(*shape, dtype=torch.float32):
+        return _FakeCuda(torch.zeros(*shape, dtype=dtype))
+
+    i32 = torch.int32
+    model = types.SimpleNamespace(h=None, cfg={"vocab": 40})
+    state = types.SimpleNamespace(h=None, batch=2)
+    tok = z(2, 9, dtype=i32)
+    samp = {"temperature": 1.0, "top_k": 4, "seed": 1}
+    cases = [
+        (lambda: rlt.rlt_replay_logprobs(model, tok, z(2, 7)), "elements"),
+        (lambda: rlt.rlt_replay_backward(model, tok, z(2, 7)), "elements"),
+        (lambda: rlt.rlt_replay_backward(model, tok, z(2, 8), logp=z(2, 7)), "elements"),
+        (lambda: rlt.rlt_replay_ratios(model, tok, z(2, 8), z(2, 8, dtype=torch.uint8), z(2, 8),
+                                       seq_logratio=z(1)), "elements"),
+        (lambda: rlt.rlt_prefill(model, state, tok, logp=z(2, 7)), "elements"),
+        (lambda: rlt.rlt_prefill(model, state, z(3, 9, dtype=i32)), "shape"),
+        (lambda: rlt.rlt_encode_prefix(model, state, z(9, dtype=i32)), "shape"),
+        (lambda: rlt.rlt_readout(model, state, logits=z(2, 39)), "elements"),
+        (lambda: rlt.rlt_decoder_step(model, state, tokens=z(1, dtype=i32)), "elements"),
+        (lambda: rlt.rlt_op_sample(z(3, 40), samp, 0, z(2, dtype=i32)), "elements"),
+        (lambda: rlt.rlt_op_linear(z(4, 8), z(3, 8), z(3, 3)), "elements"),
+        (lambda: rlt.rlt_op_linear(z(4, 8), z(3, 7), z(3, 4)), "x must be"),
+        (lambda: rlt.rlt_op_prefix_attention(z(2, 32), z(2, 2, 8, 16), z(2, 2, 8, 16), 4, z(2, 31)), "elements"),
+        (lambda: rlt.rlt_op_prefix_attention(z(2, 32), z(2, 2, 8, 16), z(2, 2, 8, 16), 4, z(2, 32),
+                                             rope_cs=z(4, 8, 2), qpos=4), "elements"),
+        (lambda: rlt.rlt_op_prefix_attention(z(2, 32), z(2, 2, 8, 16), z(2, 2, 7, 16), 4, z(2, 32)), "match"),
+    ]
+    for i, (call, msg) in enumerate(cases):
+        with pytest.raises(ValueError, match=msg):
+            call()
+    # a correctly sized call gets through the binding to the library, whose
+    # own checks then refuse the null handle
+    with pytest.raises(rlt.RltError):
+        rlt.rlt_replay_logprobs(model, tok, z(2, 8), stream=0)
