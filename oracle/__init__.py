@@ -205,7 +205,8 @@ class Model:
     def __init__(self, cfg: dict, seed: int | None = None):
         self.cfg = dict(cfg)
         self._c = _cfg_struct(cfg)
-        self.h = lib().orc_model_new(ctypes.byref(self._c))
+        self._lib = lib()  # kept for __del__, which may run after module teardown
+        self.h = self._lib.orc_model_new(ctypes.byref(self._c))
         if not self.h:
             raise ValueError("oracle rejected the configuration")
         if seed is not None:
@@ -213,7 +214,7 @@ class Model:
 
     def __del__(self):
         if getattr(self, "h", None):
-            lib().orc_model_free(self.h)
+            self._lib.orc_model_free(self.h)
             self.h = None
 
     @property
@@ -277,13 +278,14 @@ class Seq:
     def __init__(self, model: Model, max_len: int, keep_enc_cache: bool):
         self.model = model
         self.d = model.cfg["d"]
-        self.h = lib().orc_seq_new(model.h, max_len, int(keep_enc_cache))
+        self._lib = lib()
+        self.h = self._lib.orc_seq_new(model.h, max_len, int(keep_enc_cache))
         if not self.h:
             raise ValueError("bad max_len")
 
     def __del__(self):
         if getattr(self, "h", None):
-            lib().orc_seq_free(self.h)
+            self._lib.orc_seq_free(self.h)
             self.h = None
 
     def encode_prefill(self, tokens) -> None:
