@@ -7,8 +7,9 @@ functors in a host loop, in fp64, built with AddressSanitizer and
 UBSanitizer.  Every gradient entry must equal the gradient oracle
 (``oracle.bptt``, autograd over the fp64 forward); a single out-of-bounds
 index or bad stride fails the sanitizers.  The variants cover tied and
-untied stacks, both merge forms, G = 1 and G = L, W = 1, W wrapping, W >= S,
-and segment lengths from 1 to the whole sequence.
+untied stacks, both merge forms, G = 1 and G = L (up to three layers), one
+head and several, W = 1, W wrapping, W >= S, another RoPE base, and segment
+lengths from 1 to the whole sequence.
 """
 import os
 import shutil
@@ -85,11 +86,13 @@ VARIANTS = [
     (dict(tied=0, merge_kind=1, groups=2, window=3), 2),
     (dict(window=32, alpha=0.5), 31),
     (dict(dtype=1, window=5), 4),
+    (dict(n_layers=3, groups=3, window=2, n_heads=1, rope_base=500.0), 6),
 ]
 
 
 @pytest.mark.parametrize("kw,seg", VARIANTS,
-                         ids=["seg1", "seg5", "W1_seg3", "untied_convex_GL_seg2", "fullwin_oneseg", "bf16_seg4"])
+                         ids=["seg1", "seg5", "W1_seg3", "untied_convex_GL_seg2", "fullwin_oneseg", "bf16_seg4",
+                              "L3_GL_one_head_base500_seg6"])
 def test_host_engine_equals_gradient_oracle(oracle_lib, host_exe, tmp_path, kw, seg):
     from oracle import bptt
     w = synth.workload("tiny", **dict(dict(d=32, n_heads=4, ffn=48, vocab=40, prompt=12), **kw))
