@@ -302,9 +302,12 @@ int32_t rlt_replay_ratios(rlt_model* m, const int32_t* tok_dev, int32_t B, int32
  * accumulated into fp32 buffers the model owns, one per stored tensor, read
  * with rlt_grad_read and cleared with rlt_grad_zero.  logp_dev [B][S-1]
  * (may be NULL) receives the log-probs the pass computed.  Device memory
- * is allocated inside the call and freed before it returns: about
- * 4 * B * S * (L * (13d + 3F) + 4 G d + 14d) bytes, plus the fp32 weight
- * copies.  The stream is synchronised.  Head size at most 128.  The token
+ * is allocated inside the call and freed before it returns, in fp32: about
+ * 4 * B * S * (L * (12d + 3F) + 4 G d + 13d + 3F) bytes for the encoder
+ * activations, the decoder key/value history and their adjoints, plus
+ * 4 * segment * B * (L * (11d + 3F) + 6d + V) bytes for one segment's
+ * recomputed steps, plus the fp32 weight copies.  The stream is
+ * synchronised.  Head size at most 128.  The token
  * ids are copied to the host and checked against the vocabulary before any
  * work is enqueued.  Errors: RLT_E_INVAL (arguments, a token id out of
  * range), RLT_E_OOM, RLT_E_CUDA. */
