@@ -1,13 +1,22 @@
 """Benchmark of the RLT decoder hot path on B200 GPUs.
 
-Default workload (one GPU): current-policy replay of the reference-width model
-at L_E = L_D = 24 (d=2048, 16x128 heads, W=256, G=1, F=5632, V=32000), B = 256
-sequences of S = 1024 tokens.  One step = one rlt_replay_logprobs call:
-token-parallel encoder + memory projection over [B, S], then S-1 lock-step
-decoder transitions with the readout of every next-token log-prob.  The
-metric is decoder tokens/s = B x (S-1) x steps / time.  (The 48+48 model at
-B=128 with 2048+2048 tokens needs about 229 GB of state and does not fit one
-GPU; this is the largest of the benchmarked configurations that does.)
+Default workload (one GPU): the reference-depth model, L_E = L_D = 48 tied
+(d=2048, 16x128 heads, W=256, G=1, F=5632, V=32000, bf16), B = 128 sequences
+per GPU.  A 2048-token prompt is prefilled (token-parallel encoder, memory
+projection and 2048 decoder transitions) before the timed region; one step is
+then a block of 32 sampled generation transitions continuing from the state:
+for every sequence, the encoder step over the cache C^E (eq. 2.8), the memory
+append, the merge, the 48 decoder blocks and the readout with the behaviour
+sampler (temperature 0.8, top-k 50).  The metric is decoder tokens/s =
+B x 32 x steps / time.  The warm-up blocks come first, so the timed positions
+follow them (t = 2048 + 32*warmup + 1 ...).  The full 2048 + 2048 schedule at
+B = 128 needs about 229 GB of state and does not fit one GPU; the positions
+reached here stay well inside it.
+
+Other workloads (--workload): `replay` (the reference width at L = 24,
+B = 256 x 1024 tokens, one rlt_replay_logprobs call per step), `layerwise`,
+`small`, `refdepth-b64` (one whole prefill + generation per step) and
+`bptt-small` (full-BPTT backward).
 
 Multi-GPU (torchrun): sequences shard across ranks with no data-path
 collective (weak scaling, B sequences per rank); timing is the max over ranks.
@@ -17,6 +26,7 @@ collective (weak scaling, B sequences per rank); timing is the max over ranks.
 from __future__ import annotations
 
 import argparse
+import hashlib
 import json
 import os
 import statistics
@@ -34,18 +44,32 @@ import synth  # noqa: E402
 
 BENCH_WORKLOADS = {
     # name: (synth workload, overrides, kind)
+    "refdepth": ("refdepth", {"block": 32}, "block"),
     "replay": ("replay", {}, "replay"),
     "layerwise": ("layerwise", {}, "replay"),
     "small": ("small", {}, "generate"),
     "refdepth-b64": ("refdepth", {"batch": 64}, "generate"),
-    "refdepth-b128-t3072": ("refdepth", {"gen": 1024}, "generate"),
     # full-BPTT forward + backward (rlt_replay_backward) of the small model
     "bptt-small": ("small", {"prompt": 256, "gen": 0}, "backward"),
 }
+DEFAULT_WORKLOAD = "refdepth"
 BPTT_METRIC = "RLT full-BPTT tokens/s (replay forward + backward through the whole history) on 1 B200"
 BPTT_SEGMENT = 32
+# decode-attention launches recorded with CUDA events by the library in the
+# profiling pass (every 4th position), then scaled to all launches
+PROFILE_STRIDE = 4
+# profiling blocks that follow the timed ones (block workloads)
+PROFILE_BLOCKS = 2
+TRAFFIC_FILE = os.path.join(ROOT, "profiles", "traffic.json")
 
-METRIC = "RLT decoder tokens/s (B seqs, 48+48 tied) on 1 B200; % of step roofline"
+
+def metric_name(w: dict, kind: str) -> str:
+    """The metric string names the model actually run: a line never claims
+    48+48 unless the 48-layer model ran."""
+    L = w["n_layers"]
+    tie = "tied" if w.get("tied", 1) else "untied"
+    extra = ", teacher-forced replay" if kind == "replay" else ""
+    return f"RLT decoder tokens/s (B seqs, {L}+{L} {tie}{extra}) on 1 B200; % of step roofline"
 
 
 def load_peaks() -> dict:
@@ -58,34 +82,61 @@ def load_peaks() -> dict:
 
 
 # ---------------------------------------------------------------- roofline model
-def step_roofline(w: dict, kind: str, peaks: dict) -> dict:
-    """Analytic lower bound of one step: per decoder transition the slower of
-    (weights + KV bytes)/HBM and FLOPs/tensor peak, plus the token-parallel
-    encoder at tensor peak."""
-    d, L, F, V, G, W, B = w["d"], w["n_layers"], w["ffn"], w["vocab"], w["groups"], w["window"], w["batch"]
-    eb = 2 if w["dtype"] == 1 else 4
+def params(w: dict) -> tuple[int, int]:
+    """Weights streamed by one decoder transition (with its readout) and by one
+    encoder step (with the memory projection)."""
+    d, L, F, V, G = w["d"], w["n_layers"], w["ffn"], w["vocab"], w["groups"]
     merge = 3 * d * d if w.get("merge_kind", 0) == 0 else 2 * d * d
     p_dec = L * (4 * d * d + 2 * d * d + 3 * d * F) + merge + V * d
     p_enc = L * (4 * d * d + 3 * d * F) + 2 * d * d * G
-    hbm = peaks["hbm_gbs"] * 1e9
-    tc = peaks["bf16_tflops_sustained"] * 1e12
-    T = w["prompt"]
-    n_gen = w.get("gen", 0) if kind == "generate" else 0
-    total = 0.0
-    dec_steps = (T - 1 if kind == "replay" else T + n_gen - 1)
-    for t in range(1, dec_steps + 1):
-        kv = B * eb * 2 * d * (L * (min(t, W) - 1) + L + L * t)
-        wbytes = eb * p_dec
-        flops = 2 * B * p_dec + 4 * B * d * (L * min(t, W) + L * t)
-        if kind == "generate" and t > T:
-            kv += B * eb * 2 * d * (L * t + L + G)
-            wbytes += eb * p_enc
-            flops += 2 * B * p_enc + 4 * B * d * L * t
-        total += max((kv + wbytes) / hbm, flops / tc)
-    S = T
-    enc_flops = 2 * B * S * p_enc + 4 * B * L * d * S * S / 2
-    total += enc_flops / tc
-    return {"bound_ms": total * 1e3, "decoder_transitions": dec_steps}
+    return p_dec, p_enc
+
+
+def transition_bound_s(w: dict, t: int, gen: bool, peaks: dict) -> float:
+    """Analytic lower bound of one decoder transition at position t for B
+    sequences: the slower of (weights + KV bytes)/HBM and FLOPs/tensor peak.
+    KV bytes: SWA ring read (min(t,W)-1 entries) and insert, memory M_<=t
+    read; with the encoder step (gen) also the C^E_<=t read, its insert and
+    the memory append."""
+    d, L, G, W, B = w["d"], w["n_layers"], w["groups"], w["window"], w["batch"]
+    eb = 2 if w["dtype"] == 1 else 4
+    p_dec, p_enc = params(w)
+    kv = B * eb * 2 * d * (L * (min(t, W) - 1) + L + L * t)
+    wbytes = eb * p_dec
+    flops = 2 * B * p_dec + 4 * B * d * (L * min(t, W) + L * t)
+    if gen:
+        kv += B * eb * 2 * d * (L * t + L + G)
+        wbytes += eb * p_enc
+        flops += 2 * B * p_enc + 4 * B * d * L * t
+    return max((kv + wbytes) / (peaks["hbm_gbs"] * 1e9), flops / (peaks["bf16_tflops_sustained"] * 1e12))
+
+
+def encoder_bound_s(w: dict, T: int, peaks: dict) -> float:
+    """Token-parallel encoder + memory projection over T tokens at tensor peak."""
+    _, p_enc = params(w)
+    flops = 2 * w["batch"] * T * p_enc + 4 * w["batch"] * w["n_layers"] * w["d"] * T * T / 2
+    return flops / (peaks["bf16_tflops_sustained"] * 1e12)
+
+
+def step_roofline(w: dict, kind: str, peaks: dict, t_range: tuple[int, int] | None = None) -> dict:
+    """Analytic bound of one step, in ms (see transition_bound_s).
+    replay: encoder over S tokens + transitions 1..S-1; generate: encoder over
+    the prompt + transitions 1..T (prefill) and T+1..T+n_gen-1 (with encoder
+    steps); block: the generation transitions t_range[0]..t_range[1]
+    inclusive, averaged per block of w['block']."""
+    if kind == "replay":
+        S = w["prompt"]
+        total = encoder_bound_s(w, S, peaks) + sum(transition_bound_s(w, t, False, peaks) for t in range(1, S))
+        return {"bound_ms": total * 1e3, "decoder_transitions": S - 1}
+    if kind == "generate":
+        T, n_gen = w["prompt"], w["gen"]
+        total = encoder_bound_s(w, T, peaks)
+        total += sum(transition_bound_s(w, t, t > T, peaks) for t in range(1, T + n_gen))
+        return {"bound_ms": total * 1e3, "decoder_transitions": T + n_gen - 1}
+    a, b = t_range
+    total = sum(transition_bound_s(w, t, True, peaks) for t in range(a, b + 1))
+    n_blocks = (b - a + 1) / w["block"]
+    return {"bound_ms": total * 1e3 / n_blocks, "decoder_transitions": w["block"]}
 
 
 # ---------------------------------------------------------------- sharding
@@ -158,18 +209,56 @@ class ClockSampler:
                 "reasons": reasons, "samples": len(self.rows)}
 
 
+def cpu_model() -> str:
+    try:
+        for line in open("/proc/cpuinfo"):
+            if line.startswith("model name"):
+                return line.split(":", 1)[1].strip()
+    except OSError:
+        pass
+    return "unknown"
+
+
 # ---------------------------------------------------------------- CPU oracle leg
-def oracle_sample(w: dict, n_tokens: int, seed_seq: int = 0) -> tuple[float, int, str]:
-    """Times the fp64 oracle on one sequence truncated to n_tokens of the
-    workload (encoder + n_tokens-1 decoder transitions with readouts).
-    Returns (decoder tokens/s, threads, description)."""
+# Every oracle sample is bounded: the fp64 oracle streams the whole model per
+# token (about 13 GFLOP per token at the reference depth), so a sample is a
+# few short sequences, not the benchmarked batch.
+ORACLE_SAMPLE = {
+    # kind: (sequences, prompt tokens, generated tokens); replay/generate use (sequences, tokens)
+    "block": (2, 6, 6),
+}
+
+
+def oracle_model(w: dict):
     import oracle
-    om = oracle.Model(synth.model_config(w), seed=synth.WEIGHT_SEED)
-    tok = synth.tokens(w, batch=1, length=n_tokens, seed=w["data_seed"] + seed_seq)[0]
+    return oracle.Model(synth.model_config(w), seed=synth.WEIGHT_SEED)
+
+
+def oracle_sample(w: dict, kind: str, om, seed_seq: int = 0) -> tuple[float, int, str]:
+    """Times the fp64 oracle on a bounded sample of the workload and returns
+    (decoder transitions/s, threads, description).  block: a few sequences
+    with a short prompt and sampled generation (prefill, then encoder step +
+    transition + sampler per token, as the timed GPU step does); otherwise a
+    teacher-forced replay of one sequence truncated to a prefix."""
+    import oracle
+    if kind == "block":
+        n_seq, n_prompt, n_new = ORACLE_SAMPLE["block"]
+        tok = synth.tokens(w, batch=n_seq, length=n_prompt, seed=w["data_seed"] + 17 * seed_seq)
+        t0 = time.perf_counter()
+        for b in range(n_seq):
+            om.generate(tok[b], n_new, synth.TEMPERATURE, synth.TOP_K, synth.SAMPLER_SEED, b)
+        dt = time.perf_counter() - t0
+        n = n_seq * (n_prompt + n_new - 1)
+        return (n / dt, oracle.num_threads(),
+                f"{n_seq} sequences x ({n_prompt}-token prompt + {n_new} sampled tokens) from BOS = {n} transitions, "
+                f"fp64; positions t <= {n_prompt + n_new - 1}, so its attention work per token is lower than at the "
+                f"benched positions")
+    n_tok = oracle_tokens_for(w)
+    tok = synth.tokens(w, batch=1, length=n_tok, seed=w["data_seed"] + seed_seq)[0]
     t0 = time.perf_counter()
     om.replay_logprobs(tok)
     dt = time.perf_counter() - t0
-    return (n_tokens - 1) / dt, oracle.num_threads(), f"1 sequence x {n_tokens} tokens (teacher-forced replay), fp64"
+    return (n_tok - 1) / dt, oracle.num_threads(), f"1 sequence x {n_tok} tokens (teacher-forced replay), fp64"
 
 
 def oracle_bptt_sample(w: dict, n_tokens: int, seed_seq: int = 0) -> tuple[float, int, str]:
@@ -196,7 +285,7 @@ def oracle_tokens_for(w: dict) -> int:
 
 
 # ---------------------------------------------------------------- GPU leg
-def run_gpu(args, w: dict, kind: str, peaks: dict, rank: int, world: int) -> dict | None:
+def run_gpu(args, w: dict, kind: str, peaks: dict, rank: int, world: int) -> dict:
     import torch
     import torch.distributed as dist
     import stateful_decoder_b200 as rlt
@@ -207,6 +296,10 @@ def run_gpu(args, w: dict, kind: str, peaks: dict, rank: int, world: int) -> dic
     B = w["batch"]
     model = rlt.rlt_init_weights(cfg, synth.WEIGHT_SEED)
     stream = torch.cuda.current_stream()
+    samp = {"temperature": synth.TEMPERATURE, "top_k": synth.TOP_K, "seed": synth.SAMPLER_SEED}
+    setup = None  # untimed preparation before a pass (block workloads: the prompt prefill)
+    after_warmup = None  # untimed hook between the warm-up and the timed e2e steps
+    t_range = None
 
     if kind == "replay":
         S = w["prompt"]
@@ -225,7 +318,10 @@ def run_gpu(args, w: dict, kind: str, peaks: dict, rank: int, world: int) -> dic
             logp_host.copy_(logp, non_blocking=True)
 
         h2d, d2h = tok_host.numel() * 4, logp_host.numel() * 4
-    else:
+        n_prof = 1
+        # decode-attention launches of one step: prefix (memory), SWA
+        launches_per_step = (w["n_layers"] * (S - 1), w["n_layers"] * (S - 1))
+    elif kind == "generate":
         T, n_gen = w["prompt"], w["gen"]
         state = rlt.rlt_state_create(model, B, T + n_gen, rlt.STATE_ENCODER_CACHE)
         tok_host = torch.from_numpy(shard_tokens(w, rank, world)).pin_memory()
@@ -234,7 +330,6 @@ def run_gpu(args, w: dict, kind: str, peaks: dict, rank: int, world: int) -> dic
         lmu = torch.zeros(n_gen, B, device=dev)
         lps = torch.zeros(n_gen, B, device=dev)
         ids_host = torch.zeros(n_gen, B, dtype=torch.int32).pin_memory()
-        samp = {"temperature": synth.TEMPERATURE, "top_k": synth.TOP_K, "seed": synth.SAMPLER_SEED}
         tokens_per_step = B * (T + n_gen - 1)
 
         def step():
@@ -251,67 +346,129 @@ def run_gpu(args, w: dict, kind: str, peaks: dict, rank: int, world: int) -> dic
             ids_host.copy_(ids, non_blocking=True)
 
         h2d, d2h = tok_host.numel() * 4, ids_host.numel() * 4
+        n_prof = 1
+        n_dec = T + n_gen - 1
+        launches_per_step = (w["n_layers"] * n_dec + w["n_layers"] * (n_gen - 1), w["n_layers"] * n_dec)
+    else:  # block: prompt prefilled untimed, then blocks of sampled transitions
+        T, blk = w["prompt"], w["block"]
+        n_blocks = args.warmup + args.steps + PROFILE_BLOCKS
+        max_len = T + blk * n_blocks
+        state = rlt.rlt_state_create(model, B, max_len, rlt.STATE_ENCODER_CACHE)
+        tok = torch.from_numpy(shard_tokens(w, rank, world)).cuda()
+        ids = torch.zeros(blk, B, dtype=torch.int32, device=dev)
+        lmu = torch.zeros(blk, B, device=dev)
+        lps = torch.zeros(blk, B, device=dev)
+        ids_host = torch.zeros(blk, B, dtype=torch.int32).pin_memory()
+        lmu_host = torch.zeros(blk, B).pin_memory()
+        first = torch.zeros(B, dtype=torch.int32, device=dev)
+        tokens_per_step = B * blk
+        t_range = (T + blk * args.warmup + 1, T + blk * (args.warmup + args.steps))
+
+        def setup():
+            # H_T after the prompt (App. A.1) and the first sampled token,
+            # which stays pending in the state and is copied to the host
+            rlt.rlt_state_reset(state)
+            rlt.rlt_prefill(model, state, tok)
+            rlt.rlt_readout(model, state, sampling=samp, sampled=ids[blk - 1], logp_sampled=lps[blk - 1],
+                            logmu=lmu[blk - 1])
+            ids_host.copy_(ids)
+
+        def step():
+            # each transition consumes the token the previous readout sampled
+            for i in range(blk):
+                rlt.rlt_decoder_step(model, state, sampling=samp, sampled=ids[i], logp_sampled=lps[i], logmu=lmu[i])
+
+        def step_e2e():
+            # the block's first tokens come from the host (what a serving
+            # loop holds after reading back the previous block), the block's
+            # sampled ids and behaviour log-probs go back to the host
+            first.copy_(ids_host[blk - 1], non_blocking=True)
+            rlt.rlt_decoder_step(model, state, tokens=first, sampling=samp, sampled=ids[0], logp_sampled=lps[0],
+                                 logmu=lmu[0])
+            for i in range(1, blk):
+                rlt.rlt_decoder_step(model, state, sampling=samp, sampled=ids[i], logp_sampled=lps[i], logmu=lmu[i])
+            ids_host.copy_(ids, non_blocking=True)
+            lmu_host.copy_(lmu, non_blocking=True)
+
+        def after_warmup():
+            ids_host.copy_(ids)  # the host holds the last block's ids, as a serving loop would
+
+        h2d, d2h = first.numel() * 4, ids_host.numel() * 4 + lmu_host.numel() * 4
+        n_prof = PROFILE_BLOCKS
+        # prefix attention: encoder step over C^E and cross-attention over M; SWA
+        launches_per_step = (2 * w["n_layers"] * blk, w["n_layers"] * blk)
 
     def barrier():
         if world > 1:
             dist.barrier()
 
-    def timed(fn, k, profile=False):
+    def timed(fn, k):
         barrier()
         torch.cuda.synchronize()
-        if profile:
-            rlt.rlt_profile_enable(model, True)
         n0 = rlt.rlt_kernel_launches()
         e0 = torch.cuda.Event(enable_timing=True)
         e1 = torch.cuda.Event(enable_timing=True)
-        torch.cuda.nvtx.range_push("timed" if profile else "timed_e2e")  # lets ncu select the timed launches
         e0.record(stream)
         for _ in range(k):
             fn()
         e1.record(stream)
-        torch.cuda.nvtx.range_pop()
         torch.cuda.synchronize()
         launches = rlt.rlt_kernel_launches() - n0
         ms = max_over_ranks(e0.elapsed_time(e1), world, dev)
         barrier()
         return ms, launches
 
+    if setup:
+        setup()
     for _ in range(args.warmup):
         step()
     torch.cuda.synchronize()
     rlt.rlt_check_device()
 
+    # timed pass: instrumentation off
     clocks = ClockSampler(dev.index)
     clocks.start()
-    ms, launches = timed(step, args.steps, profile=True)
+    ms, launches = timed(step, args.steps)
     clk = clocks.stop()
+
+    # profiling pass (not timed): the library records CUDA events around the
+    # decode-attention launches of every 4th position
+    rlt.rlt_profile_enable(model, True)
+    for _ in range(n_prof):
+        step()
+    torch.cuda.synchronize()
     a_ms, a_n, a_bytes = rlt.rlt_profile_read(model, 0)
     s_ms, s_n, s_bytes = rlt.rlt_profile_read(model, 1)
     rlt.rlt_profile_enable(model, False)
+    rlt.rlt_check_device()
+
+    # end-to-end pass through the public API with host copies in the timed region
+    if setup:
+        setup()
+        for _ in range(args.warmup):
+            step()
+        after_warmup()
     ms_e2e, _ = timed(step_e2e, args.steps)
     rlt.rlt_check_device()
 
-    # the library times the attention launches of every 4th position; scale
-    # the sampled time up to all launches of the timed steps for the share
-    L = w["n_layers"]
-    if kind == "replay":
-        n_prefix = n_swa = L * (w["prompt"] - 1) * args.steps
-    else:
-        n_dec = w["prompt"] + w["gen"] - 1
-        n_prefix = (L * n_dec + L * (w["gen"] - 1)) * args.steps
-        n_swa = L * n_dec * args.steps
     value = world * tokens_per_step * args.steps / (ms / 1e3)
     e2e = world * tokens_per_step * args.steps / (ms_e2e / 1e3)
-    roof = step_roofline(w, kind, peaks)
+    roof = step_roofline(w, kind, peaks, t_range)
     ms_step = ms / args.steps
-    achieved = (a_bytes / a_n) / ((a_ms / a_n) / 1e3) / 1e9 if a_n else None
+
+    def share(ms_sampled, n_sampled, per_step):
+        # mean sampled launch time x launches of one step / step time
+        return (ms_sampled / n_sampled) * per_step / ms_step if n_sampled else None
+
+    def gbs(nbytes, ms_sampled, n_sampled):
+        return (nbytes / n_sampled) / ((ms_sampled / n_sampled) / 1e3) / 1e9 if n_sampled else None
+
     return {
         "value": value, "ms_per_step": ms_step, "e2e": e2e, "h2d": h2d, "d2h": d2h, "launches": launches,
-        "clocks": clk, "attn": {"ms": a_ms, "n": a_n, "bytes": a_bytes, "gbs": achieved,
-                                "ms_all": a_ms * n_prefix / a_n if a_n else None},
-        "swa": {"ms": s_ms, "n": s_n, "bytes": s_bytes,
-                "gbs": (s_bytes / s_n) / ((s_ms / s_n) / 1e3) / 1e9 if s_n else None,
-                "ms_all": s_ms * n_swa / s_n if s_n else None},
+        "clocks": clk, "t_range": t_range,
+        "attn": {"ms": a_ms, "n": a_n, "bytes": a_bytes, "gbs": gbs(a_bytes, a_ms, a_n),
+                 "share": share(a_ms, a_n, launches_per_step[0])},
+        "swa": {"gbs": gbs(s_bytes, s_ms, s_n), "share": share(s_ms, s_n, launches_per_step[1])},
         "step_roofline": {"bound_ms": roof["bound_ms"], "frac": roof["bound_ms"] / ms_step},
         "tokens_per_step": tokens_per_step,
     }
@@ -357,26 +514,41 @@ def run_backward(args, w: dict, rank: int, world: int) -> dict:
 
 
 def read_traffic_ratio() -> tuple[float | None, str]:
-    """DRAM bytes per algorithmic byte of the prefix-attention kernel from the
-    committed ncu summary, with a note.  The summary records the SHA-1 of the
-    kernel's source file at capture time; if the source has changed since,
-    the counters no longer describe the kernel and the ratio is None."""
-    import hashlib
-    p = os.path.join(ROOT, "profiles", "prefix_attn_replay.md")
-    if not os.path.exists(p):
-        return None, "no ncu summary"
-    ratio, sha = None, None
-    for line in open(p):
-        if line.startswith("traffic_per_algorithmic_byte:"):
-            v = line.split(":", 1)[1].strip()
-            ratio = None if v in ("", "null") else float(v)
-        elif line.startswith("kernel_source_sha1:"):
-            sha = line.split(":", 1)[1].strip()
-    src = os.path.join(ROOT, "stateful_decoder_b200", "csrc", "attn_decode.cu")
+    """DRAM bytes per algorithmic byte of the prefix-attention kernel, from the
+    machine-readable record of the committed ncu capture.  The record holds
+    the SHA-1 of the kernel's source file at capture time; if the source has
+    changed since, the counters no longer describe the kernel and the ratio
+    is None."""
+    if not os.path.exists(TRAFFIC_FILE):
+        return None, "no ncu traffic record"
+    rec = json.load(open(TRAFFIC_FILE)).get("prefix_attn")
+    if not rec:
+        return None, "no ncu traffic record for prefix_attn"
+    src = os.path.join(ROOT, rec["source"])
     now = hashlib.sha1(open(src, "rb").read()).hexdigest()
-    if sha != now:
-        return None, "kernel source changed since the ncu capture in profiles/prefix_attn_replay.md"
-    return ratio, "from profiles/prefix_attn_replay.md, scaled to the mean timed launch"
+    if rec["source_sha1"] != now:
+        return None, "kernel source changed since the ncu capture"
+    return rec["traffic_per_algorithmic_byte"], (f"ncu capture ({rec['case']}): DRAM bytes / algorithmic bytes, "
+                                                 f"scaled to the mean profiled launch")
+
+
+def config_desc(args, w: dict, kind: str, world: int) -> dict:
+    if kind == "replay":
+        tokens, schedule = w["prompt"], "replay (teacher-forced)"
+    elif kind == "generate":
+        tokens, schedule = f"{w['prompt']}+{w['gen']}", "prefill + sampled generation"
+    else:
+        a = w["prompt"] + w["block"] * args.warmup + 1
+        b = w["prompt"] + w["block"] * (args.warmup + args.steps)
+        tokens = f"prompt {w['prompt']} prefilled untimed; step = {w['block']} sampled transitions; timed t={a}..{b}"
+        schedule = "sampled generation (encoder step + memory append + transition + readout/sampler per token)"
+    return {"workload": args.workload, "d": w["d"], "n_heads": w["n_heads"],
+            "layers": f"{w['n_layers']}+{w['n_layers']}", "window": w["window"], "groups": w["groups"],
+            "ffn": w["ffn"], "vocab": w["vocab"], "batch_per_gpu": w["batch"], "global_batch": w["batch"] * world,
+            "tokens": tokens, "schedule": schedule, "merge": "paper eqs. 2.9-2.11",
+            "sampler": f"temperature {synth.TEMPERATURE}, top-k {synth.TOP_K}" if kind != "replay" else None,
+            "l2": "inputs larger than L2 (KV state of tens of GB read per transition)",
+            "parallelism": f"dp{world} (independent sequences, no collective)"}
 
 
 def main():
@@ -384,7 +556,7 @@ def main():
     ap.add_argument("--gpus", type=int, default=1)
     ap.add_argument("--steps", type=int, default=3)
     ap.add_argument("--warmup", type=int, default=3)
-    ap.add_argument("--workload", default="replay", choices=sorted(BENCH_WORKLOADS))
+    ap.add_argument("--workload", default=DEFAULT_WORKLOAD, choices=sorted(BENCH_WORKLOADS))
     ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
     ap.add_argument("--no-cpu-baseline", action="store_true")
     args = ap.parse_args()
@@ -394,37 +566,39 @@ def main():
     wname, over, kind = BENCH_WORKLOADS[args.workload]
     w = synth.workload(wname, **over)
     peaks = load_peaks()
-    cfg_desc = {"workload": args.workload, "d": w["d"], "n_heads": w["n_heads"], "layers": f"{w['n_layers']}+{w['n_layers']}",
-                "window": w["window"], "groups": w["groups"], "ffn": w["ffn"], "vocab": w["vocab"],
-                "batch_per_gpu": w["batch"], "global_batch": w["batch"] * world,
-                "tokens": w["prompt"] if kind == "replay" else f"{w['prompt']}+{w['gen']}",
-                "schedule": "replay (teacher-forced)" if kind == "replay" else "prefill + sampled generation",
-                "merge": "paper eqs. 2.9-2.11", "l2": "inputs larger than L2 (KV state of several GB per step)",
-                "parallelism": f"dp{world} (independent sequences, no collective)"}
+    cfg_desc = config_desc(args, w, kind, world)
+    metric = BPTT_METRIC if kind == "backward" else metric_name(w, kind)
 
     if args.impl == "reference":
         # the reference arm is the fp64 oracle on the host cores (rank 0 only)
         if rank != 0:
             return
-        n_tok = oracle_tokens_for(w)
-        sample = oracle_sample
-        if kind == "backward":
-            n_tok, sample = min(n_tok, 16), oracle_bptt_sample
-        for _ in range(args.warmup):
-            sample(w, n_tok)
         vals = []
-        t0 = time.perf_counter()
-        for i in range(args.steps):
-            v, cores, desc = sample(w, n_tok, seed_seq=i)
-            vals.append(v)
+        if kind == "backward":
+            n_tok = min(oracle_tokens_for(w), 16)
+            for _ in range(args.warmup):
+                oracle_bptt_sample(w, n_tok)
+            t0 = time.perf_counter()
+            for i in range(args.steps):
+                v, cores, desc = oracle_bptt_sample(w, n_tok, seed_seq=i)
+                vals.append(v)
+        else:
+            om = oracle_model(w)
+            for _ in range(args.warmup):
+                oracle_sample(w, kind, om)
+            t0 = time.perf_counter()
+            for i in range(args.steps):
+                v, cores, desc = oracle_sample(w, kind, om, seed_seq=i)
+                vals.append(v)
         dt = time.perf_counter() - t0
         value = statistics.mean(vals)
         print(json.dumps({
-            "impl": "reference", "metric": BPTT_METRIC if kind == "backward" else METRIC, "value": value, "unit": "tokens/s", "n_gpus": args.gpus,
+            "impl": "reference", "metric": metric, "value": value, "unit": "tokens/s", "n_gpus": args.gpus,
             "steps": args.steps, "warmup": args.warmup, "ms_per_step": dt * 1e3 / args.steps,
             "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "f64", "data": "synthetic",
             "config": cfg_desc,
-            "cpu_baseline": {"value": value, "unit": "tokens/s", "cores": cores, "kind": "oracle", "sample": desc},
+            "cpu_baseline": {"value": value, "unit": "tokens/s", "cores": cores, "kind": "oracle", "sample": desc,
+                             "cpu": cpu_model()},
             "e2e": {"value": value, "unit": "tokens/s", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0},
         }), flush=True)
         return
@@ -458,9 +632,9 @@ def main():
 
     cpu = None
     if rank == 0 and world == 1 and not args.no_cpu_baseline:
-        n_tok = oracle_tokens_for(w)
-        v, cores, desc = oracle_sample(w, n_tok)
-        cpu = {"value": v, "unit": "tokens/s", "cores": cores, "kind": "oracle", "sample": desc}
+        om = oracle_model(w)
+        v, cores, desc = oracle_sample(w, kind, om)
+        cpu = {"value": v, "unit": "tokens/s", "cores": cores, "kind": "oracle", "sample": desc, "cpu": cpu_model()}
 
     if world > 1:
         import torch.distributed as dist
@@ -472,19 +646,20 @@ def main():
     a = r["attn"]
     traffic = ratio * (a["bytes"] / a["n"]) if (ratio is not None and a["n"]) else None
     line = {
-        "metric": METRIC, "value": r["value"], "unit": "tokens/s", "n_gpus": world, "steps": args.steps,
+        "metric": metric, "value": r["value"], "unit": "tokens/s", "n_gpus": world, "steps": args.steps,
         "warmup": args.warmup, "ms_per_step": r["ms_per_step"], "higher_is_better": True, "scaling": "weak",
         "vs_baseline": None, "dtype": "bf16", "data": "synthetic (seeded Zipf(1.1) token ids, random-init weights)",
         "config": cfg_desc,
-        "roofline": {"bound": "hbm", "kernel": "prefix_attn (cross-attention over M_<=t)",
+        "roofline": {"bound": "hbm",
+                     "kernel": "prefix_attn (encoder step over C^E and cross-attention over M_<=t)",
                      "achieved": a["gbs"], "peak": peaks["hbm_gbs"], "unit": "GB/s",
                      "frac": (a["gbs"] / peaks["hbm_gbs"]) if a["gbs"] else None, "traffic": traffic,
                      "traffic_note": traffic_note,
                      "peak_source": peaks["source"] + " (copy bandwidth)",
-                     "timed_launches": a["n"], "sampling": "launches at every 4th position, CUDA events",
-                     "share_of_step": a["ms_all"] / (r["ms_per_step"] * args.steps) if a["ms_all"] else None},
-        "swa_attn": {"achieved_gbs": r["swa"]["gbs"],
-                     "share_of_step": r["swa"]["ms_all"] / (r["ms_per_step"] * args.steps) if r["swa"]["ms_all"] else None},
+                     "profiled_launches": a["n"],
+                     "sampling": f"separate untimed pass: launches at every {PROFILE_STRIDE}th position, CUDA events",
+                     "share_of_step": a["share"]},
+        "swa_attn": {"achieved_gbs": r["swa"]["gbs"], "share_of_step": r["swa"]["share"]},
         "step_roofline": r["step_roofline"],
         "cpu_baseline": cpu,
         "e2e": {"value": r["e2e"], "unit": "tokens/s", "h2d_bytes_per_step": r["h2d"], "d2h_bytes_per_step": r["d2h"]},

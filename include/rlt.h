@@ -403,6 +403,17 @@ int32_t rlt_check_device(void);
  * every attended position, plus the SWA insert). */
 int32_t rlt_profile_enable(rlt_model* m, int32_t on);
 
+/* Test hook of the failure detection above (the report has no counterpart):
+ * launches one block whose thread waits, through the same bounded mbarrier
+ * wait the tensor-core kernels use, on a barrier that no thread ever arrives
+ * at, with a limit of limit_us microseconds (1..1000000) instead of the
+ * kernels' 2 s.  The wait runs out, the kernel returns and the device error
+ * word is set: the next rlt_check_device() reports RLT_E_CUDA ("a bounded
+ * device wait ran out") and clears it; the context stays usable.
+ * Synchronises `stream`; *waited_ns receives how long the wait lasted.
+ * Errors: RLT_E_INVAL, RLT_E_CUDA. */
+int32_t rlt_test_bounded_wait(uint32_t limit_us, uint64_t* waited_ns, void* stream);
+
 /* Number of kernel launches the library has issued since it was loaded
  * (host-side counter, all devices and threads). */
 int32_t rlt_kernel_launches(int64_t* count);

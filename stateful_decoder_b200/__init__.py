@@ -45,7 +45,7 @@ EXPORTED = (
     "rlt_last_error", "rlt_check_device", "rlt_profile_enable", "rlt_profile_read", "rlt_op_linear",
     "rlt_op_sample", "rlt_kernel_launches", "rlt_op_prefix_attention", "rlt_op_prefix_attention_noalloc",
     "rlt_state_export", "rlt_state_import", "rlt_replay_ratios", "rlt_replay_backward", "rlt_grad_read",
-    "rlt_grad_zero",
+    "rlt_grad_zero", "rlt_test_bounded_wait",
 )
 
 
@@ -114,6 +114,7 @@ _sig = {
     "rlt_last_error": [ctypes.c_char_p, ctypes.c_size_t],
     "rlt_check_device": [],
     "rlt_kernel_launches": [ctypes.POINTER(ctypes.c_int64)],
+    "rlt_test_bounded_wait": [ctypes.c_uint32, ctypes.POINTER(ctypes.c_uint64), _vp],
     "rlt_profile_enable": [_vp, _i32],
     "rlt_profile_read": [_vp, _i32, ctypes.POINTER(ctypes.c_double), ctypes.POINTER(ctypes.c_int64),
                          ctypes.POINTER(ctypes.c_double)],
@@ -410,6 +411,15 @@ def rlt_op_sample(logits, sampling: dict, t: int, token, logp=None, logmu=None, 
 
 def rlt_check_device() -> None:
     _check(_lib.rlt_check_device())
+
+
+def rlt_test_bounded_wait(limit_us: int, stream=None) -> int:
+    """Runs the failure-detection probe (a bounded wait that cannot complete)
+    and returns how long it waited, in ns; the device error word is left set
+    for rlt_check_device to report."""
+    n = ctypes.c_uint64()
+    _check(_lib.rlt_test_bounded_wait(limit_us, ctypes.byref(n), _stream(stream)))
+    return n.value
 
 
 def rlt_kernel_launches() -> int:

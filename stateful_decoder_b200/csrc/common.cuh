@@ -182,7 +182,7 @@ __device__ __forceinline__ void mbar_arrive_expect_tx(uint32_t bar, uint32_t byt
 }
 // Bounded wait for the completion of the phase with the given parity.
 // Returns false (and raises the device error word) when the limit runs out.
-__device__ __forceinline__ bool mbar_wait(uint32_t bar, uint32_t parity) {
+__device__ __forceinline__ bool mbar_wait(uint32_t bar, uint32_t parity, uint64_t limit_ns = kWaitLimitNs) {
   uint64_t t0 = 0;
   for (uint32_t it = 0;; ++it) {
     uint32_t ok;
@@ -195,7 +195,7 @@ __device__ __forceinline__ bool mbar_wait(uint32_t bar, uint32_t parity) {
         : "memory");
     if (ok) return true;
     if (it == 0) t0 = globaltimer_ns();
-    else if ((it & 255u) == 0 && globaltimer_ns() - t0 > kWaitLimitNs) break;
+    else if ((it & 255u) == 0 && globaltimer_ns() - t0 > limit_ns) break;
   }
   atomicExch(&g_device_error, 1);
   return false;

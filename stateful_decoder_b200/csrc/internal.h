@@ -136,6 +136,11 @@ cudaError_t sample_topk(const float* logits, int B, int V, float temperature, in
 
 cudaError_t copy_f32(float* dst, const float* src, int64_t n, cudaStream_t st);
 
+// Failure-detection probe: one bounded mbarrier wait that can never complete
+// runs out after limit_ns and raises the device error word; synchronises
+// `st` and returns how long the wait lasted.
+cudaError_t bounded_wait_probe(uint64_t limit_ns, uint64_t* waited_ns, cudaStream_t st);
+
 // dst[b][:] = src[:] (fp32) for b < B
 template <typename WT>
 cudaError_t broadcast_row(const WT* src, int d, float* dst, int B, cudaStream_t st);

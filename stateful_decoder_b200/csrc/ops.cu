@@ -13,6 +13,8 @@
 namespace rlt {
 
 __device__ int g_device_error = 0;
+// Time the last bounded_wait_probe launch waited (ns), for the host to read.
+__device__ unsigned long long g_probe_waited_ns = 0;
 
 namespace {
 std::atomic<int64_t> g_launches{0};
@@ -567,5 +569,36 @@ RLT_INST_W(float)
 RLT_INST_W(bf16)
 template cudaError_t head_scatter<bf16, bf16>(const bf16*, int64_t, int64_t, int64_t, int, int, int, int, int, int,
                                               const float*, bf16*, int64_t, cudaStream_t);
+
+// ------------------------------------------------------------------ failure-detection probe
+namespace {
+// One thread waits on an mbarrier that expects one arrival which no thread
+// ever makes, so the bounded wait must run out after limit_ns: the same
+// mbar_wait the tensor-core kernels use, which then raises the device error
+// word and returns instead of spinning on.
+__global__ void bounded_wait_probe_kernel(uint64_t limit_ns) {
+  __shared__ __align__(8) uint64_t bar;
+  if (threadIdx.x != 0) return;
+  const uint32_t b = smem_u32(&bar);
+  mbar_init(b, 1);
+  fence_mbar_init();
+  const uint64_t t0 = globaltimer_ns();
+  const bool ok = mbar_wait(b, 0, limit_ns);
+  g_probe_waited_ns = ok ? 0ull : (unsigned long long)(globaltimer_ns() - t0);
+}
+}  // namespace
+
+cudaError_t bounded_wait_probe(uint64_t limit_ns, uint64_t* waited_ns, cudaStream_t st) {
+  bounded_wait_probe_kernel<<<1, 32, 0, st>>>(limit_ns);
+  note_launch();
+  cudaError_t e = cudaGetLastError();
+  if (e != cudaSuccess) return e;
+  e = cudaStreamSynchronize(st);
+  if (e != cudaSuccess) return e;
+  unsigned long long v = 0;
+  e = cudaMemcpyFromSymbol(&v, g_probe_waited_ns, sizeof(v));
+  *waited_ns = v;
+  return e;
+}
 
 }  // namespace rlt

@@ -1254,18 +1254,33 @@ const View* bptt_view(const rlt_model* m, const bptt::Dims& D, int i) {
   return it == m->views.end() ? nullptr : &it->second;
 }
 
-int32_t ensure_grads(rlt_model* m, const bptt::Dims& D) {
+// Allocates the model's gradient buffers on first use and zeroes them on the
+// caller's stream `st`, so the zeroing is ordered before the backward that
+// accumulates into them on the same stream.  The buffers join the model's
+// allocations only once all exist; a failure part-way frees those already
+// made, so a retry starts clean.
+int32_t ensure_grads(rlt_model* m, const bptt::Dims& D, cudaStream_t st) {
   if (!m->grad.empty()) return RLT_OK;
   const int n = bptt::n_tensors(D);
   std::vector<float*> g(n, nullptr);
-  for (int i = 0; i < n; ++i) {
+  std::vector<void*> made;
+  int32_t r = RLT_OK;
+  for (int i = 0; i < n && r == RLT_OK; ++i) {
     const View* v = bptt_view(m, D, i);
     if (!v) continue;
     void* p = nullptr;
-    RLT_TRY(dev_alloc(m->allocs, &p, (size_t)(v->rows * v->cols) * 4));
-    RLT_CUDA(cudaMemset(p, 0, (size_t)(v->rows * v->cols) * 4));
+    r = dev_alloc(made, &p, (size_t)(v->rows * v->cols) * 4);
+    if (r != RLT_OK) break;
+    const cudaError_t e = cudaMemsetAsync(p, 0, (size_t)(v->rows * v->cols) * 4, st);
+    if (e != cudaSuccess) r = fail(RLT_E_CUDA, std::string("zeroing a gradient: ") + cudaGetErrorString(e));
     g[i] = static_cast<float*>(p);
   }
+  if (r != RLT_OK) {
+    cudaStreamSynchronize(st);
+    free_all(made);
+    return r;
+  }
+  m->allocs.insert(m->allocs.end(), made.begin(), made.end());
   m->grad = g;
   return RLT_OK;
 }
@@ -1290,7 +1305,7 @@ int32_t rlt_replay_backward(rlt_model* m, const int32_t* tok_dev, int32_t B, int
       if (v < 0 || v >= m->cfg.vocab) return fail(RLT_E_INVAL, "token id " + std::to_string(v) + " out of range");
   }
   const bptt::Dims D = bptt_dims(m, B, S);
-  RLT_TRY(ensure_grads(m, D));
+  RLT_TRY(ensure_grads(m, D, st));
   // fp32 copies of the current weights, freed before returning
   const int n = bptt::n_tensors(D);
   std::vector<float*> w32(n, nullptr);
@@ -1368,6 +1383,12 @@ int32_t rlt_check_device(void) {
     RLT_CUDA(cudaMemcpyToSymbol(rlt::g_device_error, &z, sizeof(int)));
     return fail(RLT_E_CUDA, v == 1 ? "a bounded device wait ran out" : "a token id was out of range");
   }
+  return ok();
+}
+
+int32_t rlt_test_bounded_wait(uint32_t limit_us, uint64_t* waited_ns, void* stream) {
+  if (!waited_ns || limit_us < 1 || limit_us > 1000000u) return fail(RLT_E_INVAL, "limit_us must be in 1..1000000");
+  RLT_CUDA(bounded_wait_probe((uint64_t)limit_us * 1000ull, waited_ns, (cudaStream_t)stream));
   return ok();
 }
 

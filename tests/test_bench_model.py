@@ -2,9 +2,11 @@
 workload: the mean bytes one decoder transition must move are the weights
 (about 3.03 GB at bf16) plus the ring, the cross-attention memory reads and
 the ring insert (about 37.1 GB averaged over t = 1..1023), which at the
-measured copy bandwidth is about 6.1 ms per transition.  Also checks that the
-bound scales with the work it counts, and that the reported DRAM traffic is
-taken from an ncu summary only while the kernel source is the one captured."""
+measured copy bandwidth is about 6.1 ms per transition.  The generation block
+of the reference-depth model adds the encoder step's cache read.  Also checks
+that the bound scales with the work it counts, that the metric string names
+the model that ran, and that the reported DRAM traffic is taken from the ncu
+record only while the kernel source is the one captured."""
 import bench
 import synth
 
@@ -38,10 +40,38 @@ def test_bound_grows_with_work():
     assert bench.step_roofline(g, "generate", PEAKS)["decoder_transitions"] == g["prompt"] + g["gen"] - 1
 
 
+def test_generation_block_bound():
+    """One block of 32 generation transitions of the 48+48 model at B = 128:
+    weights of the decoder transition and of the encoder step (10.8 GB),
+    plus per position t the ring (255 entries once t > 256), the memory and
+    encoder-cache reads of t positions and the inserts.  At t = 2400 that
+    is about 256 GB, so about 39 ms per transition."""
+    w = synth.workload("refdepth", block=32)
+    d, L, F, V, B = w["d"], w["n_layers"], w["ffn"], w["vocab"], w["batch"]
+    weights = 2 * (L * (6 * d * d + 3 * d * F) + 3 * d * d + V * d) + 2 * (L * (4 * d * d + 3 * d * F) + 2 * d * d)
+    assert abs(weights / 1e9 - 10.8) < 0.1
+    r = bench.step_roofline(w, "block", PEAKS, (2385, 2416))
+    assert r["decoder_transitions"] == 32
+    kv = sum(B * 4 * d * (L * 255 + L + L * t + L * t + L + 1) for t in range(2385, 2417))
+    assert abs(r["bound_ms"] - (32 * weights + kv) / 6557.8e9 * 1e3) < 1e-6 * r["bound_ms"]
+    assert 37 * 32 < r["bound_ms"] < 41 * 32
+    # the mean over several blocks is per block
+    r2 = bench.step_roofline(w, "block", PEAKS, (2385, 2448))
+    assert r["bound_ms"] < r2["bound_ms"] < 1.05 * r["bound_ms"]
+
+
+def test_metric_names_the_model_that_ran():
+    assert bench.metric_name(synth.workload("refdepth"), "block") == \
+        "RLT decoder tokens/s (B seqs, 48+48 tied) on 1 B200; % of step roofline"
+    name = bench.metric_name(synth.workload("replay"), "replay")
+    assert "24+24" in name and "48+48" not in name
+
+
 def test_traffic_ratio_only_for_the_captured_source(tmp_path, monkeypatch):
-    """roofline.traffic comes from the committed ncu summary only while the
+    """roofline.traffic comes from the committed ncu record only while the
     kernel source still has the SHA-1 recorded at capture time."""
     import hashlib
+    import json
 
     import bench
     (tmp_path / "profiles").mkdir()
@@ -49,9 +79,12 @@ def test_traffic_ratio_only_for_the_captured_source(tmp_path, monkeypatch):
     src.mkdir(parents=True)
     (src / "attn_decode.cu").write_bytes(b"// kernel v1\n")
     sha = hashlib.sha1(b"// kernel v1\n").hexdigest()
-    (tmp_path / "profiles" / "prefix_attn_replay.md").write_text(
-        f"x\ntraffic_per_algorithmic_byte: 1.015\nkernel_source_sha1: {sha}\n")
+    rec = tmp_path / "profiles" / "traffic.json"
+    rec.write_text(json.dumps({"prefix_attn": {"source": "stateful_decoder_b200/csrc/attn_decode.cu",
+                                               "source_sha1": sha, "traffic_per_algorithmic_byte": 1.015,
+                                               "case": "test"}}))
     monkeypatch.setattr(bench, "ROOT", str(tmp_path))
+    monkeypatch.setattr(bench, "TRAFFIC_FILE", str(rec))
     assert bench.read_traffic_ratio()[0] == 1.015
     (src / "attn_decode.cu").write_bytes(b"// kernel v2\n")
     ratio, note = bench.read_traffic_ratio()

@@ -81,3 +81,33 @@ def test_backward_accumulates_and_zeroes(rlt):
         rlt.rlt_replay_backward(m, bad, wts, segment=2)
     assert e.value.code == rlt.RLT_E_INVAL and "out of range" in str(e.value)
     rlt.rlt_check_device()
+
+
+def test_backward_on_a_side_stream(rlt, oracle_lib):
+    """The first backward of a model zeroes the fresh gradient buffers on the
+    caller's stream: run on a non-blocking side stream, its gradients still
+    equal the oracle's."""
+    import torch
+
+    from oracle import bptt
+    w = synth.workload("tiny", d=32, n_heads=2, ffn=48, vocab=40, prompt=9)
+    cfg = synth.model_config(w)
+    m = rlt.rlt_init_weights(cfg, synth.WEIGHT_SEED)
+    tok = synth.tokens(w, batch=2)
+    wts = np.full((2, 8), 0.125, dtype=np.float32)
+    side = torch.cuda.Stream()
+    with torch.cuda.stream(side):
+        t = torch.from_numpy(tok).cuda(non_blocking=False)
+        wd = torch.from_numpy(wts).cuda(non_blocking=False)
+        side.synchronize()
+        rlt.rlt_replay_backward(m, t, wd, segment=3, stream=side)
+    side.synchronize()
+    om = oracle_lib.Model(cfg, seed=synth.WEIGHT_SEED)
+    want = None
+    for b in range(2):
+        _, g = bptt.loss_and_grads(om, tok[b], wts[b].astype(np.float64))
+        want = g if want is None else {k: want[k] + g[k] for k in want}
+    for name in ("emb", "s_star", "w_gate", "wq.0", "w2.1", "w_out"):
+        ref = want[name]
+        assert np.max(np.abs(m.grad(name) - ref)) <= 1e-4 * float(np.max(np.abs(ref))) + 1e-6, name
+    rlt.rlt_check_device()

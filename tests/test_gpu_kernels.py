@@ -1,7 +1,7 @@
 """Kernel-level numerics of the decode attention (eq. 2.15 / eq. 2.8) against
 a plain PyTorch fp32 reference of the same operation, through the C ABI's
 op-level entry point.  Cases span one key, exact chunk boundaries (256),
-ragged tails, several chunks, head sizes 16/64/128 and both storage types,
+ragged tails, several chunks, head sizes 16/64/128/256 and both storage types,
 with and without the rotary map on the query."""
 import math
 
@@ -46,6 +46,8 @@ CASES = [  # B, H, hd, n, ld_t, dtype, rope
     (5, 2, 64, 700, 1024, "bf16", True),
     (1, 16, 128, 1023, 1024, "bf16", True),
     (2, 4, 16, 513, 600, "f32", True),
+    (2, 2, 256, 300, 320, "bf16", True),
+    (3, 1, 256, 100, 128, "f32", False),
 ]
 
 
