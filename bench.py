@@ -474,6 +474,17 @@ def run_gpu(args, w: dict, kind: str, peaks: dict, rank: int, world: int) -> dic
     }
 
 
+def backward_flops(w: dict, B: int, S: int) -> float:
+    """Contraction FLOPs of one full-BPTT call (rlt_replay_backward) over B
+    sequences of S tokens: the encoder and memory projection forward once and
+    backward once (dX and dW: twice the forward), the S-1 decoder transitions
+    forward twice (the sweep and the segment recompute) and backward once
+    (dX and dW)."""
+    p_dec, p_enc = params(w)
+    n = B * S
+    return 2.0 * n * p_enc * 3 + 2.0 * B * (S - 1) * p_dec * 4
+
+
 def run_backward(args, w: dict, rank: int, world: int) -> dict:
     """Times rlt_replay_backward (eq. 5.1 weights) over the workload's token
     ids, already resident on the device: K calls after W warm-up calls."""
@@ -612,6 +623,12 @@ def main():
 
     if kind == "backward":
         r = run_backward(args, w, rank, world)
+        fl = backward_flops(w, r["B"], r["S"])
+        tf = fl / (r["ms_per_step"] / 1e3) / 1e12
+        pk = peaks["bf16_tflops_sustained"]
+        roof = {"bound": "tensor", "kernel": "whole backward: contraction FLOPs at the bf16 tensor peak",
+                "flops_per_step": fl, "achieved": tf, "peak": pk, "unit": "TFLOP/s", "frac": tf / pk,
+                "traffic": None, "peak_source": peaks["source"] + " (sustained bf16 GEMM)"}
         if world > 1:
             import torch.distributed as dist
             dist.barrier()
@@ -620,12 +637,13 @@ def main():
             print(json.dumps({
                 "metric": BPTT_METRIC, "value": r["value"], "unit": "tokens/s", "n_gpus": world,
                 "steps": args.steps, "warmup": args.warmup, "ms_per_step": r["ms_per_step"],
-                "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "f32",
+                "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "bf16",
                 "data": "synthetic (seeded Zipf(1.1) token ids, random-init weights)",
                 "config": dict(cfg_desc, tokens=r["S"], schedule=f"full BPTT, segments of {BPTT_SEGMENT}",
-                               objective="eq. 5.1 weights"),
-                "roofline": None, "note": "first backward engine (CUDA-core functor kernels), not yet characterised",
-                "gpu_launches": r["launches"], "clocks": r["clocks"]}), flush=True)
+                               objective="eq. 5.1 weights",
+                               arithmetic="contractions on tcgen05 with bf16 operands, fp32 accumulation; "
+                                          "attention, norms and elementwise adjoints on CUDA cores in fp32"),
+                "roofline": roof, "gpu_launches": r["launches"], "clocks": r["clocks"]}), flush=True)
         return
 
     r = run_gpu(args, w, kind, peaks, rank, world)

@@ -34,8 +34,12 @@
  *  - A state remembers the model version it was built under.  Loading weights
  *    bumps the version; using an older state then fails with RLT_E_STALE
  *    (report §5.4 and App. C: caches built under other weights are invalid).
- *  - All sequences of one state advance in lock step (report §4.1 batching of
- *    ready transitions): they share positions n_enc and n_dec.
+ *  - Every sequence of a state has its own positions n_enc[b] and n_dec[b]
+ *    (report §4.1: the batch gathers ready transitions of independent
+ *    sequences, each with its own memory, cache, s and position).  A
+ *    transition advances every sequence of the batch by one, each at its own
+ *    position; rlt_append_spans appends spans of different lengths and lets
+ *    each sequence sit out the transitions its span does not need.
  *  - A model and its states are used from one host thread at a time: calls
  *    on one model, or on its states, must not overlap across threads (the
  *    model holds the state of rlt_replay_logprobs and the profiling record).
@@ -107,16 +111,19 @@ typedef struct rlt_readout_out {
   float* logits;        /* [B, V] raw logits */
 } rlt_readout_out;
 
-/* State inspection (test hooks, report §6 snapshot contents). */
+/* State inspection (test hooks, report §6 snapshot contents).  The position
+ * fields are those of the furthest sequence; rlt_state_positions gives every
+ * sequence's own. */
 typedef struct rlt_state_info {
   int32_t batch, max_len;
-  int32_t n_enc;        /* tokens encoded: e_1..e_n_enc and M_<=n_enc exist */
-  int32_t n_dec;        /* decoder transitions applied: the state is H_n_dec */
+  int32_t n_enc;        /* tokens encoded: e_1..e_n_enc and M_<=n_enc exist (maximum over sequences) */
+  int32_t n_dec;        /* decoder transitions applied: the state is H_n_dec (maximum over sequences) */
   int32_t ring_valid;   /* retained SWA entries per layer: min(n_dec, W-1) */
   int32_t ring_head;    /* slot the next transition writes: n_dec mod (W-1), 0 if W = 1 */
   int32_t has_encoder_cache;
   uint64_t model_version;
   int32_t has_pending;  /* a sampled x_{t+1} awaits its transition (App. A, pending token) */
+  int32_t uniform;      /* 1: every sequence stands at the same n_enc and n_dec */
 } rlt_state_info;
 
 #define RLT_STATE_ENCODER_CACHE 1   /* keep C^E (needed for incremental encoding, eq. 2.8) */
@@ -186,6 +193,14 @@ int32_t rlt_state_reset(rlt_state* s, void* stream);
 
 int32_t rlt_state_info_get(const rlt_state* s, rlt_state_info* out);
 
+/* Per-sequence positions (report §2.1, §4.1) into caller-owned host arrays
+ * of `batch` entries, each of which may be NULL: n_enc[b], n_dec[b], the
+ * retained SWA entries ring_valid[b] = min(n_dec[b], W-1) and the slot the
+ * next transition of sequence b writes, ring_head[b] = n_dec[b] mod (W-1)
+ * (0 if W = 1).  Errors: RLT_E_INVAL. */
+int32_t rlt_state_positions(const rlt_state* s, int32_t* n_enc, int32_t* n_dec, int32_t* ring_valid,
+                            int32_t* ring_head);
+
 /* Copies one state component to host memory (synchronous); layouts above. */
 int32_t rlt_state_read(const rlt_state* s, int32_t what, int32_t index, void* host, size_t bytes);
 
@@ -196,7 +211,10 @@ int32_t rlt_state_read(const rlt_state* s, int32_t what, int32_t index, void* ho
  * H_t = (s_t, C^D_t) with the whole SWA ring, the positions n_enc and n_dec,
  * the pending sampled token (App. A) if any, the model configuration
  * (window convention included) and the identity of the weights (generator
- * seed and model version).  bf16 models also store the readout operand the
+ * seed and model version).  The header holds the furthest sequence's
+ * positions and the rows up to them are stored for every sequence; when the
+ * sequences stand at different positions a last section holds n_enc[B] and
+ * n_dec[B] (int32).  bf16 models also store the readout operand the
  * last transition left (gamma_o * s_t in bf16 and its sums of squares), so
  * that a restored state reads out bit-identically.  Layout: a 120-byte
  * little-endian header ("RLTSNAP1") followed by the sections in that order.
@@ -221,7 +239,8 @@ int32_t rlt_state_import(rlt_state* s, const void* host, size_t bytes, void* str
 
 /* Token-parallel causal encoder (eq. 2.1) and memory projection (eq. 2.2) for
  * T tokens per sequence, tok_dev [B][T] int32 (row-major), placed at positions
- * n_enc+1..n_enc+T.  With n_enc > 0 the tokens attend to the encoded prefix
+ * n_enc+1..n_enc+T (every sequence must stand at the same n_enc, else
+ * RLT_E_STATE: rlt_append_spans takes spans at different positions).  With n_enc > 0 the tokens attend to the encoded prefix
  * through the encoder cache: the chunked schedule of App. A.2 (an appended
  * span -- a user turn or a tool result -- is encoded in one pass; every
  * token still receives its decoder transition through rlt_decoder_step).
@@ -230,18 +249,40 @@ int32_t rlt_state_import(rlt_state* s, const void* host, size_t bytes, void* str
  * RLT_E_INVAL. */
 int32_t rlt_encode_prefix(rlt_model* m, rlt_state* s, const int32_t* tok_dev, int32_t T, void* stream);
 
+/* Appends a span of lens[b] tokens to every sequence b (report §6 multi-turn
+ * serving: a user turn or tool result; App. A.1 prefill when the state is
+ * fresh): span b is tok_dev[b * ld_tok + 0 .. lens[b]-1] (int32, device),
+ * lens is a host array of B entries >= 0 (0: the sequence takes no part).
+ * Each span is encoded token-parallel over its sequence's cached prefix
+ * (eq. 2.1, the chunked schedule of App. A.2; runs of consecutive sequences
+ * with the same position and length share one pass), then every span token
+ * receives its decoder transition: max(lens) transitions in lock step, in
+ * which sequence b takes part only while its span lasts (its state is
+ * otherwise left unchanged).  If logp_dev != NULL, logp_dev[b * ld_logp + i]
+ * receives log p(span_b[i+1] | history) for i = 0..lens[b]-2 (other entries
+ * are not written).  Afterwards n_enc[b] = n_dec[b] = old + lens[b].
+ * Requires every encoded token to be consumed (n_enc[b] = n_dec[b]) and no
+ * pending sampled token; a non-empty span after an encoded prefix needs the
+ * encoder cache.  Copies lens to the device with an ordinary host copy, so
+ * the call waits for `stream` once.  Errors: RLT_E_INVAL, RLT_E_CAPACITY
+ * (n_enc[b] + lens[b] > max_len), RLT_E_STATE, RLT_E_STALE. */
+int32_t rlt_append_spans(rlt_model* m, rlt_state* s, const int32_t* tok_dev, int64_t ld_tok, const int32_t* lens,
+                         float* logp_dev, int64_t ld_logp, void* stream);
+
 /* Readout of the current s_t (eq. 2.6): log p of next_dev [B] (may be NULL),
- * and/or a sample from the behaviour sampler (samp may be NULL).  A sample
- * is also recorded in the state as the pending token x_{t+1} (App. A): the
- * state represents the consumed prefix only, and the next rlt_decoder_step
- * consumes the pending token when it is given no tokens.  Requires
- * n_dec >= 1. */
+ * and/or a sample from the behaviour sampler (samp may be NULL; its counter
+ * position t is each sequence's own n_dec).  A sample is also recorded in
+ * the state as the pending token x_{t+1} (App. A): the state represents the
+ * consumed prefix only, and the next rlt_decoder_step consumes the pending
+ * token when it is given no tokens.  Requires n_dec[b] >= 1 for every
+ * sequence. */
 int32_t rlt_readout(rlt_model* m, rlt_state* s, const int32_t* next_dev, const rlt_sampling* samp,
                     const rlt_readout_out* out, void* stream);
 
-/* Consumes x_t for every sequence, t = n_dec+1 (App. A.2): if x_t is not yet
- * encoded (n_enc < t), runs the encoder step (eq. 2.8, needs the encoder
- * cache) and the memory append; then the merge and the L_D decoder blocks
+/* Consumes x_t for every sequence b, at its own t = n_dec[b]+1 (App. A.2):
+ * for the sequences whose x_t is not yet encoded (n_enc[b] < t), runs the
+ * encoder step (eq. 2.8, needs the encoder cache) and the memory append;
+ * then the merge and the L_D decoder blocks
  * (eqs. 2.4, 2.5, 2.12-2.16) with one SWA insert per layer; then the readout
  * as rlt_readout does (skipped when next_dev, samp and out are all NULL).
  * tok_dev [B] int32 is read only when the token is encoded here; NULL takes

@@ -20,6 +20,10 @@ shape of the workload's model but holds fewer layers' state.
       tokens of `batch` sequences (GEMMs with B*len activation rows, causal
       attention on the tensor cores).
 
+  python profile_case.py bptt --workload small --batch 16 --len 64 [--layers 2]
+      Profiles one full-BPTT backward (rlt_replay_backward, eq. 5.1 weights,
+      segments of 32) of `batch` sequences of `len` tokens.
+
   python profile_case.py summarize launches.csv [S]
       Per-kernel summary of an ncu launch list (gpu__time_duration.sum, --csv)
       captured with `--nvtx --nvtx-include "rlt_sample]"` on a replay of S
@@ -115,6 +119,24 @@ def encoder(args) -> None:
     print("profiled encoder over", args.batch, "x", args.len, "tokens")
 
 
+def bptt(args) -> None:
+    import torch
+
+    import synth
+    rlt, w, m = _model(args)
+    tok = torch.from_numpy(synth.tokens(w)).cuda()
+    B, S = tok.shape
+    wts = torch.full((B, S - 1), 1.0 / (B * (S - 1)), device="cuda")
+    rlt.rlt_replay_backward(m, tok, wts, segment=32)  # warm-up
+    torch.cuda.synchronize()
+    torch.cuda.cudart().cudaProfilerStart()
+    rlt.rlt_replay_backward(m, tok, wts, segment=32)
+    torch.cuda.synchronize()
+    torch.cuda.cudart().cudaProfilerStop()
+    rlt.rlt_check_device()
+    print("profiled backward over", B, "x", S, "tokens")
+
+
 def summarize(path: str, S: int) -> str:
     rows = list(csv.reader(open(path)))
     hdr_i = next(i for i, r in enumerate(rows) if "Kernel Name" in r)
@@ -164,6 +186,11 @@ def main() -> None:
     e.add_argument("--batch", type=int, default=4)
     e.add_argument("--len", type=int, default=2048)
     e.add_argument("--layers", type=int, default=0)
+    p = sub.add_parser("bptt")
+    p.add_argument("--workload", default="small")
+    p.add_argument("--batch", type=int, default=16)
+    p.add_argument("--len", type=int, default=64)
+    p.add_argument("--layers", type=int, default=0)
     b = sub.add_parser("summarize")
     b.add_argument("csv")
     b.add_argument("S", type=int, nargs="?", default=1024)
@@ -174,6 +201,8 @@ def main() -> None:
         gen(args)
     elif args.cmd == "encoder":
         encoder(args)
+    elif args.cmd == "bptt":
+        bptt(args)
     else:
         print(summarize(args.csv, args.S))
 

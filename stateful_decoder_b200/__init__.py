@@ -45,7 +45,7 @@ EXPORTED = (
     "rlt_last_error", "rlt_check_device", "rlt_profile_enable", "rlt_profile_read", "rlt_op_linear",
     "rlt_op_sample", "rlt_kernel_launches", "rlt_op_prefix_attention", "rlt_op_prefix_attention_noalloc",
     "rlt_state_export", "rlt_state_import", "rlt_replay_ratios", "rlt_replay_backward", "rlt_grad_read",
-    "rlt_grad_zero", "rlt_test_bounded_wait",
+    "rlt_grad_zero", "rlt_test_bounded_wait", "rlt_state_positions", "rlt_append_spans",
 )
 
 
@@ -78,7 +78,7 @@ class StateInfo(ctypes.Structure):
     _fields_ = [("batch", ctypes.c_int32), ("max_len", ctypes.c_int32), ("n_enc", ctypes.c_int32),
                 ("n_dec", ctypes.c_int32), ("ring_valid", ctypes.c_int32), ("ring_head", ctypes.c_int32),
                 ("has_encoder_cache", ctypes.c_int32), ("model_version", ctypes.c_uint64),
-                ("has_pending", ctypes.c_int32)]
+                ("has_pending", ctypes.c_int32), ("uniform", ctypes.c_int32)]
 
 
 _vp = ctypes.c_void_p
@@ -115,6 +115,8 @@ _sig = {
     "rlt_check_device": [],
     "rlt_kernel_launches": [ctypes.POINTER(ctypes.c_int64)],
     "rlt_test_bounded_wait": [ctypes.c_uint32, ctypes.POINTER(ctypes.c_uint64), _vp],
+    "rlt_state_positions": [_vp, _vp, _vp, _vp, _vp],
+    "rlt_append_spans": [_vp, _vp, _vp, ctypes.c_int64, _vp, _vp, ctypes.c_int64, _vp],
     "rlt_profile_enable": [_vp, _i32],
     "rlt_profile_read": [_vp, _i32, ctypes.POINTER(ctypes.c_double), ctypes.POINTER(ctypes.c_int64),
                          ctypes.POINTER(ctypes.c_double)],
@@ -238,6 +240,13 @@ class State:
         _check(_lib.rlt_state_info_get(self.h, ctypes.byref(i)))
         return {f: getattr(i, f) for f, _ in StateInfo._fields_}
 
+    def positions(self) -> dict:
+        """Per-sequence n_enc, n_dec, ring_valid and ring_head (int32 [B])."""
+        out = {k: np.zeros(self.batch, np.int32) for k in ("n_enc", "n_dec", "ring_valid", "ring_head")}
+        _check(_lib.rlt_state_positions(self.h, *(out[k].ctypes.data for k in ("n_enc", "n_dec", "ring_valid",
+                                                                                 "ring_head"))))
+        return out
+
     def read(self, what: int, index: int = 0) -> np.ndarray:
         c = self.model.cfg
         d, B, L = c["d"], self.batch, self.max_len
@@ -311,6 +320,26 @@ def _sampling(sampling):
     if sampling is None:
         return None
     return ctypes.byref(Sampling(temperature=sampling["temperature"], top_k=sampling["top_k"], seed=sampling["seed"]))
+
+
+def rlt_append_spans(model: Model, state: State, tokens, lens, logp=None, stream=None) -> None:
+    """Appends span b = tokens[b, :lens[b]] to every sequence b: tokens int32
+    CUDA tensor [B, L] (L >= max(lens)), lens host ints; logp (optional)
+    float32 CUDA tensor [B, L-1] receives log p(span_b[i+1] | history) for
+    i < lens[b]-1."""
+    B = state.batch
+    if tokens.dim() != 2 or tokens.shape[0] != B:
+        raise ValueError(f"expected tokens of shape [{B}, L]")
+    ln = np.ascontiguousarray(np.asarray(lens, dtype=np.int32))
+    if ln.shape != (B,):
+        raise ValueError(f"expected {B} span lengths")
+    ld = tokens.shape[1]
+    if logp is not None and (logp.dim() != 2 or logp.shape[0] != B):
+        raise ValueError(f"expected logp of shape [{B}, L-1]")
+    ld_lp = logp.shape[1] if logp is not None else 0
+    _check(_lib.rlt_append_spans(model.h, state.h, _dev(tokens, "torch.int32"), ld, ln.ctypes.data,
+                                 _dev(logp, "torch.float32", B * ld_lp) if logp is not None else None, ld_lp,
+                                 _stream(stream)))
 
 
 def rlt_readout(model: Model, state: State, next_tokens=None, sampling: dict | None = None, stream=None,

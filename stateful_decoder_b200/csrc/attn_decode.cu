@@ -102,13 +102,17 @@ __device__ __forceinline__ float2 softmax_inplace(float* sc, int n, float* red) 
 // ------------------------------------------------------------------ SWA
 template <typename KT, int HD>
 __global__ void __launch_bounds__(kThreads, 9) swa_attn_kernel(const float* __restrict__ qkv, int64_t ld_qkv, KT* ring_k,
-                                                            KT* ring_v, int H, int t, int W,
+                                                            KT* ring_v, int H, int t_all, SeqPos sp, int W,
                                                             const float* __restrict__ rope_cs, KT* out,
                                                             int64_t ld_out, float scale_log2) {
   // Dependents (the next GEMM) are released only once this block has issued
   // all its ring loads: released at the start, their CTAs would take SMs
   // (shared memory, registers) from the blocks of this HBM-bound kernel.
   griddep_wait();
+  // position of this sequence's transition; an idle sequence (masked phase)
+  // reads its ring but inserts nothing
+  const int t = sp.on() ? sp.dec[blockIdx.y] + 1 : t_all;
+  const bool insert = !sp.on() || sp.active(blockIdx.y);
   constexpr int LPK = HD / 8, KPW = 32 / LPK, NKG = (kThreads / 32) * KPW, HALF = HD / 2;
   extern __shared__ float sm[];
   float* sq = sm;            // rotated, scaled query
@@ -169,7 +173,7 @@ __global__ void __launch_bounds__(kThreads, 9) swa_attn_kernel(const float* __re
   }
   // Ring insert after every read of the ring above: the slot of position t is
   // the one that held t-W+1, which this step still attended to (§2.5).
-  if (Wm1 > 0) {
+  if (Wm1 > 0 && insert) {
     const int slot = (t - 1) % Wm1;
     for (int i = threadIdx.x; i < HD; i += kThreads) {
       kb[(int64_t)slot * HD + i] = from_f32<KT>(sk[i]);
@@ -182,9 +186,9 @@ __global__ void __launch_bounds__(kThreads, 9) swa_attn_kernel(const float* __re
 template <typename KT, int HD>
 __global__ void __launch_bounds__(kThreads) prefix_attn_kernel(const float* __restrict__ q, int64_t ld_q,
                                                                const KT* __restrict__ kc, const KT* __restrict__ vc,
-                                                               int64_t ld_t, int H, int n, int qpos,
-                                                               const float* __restrict__ rope_cs, KT* out,
-                                                               int64_t ld_out, float* ws, int nchunks,
+                                                               int64_t ld_t, int H, int n_all, int qpos_all,
+                                                               SeqPos sp, const float* __restrict__ rope_cs, KT* out,
+                                                               int64_t ld_out, float* ws, int nchunks, int* counters,
                                                                float scale_log2) {
   griddep_wait();  // dependents are released after the last K/V load, as in swa_attn_kernel
   constexpr int LPK = HD / 8, KPW = 32 / LPK, NKG = (kThreads / 32) * KPW, HALF = HD / 2;
@@ -194,6 +198,12 @@ __global__ void __launch_bounds__(kThreads) prefix_attn_kernel(const float* __re
   float* sc = red_o + NKG * HD;
   __shared__ float red[32];
   const int c = blockIdx.x, h = blockIdx.y, b = blockIdx.z;
+  // keys 0..n-1 of this sequence (its own position when the state has
+  // per-sequence positions); the grid covers the longest sequence
+  const int n = sp.on() ? sp.n_keys(b) : n_all;
+  const int qpos = sp.on() ? n - 1 : qpos_all;
+  const int nch = (n + kPrefixChunk - 1) / kPrefixChunk;
+  if (c >= nch) return;
   const int j0 = c * kPrefixChunk, j1 = min(n, j0 + kPrefixChunk);
   const float* qrow = q + (int64_t)b * ld_q + h * HD;
   if (rope_cs != nullptr) {
@@ -223,7 +233,7 @@ __global__ void __launch_bounds__(kThreads) prefix_attn_kernel(const float* __re
 #pragma unroll
   for (int i = 0; i < 8; ++i) red_o[kg * HD + sub * 8 + i] = o[i];
   __syncthreads();
-  if (nchunks == 1) {
+  if (nch == 1) {
     const float inv = 1.0f / ml.y;
     for (int i = threadIdx.x; i < HD; i += kThreads) {
       float acc = 0.f;
@@ -242,23 +252,59 @@ __global__ void __launch_bounds__(kThreads) prefix_attn_kernel(const float* __re
       po[HD] = ml.x;
       po[HD + 1] = ml.y;
     }
+    if (counters != nullptr) {
+      // The last of this (sequence, head)'s chunk blocks to finish combines
+      // the partials in chunk order (the arithmetic of
+      // prefix_combine_kernel, so the result does not depend on which block
+      // it is) and resets the counter for the next launch.
+      __shared__ int s_last;
+      __threadfence();
+      __syncthreads();
+      if (threadIdx.x == 0) {
+        const int prev = atomicAdd(&counters[b * H + h], 1);
+        s_last = prev == nch - 1;
+        if (s_last) counters[b * H + h] = 0;
+      }
+      __syncthreads();
+      if (s_last) {
+        __threadfence();
+        const float* p = ws + ((int64_t)b * H + h) * nchunks * (HD + 2);
+        float mx = -INFINITY;
+        for (int cc = 0; cc < nch; ++cc) mx = fmaxf(mx, __ldcg(p + cc * (HD + 2) + HD));
+        float l = 0.f;
+        for (int cc = 0; cc < nch; ++cc)
+          l += __ldcg(p + cc * (HD + 2) + HD + 1) * exp2f(__ldcg(p + cc * (HD + 2) + HD) - mx);
+        const float inv = 1.0f / l;
+        for (int i = threadIdx.x; i < HD; i += kThreads) {
+          float acc = 0.f;
+          for (int cc = 0; cc < nch; ++cc)
+            acc += __ldcg(p + cc * (HD + 2) + i) * exp2f(__ldcg(p + cc * (HD + 2) + HD) - mx);
+          out[(int64_t)b * ld_out + h * HD + i] = from_f32<KT>(acc * inv);
+        }
+      }
+    }
   }
 }
 
-// Combines the chunk partials of one (sequence, head) in chunk order.
+// Combines the chunk partials of one (sequence, head) in chunk order; a
+// sequence whose keys fit one chunk was finished by prefix_attn_kernel.
 template <typename KT, int HD>
-__global__ void prefix_combine_kernel(const float* __restrict__ ws, int H, int nchunks, KT* out, int64_t ld_out) {
+__global__ void prefix_combine_kernel(const float* __restrict__ ws, int H, int nchunks, int n_all, SeqPos sp, KT* out,
+                                      int64_t ld_out) {
   griddep_enter();
   const int h = blockIdx.x, b = blockIdx.y;
+  const int n = sp.on() ? sp.n_keys(b) : n_all;
+  const int nch = (n + kPrefixChunk - 1) / kPrefixChunk;
+  if (nch <= 1) return;
   const float* p = ws + ((int64_t)b * H + h) * nchunks * (HD + 2);
   float mx = -INFINITY;
-  for (int c = 0; c < nchunks; ++c) mx = fmaxf(mx, p[c * (HD + 2) + HD]);
+  for (int c = 0; c < nch; ++c) mx = fmaxf(mx, p[c * (HD + 2) + HD]);
   float l = 0.f;
-  for (int c = 0; c < nchunks; ++c) l += p[c * (HD + 2) + HD + 1] * exp2f(p[c * (HD + 2) + HD] - mx);
+  for (int c = 0; c < nch; ++c) l += p[c * (HD + 2) + HD + 1] * exp2f(p[c * (HD + 2) + HD] - mx);
   const float inv = 1.0f / l;
   for (int i = threadIdx.x; i < HD; i += blockDim.x) {
     float acc = 0.f;
-    for (int c = 0; c < nchunks; ++c) acc += p[c * (HD + 2) + i] * exp2f(p[c * (HD + 2) + HD] - mx);
+    for (int c = 0; c < nch; ++c) acc += p[c * (HD + 2) + i] * exp2f(p[c * (HD + 2) + HD] - mx);
     out[(int64_t)b * ld_out + h * HD + i] = from_f32<KT>(acc * inv);
   }
 }
@@ -269,7 +315,7 @@ constexpr int nkg_of() {
 }
 
 template <typename KT, int HD>
-cudaError_t swa_launch(const float* qkv, int64_t ld_qkv, KT* rk, KT* rv, int B, int H, int t, int W,
+cudaError_t swa_launch(const float* qkv, int64_t ld_qkv, KT* rk, KT* rv, int B, int H, int t, const SeqPos& sp, int W,
                        const float* rope_cs, KT* out, int64_t ld_out, cudaStream_t st) {
   const size_t smem = sizeof(float) * (3 * HD + nkg_of<HD>() * HD + W + 1);
   if (smem > 48 * 1024) {
@@ -278,7 +324,7 @@ cudaError_t swa_launch(const float* qkv, int64_t ld_qkv, KT* rk, KT* rv, int B, 
   }
   const float scale_log2 = 1.4426950408889634f / sqrtf((float)HD);
   {
-    const cudaError_t e_l = launch_pdl(swa_attn_kernel<KT, HD>, dim3(dim3(H, B)), dim3(kThreads), smem, st, qkv, ld_qkv, rk, rv, H, t, W, rope_cs, out, ld_out,
+    const cudaError_t e_l = launch_pdl(swa_attn_kernel<KT, HD>, dim3(dim3(H, B)), dim3(kThreads), smem, st, qkv, ld_qkv, rk, rv, H, t, sp, W, rope_cs, out, ld_out,
                                                                scale_log2);
     if (e_l != cudaSuccess) return e_l;
   }
@@ -287,21 +333,21 @@ cudaError_t swa_launch(const float* qkv, int64_t ld_qkv, KT* rk, KT* rv, int B, 
 
 template <typename KT, int HD>
 cudaError_t prefix_launch(const float* q, int64_t ld_q, const KT* k, const KT* v, int64_t ld_t, int B, int H, int n,
-                          int qpos, const float* rope_cs, KT* out, int64_t ld_out, float* ws, size_t ws_floats,
-                          cudaStream_t st) {
+                          int qpos, const SeqPos& sp, const float* rope_cs, KT* out, int64_t ld_out, float* ws,
+                          size_t ws_floats, int* counters, cudaStream_t st) {
   const int nchunks = (n + kPrefixChunk - 1) / kPrefixChunk;
   if (nchunks > 1 && (!ws || ws_floats < (size_t)B * H * nchunks * (HD + 2))) return cudaErrorInvalidValue;
   const size_t smem = sizeof(float) * (HD + nkg_of<HD>() * HD + kPrefixChunk);
   const float scale_log2 = 1.4426950408889634f / sqrtf((float)HD);
   {
-    const cudaError_t e_l = launch_pdl(prefix_attn_kernel<KT, HD>, dim3(dim3(nchunks, H, B)), dim3(kThreads), smem, st, q, ld_q, k, v, ld_t, H, n, qpos, rope_cs,
-                                                                          out, ld_out, ws, nchunks, scale_log2);
+    const cudaError_t e_l = launch_pdl(prefix_attn_kernel<KT, HD>, dim3(dim3(nchunks, H, B)), dim3(kThreads), smem, st, q, ld_q, k, v, ld_t, H, n, qpos, sp, rope_cs,
+                                                                          out, ld_out, ws, nchunks, counters, scale_log2);
     if (e_l != cudaSuccess) return e_l;
   }
   cudaError_t e = cudaGetLastError();
-  if (e != cudaSuccess || nchunks == 1) return e;
+  if (e != cudaSuccess || nchunks == 1 || counters != nullptr) return e;
   {
-    const cudaError_t e_l = launch_pdl(prefix_combine_kernel<KT, HD>, dim3(dim3(H, B)), dim3(HD < 128 ? HD : 128), 0, st, ws, H, nchunks, out, ld_out);
+    const cudaError_t e_l = launch_pdl(prefix_combine_kernel<KT, HD>, dim3(dim3(H, B)), dim3(HD < 128 ? HD : 128), 0, st, ws, H, nchunks, n, sp, out, ld_out);
     if (e_l != cudaSuccess) return e_l;
   }
   return cudaGetLastError();
@@ -310,31 +356,34 @@ cudaError_t prefix_launch(const float* q, int64_t ld_q, const KT* k, const KT* v
 }  // namespace
 
 template <typename KT>
-cudaError_t swa_attn(const float* qkv, int64_t ld_qkv, KT* ring_k, KT* ring_v, int B, int H, int hd, int t, int W,
-                     const float* rope_cs, KT* out, int64_t ld_out, cudaStream_t st) {
-  if (t < 1 || W < 1 || B <= 0) return cudaErrorInvalidValue;
+cudaError_t swa_attn(const float* qkv, int64_t ld_qkv, KT* ring_k, KT* ring_v, int B, int H, int hd, int t,
+                     const SeqPos& sp, int W, const float* rope_cs, KT* out, int64_t ld_out, cudaStream_t st) {
+  if ((!sp.on() && t < 1) || W < 1 || B <= 0) return cudaErrorInvalidValue;
   switch (hd) {
-    case 16: return swa_launch<KT, 16>(qkv, ld_qkv, ring_k, ring_v, B, H, t, W, rope_cs, out, ld_out, st);
-    case 32: return swa_launch<KT, 32>(qkv, ld_qkv, ring_k, ring_v, B, H, t, W, rope_cs, out, ld_out, st);
-    case 64: return swa_launch<KT, 64>(qkv, ld_qkv, ring_k, ring_v, B, H, t, W, rope_cs, out, ld_out, st);
-    case 128: return swa_launch<KT, 128>(qkv, ld_qkv, ring_k, ring_v, B, H, t, W, rope_cs, out, ld_out, st);
-    case 256: return swa_launch<KT, 256>(qkv, ld_qkv, ring_k, ring_v, B, H, t, W, rope_cs, out, ld_out, st);
+    case 16: return swa_launch<KT, 16>(qkv, ld_qkv, ring_k, ring_v, B, H, t, sp, W, rope_cs, out, ld_out, st);
+    case 32: return swa_launch<KT, 32>(qkv, ld_qkv, ring_k, ring_v, B, H, t, sp, W, rope_cs, out, ld_out, st);
+    case 64: return swa_launch<KT, 64>(qkv, ld_qkv, ring_k, ring_v, B, H, t, sp, W, rope_cs, out, ld_out, st);
+    case 128: return swa_launch<KT, 128>(qkv, ld_qkv, ring_k, ring_v, B, H, t, sp, W, rope_cs, out, ld_out, st);
+    case 256: return swa_launch<KT, 256>(qkv, ld_qkv, ring_k, ring_v, B, H, t, sp, W, rope_cs, out, ld_out, st);
   }
   return cudaErrorInvalidValue;
 }
 
 template <typename KT>
 cudaError_t prefix_attn(const float* q, int64_t ld_q, const KT* k, const KT* v, int64_t ld_t, int B, int H, int hd,
-                        int n, int qpos, const float* rope_cs, KT* out, int64_t ld_out, float* ws, size_t ws_floats,
-                        cudaStream_t st) {
+                        int n, int qpos, const SeqPos& sp, const float* rope_cs, KT* out, int64_t ld_out, float* ws,
+                        size_t ws_floats, int* counters, cudaStream_t st) {
   if (n < 1 || B <= 0) return cudaErrorInvalidValue;
+#define RLT_PFX(HD) \
+  prefix_launch<KT, HD>(q, ld_q, k, v, ld_t, B, H, n, qpos, sp, rope_cs, out, ld_out, ws, ws_floats, counters, st)
   switch (hd) {
-    case 16: return prefix_launch<KT, 16>(q, ld_q, k, v, ld_t, B, H, n, qpos, rope_cs, out, ld_out, ws, ws_floats, st);
-    case 32: return prefix_launch<KT, 32>(q, ld_q, k, v, ld_t, B, H, n, qpos, rope_cs, out, ld_out, ws, ws_floats, st);
-    case 64: return prefix_launch<KT, 64>(q, ld_q, k, v, ld_t, B, H, n, qpos, rope_cs, out, ld_out, ws, ws_floats, st);
-    case 128: return prefix_launch<KT, 128>(q, ld_q, k, v, ld_t, B, H, n, qpos, rope_cs, out, ld_out, ws, ws_floats, st);
-    case 256: return prefix_launch<KT, 256>(q, ld_q, k, v, ld_t, B, H, n, qpos, rope_cs, out, ld_out, ws, ws_floats, st);
+    case 16: return RLT_PFX(16);
+    case 32: return RLT_PFX(32);
+    case 64: return RLT_PFX(64);
+    case 128: return RLT_PFX(128);
+    case 256: return RLT_PFX(256);
   }
+#undef RLT_PFX
   return cudaErrorInvalidValue;
 }
 
@@ -343,13 +392,15 @@ size_t prefix_attn_workspace_floats(int B, int H, int hd, int n) {
   return nchunks > 1 ? (size_t)B * H * nchunks * (hd + 2) : 0;
 }
 
-template cudaError_t swa_attn<float>(const float*, int64_t, float*, float*, int, int, int, int, int, const float*,
-                                     float*, int64_t, cudaStream_t);
-template cudaError_t swa_attn<bf16>(const float*, int64_t, bf16*, bf16*, int, int, int, int, int, const float*, bf16*,
-                                    int64_t, cudaStream_t);
+template cudaError_t swa_attn<float>(const float*, int64_t, float*, float*, int, int, int, int, const SeqPos&, int,
+                                     const float*, float*, int64_t, cudaStream_t);
+template cudaError_t swa_attn<bf16>(const float*, int64_t, bf16*, bf16*, int, int, int, int, const SeqPos&, int,
+                                    const float*, bf16*, int64_t, cudaStream_t);
 template cudaError_t prefix_attn<float>(const float*, int64_t, const float*, const float*, int64_t, int, int, int, int,
-                                        int, const float*, float*, int64_t, float*, size_t, cudaStream_t);
+                                        int, const SeqPos&, const float*, float*, int64_t, float*, size_t, int*,
+                                        cudaStream_t);
 template cudaError_t prefix_attn<bf16>(const float*, int64_t, const bf16*, const bf16*, int64_t, int, int, int, int,
-                                       int, const float*, bf16*, int64_t, float*, size_t, cudaStream_t);
+                                       int, const SeqPos&, const float*, bf16*, int64_t, float*, size_t, int*,
+                                       cudaStream_t);
 
 }  // namespace rlt

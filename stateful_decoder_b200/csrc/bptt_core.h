@@ -19,8 +19,11 @@
 //             before and de_t to the encoder.  SWA key/value adjoints are
 //             accumulated per position and are complete when their own
 //             step is reversed (the later steps that read them come first).
-//             The memory key/value adjoints of a segment's queries are
-//             gathered after its reversal, off the serial chain;
+//             Off the serial chain, after the segment's reversal: every
+//             weight gradient of the segment as one contraction over its
+//             seg*B rows (dW += dY^T X, the adjoints dY of each step kept per
+//             step), and the memory key/value adjoints of the segment's
+//             queries as one masked token-parallel pass per layer;
 //   encoder   the encoder backward runs token-parallel at the end.
 //
 // Every operation is a functor whose operator()(i) computes output element
@@ -537,6 +540,7 @@ class Engine {
         bk_.copy(s_cur_, rec(t - t0).zout, (size_t)D.B * D.d);
       }
       for (int t = t1 - 1; t >= t0; --t) step_backward(t, t - t0, tok, wts);
+      segment_grads(t0, t1);
       memory_pass(t0, t1);
     }
     launch(ColSum<Real>{ds_, D.d, G(T_SSTAR), D.B}, D.d);
@@ -545,11 +549,18 @@ class Engine {
   }
 
  private:
+  // Step records of a segment.  Every field is a slice of a [seg][B][width]
+  // block, so that the rows of one field over the whole segment are one
+  // contiguous matrix (the weight-gradient contractions and the memory pass
+  // run over them).  The d* fields are the step's adjoints at the points
+  // where a weight gradient needs them.
   struct LayerRec {
     Real *z, *x, *r1, *q, *o, *lse_sa, *b, *xm, *r2, *qm, *om, *lse_m, *dom, *a, *y, *r3, *u1, *u3, *hs;
+    Real *dz, *du1, *du3, *da, *dqm, *db, *dq, *dk, *dv;
   };
   struct StepRec {
-    Real *sprev, *rm, *rr, *gate, *ws, *zout, *nrm, *rn, *logits;
+    Real *sprev, *rm, *rr, *gate, *ws, *zout, *nrm, *rn, *logits, *et;
+    Real *dlog, *dgp, *dws;
     std::vector<LayerRec> lay;
   };
   struct EncRec {
@@ -569,8 +580,7 @@ class Engine {
   std::vector<StepRec> recs_;
   Real *ckpt_ = nullptr, *s_cur_ = nullptr, *ds_ = nullptr, *de_ = nullptr;
   // step scratch
-  Real *dz_, *da_, *db_, *dx_, *dq_, *dk_, *dv_, *dlog_, *dn_, *dqm_, *dxm_, *dhs_, *du1_, *du3_, *dy_, *dws_, *dgp_,
-      *drm_;
+  Real *dz_, *dx_, *dn_, *dxm_, *dhs_, *dy_, *drm_;
   // encoder scratch
   Real *edh_, *edh2_, *edhs_, *edu1_, *edu3_, *edy_, *edq_, *edk_, *edv_, *edo_, *edx_, *edn_, *edk2_;
 
@@ -612,22 +622,35 @@ class Engine {
       dkh_.push_back(A(N * d)); dvh_.push_back(A(N * d));
     }
     recs_.resize(seg_);
-    for (auto& s : recs_) {
-      s.sprev = A(B * d); s.rm = A(B * d); s.rr = A(B); s.gate = A(B * d); s.ws = A(B * d); s.zout = A(B * d);
-      s.nrm = A(B * d); s.rn = A(B); s.logits = A(B * D.V);
-      s.lay.resize(D.L);
-      for (auto& r : s.lay) {
-        r.z = A(B * d); r.x = A(B * d); r.r1 = A(B); r.q = A(B * d); r.o = A(B * d); r.lse_sa = A(B * H);
-        r.b = A(B * d); r.xm = A(B * d); r.r2 = A(B); r.qm = A(B * d); r.om = A(B * d); r.lse_m = A(B * H);
-        r.dom = A(B * d); r.a = A(B * d); r.y = A(B * d); r.r3 = A(B); r.u1 = A(B * F); r.u3 = A(B * F);
-        r.hs = A(B * F);
+    // one [seg][B][width] block per field; step `slot` takes rows slot*B..
+    auto field = [&](Real* StepRec::*f, size_t w) {
+      Real* blk = A((size_t)seg_ * B * w);
+      for (int k = 0; k < seg_; ++k) recs_[k].*f = blk + (size_t)k * B * w;
+    };
+    auto lfield = [&](Real* LayerRec::*f, size_t w) {
+      for (int l = 0; l < D.L; ++l) {
+        Real* blk = A((size_t)seg_ * B * w);
+        for (int k = 0; k < seg_; ++k) recs_[k].lay[l].*f = blk + (size_t)k * B * w;
       }
-    }
+    };
+    for (auto& r : recs_) r.lay.resize(D.L);
+    field(&StepRec::sprev, d); field(&StepRec::rm, d); field(&StepRec::rr, 1); field(&StepRec::gate, d);
+    field(&StepRec::ws, d); field(&StepRec::zout, d); field(&StepRec::nrm, d); field(&StepRec::rn, 1);
+    field(&StepRec::logits, D.V); field(&StepRec::et, d); field(&StepRec::dlog, D.V); field(&StepRec::dgp, d);
+    field(&StepRec::dws, d);
+    for (Real* LayerRec::*f : {&LayerRec::z, &LayerRec::x, &LayerRec::q, &LayerRec::o, &LayerRec::b, &LayerRec::xm,
+                               &LayerRec::qm, &LayerRec::om, &LayerRec::dom, &LayerRec::a, &LayerRec::y,
+                               &LayerRec::dz, &LayerRec::da, &LayerRec::dqm, &LayerRec::db, &LayerRec::dq,
+                               &LayerRec::dk, &LayerRec::dv})
+      lfield(f, d);
+    for (Real* LayerRec::*f : {&LayerRec::r1, &LayerRec::r2, &LayerRec::r3}) lfield(f, 1);
+    for (Real* LayerRec::*f : {&LayerRec::lse_sa, &LayerRec::lse_m}) lfield(f, H);
+    for (Real* LayerRec::*f : {&LayerRec::u1, &LayerRec::u3, &LayerRec::hs, &LayerRec::du1, &LayerRec::du3})
+      lfield(f, F);
     const size_t nseg = (S - 1 + seg_ - 1) / seg_;
     ckpt_ = A(nseg * B * d); s_cur_ = A(B * d); ds_ = A(B * d);
-    dz_ = A(B * d); da_ = A(B * d); db_ = A(B * d); dx_ = A(B * d); dq_ = A(B * d); dk_ = A(B * d); dv_ = A(B * d);
-    dlog_ = A(B * D.V); dn_ = A(B * d); dqm_ = A(B * d); dxm_ = A(B * d); dhs_ = A(B * F); du1_ = A(B * F);
-    du3_ = A(B * F); dy_ = A(B * d); dws_ = A(B * d); dgp_ = A(B * d); drm_ = A(B * d);
+    dz_ = A(B * d); dx_ = A(B * d); dn_ = A(B * d); dxm_ = A(B * d); dhs_ = A(B * F); dy_ = A(B * d);
+    drm_ = A(B * d);
     edh_ = A(N * d); edh2_ = A(N * d); edhs_ = A(N * F); edu1_ = A(N * F); edu3_ = A(N * F); edy_ = A(N * d);
     edq_ = A(N * d); edk_ = A(N * d); edv_ = A(N * d); edo_ = A(N * d); edx_ = A(N * d); edn_ = A(N * d);
     edk2_ = A(N * d);
@@ -711,19 +734,20 @@ class Engine {
     const Dims& D = D_;
     const int d = D.d, F = D.F, B = D.B;
     const int64_t lde = (int64_t)D.S * d;
-    const Real* et = e_ + (int64_t)t * d;
     StepRec& R = rec(slot);
+    copy2(e_ + (int64_t)t * d, lde, R.et, d, B, d);  // e_t rows of the step, contiguous
+    const Real* et = R.et;
     copy2(s_in, d, R.sprev, d, B, d);
     if (D.merge_kind == 0) {
       rms_f(R.sprev, d, Wt(T_GMERGE), R.rm, R.rr, B);
-      mm_nt(et, lde, Wt(T_WGATE), 2 * d, R.gate, d, B, d, d, 0);
+      mm_nt(et, d, Wt(T_WGATE), 2 * d, R.gate, d, B, d, d, 0);
       mm_nt(R.rm, d, Wt(T_WGATE) + d, 2 * d, R.gate, d, B, d, d, 1);
       mm_nt(R.rm, d, Wt(T_WSTATE), d, R.ws, d, B, d, d, 0);
     } else {
-      mm_nt(et, lde, Wt(T_WGATE), 2 * d, R.gate, d, B, d, d, 0);
+      mm_nt(et, d, Wt(T_WGATE), 2 * d, R.gate, d, B, d, d, 0);
       mm_nt(R.sprev, d, Wt(T_WGATE) + d, 2 * d, R.gate, d, B, d, d, 1);
     }
-    launch(MergeF<Real>{et, lde, R.sprev, Wt(T_BGATE), R.ws, R.gate, R.lay[0].z, d, D.merge_kind, (Real)D.alpha},
+    launch(MergeF<Real>{et, d, R.sprev, Wt(T_BGATE), R.ws, R.gate, R.lay[0].z, d, D.merge_kind, (Real)D.alpha},
            (int64_t)B * d);
     for (int l = 0; l < D.L; ++l) {
       LayerRec& r = R.lay[l];
@@ -759,97 +783,117 @@ class Engine {
   }
 
   // ---- reverse of the transition at position t; ds_ holds dL/ds_t on entry
-  // and dL/ds_{t-1} on exit
+  // and dL/ds_{t-1} on exit.  The adjoints a weight gradient needs are left
+  // in the step's record; segment_grads turns them into the gradients.
   void step_backward(int t, int slot, const int32_t* tok, const Real* wts) {
     const Dims& D = D_;
     const int d = D.d, F = D.F, B = D.B;
     const int64_t lde = (int64_t)D.S * d;
     StepRec& R = rec(slot);
-    launch(Xent<Real>{R.logits, D.V, tok, D.S, t, wts, D.S - 1, nullptr, dlog_}, B);
-    mm_tn(dlog_, D.V, R.nrm, d, G(T_WOUT), d, B, D.V, d);
-    mm_nn(dlog_, D.V, Wt(T_WOUT), d, dn_, d, B, D.V, d, 0);
-    copy2(ds_, d, dz_, d, B, d);
-    rms_b(dn_, R.zout, d, R.rn, Wt(T_GOUT), dz_, G(T_GOUT), B);
+    launch(Xent<Real>{R.logits, D.V, tok, D.S, t, wts, D.S - 1, nullptr, R.dlog}, B);
+    mm_nn(R.dlog, D.V, Wt(T_WOUT), d, dn_, d, B, D.V, d, 0);
+    Real* dz = R.lay[D.L - 1].dz;
+    copy2(ds_, d, dz, d, B, d);
+    rms_b(dn_, R.zout, d, R.rn, Wt(T_GOUT), dz, G(T_GOUT), B);
     for (int l = D.L - 1; l >= 0; --l) {
       LayerRec& r = R.lay[l];
       const int grp = D.G == 1 ? 0 : l;
       // FFN (eq. 2.16): z_out = a + W2 (silu(W1 y) * W3 y), y = RMSNorm(a)
-      mm_tn(dz_, d, r.hs, F, Gl(l, dslot(L_W2)), F, B, d, F);
-      mm_nn(dz_, d, Wl(l, dslot(L_W2)), F, dhs_, F, B, d, F, 0);
-      launch(SwiB<Real>{dhs_, r.u1, r.u3, du1_, du3_}, (int64_t)B * F);
-      mm_tn(du1_, F, r.y, d, Gl(l, dslot(L_W1)), d, B, F, d);
-      mm_tn(du3_, F, r.y, d, Gl(l, dslot(L_W3)), d, B, F, d);
-      mm_nn(du1_, F, Wl(l, dslot(L_W1)), d, dy_, d, B, F, d, 0);
-      mm_nn(du3_, F, Wl(l, dslot(L_W3)), d, dy_, d, B, F, d, 1);
-      copy2(dz_, d, da_, d, B, d);
-      rms_b(dy_, r.a, d, r.r3, Wl(l, L_GDFFN), da_, Gl(l, L_GDFFN), B);
+      mm_nn(r.dz, d, Wl(l, dslot(L_W2)), F, dhs_, F, B, d, F, 0);
+      launch(SwiB<Real>{dhs_, r.u1, r.u3, r.du1, r.du3}, (int64_t)B * F);
+      mm_nn(r.du1, F, Wl(l, dslot(L_W1)), d, dy_, d, B, F, d, 0);
+      mm_nn(r.du3, F, Wl(l, dslot(L_W3)), d, dy_, d, B, F, d, 1);
+      copy2(r.dz, d, r.da, d, B, d);
+      rms_b(dy_, r.a, d, r.r3, Wl(l, L_GDFFN), r.da, Gl(l, L_GDFFN), B);
       // memory cross-attention (eq. 2.15): a = b + W_om attn(q_m, M_<=t)
-      mm_tn(da_, d, r.om, d, Gl(l, L_WOM), d, B, d, d);
-      mm_nn(da_, d, Wl(l, L_WOM), d, r.dom, d, B, d, d, 0);
-      launch(AttnBQ<Real>{step_geom(t, full_win()), r.qm, memk_[grp], memv_[grp], r.om, r.dom, r.lse_m, dqm_,
+      mm_nn(r.da, d, Wl(l, L_WOM), d, r.dom, d, B, d, d, 0);
+      launch(AttnBQ<Real>{step_geom(t, full_win()), r.qm, memk_[grp], memv_[grp], r.om, r.dom, r.lse_m, r.dqm,
                           scale()},
              (int64_t)B * D.H);
-      rope(dqm_, d, B, 1, t, -1.0);
-      mm_tn(dqm_, d, r.xm, d, Gl(l, L_WQM), d, B, d, d);
-      mm_nn(dqm_, d, Wl(l, L_WQM), d, dxm_, d, B, d, d, 0);
-      copy2(da_, d, db_, d, B, d);
-      rms_b(dxm_, r.b, d, r.r2, Wl(l, L_GDMEM), db_, Gl(l, L_GDMEM), B);
+      rope(r.dqm, d, B, 1, t, -1.0);
+      mm_nn(r.dqm, d, Wl(l, L_WQM), d, dxm_, d, B, d, d, 0);
+      copy2(r.da, d, r.db, d, B, d);
+      rms_b(dxm_, r.b, d, r.r2, Wl(l, L_GDMEM), r.db, Gl(l, L_GDMEM), B);
       // SWA (eqs. 2.12-2.14): b = z + W_o attn(q, window of K/V)
-      mm_tn(db_, d, r.o, d, Gl(l, dslot(L_WO)), d, B, d, d);
-      mm_nn(db_, d, Wl(l, dslot(L_WO)), d, dx_, d, B, d, d, 0);  // dx_ = adjoint of the attention output
+      mm_nn(r.db, d, Wl(l, dslot(L_WO)), d, dx_, d, B, d, d, 0);  // dx_ = adjoint of the attention output
       const AttnGeom<Real> gw = step_geom(t, D.W);
-      launch(AttnBQ<Real>{gw, r.q, kh_[l], vh_[l], r.o, dx_, r.lse_sa, dq_, scale()}, (int64_t)B * D.H);
+      launch(AttnBQ<Real>{gw, r.q, kh_[l], vh_[l], r.o, dx_, r.lse_sa, r.dq, scale()}, (int64_t)B * D.H);
       const int p0 = gw.lo(0), np = t - p0 + 1;
       launch(AttnBKV<Real>{gw, r.q, kh_[l], vh_[l], r.o, dx_, r.lse_sa, dkh_[l], dvh_[l], scale(), p0, np},
              (int64_t)B * np * D.H);
       // the adjoints of this position's key and value are complete now
-      copy2(dkh_[l] + (int64_t)t * d, lde, dk_, d, B, d);
-      copy2(dvh_[l] + (int64_t)t * d, lde, dv_, d, B, d);
-      rope(dk_, d, B, 1, t, -1.0);
-      rope(dq_, d, B, 1, t, -1.0);
-      mm_tn(dq_, d, r.x, d, Gl(l, dslot(L_WQ)), d, B, d, d);
-      mm_tn(dk_, d, r.x, d, Gl(l, dslot(L_WK)), d, B, d, d);
-      mm_tn(dv_, d, r.x, d, Gl(l, dslot(L_WV)), d, B, d, d);
-      mm_nn(dq_, d, Wl(l, dslot(L_WQ)), d, dx_, d, B, d, d, 0);
-      mm_nn(dk_, d, Wl(l, dslot(L_WK)), d, dx_, d, B, d, d, 1);
-      mm_nn(dv_, d, Wl(l, dslot(L_WV)), d, dx_, d, B, d, d, 1);
-      copy2(db_, d, dz_, d, B, d);
-      rms_b(dx_, r.z, d, r.r1, Wl(l, L_GDSA), dz_, Gl(l, L_GDSA), B);
+      copy2(dkh_[l] + (int64_t)t * d, lde, r.dk, d, B, d);
+      copy2(dvh_[l] + (int64_t)t * d, lde, r.dv, d, B, d);
+      rope(r.dk, d, B, 1, t, -1.0);
+      rope(r.dq, d, B, 1, t, -1.0);
+      mm_nn(r.dq, d, Wl(l, dslot(L_WQ)), d, dx_, d, B, d, d, 0);
+      mm_nn(r.dk, d, Wl(l, dslot(L_WK)), d, dx_, d, B, d, d, 1);
+      mm_nn(r.dv, d, Wl(l, dslot(L_WV)), d, dx_, d, B, d, d, 1);
+      Real* dz_in = l > 0 ? R.lay[l - 1].dz : dz_;  // adjoint of this layer's input
+      copy2(r.db, d, dz_in, d, B, d);
+      rms_b(dx_, r.z, d, r.r1, Wl(l, L_GDSA), dz_in, Gl(l, L_GDSA), B);
     }
     // merge (eqs. 2.9-2.11 or the convex gate); dz_ = dL/du_t
     Real* det = de_ + (int64_t)t * d;
-    const Real* et = e_ + (int64_t)t * d;
-    launch(MergeB<Real>{dz_, et, lde, R.sprev, R.gate, R.ws, det, dws_, dgp_, ds_, d, D.merge_kind, (Real)D.alpha},
+    // (e_t and its adjoint share MergeB's row stride: both in the [B][S][d] layout)
+    launch(MergeB<Real>{dz_, e_ + (int64_t)t * d, lde, R.sprev, R.gate, R.ws, det, R.dws, R.dgp, ds_, d, D.merge_kind,
+                        (Real)D.alpha},
            (int64_t)B * d);
-    mm_tn(dgp_, d, et, lde, G(T_WGATE), 2 * d, B, d, d);
-    mm_nn(dgp_, d, Wt(T_WGATE), 2 * d, det, lde, B, d, d, 1);
+    mm_nn(R.dgp, d, Wt(T_WGATE), 2 * d, det, lde, B, d, d, 1);
     if (D.merge_kind == 0) {
-      launch(ColSum<Real>{dgp_, d, G(T_BGATE), B}, d);
-      mm_tn(dgp_, d, R.rm, d, G(T_WGATE) + d, 2 * d, B, d, d);
-      mm_tn(dws_, d, R.rm, d, G(T_WSTATE), d, B, d, d);
-      mm_nn(dws_, d, Wt(T_WSTATE), d, drm_, d, B, d, d, 0);
-      mm_nn(dgp_, d, Wt(T_WGATE) + d, 2 * d, drm_, d, B, d, d, 1);
+      mm_nn(R.dws, d, Wt(T_WSTATE), d, drm_, d, B, d, d, 0);
+      mm_nn(R.dgp, d, Wt(T_WGATE) + d, 2 * d, drm_, d, B, d, d, 1);
       bk_.zero(ds_, (size_t)B * d);
       rms_b(drm_, R.sprev, d, R.rr, Wt(T_GMERGE), ds_, G(T_GMERGE), B);
     } else {
-      mm_tn(dgp_, d, R.sprev, d, G(T_WGATE) + d, 2 * d, B, d, d);
-      mm_nn(dgp_, d, Wt(T_WGATE) + d, 2 * d, ds_, d, B, d, d, 1);
+      mm_nn(R.dgp, d, Wt(T_WGATE) + d, 2 * d, ds_, d, B, d, d, 1);
     }
   }
 
-  // ---- memory key/value adjoints of the segment's queries t0..t1-1 (deferred)
-  // (one launch per step and layer, each over the memory positions 0..t its
-  // query saw; they run after the segment's reversal, off the serial chain)
+  // ---- weight gradients of the segment's steps t0..t1-1: dW += dY^T X, one
+  // contraction per weight over the (t1-t0)*B rows of the step records
+  void segment_grads(int t0, int t1) {
+    const Dims& D = D_;
+    const int d = D.d, F = D.F;
+    const int R = (t1 - t0) * D.B;
+    const StepRec& S0 = rec(0);
+    mm_tn(S0.dlog, D.V, S0.nrm, d, G(T_WOUT), d, R, D.V, d);
+    mm_tn(S0.dgp, d, S0.et, d, G(T_WGATE), 2 * d, R, d, d);
+    if (D.merge_kind == 0) {
+      launch(ColSum<Real>{S0.dgp, d, G(T_BGATE), R}, d);
+      mm_tn(S0.dgp, d, S0.rm, d, G(T_WGATE) + d, 2 * d, R, d, d);
+      mm_tn(S0.dws, d, S0.rm, d, G(T_WSTATE), d, R, d, d);
+    } else {
+      mm_tn(S0.dgp, d, S0.sprev, d, G(T_WGATE) + d, 2 * d, R, d, d);
+    }
+    for (int l = 0; l < D.L; ++l) {
+      const LayerRec& r = S0.lay[l];
+      mm_tn(r.dz, d, r.hs, F, Gl(l, dslot(L_W2)), F, R, d, F);
+      mm_tn(r.du1, F, r.y, d, Gl(l, dslot(L_W1)), d, R, F, d);
+      mm_tn(r.du3, F, r.y, d, Gl(l, dslot(L_W3)), d, R, F, d);
+      mm_tn(r.da, d, r.om, d, Gl(l, L_WOM), d, R, d, d);
+      mm_tn(r.dqm, d, r.xm, d, Gl(l, L_WQM), d, R, d, d);
+      mm_tn(r.db, d, r.o, d, Gl(l, dslot(L_WO)), d, R, d, d);
+      mm_tn(r.dq, d, r.x, d, Gl(l, dslot(L_WQ)), d, R, d, d);
+      mm_tn(r.dk, d, r.x, d, Gl(l, dslot(L_WK)), d, R, d, d);
+      mm_tn(r.dv, d, r.x, d, Gl(l, dslot(L_WV)), d, R, d, d);
+    }
+  }
+
+  // ---- memory key/value adjoints of the segment's queries t0..t1-1: per
+  // layer one token-parallel pass over the memory positions 0..t1-1, each
+  // position gathering the queries of the segment that see it (p <= t)
   void memory_pass(int t0, int t1) {
     const Dims& D = D_;
+    const int d = D.d, B = D.B;
     for (int l = 0; l < D.L; ++l) {
       const int grp = D.G == 1 ? 0 : l;
-      for (int t = t0; t < t1; ++t) {
-        const LayerRec& r = rec(t - t0).lay[l];
-        launch(AttnBKV<Real>{step_geom(t, full_win()), r.qm, memk_[grp], memv_[grp], r.om, r.dom, r.lse_m,
-                             dmemk_[grp], dmemv_[grp], scale(), 0, t + 1},
-               (int64_t)D.B * (t + 1) * D.H);
-      }
+      const LayerRec& r = rec(0).lay[l];
+      const AttnGeom<Real> g{(int64_t)d, (int64_t)B * d, (int64_t)D.S * d, (int64_t)d, (int64_t)D.H,
+                             (int64_t)B * D.H, t1 - t0, D.H, D.hd(), t0, full_win()};
+      launch(AttnBKV<Real>{g, r.qm, memk_[grp], memv_[grp], r.om, r.dom, r.lse_m, dmemk_[grp], dmemv_[grp], scale(),
+                           0, t1},
+             (int64_t)B * t1 * D.H);
     }
   }
 

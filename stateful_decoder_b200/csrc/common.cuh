@@ -167,6 +167,29 @@ struct RowMap {
 };
 __host__ __device__ inline RowMap plain_rows(int64_t ld) { return RowMap{ld, 0, 0}; }
 
+// ---------------------------------------------------------------- positions
+// Per-sequence positions of a state, as device arrays of B entries (report
+// §4.1: every sequence of a batch has its own position).  `dec` counts the
+// decoder transitions applied (n_dec), `enc` the tokens encoded (n_enc); the
+// transition in flight for sequence b is at t_b = dec[b] + 1.  In a masked
+// phase (catching up over appended spans of different lengths) `lim` is set
+// and sequence b takes part in a transition only while dec[b] < lim[b]; an
+// idle sequence reads only rows that exist and writes nothing.  All pointers
+// null: the kernel takes the scalar position it is given instead.
+struct SeqPos {
+  const int32_t* dec;
+  const int32_t* enc;
+  const int32_t* lim;
+  __host__ __device__ bool on() const { return dec != nullptr; }
+  __device__ __forceinline__ bool active(int b) const { return lim == nullptr || dec[b] < lim[b]; }
+  // keys an attention query of sequence b reads: 1..t_b when active, else
+  // the rows an idle sequence already holds (at least one)
+  __device__ __forceinline__ int n_keys(int b) const { return active(b) ? dec[b] + 1 : max(1, dec[b]); }
+  // the transition's encoder step writes position t_b of sequence b
+  __device__ __forceinline__ bool encodes(int b) const { return active(b) && enc[b] <= dec[b]; }
+};
+__host__ __device__ inline SeqPos no_pos() { return SeqPos{nullptr, nullptr, nullptr}; }
+
 // ---------------------------------------------------------------- mbarrier / PTX
 __device__ __forceinline__ uint32_t smem_u32(const void* p) {
   return static_cast<uint32_t>(__cvta_generic_to_shared(p));

@@ -59,20 +59,24 @@ cudaError_t gemm_simt(const WT* W, int64_t ldw, const XT* X, int64_t ldx, int M,
 
 // ---------------------------------------------------------------- attention
 // SWA decode attention of one decoder layer (eq. 2.14) over the ring of
-// retained entries plus the current key/value, then the ring insert.
+// retained entries plus the current key/value, then the ring insert; at
+// position t, or at each sequence's own position when sp is on.
 template <typename KT>
-cudaError_t swa_attn(const float* qkv, int64_t ld_qkv, KT* ring_k, KT* ring_v, int B, int H, int hd, int t, int W,
-                     const float* rope_cs, KT* out, int64_t ld_out, cudaStream_t st);
+cudaError_t swa_attn(const float* qkv, int64_t ld_qkv, KT* ring_k, KT* ring_v, int B, int H, int hd, int t,
+                     const SeqPos& sp, int W, const float* rope_cs, KT* out, int64_t ld_out, cudaStream_t st);
 
 // Decode attention of one query per (sequence, head) over key/value rows
 // 0..n-1 of a [B][H][ld_t][hd] cache; the query is rotated at position
-// qpos (0-based) first unless rope_cs is null.  Split over fixed chunks of
-// keys when n is large; the chunk partials go to `ws`
-// (prefix_attn_workspace_floats).
+// qpos (0-based) first unless rope_cs is null.  With sp on, sequence b reads
+// its own sp.n_keys(b) rows (query at n_keys - 1) and n only bounds them.
+// Split over fixed chunks of keys when n is large; the chunk partials go to
+// `ws` (prefix_attn_workspace_floats).  With `counters` (B*H ints, zero
+// between launches) the last chunk block of each (sequence, head) combines
+// them; without, a second kernel does.
 template <typename KT>
 cudaError_t prefix_attn(const float* q, int64_t ld_q, const KT* k, const KT* v, int64_t ld_t, int B, int H, int hd,
-                        int n, int qpos, const float* rope_cs, KT* out, int64_t ld_out, float* ws, size_t ws_floats,
-                        cudaStream_t st);
+                        int n, int qpos, const SeqPos& sp, const float* rope_cs, KT* out, int64_t ld_out, float* ws,
+                        size_t ws_floats, int* counters, cudaStream_t st);
 size_t prefix_attn_workspace_floats(int B, int H, int hd, int n);
 constexpr int kPrefixChunk = 256;
 
@@ -125,14 +129,42 @@ template <typename XT, typename KT>
 cudaError_t head_scatter(const XT* x, int64_t ld_x, int64_t col0, int64_t rows, int rows_per_seq, int pos0,
                          int dst_row0, int H, int hd, int rope, const float* rope_cs, KT* dst, int64_t ld_t,
                          cudaStream_t st);
+// The encoder step's insert of one row per sequence at its own position:
+// row b goes to store row t_b - 1 (rotated at t_b - 1) for the sequences
+// whose transition encodes its token (sp.encodes(b)); the others are left.
+template <typename XT, typename KT>
+cudaError_t head_insert(const XT* x, int64_t ld_x, int64_t col0, int B, const SeqPos& sp, int H, int hd, int rope,
+                        const float* rope_cs, KT* dst, int64_t ld_t, cudaStream_t st);
 
-// logp[b*ld_logp] = logits[b][next[b*next_stride]] - logsumexp(logits[b])
+// et[b] = e[b][t_b - 1] ([B][max_len][d] -> [B][d]; idle sequences copy a
+// row they hold), and its inverse for the sequences whose transition encoded
+// their token.
+cudaError_t erow_gather(const float* e, int max_len, int d, int B, const SeqPos& sp, float* et, cudaStream_t st);
+cudaError_t erow_scatter(const float* et, int max_len, int d, int B, const SeqPos& sp, float* e, cudaStream_t st);
+
+// Position bookkeeping after a transition (report §2.1): every active
+// sequence b moves to n_dec = t_b (and n_enc = max(n_enc, t_b)).  In a
+// masked phase, the idle sequences get back the recurrent output and the
+// folded-norm operand saved by save_rows before the transition, so that a
+// transition they took no part in leaves them unchanged.
+cudaError_t advance_positions(int32_t* dec, int32_t* enc, const int32_t* lim, int B, int d, float* s,
+                              const float* s_save, bf16* zb, const bf16* zb_save, float* ss, const float* ss_save,
+                              int n_ss, cudaStream_t st);
+cudaError_t save_rows(const float* s, float* s_save, const bf16* zb, bf16* zb_save, const float* ss, float* ss_save,
+                      int B, int d, int n_ss, cudaStream_t st);
+// n[b] = value for b in [b0, b1)
+cudaError_t set_positions(int32_t* n, int b0, int b1, int32_t value, cudaStream_t st);
+
+// logp[b*ld_logp] = logits[b][next[b*next_stride]] - logsumexp(logits[b]);
+// with `lim`, only for the sequences whose (advanced) dec[b] < lim[b], i.e.
+// whose masked phase has a next token left.
 cudaError_t logp_gather(const float* logits, int B, int V, const int32_t* next, int64_t next_stride, float* logp,
-                        int64_t ld_logp, cudaStream_t st);
+                        int64_t ld_logp, const int32_t* dec, const int32_t* lim, cudaStream_t st);
 
-// Top-k / temperature behaviour sampler (report §5.3).
+// Top-k / temperature behaviour sampler (report §5.3); the Philox counter's
+// position is t, or t_rows[b] per sequence when t_rows is not null.
 cudaError_t sample_topk(const float* logits, int B, int V, float temperature, int top_k, uint64_t seed, uint32_t t,
-                        int32_t* token, float* logp_tok, float* logmu, cudaStream_t st);
+                        const int32_t* t_rows, int32_t* token, float* logp_tok, float* logmu, cudaStream_t st);
 
 cudaError_t copy_f32(float* dst, const float* src, int64_t n, cudaStream_t st);
 
@@ -152,9 +184,10 @@ cudaError_t widen_to_f32(const void* src, int dtype, int64_t rows, int64_t cols,
                          cudaStream_t st);
 // Full-BPTT gradient of the weighted replay loss (bptt_core.h) on fp32
 // weights W32 into G32 (per catalogue index; null where a tensor is absent).
-// Drains the stream before it returns.
+// tensor_cores: run the contractions whose shapes allow it on tcgen05 with
+// bf16 operands (bf16 models).  Drains the stream before it returns.
 cudaError_t replay_backward_f32(const Dims& D, const float* const* W32, float* const* G32, const int32_t* tok,
-                                const float* wts, int seg, float* logp, cudaStream_t st);
+                                const float* wts, int seg, float* logp, bool tensor_cores, cudaStream_t st);
 }  // namespace bptt
 
 }  // namespace rlt

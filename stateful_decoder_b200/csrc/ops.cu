@@ -196,12 +196,116 @@ __global__ void head_scatter_kernel(const XT* __restrict__ x, int64_t ld_x, int6
   }
 }
 
+// One row per sequence (the encoder step's keys/values or memory row of the
+// token at t_b), written to store row t_b - 1 and rotated at t_b - 1, for the
+// sequences whose transition encodes its token; the same 16-byte moves as
+// head_scatter_kernel.
+template <typename XT, typename KT>
+__global__ void head_insert_kernel(const XT* __restrict__ x, int64_t ld_x, int64_t col0, int B, SeqPos sp, int H,
+                                   int hd, int rope, const float* __restrict__ rope_cs, KT* dst, int64_t ld_t) {
+  griddep_enter();
+  const int half = hd / 2, oct = half / 8;
+  const int64_t n = (int64_t)B * H * oct;
+  for (int64_t idx = (int64_t)blockIdx.x * blockDim.x + threadIdx.x; idx < n; idx += (int64_t)gridDim.x * blockDim.x) {
+    const int i = (int)(idx % oct) * 8;
+    const int h = (int)((idx / oct) % H);
+    const int b = (int)(idx / ((int64_t)oct * H));
+    if (!sp.encodes(b)) continue;
+    const int pos = sp.dec[b];  // t_b - 1
+    const XT* xr = x + (int64_t)b * ld_x + col0 + (int64_t)h * hd;
+    float a[8], c[8];
+    load8(xr + i, a);
+    load8(xr + i + half, c);
+    if (rope) {
+      const float4* cs = reinterpret_cast<const float4*>(rope_cs + ((int64_t)pos * half + i) * 2);
+#pragma unroll
+      for (int u = 0; u < 4; ++u) {
+        const float4 t = cs[u];
+        const float a0 = a[2 * u] * t.x - c[2 * u] * t.y, c0 = a[2 * u] * t.y + c[2 * u] * t.x;
+        const float a1 = a[2 * u + 1] * t.z - c[2 * u + 1] * t.w, c1 = a[2 * u + 1] * t.w + c[2 * u + 1] * t.z;
+        a[2 * u] = a0;
+        c[2 * u] = c0;
+        a[2 * u + 1] = a1;
+        c[2 * u + 1] = c1;
+      }
+    }
+    KT* o = dst + (((int64_t)b * H + h) * ld_t + pos) * hd;
+    store8(o + i, a);
+    store8(o + i + half, c);
+  }
+}
+
+// ------------------------------------------------------------------ positions
+// et[b] = e[b][row_b]: the encoder output the merge of sequence b's
+// transition reads (row t_b - 1; an idle sequence copies a row it holds).
+__global__ void erow_gather_kernel(const float* __restrict__ e, int max_len, int d, SeqPos sp, float* et) {
+  griddep_enter();
+  const int b = blockIdx.x;
+  const int row = min(sp.dec[b], max_len - 1);
+  const float4* src = reinterpret_cast<const float4*>(e + ((int64_t)b * max_len + row) * d);
+  float4* dst = reinterpret_cast<float4*>(et + (int64_t)b * d);
+  for (int i = threadIdx.x; i < d / 4; i += blockDim.x) dst[i] = src[i];
+}
+
+// e[b][t_b - 1] = et[b] for the sequences whose transition encoded their token.
+__global__ void erow_scatter_kernel(const float* __restrict__ et, int max_len, int d, SeqPos sp, float* e) {
+  griddep_enter();
+  const int b = blockIdx.x;
+  if (!sp.encodes(b)) return;
+  const float4* src = reinterpret_cast<const float4*>(et + (int64_t)b * d);
+  float4* dst = reinterpret_cast<float4*>(e + ((int64_t)b * max_len + sp.dec[b]) * d);
+  for (int i = threadIdx.x; i < d / 4; i += blockDim.x) dst[i] = src[i];
+}
+
+__global__ void save_rows_kernel(const float* __restrict__ s, float* s_save, const bf16* __restrict__ zb,
+                                 bf16* zb_save, const float* __restrict__ ss, float* ss_save, int B, int d, int n_ss) {
+  griddep_enter();
+  const int b = blockIdx.x;
+  for (int i = threadIdx.x; i < d; i += blockDim.x) s_save[(int64_t)b * d + i] = s[(int64_t)b * d + i];
+  if (zb)
+    for (int i = threadIdx.x; i < d; i += blockDim.x) zb_save[(int64_t)b * d + i] = zb[(int64_t)b * d + i];
+  if (ss)
+    for (int i = threadIdx.x; i < n_ss; i += blockDim.x) ss_save[(int64_t)i * B + b] = ss[(int64_t)i * B + b];
+}
+
+// One block per sequence: the active ones advance (n_dec = t_b, n_enc at
+// least t_b); in a masked phase the idle ones get their saved rows back.
+__global__ void advance_kernel(int32_t* dec, int32_t* enc, const int32_t* __restrict__ lim, int B, int d, float* s,
+                               const float* __restrict__ s_save, bf16* zb, const bf16* __restrict__ zb_save, float* ss,
+                               const float* __restrict__ ss_save, int n_ss) {
+  griddep_wait();
+  const int b = blockIdx.x;
+  const int db = dec[b];
+  const bool act = lim == nullptr || db < lim[b];
+  if (!act && s_save) {
+    for (int i = threadIdx.x; i < d; i += blockDim.x) s[(int64_t)b * d + i] = s_save[(int64_t)b * d + i];
+    if (zb)
+      for (int i = threadIdx.x; i < d; i += blockDim.x) zb[(int64_t)b * d + i] = zb_save[(int64_t)b * d + i];
+    if (ss)
+      for (int i = threadIdx.x; i < n_ss; i += blockDim.x) ss[(int64_t)i * B + b] = ss_save[(int64_t)i * B + b];
+  }
+  __syncthreads();  // every thread has read dec[b] before it changes
+  if (threadIdx.x == 0 && act) {
+    dec[b] = db + 1;
+    if (enc[b] < db + 1) enc[b] = db + 1;
+  }
+  griddep_launch_dependents();
+}
+
+__global__ void set_positions_kernel(int32_t* n, int b0, int b1, int32_t value) {
+  griddep_enter();
+  for (int b = b0 + (int)(blockIdx.x * blockDim.x + threadIdx.x); b < b1; b += (int)(gridDim.x * blockDim.x))
+    n[b] = value;
+}
+
 // ------------------------------------------------------------------ readout
 __global__ void logp_gather_kernel(const float* __restrict__ logits, int V, const int32_t* __restrict__ next,
-                                   int64_t next_stride, float* logp, int64_t ld_logp) {
+                                   int64_t next_stride, float* logp, int64_t ld_logp, const int32_t* __restrict__ dec,
+                                   const int32_t* __restrict__ lim) {
   griddep_enter();
   __shared__ float red[32];
   const int b = blockIdx.x;
+  if (lim != nullptr && !(dec[b] < lim[b])) return;  // this sequence's phase has no next token here
   const float* l = logits + (int64_t)b * V;
   // 16-byte loads when every row starts 16-byte aligned (V % 4 == 0); the
   // second pass finds the row in L1/L2
@@ -283,7 +387,7 @@ constexpr int kMaxTopK = 256;
 // running sum exceeds u * total.
 __global__ void __launch_bounds__(kSampleThreads)
     sample_kernel(const float* __restrict__ logits, int V, float temperature, int top_k, uint32_t k0, uint32_t k1,
-                  uint32_t t, int32_t* token, float* logp_tok, float* logmu) {
+                  uint32_t t, const int32_t* __restrict__ t_rows, int32_t* token, float* logp_tok, float* logmu) {
   griddep_enter();
   __shared__ uint32_t hist[256];
   __shared__ uint32_t s_sel[2];
@@ -389,7 +493,7 @@ __global__ void __launch_bounds__(kSampleThreads)
       w[r] = expf(l[cand_id[r]] / temperature - z0);
       total += w[r];
     }
-    uint32_t c[4] = {t, (uint32_t)b, 0u, 0u};
+    uint32_t c[4] = {t_rows ? (uint32_t)t_rows[b] : t, (uint32_t)b, 0u, 0u};
     philox4x32_10(c, k0, k1);
     const float u = (float)(c[0] >> 8) * (1.0f / 16777216.0f);
     const float target = u * total;
@@ -505,10 +609,55 @@ cudaError_t head_scatter(const XT* x, int64_t ld_x, int64_t col0, int64_t rows, 
   return cudaGetLastError();
 }
 
+template <typename XT, typename KT>
+cudaError_t head_insert(const XT* x, int64_t ld_x, int64_t col0, int B, const SeqPos& sp, int H, int hd, int rope,
+                        const float* rope_cs, KT* dst, int64_t ld_t, cudaStream_t st) {
+  if (hd % 16 || !sp.on()) return cudaErrorInvalidValue;
+  const int64_t n = (int64_t)B * H * (hd / 16);
+  const cudaError_t e_l = launch_pdl(head_insert_kernel<XT, KT>, dim3(grid_for(n, 256, 148 * 32)), dim3(256), 0, st, x,
+                                     ld_x, col0, B, sp, H, hd, rope, rope_cs, dst, ld_t);
+  return e_l != cudaSuccess ? e_l : cudaGetLastError();
+}
+
+cudaError_t erow_gather(const float* e, int max_len, int d, int B, const SeqPos& sp, float* et, cudaStream_t st) {
+  if (d % 4 || !sp.on()) return cudaErrorInvalidValue;
+  const cudaError_t e_l = launch_pdl(erow_gather_kernel, dim3(B), dim3(128), 0, st, e, max_len, d, sp, et);
+  return e_l != cudaSuccess ? e_l : cudaGetLastError();
+}
+
+cudaError_t erow_scatter(const float* et, int max_len, int d, int B, const SeqPos& sp, float* e, cudaStream_t st) {
+  if (d % 4 || !sp.on()) return cudaErrorInvalidValue;
+  const cudaError_t e_l = launch_pdl(erow_scatter_kernel, dim3(B), dim3(128), 0, st, et, max_len, d, sp, e);
+  return e_l != cudaSuccess ? e_l : cudaGetLastError();
+}
+
+cudaError_t advance_positions(int32_t* dec, int32_t* enc, const int32_t* lim, int B, int d, float* s,
+                              const float* s_save, bf16* zb, const bf16* zb_save, float* ss, const float* ss_save,
+                              int n_ss, cudaStream_t st) {
+  const cudaError_t e_l = launch_pdl(advance_kernel, dim3(B), dim3(128), 0, st, dec, enc, lim, B, d, s, s_save, zb,
+                                     zb_save, ss, ss_save, n_ss);
+  return e_l != cudaSuccess ? e_l : cudaGetLastError();
+}
+
+cudaError_t save_rows(const float* s, float* s_save, const bf16* zb, bf16* zb_save, const float* ss, float* ss_save,
+                      int B, int d, int n_ss, cudaStream_t st) {
+  const cudaError_t e_l =
+      launch_pdl(save_rows_kernel, dim3(B), dim3(128), 0, st, s, s_save, zb, zb_save, ss, ss_save, B, d, n_ss);
+  return e_l != cudaSuccess ? e_l : cudaGetLastError();
+}
+
+cudaError_t set_positions(int32_t* n, int b0, int b1, int32_t value, cudaStream_t st) {
+  if (b1 <= b0) return cudaSuccess;
+  const cudaError_t e_l = launch_pdl(set_positions_kernel, dim3(grid_for(b1 - b0, 128)), dim3(128), 0, st, n, b0, b1,
+                                     value);
+  return e_l != cudaSuccess ? e_l : cudaGetLastError();
+}
+
 cudaError_t logp_gather(const float* logits, int B, int V, const int32_t* next, int64_t next_stride, float* logp,
-                        int64_t ld_logp, cudaStream_t st) {
+                        int64_t ld_logp, const int32_t* dec, const int32_t* lim, cudaStream_t st) {
   {
-    const cudaError_t e_l = launch_pdl(logp_gather_kernel, dim3(B), dim3(256), 0, st, logits, V, next, next_stride, logp, ld_logp);
+    const cudaError_t e_l = launch_pdl(logp_gather_kernel, dim3(B), dim3(256), 0, st, logits, V, next, next_stride, logp, ld_logp,
+                                       dec, lim);
     if (e_l != cudaSuccess) return e_l;
   }
   return cudaGetLastError();
@@ -525,11 +674,11 @@ cudaError_t replay_ratios(const float* logp, const float* logmu, const uint8_t* 
 }
 
 cudaError_t sample_topk(const float* logits, int B, int V, float temperature, int top_k, uint64_t seed, uint32_t t,
-                        int32_t* token, float* logp_tok, float* logmu, cudaStream_t st) {
+                        const int32_t* t_rows, int32_t* token, float* logp_tok, float* logmu, cudaStream_t st) {
   if (top_k < 1 || top_k > kMaxTopK || !(temperature > 0.f)) return cudaErrorInvalidValue;
   {
     const cudaError_t e_l = launch_pdl(sample_kernel, dim3(B), dim3(kSampleThreads), 0, st, logits, V, temperature, top_k, (uint32_t)seed, (uint32_t)(seed >> 32), t,
-                                             token, logp_tok, logmu);
+                                             t_rows, token, logp_tok, logmu);
     if (e_l != cudaSuccess) return e_l;
   }
   return cudaGetLastError();
@@ -563,6 +712,8 @@ cudaError_t copy_f32(float* dst, const float* src, int64_t n, cudaStream_t st) {
                                           WT*, cudaStream_t);                                                     \
   template cudaError_t head_scatter<float, WT>(const float*, int64_t, int64_t, int64_t, int, int, int, int, int, int,   \
                                                const float*, WT*, int64_t, cudaStream_t);                         \
+  template cudaError_t head_insert<float, WT>(const float*, int64_t, int64_t, int, const SeqPos&, int, int, int,  \
+                                              const float*, WT*, int64_t, cudaStream_t);                          \
   template cudaError_t broadcast_row<WT>(const WT*, int, float*, int, cudaStream_t);
 
 RLT_INST_W(float)

@@ -18,6 +18,7 @@
 #include <cuda_runtime.h>
 #include <nvtx3/nvToolsExt.h>
 
+#include <algorithm>
 #include <cmath>
 #include <type_traits>
 #include <cstdio>
@@ -110,9 +111,20 @@ struct rlt_state {
   rlt_model* m = nullptr;
   int32_t B = 0, max_len = 0, flags = 0;
   uint64_t version = 0;
-  int32_t n_enc = 0, n_dec = 0;
+  // Per-sequence positions (report §4.1: each sequence of a batch has its
+  // own position): n_enc[b] tokens encoded, n_dec[b] transitions applied.
+  // The host copies decide shapes and validate calls; the device copy `pos`
+  // ([3][B]: n_enc, n_dec, lim) is what the kernels read and advance, so
+  // no host-to-device copy is needed per transition.  lim is the end of a
+  // masked phase (rlt_append_spans).
+  std::vector<int32_t> enc_h, dec_h, lim_h;
+  int32_t* pos = nullptr;
   std::vector<void*> allocs;
   float* e = nullptr;          // [B][max_len][d]
+  float* et = nullptr;         // [B][d] encoder output of each sequence's position in flight
+  float* s_save = nullptr;     // [B][d] masked phases: rows of idle sequences, restored after a transition
+  void* zb_save = nullptr;     // [B][d] bf16
+  float* ss_save = nullptr;    // [d/128][B]
   void* mem_k = nullptr; void* mem_v = nullptr;  // [G][B][H][max_len][hd]
   void* ce_k = nullptr; void* ce_v = nullptr;    // [L][B][H][max_len][hd]
   void* ring_k = nullptr; void* ring_v = nullptr;  // [L][B][H][W-1][hd]
@@ -127,6 +139,7 @@ struct rlt_state {
   float* gate = nullptr;       // [B][d]
   float* logits = nullptr;     // [B][V]
   float* attn_ws = nullptr; size_t attn_ws_floats = 0;
+  int* attn_cnt = nullptr;     // [B][H] chunk counters of the decode attention (zero between launches)
   float* gemm_ws = nullptr; size_t gemm_ws_floats = 0;  // split-K exchange of the decode GEMMs (bf16)
   int32_t* pending = nullptr;  // [B] last sampled x_{t+1}, not yet consumed (report App. A, pending token)
   bool has_pending = false;
@@ -407,12 +420,24 @@ int32_t make_state(rlt_model* m, int32_t B, int32_t max_len, int32_t flags, rlt_
   }
   if ((r = A(&p, (int64_t)B * d * 4))) goto fail_;
   S->s = static_cast<float*>(p);
+  if ((r = A(&p, (int64_t)B * d * 4))) goto fail_;
+  S->et = static_cast<float*>(p);
+  if ((r = A(&p, (int64_t)B * d * 4))) goto fail_;
+  S->s_save = static_cast<float*>(p);
+  if ((r = A(&p, (int64_t)3 * B * 4))) goto fail_;
+  S->pos = static_cast<int32_t*>(p);
   if ((r = A(&S->xb, (int64_t)B * 2 * d * es))) goto fail_;
   if (c.dtype == RLT_DTYPE_BF16) {
     if ((r = A(&S->zb, (int64_t)B * d * 2))) goto fail_;
+    if ((r = A(&S->zb_save, (int64_t)B * d * 2))) goto fail_;
     if ((r = A(&p, (int64_t)(d / 128) * B * 4))) goto fail_;
     S->ss = static_cast<float*>(p);
+    if ((r = A(&p, (int64_t)(d / 128) * B * 4))) goto fail_;
+    S->ss_save = static_cast<float*>(p);
   }
+  S->enc_h.assign(B, 0);
+  S->dec_h.assign(B, 0);
+  S->lim_h.assign(B, 0);
   S->ld_qkv = std::max<int64_t>(3 * d, 2 * d * G);
   if ((r = A(&p, (int64_t)B * S->ld_qkv * 4))) goto fail_;
   S->qkv = static_cast<float*>(p);
@@ -425,6 +450,8 @@ int32_t make_state(rlt_model* m, int32_t B, int32_t max_len, int32_t flags, rlt_
   S->attn_ws_floats = prefix_attn_workspace_floats(B, c.n_heads, (int)(d / c.n_heads), max_len);
   if ((r = A(&p, (int64_t)S->attn_ws_floats * 4))) goto fail_;
   S->attn_ws = static_cast<float*>(p);
+  if ((r = A(&p, (int64_t)B * c.n_heads * 4))) goto fail_;
+  S->attn_cnt = static_cast<int*>(p);  // zeroed by reset_state
   if ((r = A(&p, (int64_t)B * 4))) goto fail_;
   S->pending = static_cast<int32_t*>(p);
   if (c.dtype == RLT_DTYPE_BF16) {
@@ -446,8 +473,10 @@ fail_:
 template <typename T>
 int32_t reset_state(rlt_state* S, cudaStream_t st) {
   RLT_CUDA(broadcast_row<T>(static_cast<const T*>(S->m->s_star), S->m->cfg.d_model, S->s, S->B, st));
-  S->n_enc = 0;
-  S->n_dec = 0;
+  RLT_CUDA(cudaMemsetAsync(S->pos, 0, (size_t)3 * S->B * 4, st));
+  RLT_CUDA(cudaMemsetAsync(S->attn_cnt, 0, (size_t)S->B * S->m->cfg.n_heads * 4, st));
+  std::fill(S->enc_h.begin(), S->enc_h.end(), 0);
+  std::fill(S->dec_h.begin(), S->dec_h.end(), 0);
   S->has_pending = false;
   S->version = S->m->version;
   return RLT_OK;
@@ -496,13 +525,30 @@ int32_t check_state(rlt_model* m, rlt_state* S) {
 }
 
 // ------------------------------------------------------------------ schedules
-// Token-parallel encoder over T tokens of every sequence (eq. 2.1) and the
-// memory projection of eq. 2.2, chunked over sequences.  With an encoded
-// prefix (n_enc > 0, keys and values in the encoder cache) the tokens are
-// positions n_enc+1..n_enc+T and attend to the cached prefix too: the
-// chunked schedule of the same causal computation (App. A.2).
+// Device views of a state's per-sequence positions.
+SeqPos seq_pos(const rlt_state* S, bool masked) {
+  return SeqPos{S->pos + S->B, S->pos, masked ? S->pos + 2 * S->B : nullptr};
+}
+bool active_h(const rlt_state* S, bool masked, int b) { return !masked || S->dec_h[b] < S->lim_h[b]; }
+// Keys an attention query of sequence b reads in the transition in flight
+// (the host image of SeqPos::n_keys).
+int n_keys_h(const rlt_state* S, bool masked, int b) {
+  return active_h(S, masked, b) ? S->dec_h[b] + 1 : std::max(1, S->dec_h[b]);
+}
+int max_of(const std::vector<int32_t>& v) { return v.empty() ? 0 : *std::max_element(v.begin(), v.end()); }
+bool uniform(const std::vector<int32_t>& v) {
+  return std::all_of(v.begin(), v.end(), [&](int32_t x) { return x == v[0]; });
+}
+
+// Token-parallel encoder (eq. 2.1) and the memory projection of eq. 2.2 over
+// Tn tokens of sequences [b_begin, b_end), which all stand at n_enc = p0;
+// sequence b's tokens are tok[b * ld_tok + 0..Tn-1].  Chunked over
+// sequences.  With p0 > 0 (keys and values of the prefix in the encoder
+// cache) the tokens are positions p0+1..p0+Tn and attend to the cached
+// prefix too: the chunked schedule of the same causal computation (App. A.2).
 template <typename T>
-int32_t encode_prefix_impl(rlt_model* m, rlt_state* S, const int32_t* tok, int32_t Tn, cudaStream_t st) {
+int32_t encode_prefix_impl(rlt_model* m, rlt_state* S, const int32_t* tok, int64_t ld_tok, int32_t Tn, int b_begin,
+                           int b_end, int p0, cudaStream_t st) {
   struct Range {
     bool on;
     explicit Range(bool o) : on(o) { if (on) nvtxRangePushA("rlt_sample"); }
@@ -513,14 +559,13 @@ int32_t encode_prefix_impl(rlt_model* m, rlt_state* S, const int32_t* tok, int32
   const int is_bf16 = c.dtype == RLT_DTYPE_BF16;
   const bool cache = (S->flags & RLT_STATE_ENCODER_CACHE) != 0;
   RLT_TRY(ensure_prefill_ws(S, Tn));
-  const int p0 = S->n_enc;  // positions p0+1..p0+Tn; p0 > 0 continues an encoded prefix (keys in the cache)
   const int64_t seqs_per_chunk = S->pf_rows / Tn;
-  for (int64_t b0 = 0; b0 < S->B; b0 += seqs_per_chunk) {
-    const int Bc = (int)std::min<int64_t>(seqs_per_chunk, S->B - b0);
+  for (int64_t b0 = b_begin; b0 < b_end; b0 += seqs_per_chunk) {
+    const int Bc = (int)std::min<int64_t>(seqs_per_chunk, b_end - b0);
     const int64_t rows = (int64_t)Bc * Tn;
     float* e0 = S->e + b0 * S->max_len * d + (int64_t)p0 * d;
     const RowMap emap{d, Tn, (int64_t)S->max_len * d};
-    RLT_CUDA(embed<T>(tok + b0 * Tn, rows, Tn, Tn, static_cast<const T*>(m->emb), d, c.vocab, e0, emap, st));
+    RLT_CUDA(embed<T>(tok + b0 * ld_tok, rows, Tn, ld_tok, static_cast<const T*>(m->emb), d, c.vocab, e0, emap, st));
     for (int l = 0; l < L; ++l) {
       const LayerW& w = m->layers[l];
       RLT_CUDA(rmsnorm<T, T>(e0, emap, static_cast<const T*>(w.g_ea), rows, d, c.rms_eps, static_cast<T*>(S->pf_x), d, st));
@@ -575,56 +620,87 @@ int32_t encode_prefix_impl(rlt_model* m, rlt_state* S, const int32_t* tok, int32
                                    static_cast<T*>(S->mem_v) + grp, S->max_len, st)));
     }
   }
-  S->n_enc = p0 + Tn;
+  RLT_CUDA(set_positions(S->pos, b_begin, b_end, p0 + Tn, st));
+  for (int b = b_begin; b < b_end; ++b) S->enc_h[b] = p0 + Tn;
   return RLT_OK;
 }
 
-// Encoder step (eq. 2.8) for x_t, t = n_enc + 1, and the memory append.
+// Encoder step (eq. 2.8) and memory append for the token x_t of every
+// sequence whose position t = n_dec + 1 is not yet encoded (n_enc < t); the
+// other sequences' rows are computed but written nowhere.  The step works on
+// S->et (one row per sequence) and then stores the encoded rows into e.
 template <typename T>
-int32_t encode_step_impl(rlt_model* m, rlt_state* S, const int32_t* tok, cudaStream_t st) {
+int32_t encode_step_impl(rlt_model* m, rlt_state* S, const int32_t* tok, bool masked, cudaStream_t st) {
   const rlt_config& c = m->cfg;
   const int d = c.d_model, H = c.n_heads, hd = m->hd, F = c.ffn, G = c.groups, L = c.n_layers, B = S->B;
   const int is_bf16 = c.dtype == RLT_DTYPE_BF16;
-  const int t = S->n_enc + 1;
-  m->prof.sample_now = (t % 4) == 0;
-  float* et = S->e + (int64_t)(t - 1) * d;
-  const RowMap emap = plain_rows((int64_t)S->max_len * d);
-  RLT_CUDA(embed<T>(tok, B, 1, 1, static_cast<const T*>(m->emb), d, c.vocab, et, emap, st));
+  const SeqPos sp = seq_pos(S, masked);
+  int n_max = 1;
+  double key_rows = 0;
+  for (int b = 0; b < B; ++b) {
+    n_max = std::max(n_max, n_keys_h(S, masked, b));
+    key_rows += n_keys_h(S, masked, b);
+  }
+  m->prof.sample_now = ((max_of(S->dec_h) + 1) % 4) == 0;
+  float* et = S->et;
+  const RowMap erow = plain_rows(d);
+  // bf16 models fold the pre-norms after the first into the GEMMs, as the
+  // decoder does: each residual epilogue leaves gamma_next * e and the sums of
+  // squares, and the next GEMM scales its accumulators by 1/rms.  The folded
+  // operand lives in the state's zb/ss, which the transition that follows
+  // overwrites.
+  constexpr bool fused = std::is_same<T, bf16>::value;
+  auto normed_in = [&](const void* gamma, bool first) -> int32_t {
+    if (fused && !first) return RLT_OK;
+    RLT_CUDA(rmsnorm<T, T>(et, erow, static_cast<const T*>(gamma), B, d, c.rms_eps, static_cast<T*>(S->xb), d, st));
+    return RLT_OK;
+  };
+  auto xin = [&](bool first) -> const void* { return (fused && !first) ? S->zb : S->xb; };
+  auto cin = [&](EpiParams p, bool first) { return (fused && !first) ? norm_in(p, S) : p; };
+  auto cout_ = [&](EpiParams p, const void* gamma_next) { return fused ? norm_out(p, S, gamma_next) : p; };
+  RLT_CUDA(embed<T>(tok, B, 1, 1, static_cast<const T*>(m->emb), d, c.vocab, et, erow, st));
   for (int l = 0; l < L; ++l) {
     const LayerW& w = m->layers[l];
     const int64_t lay = (int64_t)l * B * H * S->max_len * hd;
     T* ck = static_cast<T*>(S->ce_k) + lay;
     T* cv = static_cast<T*>(S->ce_v) + lay;
-    RLT_CUDA(rmsnorm<T, T>(et, emap, static_cast<const T*>(w.g_ea), B, d, c.rms_eps, static_cast<T*>(S->xb), d, st));
-    RLT_TRY(gemm<T>(S, w.qkv, d, S->xb, d, 3 * d, B, d, EPI_STORE, epi_out(S->qkv, plain_rows(S->ld_qkv), 0), true, st));
-    RLT_CUDA((head_scatter<float, T>(S->qkv, S->ld_qkv, d, B, 1, t - 1, t - 1, H, hd, 1, m->rope_cs, ck, S->max_len, st)));
-    RLT_CUDA((head_scatter<float, T>(S->qkv, S->ld_qkv, 2 * d, B, 1, t - 1, t - 1, H, hd, 0, m->rope_cs, cv, S->max_len, st)));
+    const void* g_next = l + 1 < L ? m->layers[l + 1].g_ea : m->g_mem;
+    RLT_TRY(normed_in(w.g_ea, l == 0));
+    RLT_TRY(gemm<T>(S, w.qkv, d, xin(l == 0), d, 3 * d, B, d, EPI_STORE,
+                    cin(epi_out(S->qkv, plain_rows(S->ld_qkv), 0), l == 0), true, st));
+    RLT_CUDA((head_insert<float, T>(S->qkv, S->ld_qkv, d, B, sp, H, hd, 1, m->rope_cs, ck, S->max_len, st)));
+    RLT_CUDA((head_insert<float, T>(S->qkv, S->ld_qkv, 2 * d, B, sp, H, hd, 0, m->rope_cs, cv, S->max_len, st)));
     prof_begin(m, st);
-    RLT_CUDA(prefix_attn<T>(S->qkv, S->ld_qkv, ck, cv, S->max_len, B, H, hd, t, t - 1, m->rope_cs,
-                            static_cast<T*>(S->attn), d, S->attn_ws, S->attn_ws_floats, st));
-    prof_end(m, st, 0, (double)B * H * t * hd * 2 * m->esz);
-    RLT_TRY(gemm<T>(S, w.wo, d, S->attn, d, d, B, d, EPI_RESID, epi_out(et, emap, 0), true, st));
-    RLT_CUDA(rmsnorm<T, T>(et, emap, static_cast<const T*>(w.g_ef), B, d, c.rms_eps, static_cast<T*>(S->xb), d, st));
-    RLT_TRY(gemm<T>(S, w.w13, d, S->xb, d, 2 * F, B, d, EPI_SWIGLU, epi_out(S->hbuf, plain_rows(F), is_bf16), true, st));
-    RLT_TRY(gemm<T>(S, w.w2, F, S->hbuf, F, d, B, F, EPI_RESID, epi_out(et, emap, 0), true, st));
+    RLT_CUDA(prefix_attn<T>(S->qkv, S->ld_qkv, ck, cv, S->max_len, B, H, hd, n_max, n_max - 1, sp, m->rope_cs,
+                            static_cast<T*>(S->attn), d, S->attn_ws, S->attn_ws_floats, S->attn_cnt, st));
+    prof_end(m, st, 0, key_rows * H * hd * 2 * m->esz);
+    RLT_TRY(gemm<T>(S, w.wo, d, S->attn, d, d, B, d, EPI_RESID, cout_(epi_out(et, erow, 0), w.g_ef), true, st));
+    RLT_TRY(normed_in(w.g_ef, false));
+    RLT_TRY(gemm<T>(S, w.w13, d, xin(false), d, 2 * F, B, d, EPI_SWIGLU,
+                    cin(epi_out(S->hbuf, plain_rows(F), is_bf16), false), true, st));
+    RLT_TRY(gemm<T>(S, w.w2, F, S->hbuf, F, d, B, F, EPI_RESID, cout_(epi_out(et, erow, 0), g_next), true, st));
   }
-  RLT_CUDA(rmsnorm<T, T>(et, emap, static_cast<const T*>(m->g_mem), B, d, c.rms_eps, static_cast<T*>(S->xb), d, st));
-  RLT_TRY(gemm<T>(S, m->w_kvm, d, S->xb, d, 2 * d * G, B, d, EPI_STORE, epi_out(S->qkv, plain_rows(S->ld_qkv), 0),
-                  true, st));
+  RLT_TRY(normed_in(m->g_mem, false));
+  RLT_TRY(gemm<T>(S, m->w_kvm, d, xin(false), d, 2 * d * G, B, d, EPI_STORE,
+                  cin(epi_out(S->qkv, plain_rows(S->ld_qkv), 0), false), true, st));
   for (int g = 0; g < G; ++g) {
     const int64_t grp = (int64_t)g * B * H * S->max_len * hd;
-    RLT_CUDA((head_scatter<float, T>(S->qkv, S->ld_qkv, (int64_t)2 * d * g, B, 1, t - 1, t - 1, H, hd, 1, m->rope_cs,
-                                     static_cast<T*>(S->mem_k) + grp, S->max_len, st)));
-    RLT_CUDA((head_scatter<float, T>(S->qkv, S->ld_qkv, (int64_t)2 * d * g + d, B, 1, t - 1, t - 1, H, hd, 0, m->rope_cs,
-                                     static_cast<T*>(S->mem_v) + grp, S->max_len, st)));
+    RLT_CUDA((head_insert<float, T>(S->qkv, S->ld_qkv, (int64_t)2 * d * g, B, sp, H, hd, 1, m->rope_cs,
+                                    static_cast<T*>(S->mem_k) + grp, S->max_len, st)));
+    RLT_CUDA((head_insert<float, T>(S->qkv, S->ld_qkv, (int64_t)2 * d * g + d, B, sp, H, hd, 0, m->rope_cs,
+                                    static_cast<T*>(S->mem_v) + grp, S->max_len, st)));
   }
-  S->n_enc = t;
+  RLT_CUDA(erow_scatter(et, S->max_len, d, B, sp, S->e, st));
   return RLT_OK;
 }
 
 // One decoder transition H_t = D_phi(Merge(e_t, s_{t-1}); M_<=t, C^D_{t-1}, t)
-// (eqs. 2.4-2.5, 2.9-2.16) for t = n_dec + 1.  s is updated in place: it
-// holds u_t after the merge, then z^l after every block, and s_t at the end.
+// (eqs. 2.4-2.5, 2.9-2.16) for every sequence b at its own t_b = n_dec[b] + 1.
+// s is updated in place: it holds u_t after the merge, then z^l after every
+// block, and s_t at the end.  In a masked phase only the sequences with
+// n_dec < lim take part: the others' rows are computed, their ring and
+// positions left as they were, and their s restored at the end.  `et_ready`:
+// S->et already holds e_t of every sequence (the encoder step ran for all).
 // While profiling is on, every 4th transition records kernel events
 // (prof_begin/prof_end), and each position with t = 64 (mod 128) -- its
 // encoder step, transition and readout -- is wrapped in an NVTX range named
@@ -644,18 +720,30 @@ struct StepRange {
 };
 
 template <typename T>
-int32_t transition_impl(rlt_model* m, rlt_state* S, cudaStream_t st) {
+int32_t transition_impl(rlt_model* m, rlt_state* S, bool masked, bool et_ready, cudaStream_t st) {
   const rlt_config& c = m->cfg;
   const int d = c.d_model, H = c.n_heads, hd = m->hd, F = c.ffn, L = c.n_layers, B = S->B, W = c.window;
   const int is_bf16 = c.dtype == RLT_DTYPE_BF16;
-  const int t = S->n_dec + 1;
-  m->prof.sample_now = (t % 4) == 0;
-  const float* et = S->e + (int64_t)(t - 1) * d;
-  const RowMap emap = plain_rows((int64_t)S->max_len * d);
+  const SeqPos sp = seq_pos(S, masked);
+  int n_max = 1;
+  double key_rows = 0, ring_rows = 0;
+  for (int b = 0; b < B; ++b) {
+    const int n = n_keys_h(S, masked, b);
+    n_max = std::max(n_max, n);
+    key_rows += n;
+    ring_rows += std::min(S->dec_h[b], W - 1) + ((W > 1 && active_h(S, masked, b)) ? 1 : 0);
+  }
+  m->prof.sample_now = ((max_of(S->dec_h) + 1) % 4) == 0;
   const RowMap srow = plain_rows(d);
   constexpr bool fused = std::is_same<T, bf16>::value;  // folded RMSNorm on the tensor-core path
+  const int n_ss = fused ? d / 128 : 0;
+  if (masked)
+    RLT_CUDA(save_rows(S->s, S->s_save, static_cast<const bf16*>(S->zb), static_cast<bf16*>(S->zb_save), S->ss,
+                       S->ss_save, B, d, n_ss, st));
+  if (!et_ready) RLT_CUDA(erow_gather(S->e, S->max_len, d, B, sp, S->et, st));
+  const float* et = S->et;
   // merge
-  RLT_CUDA((merge_prep<T, T>(et, emap, S->s, static_cast<const T*>(m->g_merge), B, d, c.rms_eps, c.merge_kind,
+  RLT_CUDA((merge_prep<T, T>(et, srow, S->s, static_cast<const T*>(m->g_merge), B, d, c.rms_eps, c.merge_kind,
                              static_cast<T*>(S->xb), st)));
   if (c.merge_kind == RLT_MERGE_PAPER) {
     EpiParams g = epi_out(S->gate, srow, 0);
@@ -664,7 +752,7 @@ int32_t transition_impl(rlt_model* m, rlt_state* S, cudaStream_t st) {
     RLT_TRY(gemm<T>(S, m->w_gate, 2 * d, S->xb, 2 * d, d, B, 2 * d, EPI_GATE, g, true, st));
     EpiParams u = epi_out(S->s, srow, 0);
     u.aux0 = et;
-    u.aux0_map = emap;
+    u.aux0_map = srow;
     u.aux1 = S->gate;
     u.ld_aux1 = d;
     u.alpha = c.alpha;
@@ -673,7 +761,7 @@ int32_t transition_impl(rlt_model* m, rlt_state* S, cudaStream_t st) {
   } else {
     EpiParams u = epi_out(S->s, srow, 0);
     u.aux0 = et;
-    u.aux0_map = emap;
+    u.aux0_map = srow;
     if (fused) u = norm_out(u, S, m->layers[0].g_dsa);
     RLT_TRY(gemm<T>(S, m->w_gate, 2 * d, S->xb, 2 * d, d, B, 2 * d, EPI_CONVEX, u, true, st));
   }
@@ -687,7 +775,6 @@ int32_t transition_impl(rlt_model* m, rlt_state* S, cudaStream_t st) {
   const void* xin = fused ? S->zb : S->xb;
   auto cin = [&](EpiParams p) { return fused ? norm_in(p, S) : p; };
   auto cout_ = [&](EpiParams p, const void* gamma_next) { return fused ? norm_out(p, S, gamma_next) : p; };
-  const int n_ring = std::min(t - 1, W - 1);
   for (int l = 0; l < L; ++l) {
     const LayerW& w = m->layers[l];
     const int grp = c.groups == 1 ? 0 : l;
@@ -699,8 +786,8 @@ int32_t transition_impl(rlt_model* m, rlt_state* S, cudaStream_t st) {
     T* rk = W > 1 ? static_cast<T*>(S->ring_k) + rlay : nullptr;
     T* rv = W > 1 ? static_cast<T*>(S->ring_v) + rlay : nullptr;
     prof_begin(m, st);
-    RLT_CUDA(swa_attn<T>(S->qkv, 3 * d, rk, rv, B, H, hd, t, W, m->rope_cs, static_cast<T*>(S->attn), d, st));
-    prof_end(m, st, 1, (double)B * H * hd * m->esz * (2.0 * n_ring + (W > 1 ? 2.0 : 0.0)));
+    RLT_CUDA(swa_attn<T>(S->qkv, 3 * d, rk, rv, B, H, hd, 0, sp, W, m->rope_cs, static_cast<T*>(S->attn), d, st));
+    prof_end(m, st, 1, ring_rows * H * hd * m->esz * 2.0);
     RLT_TRY(gemm<T>(S, w.dwo, d, S->attn, d, d, B, d, EPI_RESID, cout_(epi_out(S->s, srow, 0), w.g_dmem), true, st));
     // cross-attention to M^{g(l)}_{<=t} (eq. 2.15)
     RLT_TRY(normed(w.g_dmem));
@@ -708,9 +795,9 @@ int32_t transition_impl(rlt_model* m, rlt_state* S, cudaStream_t st) {
     const int64_t mg = (int64_t)grp * B * H * S->max_len * hd;
     prof_begin(m, st);
     RLT_CUDA(prefix_attn<T>(S->qkv, d, static_cast<const T*>(S->mem_k) + mg, static_cast<const T*>(S->mem_v) + mg,
-                            S->max_len, B, H, hd, t, t - 1, m->rope_cs, static_cast<T*>(S->attn), d, S->attn_ws,
-                            S->attn_ws_floats, st));
-    prof_end(m, st, 0, (double)B * H * t * hd * 2 * m->esz);
+                            S->max_len, B, H, hd, n_max, n_max - 1, sp, m->rope_cs, static_cast<T*>(S->attn), d,
+                            S->attn_ws, S->attn_ws_floats, S->attn_cnt, st));
+    prof_end(m, st, 0, key_rows * H * hd * 2 * m->esz);
     RLT_TRY(gemm<T>(S, w.wo_mem, d, S->attn, d, d, B, d, EPI_RESID, cout_(epi_out(S->s, srow, 0), w.g_dffn), true, st));
     // FFN (eq. 2.16)
     RLT_TRY(normed(w.g_dffn));
@@ -718,15 +805,25 @@ int32_t transition_impl(rlt_model* m, rlt_state* S, cudaStream_t st) {
                     st));
     RLT_TRY(gemm<T>(S, w.dw2, F, S->hbuf, F, d, B, F, EPI_RESID, cout_(epi_out(S->s, srow, 0), g_next), true, st));
   }
-  S->n_dec = t;
+  // positions (and, for idle sequences of a masked phase, their saved rows)
+  RLT_CUDA(advance_positions(S->pos + B, S->pos, masked ? S->pos + 2 * B : nullptr, B, d, S->s,
+                             masked ? S->s_save : nullptr, static_cast<bf16*>(S->zb),
+                             static_cast<const bf16*>(S->zb_save), S->ss, S->ss_save, n_ss, st));
+  for (int b = 0; b < B; ++b) {
+    if (!active_h(S, masked, b)) continue;
+    S->dec_h[b] += 1;
+    S->enc_h[b] = std::max(S->enc_h[b], S->dec_h[b]);
+  }
   return RLT_OK;
 }
 
 // Readout (eq. 2.6) of s_t: logits = W_o RMSNorm_o(s_t), then the teacher
-// log-prob and/or the behaviour sample.
+// log-prob and/or the behaviour sample (the sampler's position is each
+// sequence's own n_dec).  In a masked phase the log-prob is written only for
+// the sequences whose phase has a next token left.
 template <typename T>
 int32_t readout_impl(rlt_model* m, rlt_state* S, const int32_t* next, int64_t next_stride, float* logp, int64_t ld_logp,
-                     const rlt_sampling* samp, const rlt_readout_out* out, cudaStream_t st) {
+                     const rlt_sampling* samp, const rlt_readout_out* out, bool masked, cudaStream_t st) {
   const rlt_config& c = m->cfg;
   const int d = c.d_model, V = c.vocab, B = S->B;
   if constexpr (std::is_same<T, bf16>::value) {
@@ -738,10 +835,12 @@ int32_t readout_impl(rlt_model* m, rlt_state* S, const int32_t* next, int64_t ne
                            static_cast<T*>(S->xb), d, st));
     RLT_TRY(gemm<T>(S, m->w_out, d, S->xb, d, V, B, d, EPI_STORE, epi_out(S->logits, plain_rows(V), 0), true, st));
   }
-  if (next && logp) RLT_CUDA(logp_gather(S->logits, B, V, next, next_stride, logp, ld_logp, st));
+  if (next && logp)
+    RLT_CUDA(logp_gather(S->logits, B, V, next, next_stride, logp, ld_logp, S->pos + B,
+                         masked ? S->pos + 2 * B : nullptr, st));
   if (samp) {
     int32_t* tok_out = out && out->sampled ? out->sampled : S->pending;
-    RLT_CUDA(sample_topk(S->logits, B, V, samp->temperature, samp->top_k, samp->seed, (uint32_t)S->n_dec, tok_out,
+    RLT_CUDA(sample_topk(S->logits, B, V, samp->temperature, samp->top_k, samp->seed, 0, S->pos + B, tok_out,
                          out ? out->logp_sampled : nullptr, out ? out->logmu : nullptr, st));
     if (tok_out != S->pending)
       RLT_CUDA(cudaMemcpyAsync(S->pending, tok_out, (size_t)B * 4, cudaMemcpyDeviceToDevice, st));
@@ -880,13 +979,28 @@ int32_t rlt_state_info_get(const rlt_state* s, rlt_state_info* out) {
   const int Wm1 = s->m->cfg.window - 1;
   out->batch = s->B;
   out->max_len = s->max_len;
-  out->n_enc = s->n_enc;
-  out->n_dec = s->n_dec;
-  out->ring_valid = std::min(s->n_dec, Wm1);
-  out->ring_head = Wm1 > 0 ? s->n_dec % Wm1 : 0;
+  const int n_enc = max_of(s->enc_h), n_dec = max_of(s->dec_h);
+  out->n_enc = n_enc;
+  out->n_dec = n_dec;
+  out->ring_valid = std::min(n_dec, Wm1);
+  out->ring_head = Wm1 > 0 ? n_dec % Wm1 : 0;
   out->has_encoder_cache = (s->flags & RLT_STATE_ENCODER_CACHE) ? 1 : 0;
   out->model_version = s->version;
   out->has_pending = s->has_pending ? 1 : 0;
+  out->uniform = (uniform(s->enc_h) && uniform(s->dec_h)) ? 1 : 0;
+  return ok();
+}
+
+int32_t rlt_state_positions(const rlt_state* s, int32_t* n_enc, int32_t* n_dec, int32_t* ring_valid,
+                            int32_t* ring_head) {
+  if (!s) return fail(RLT_E_INVAL, "null state");
+  const int Wm1 = s->m->cfg.window - 1;
+  for (int b = 0; b < s->B; ++b) {
+    if (n_enc) n_enc[b] = s->enc_h[b];
+    if (n_dec) n_dec[b] = s->dec_h[b];
+    if (ring_valid) ring_valid[b] = std::min(s->dec_h[b], Wm1);
+    if (ring_head) ring_head[b] = Wm1 > 0 ? s->dec_h[b] % Wm1 : 0;
+  }
   return ok();
 }
 
@@ -904,7 +1018,7 @@ struct SnapHeader {
   int32_t n_enc, n_dec, reserved0, reserved1;
   uint64_t weight_seed, model_version, payload_bytes;
 };
-constexpr uint32_t kSnapCache = 1, kSnapPending = 2, kSnapFold = 4;
+constexpr uint32_t kSnapCache = 1, kSnapPending = 2, kSnapFold = 4, kSnapRagged = 8;
 
 struct SnapSection {
   void* dev;      // first byte on the device
@@ -938,6 +1052,8 @@ std::vector<SnapSection> snapshot_sections(rlt_state* S, int n_enc, uint32_t fla
     v.push_back({S->zb, B * d * 2, B * d * 2, 1});
     v.push_back({S->ss, (d / 128) * B * 4, (d / 128) * B * 4, 1});
   }
+  // per-sequence positions n_enc[B], n_dec[B] (the first 2B entries of pos)
+  if (flags & kSnapRagged) v.push_back({S->pos, 2 * B * 4, 2 * B * 4, 1});
   return v;
 }
 
@@ -949,9 +1065,10 @@ size_t payload_bytes(const std::vector<SnapSection>& v) {
 
 uint32_t snapshot_flags(const rlt_state* S) {
   uint32_t f = 0;
-  if ((S->flags & RLT_STATE_ENCODER_CACHE) && S->n_enc > 0) f |= kSnapCache;
+  if ((S->flags & RLT_STATE_ENCODER_CACHE) && max_of(S->enc_h) > 0) f |= kSnapCache;
   if (S->has_pending) f |= kSnapPending;
-  if (S->m->cfg.dtype == RLT_DTYPE_BF16 && S->n_dec > 0) f |= kSnapFold;
+  if (S->m->cfg.dtype == RLT_DTYPE_BF16 && max_of(S->dec_h) > 0) f |= kSnapFold;
+  if (!uniform(S->enc_h) || !uniform(S->dec_h)) f |= kSnapRagged;
   return f;
 }
 
@@ -1000,7 +1117,7 @@ int32_t rlt_state_export(const rlt_state* s_const, void* host, size_t cap, size_
   rlt_state* S = const_cast<rlt_state*>(s_const);
   const rlt_model* m = S->m;
   const uint32_t flags = snapshot_flags(S);
-  const std::vector<SnapSection> secs = snapshot_sections(S, S->n_enc, flags);
+  const std::vector<SnapSection> secs = snapshot_sections(S, max_of(S->enc_h), flags);
   const size_t total = sizeof(SnapHeader) + payload_bytes(secs);
   *used = total;
   if (!host) return ok();
@@ -1014,7 +1131,7 @@ int32_t rlt_state_export(const rlt_state* s_const, void* host, size_t cap, size_
   h.ffn = c.ffn; h.vocab = c.vocab; h.tied = c.tied; h.merge_kind = c.merge_kind; h.dtype = c.dtype;
   h.bos_id = c.bos_id; h.batch = S->B;
   h.alpha = c.alpha; h.rms_eps = c.rms_eps; h.rope_base = c.rope_base;
-  h.n_enc = S->n_enc; h.n_dec = S->n_dec;
+  h.n_enc = max_of(S->enc_h); h.n_dec = max_of(S->dec_h);
   h.weight_seed = m->seed; h.model_version = S->version;
   h.payload_bytes = total - sizeof(SnapHeader);
   std::memcpy(host, &h, sizeof h);
@@ -1026,6 +1143,27 @@ int32_t rlt_state_export(const rlt_state* s_const, void* host, size_t cap, size_
     dst += x.width * x.rows;
   }
   RLT_CUDA(cudaStreamSynchronize(st));
+  if (flags & kSnapRagged) {
+    // The per-position sections hold the furthest sequence's rows for every
+    // sequence; the rows a shorter sequence has not reached were never
+    // written, so the snapshot carries zeros there (its contents then depend
+    // only on the state's history).
+    const size_t d = c.d_model, hd = m->hd, es = m->esz, B = S->B, H = c.n_heads;
+    dst = static_cast<uint8_t*>(host) + sizeof h;
+    for (const auto& x : secs) {
+      const bool e_sec = x.dev == S->e;
+      const bool kv_sec = x.dev == S->mem_k || x.dev == S->mem_v || x.dev == S->ce_k || x.dev == S->ce_v;
+      if (e_sec || kv_sec) {
+        const size_t row_bytes = e_sec ? d * 4 : hd * es;
+        for (size_t r = 0; r < x.rows; ++r) {
+          const size_t b = e_sec ? r : (r / H) % B;
+          const size_t keep = (size_t)S->enc_h[b] * row_bytes;
+          if (keep < x.width) std::memset(dst + r * x.width + keep, 0, x.width - keep);
+        }
+      }
+      dst += x.width * x.rows;
+    }
+  }
   return ok();
 }
 
@@ -1056,6 +1194,16 @@ int32_t rlt_state_import(rlt_state* S, const void* host, size_t bytes, void* str
   const std::vector<SnapSection> secs = snapshot_sections(S, h.n_enc, h.flags);
   if (h.payload_bytes != payload_bytes(secs) || bytes < sizeof(SnapHeader) + h.payload_bytes)
     return fail(RLT_E_INVAL, "snapshot payload size mismatch");
+  // per-sequence positions: the ragged section (the payload's last), else
+  // every sequence at the header's positions
+  std::vector<int32_t> enc(S->B, h.n_enc), dec(S->B, h.n_dec);
+  if (h.flags & kSnapRagged) {
+    const uint8_t* pp = static_cast<const uint8_t*>(host) + sizeof h + h.payload_bytes - (size_t)2 * S->B * 4;
+    std::memcpy(enc.data(), pp, (size_t)S->B * 4);
+    std::memcpy(dec.data(), pp + (size_t)S->B * 4, (size_t)S->B * 4);
+    for (int b = 0; b < S->B; ++b)
+      if (dec[b] < 0 || dec[b] > enc[b] || enc[b] > h.n_enc) return fail(RLT_E_INVAL, "bad positions in snapshot");
+  }
   RLT_CUDA(cudaSetDevice(m->device));
   cudaStream_t st = (cudaStream_t)stream;
   const uint8_t* src = static_cast<const uint8_t*>(host) + sizeof h;
@@ -1066,9 +1214,13 @@ int32_t rlt_state_import(rlt_state* S, const void* host, size_t bytes, void* str
       RLT_CUDA(cudaMemcpy2DAsync(x.dev, x.pitch, src, x.width, x.width, x.rows, cudaMemcpyHostToDevice, st));
     src += x.width * x.rows;
   }
+  if (!(h.flags & kSnapRagged)) {
+    RLT_CUDA(set_positions(S->pos, 0, S->B, h.n_enc, st));
+    RLT_CUDA(set_positions(S->pos + S->B, 0, S->B, h.n_dec, st));
+  }
   RLT_CUDA(cudaStreamSynchronize(st));
-  S->n_enc = h.n_enc;
-  S->n_dec = h.n_dec;
+  S->enc_h = enc;
+  S->dec_h = dec;
   S->has_pending = (h.flags & kSnapPending) != 0;
   S->version = m->version;
   return ok();
@@ -1077,55 +1229,114 @@ int32_t rlt_state_import(rlt_state* S, const void* host, size_t bytes, void* str
 int32_t rlt_encode_prefix(rlt_model* m, rlt_state* s, const int32_t* tok_dev, int32_t T, void* stream) {
   RLT_TRY(check_state(m, s));
   if (!tok_dev || T <= 0) return fail(RLT_E_INVAL, "need tokens and T > 0");
-  if (s->n_enc != 0 && !(s->flags & RLT_STATE_ENCODER_CACHE))
+  if (!uniform(s->enc_h))
+    return fail(RLT_E_STATE, "the sequences have encoded different numbers of tokens: use rlt_append_spans");
+  const int p0 = s->enc_h[0];
+  if (p0 != 0 && !(s->flags & RLT_STATE_ENCODER_CACHE))
     return fail(RLT_E_STATE, "continuing an encoded prefix needs the encoder cache");
-  if ((int64_t)s->n_enc + T > s->max_len) return fail(RLT_E_CAPACITY, "n_enc + T exceeds max_len");
-  return RLT_DISPATCH(m, encode_prefix_impl, m, s, tok_dev, T, (cudaStream_t)stream);
+  if ((int64_t)p0 + T > s->max_len) return fail(RLT_E_CAPACITY, "n_enc + T exceeds max_len");
+  return RLT_DISPATCH(m, encode_prefix_impl, m, s, tok_dev, (int64_t)T, T, 0, s->B, p0, (cudaStream_t)stream);
+}
+
+int32_t rlt_append_spans(rlt_model* m, rlt_state* s, const int32_t* tok_dev, int64_t ld_tok, const int32_t* lens,
+                         float* logp_dev, int64_t ld_logp, void* stream) {
+  RLT_TRY(check_state(m, s));
+  if (!tok_dev || !lens) return fail(RLT_E_INVAL, "null tokens or lengths");
+  int max_len_span = 0;
+  for (int b = 0; b < s->B; ++b) {
+    if (lens[b] < 0) return fail(RLT_E_INVAL, "negative span length");
+    max_len_span = std::max(max_len_span, (int)lens[b]);
+  }
+  if (max_len_span == 0) return fail(RLT_E_INVAL, "every span is empty");
+  if (ld_tok < max_len_span) return fail(RLT_E_INVAL, "ld_tok is shorter than the longest span");
+  if (logp_dev && ld_logp < max_len_span - 1) return fail(RLT_E_INVAL, "ld_logp is shorter than the longest span - 1");
+  if (s->has_pending) return fail(RLT_E_STATE, "a sampled token is pending: consume it with rlt_decoder_step first");
+  for (int b = 0; b < s->B; ++b) {
+    if (s->enc_h[b] != s->dec_h[b])
+      return fail(RLT_E_STATE, "sequence " + std::to_string(b) + " has encoded tokens not yet consumed");
+    if ((int64_t)s->enc_h[b] + lens[b] > s->max_len)
+      return fail(RLT_E_CAPACITY, "sequence " + std::to_string(b) + ": n_enc + span exceeds max_len");
+    if (lens[b] > 0 && s->enc_h[b] > 0 && !(s->flags & RLT_STATE_ENCODER_CACHE))
+      return fail(RLT_E_STATE, "appending to an encoded prefix needs the encoder cache");
+  }
+  cudaStream_t st = (cudaStream_t)stream;
+  // token-parallel encoding of each run of consecutive sequences with the
+  // same position and span length (App. A.2, chunked encoder)
+  for (int b0 = 0; b0 < s->B;) {
+    int b1 = b0 + 1;
+    while (b1 < s->B && lens[b1] == lens[b0] && s->enc_h[b1] == s->enc_h[b0]) ++b1;
+    if (lens[b0] > 0)
+      RLT_TRY(RLT_DISPATCH(m, encode_prefix_impl, m, s, tok_dev, ld_tok, (int32_t)lens[b0], b0, b1, s->enc_h[b0], st));
+    b0 = b1;
+  }
+  // then every span token gets its transition, in lock step; a sequence
+  // whose span is over sits out the remaining transitions (masked phase)
+  for (int b = 0; b < s->B; ++b) s->lim_h[b] = s->dec_h[b] + lens[b];
+  RLT_CUDA(cudaMemcpyAsync(s->pos + 2 * s->B, s->lim_h.data(), (size_t)s->B * 4, cudaMemcpyHostToDevice, st));
+  for (int k = 1; k <= max_len_span; ++k) {
+    StepRange range(m, max_of(s->dec_h) + 1);
+    RLT_TRY(RLT_DISPATCH(m, transition_impl, m, s, true, false, st));
+    if (logp_dev && k < max_len_span)
+      RLT_TRY(RLT_DISPATCH(m, readout_impl, m, s, tok_dev + k, ld_tok, logp_dev + (k - 1), ld_logp,
+                           (const rlt_sampling*)nullptr, (const rlt_readout_out*)nullptr, true, st));
+  }
+  return ok();
 }
 
 int32_t rlt_readout(rlt_model* m, rlt_state* s, const int32_t* next_dev, const rlt_sampling* samp,
                     const rlt_readout_out* out, void* stream) {
   RLT_TRY(check_state(m, s));
-  if (s->n_dec < 1) return fail(RLT_E_STATE, "readout needs at least one transition");
+  if (*std::min_element(s->dec_h.begin(), s->dec_h.end()) < 1)
+    return fail(RLT_E_STATE, "readout needs at least one transition of every sequence");
   RLT_TRY(check_sampling(samp, out));
   return RLT_DISPATCH(m, readout_impl, m, s, next_dev, (int64_t)1, out ? out->logp : nullptr, (int64_t)1, samp, out,
-                      (cudaStream_t)stream);
+                      false, (cudaStream_t)stream);
 }
 
 int32_t rlt_decoder_step(rlt_model* m, rlt_state* s, const int32_t* tok_dev, const int32_t* next_dev,
                          const rlt_sampling* samp, const rlt_readout_out* out, void* stream) {
   RLT_TRY(check_state(m, s));
   RLT_TRY(check_sampling(samp, out));
-  const int t = s->n_dec + 1;
-  if (t > s->max_len) return fail(RLT_E_CAPACITY, "position would pass max_len");
+  // every sequence takes its transition at its own t_b = n_dec[b] + 1; the
+  // ones whose x_t is not yet encoded run the encoder step first
+  int t_max = 0;
+  bool any_enc = false, all_enc = true;
+  for (int b = 0; b < s->B; ++b) {
+    const int t = s->dec_h[b] + 1;
+    t_max = std::max(t_max, t);
+    if (s->enc_h[b] < t) any_enc = true;
+    else all_enc = false;
+  }
+  if (t_max > s->max_len) return fail(RLT_E_CAPACITY, "position would pass max_len");
   cudaStream_t st = (cudaStream_t)stream;
-  StepRange range(m, t);
-  if (s->n_enc < t) {
+  StepRange range(m, t_max);
+  if (any_enc) {
     if (!(s->flags & RLT_STATE_ENCODER_CACHE)) return fail(RLT_E_STATE, "x_t not encoded and the state has no encoder cache");
     if (!tok_dev && !s->has_pending)
       return fail(RLT_E_STATE, "x_t must be given: it is not yet encoded and no sampled token is pending");
-    RLT_TRY(RLT_DISPATCH(m, encode_step_impl, m, s, tok_dev ? tok_dev : s->pending, st));
+    RLT_TRY(RLT_DISPATCH(m, encode_step_impl, m, s, tok_dev ? tok_dev : s->pending, false, st));
   }
-  RLT_TRY(RLT_DISPATCH(m, transition_impl, m, s, st));
+  RLT_TRY(RLT_DISPATCH(m, transition_impl, m, s, false, any_enc && all_enc, st));
   s->has_pending = false;
   if (next_dev || samp || (out && out->logits))
-    RLT_TRY(RLT_DISPATCH(m, readout_impl, m, s, next_dev, (int64_t)1, out ? out->logp : nullptr, (int64_t)1, samp, out, st));
+    RLT_TRY(RLT_DISPATCH(m, readout_impl, m, s, next_dev, (int64_t)1, out ? out->logp : nullptr, (int64_t)1, samp, out,
+                         false, st));
   return ok();
 }
 
 int32_t rlt_prefill(rlt_model* m, rlt_state* s, const int32_t* tok_dev, int32_t T, float* logp_dev, void* stream) {
   RLT_TRY(check_state(m, s));
   if (!tok_dev || T <= 0) return fail(RLT_E_INVAL, "need tokens and T > 0");
-  if (s->n_enc != 0 || s->n_dec != 0) return fail(RLT_E_STATE, "prefill starts from H_0");
+  if (max_of(s->enc_h) != 0 || max_of(s->dec_h) != 0) return fail(RLT_E_STATE, "prefill starts from H_0");
   if (T > s->max_len) return fail(RLT_E_CAPACITY, "T exceeds max_len");
   cudaStream_t st = (cudaStream_t)stream;
-  RLT_TRY(RLT_DISPATCH(m, encode_prefix_impl, m, s, tok_dev, T, st));
+  RLT_TRY(RLT_DISPATCH(m, encode_prefix_impl, m, s, tok_dev, (int64_t)T, T, 0, s->B, 0, st));
   for (int t = 1; t <= T; ++t) {
     StepRange range(m, t);
-    RLT_TRY(RLT_DISPATCH(m, transition_impl, m, s, st));
+    RLT_TRY(RLT_DISPATCH(m, transition_impl, m, s, false, false, st));
     if (logp_dev && t < T)
       RLT_TRY(RLT_DISPATCH(m, readout_impl, m, s, tok_dev + t, (int64_t)T, logp_dev + (t - 1), (int64_t)(T - 1),
-                           (const rlt_sampling*)nullptr, (const rlt_readout_out*)nullptr, st));
+                           (const rlt_sampling*)nullptr, (const rlt_readout_out*)nullptr, false, st));
   }
   return ok();
 }
@@ -1142,12 +1353,12 @@ int32_t rlt_replay_logprobs(rlt_model* m, const int32_t* tok_dev, int32_t B, int
   rlt_state* st_ = m->replay;
   cudaStream_t st = (cudaStream_t)stream;
   RLT_TRY(RLT_DISPATCH(m, reset_state, st_, st));
-  RLT_TRY(RLT_DISPATCH(m, encode_prefix_impl, m, st_, tok_dev, S, st));
+  RLT_TRY(RLT_DISPATCH(m, encode_prefix_impl, m, st_, tok_dev, (int64_t)S, S, 0, B, 0, st));
   for (int t = 1; t <= S - 1; ++t) {
     StepRange range(m, t);
-    RLT_TRY(RLT_DISPATCH(m, transition_impl, m, st_, st));
+    RLT_TRY(RLT_DISPATCH(m, transition_impl, m, st_, false, false, st));
     RLT_TRY(RLT_DISPATCH(m, readout_impl, m, st_, tok_dev + t, (int64_t)S, logp_dev + (t - 1), (int64_t)(S - 1),
-                         (const rlt_sampling*)nullptr, (const rlt_readout_out*)nullptr, st));
+                         (const rlt_sampling*)nullptr, (const rlt_readout_out*)nullptr, false, st));
   }
   return ok();
 }
@@ -1210,11 +1421,12 @@ int32_t rlt_op_prefix_attention(const float* q_dev, const void* k_dev, const voi
   cudaError_t e;
   if (dtype == RLT_DTYPE_BF16)
     e = prefix_attn<bf16>(q_dev, (int64_t)H * hd, static_cast<const bf16*>(k_dev), static_cast<const bf16*>(v_dev), ld_t,
-                          B, H, hd, n, qpos, rope_cs_dev, static_cast<bf16*>(out_dev), (int64_t)H * hd, ws, wsf, st);
+                          B, H, hd, n, qpos, no_pos(), rope_cs_dev, static_cast<bf16*>(out_dev), (int64_t)H * hd, ws,
+                          wsf, nullptr, st);
   else
     e = prefix_attn<float>(q_dev, (int64_t)H * hd, static_cast<const float*>(k_dev), static_cast<const float*>(v_dev),
-                           ld_t, B, H, hd, n, qpos, rope_cs_dev, static_cast<float*>(out_dev), (int64_t)H * hd, ws, wsf,
-                           st);
+                           ld_t, B, H, hd, n, qpos, no_pos(), rope_cs_dev, static_cast<float*>(out_dev),
+                           (int64_t)H * hd, ws, wsf, nullptr, st);
   if (ws) {
     cudaStreamSynchronize(st);
     cudaFree(ws);
@@ -1228,8 +1440,8 @@ int32_t rlt_op_sample(const float* logits_dev, int32_t B, int32_t V, const rlt_s
   if (!logits_dev || !samp || !token_dev || B <= 0 || V <= 0) return fail(RLT_E_INVAL, "bad sample arguments");
   if (!(samp->temperature > 0.f) || samp->top_k < 1 || samp->top_k > 256)
     return fail(RLT_E_INVAL, "sampler needs temperature > 0 and 1 <= top_k <= 256");
-  RLT_CUDA(sample_topk(logits_dev, B, V, samp->temperature, samp->top_k, samp->seed, t, token_dev, logp_dev, logmu_dev,
-                       (cudaStream_t)stream));
+  RLT_CUDA(sample_topk(logits_dev, B, V, samp->temperature, samp->top_k, samp->seed, t, nullptr, token_dev, logp_dev,
+                       logmu_dev, (cudaStream_t)stream));
   return ok();
 }
 
@@ -1322,7 +1534,8 @@ int32_t rlt_replay_backward(rlt_model* m, const int32_t* tok_dev, int32_t B, int
     if (e != cudaSuccess) r = fail(RLT_E_CUDA, std::string("widen: ") + cudaGetErrorString(e));
   }
   if (r == RLT_OK) {
-    const cudaError_t e = bptt::replay_backward_f32(D, w32.data(), m->grad.data(), tok_dev, w_dev, segment, logp_dev, st);
+    const cudaError_t e = bptt::replay_backward_f32(D, w32.data(), m->grad.data(), tok_dev, w_dev, segment, logp_dev,
+                                                    m->cfg.dtype == RLT_DTYPE_BF16, st);
     if (e == cudaErrorMemoryAllocation) r = fail(RLT_E_OOM, "backward buffers: out of device memory");
     else if (e != cudaSuccess) r = fail(RLT_E_CUDA, std::string("backward: ") + cudaGetErrorString(e));
   }
@@ -1475,12 +1688,12 @@ extern "C" int32_t rlt_op_prefix_attention_noalloc(const float* q_dev, const voi
   cudaError_t e;
   if (dtype == RLT_DTYPE_BF16)
     e = prefix_attn<bf16>(q_dev, (int64_t)H * hd, static_cast<const bf16*>(k_dev), static_cast<const bf16*>(v_dev), ld_t,
-                          B, H, hd, n, qpos, rope_cs_dev, static_cast<bf16*>(out_dev), (int64_t)H * hd, ws,
-                          kNoallocScratchFloats, st);
+                          B, H, hd, n, qpos, no_pos(), rope_cs_dev, static_cast<bf16*>(out_dev), (int64_t)H * hd, ws,
+                          kNoallocScratchFloats, nullptr, st);
   else
     e = prefix_attn<float>(q_dev, (int64_t)H * hd, static_cast<const float*>(k_dev), static_cast<const float*>(v_dev),
-                           ld_t, B, H, hd, n, qpos, rope_cs_dev, static_cast<float*>(out_dev), (int64_t)H * hd, ws,
-                           kNoallocScratchFloats, st);
+                           ld_t, B, H, hd, n, qpos, no_pos(), rope_cs_dev, static_cast<float*>(out_dev),
+                           (int64_t)H * hd, ws, kNoallocScratchFloats, nullptr, st);
   if (e != cudaSuccess) return fail(RLT_E_CUDA, std::string("prefix attention: ") + cudaGetErrorString(e));
   return ok();
 }

@@ -2,11 +2,26 @@
 against the gradient oracle (``oracle.bptt``: autograd over the fp64
 forward, itself pinned by finite differences).
 
-The engine differentiates fp32 copies of the stored weights, so the bar is
-fp32 accumulation error.  Per tensor, the largest deviation must stay within
-1e-4 of the tensor's largest gradient entry, plus 1e-6.  The host build of
-the same engine meets the oracle to 1e-10 in fp64 (``test_bptt_host.py``).
+fp32 models: the engine differentiates fp32 copies of the stored weights on
+CUDA cores, so the bar is fp32 accumulation error: per tensor, the largest
+deviation within 1e-4 of the tensor's largest gradient entry, plus 1e-6, and
+log-probs within 1e-4.
+
+bf16 models: the contractions run on the tensor cores with bf16 operands
+(activations and adjoints rounded to bf16, relative error 2^-9 each, fp32
+accumulation), the precision of the model's forward.  Log-probs meet the
+bf16 bar of the forward (5e-2); per tensor the largest gradient deviation
+must stay within 5e-2 of the tensor's largest entry (the same relative
+budget as the log-probs: a handful of bf16 roundings compounded through the
+layers and the recurrence).  With RLT_GRAD_REPORT set to a file name, each
+case appends its relative errors there.
+
+The host build of the same engine meets the oracle to 1e-10 in fp64
+(``test_bptt_host.py``).
 """
+import json
+import os
+
 import numpy as np
 import pytest
 
@@ -27,10 +42,12 @@ VARIANTS = [
     (dict(d=32, n_heads=2, ffn=48, vocab=40, prompt=12), 4),
     (dict(d=32, n_heads=2, ffn=48, vocab=40, prompt=12, tied=0, merge_kind=1, groups=2, window=3), 3),
     (dict(d=128, n_heads=2, ffn=192, vocab=256, prompt=10, dtype=1, window=3), 9),
+    # every contraction on the tensor cores (d, F and V multiples of 128), hd 128
+    (dict(d=256, n_heads=2, n_layers=2, ffn=384, vocab=256, prompt=40, dtype=1, window=8), 8),
 ]
 
 
-@pytest.mark.parametrize("kw,seg", VARIANTS, ids=["f32_tied", "f32_untied_convex_GL", "bf16_hd64"])
+@pytest.mark.parametrize("kw,seg", VARIANTS, ids=["f32_tied", "f32_untied_convex_GL", "bf16_hd64", "bf16_tc_hd128"])
 def test_backward_matches_gradient_oracle(rlt, oracle_lib, kw, seg):
     import torch
 
@@ -44,15 +61,28 @@ def test_backward_matches_gradient_oracle(rlt, oracle_lib, kw, seg):
     wts = np.random.default_rng(7).uniform(-1.0, 1.0, (B, S - 1)).astype(np.float32)
     lp = torch.zeros((B, S - 1), dtype=torch.float32, device="cuda")
     rlt.rlt_replay_backward(m, torch.from_numpy(tok).cuda(), torch.from_numpy(wts).cuda(), segment=seg, logp=lp)
+    bf16 = cfg["dtype"] == 1
+    lp_tol, g_rel = (5e-2, 5e-2) if bf16 else (1e-4, 1e-4)
     want = None
+    lp_err = 0.0
     for b in range(B):
-        assert np.max(np.abs(lp[b].cpu().numpy() - om.replay_logprobs(tok[b]))) < 1e-4
+        lp_err = max(lp_err, float(np.max(np.abs(lp[b].cpu().numpy() - om.replay_logprobs(tok[b])))))
         _, g = bptt.loss_and_grads(om, tok[b], wts[b].astype(np.float64))
         want = g if want is None else {k: want[k] + g[k] for k in want}
+    rel = {}
     for name, ref in want.items():
         got = m.grad(name)
         scale = float(np.max(np.abs(ref)))
-        assert np.max(np.abs(got - ref)) <= 1e-4 * scale + 1e-6, name
+        rel[name] = float(np.max(np.abs(got - ref))) / max(scale, 1e-30)
+    report = os.environ.get("RLT_GRAD_REPORT")
+    if report:
+        worst = sorted(rel.items(), key=lambda x: -x[1])[:5]
+        with open(report, "a") as f:
+            f.write(json.dumps({"case": kw, "logp_err": lp_err, "worst_rel": worst}) + "\n")
+    assert lp_err <= lp_tol
+    for name, ref in want.items():
+        scale = float(np.max(np.abs(ref)))
+        assert rel[name] * scale <= g_rel * scale + 1e-6, (name, rel[name])
     rlt.rlt_check_device()
 
 
