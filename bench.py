@@ -544,7 +544,7 @@ def read_traffic_ratio() -> tuple[float | None, str]:
 
 
 def config_desc(args, w: dict, kind: str, world: int) -> dict:
-    if kind == "replay":
+    if kind in ("replay", "backward"):
         tokens, schedule = w["prompt"], "replay (teacher-forced)"
     elif kind == "generate":
         tokens, schedule = f"{w['prompt']}+{w['gen']}", "prefill + sampled generation"

@@ -127,6 +127,7 @@ typedef struct rlt_state_info {
 } rlt_state_info;
 
 #define RLT_STATE_ENCODER_CACHE 1   /* keep C^E (needed for incremental encoding, eq. 2.8) */
+#define RLT_STATE_GRAPHS 2          /* replay rlt_decoder_step's kernels as CUDA graphs, one per step shape */
 
 /* what for rlt_state_read: */
 #define RLT_READ_S 0        /* [B][d] fp32 recurrent output s_t */
@@ -279,6 +280,16 @@ int32_t rlt_append_spans(rlt_model* m, rlt_state* s, const int32_t* tok_dev, int
 int32_t rlt_readout(rlt_model* m, rlt_state* s, const int32_t* next_dev, const rlt_sampling* samp,
                     const rlt_readout_out* out, void* stream);
 
+/* Consumes x_t for every sequence b, at its own t = n_dec[b]+1 (App. A.2).
+ * With RLT_STATE_GRAPHS the step's kernels (encoder step and transition,
+ * not the readout) run as a CUDA graph: one graph per step shape (which
+ * sequences run the encoder step, the token source, and the number of
+ * 256-key attention chunks), captured the second time a shape occurs and
+ * launched on a stream private to the state, ordered after `stream` by
+ * events.  Results are bit-identical to plain launches; if a capture fails
+ * the state falls back to plain launches for good.  Graphs are not used
+ * while profiling is enabled.
+ */
 /* Consumes x_t for every sequence b, at its own t = n_dec[b]+1 (App. A.2):
  * for the sequences whose x_t is not yet encoded (n_enc[b] < t), runs the
  * encoder step (eq. 2.8, needs the encoder cache) and the memory append;

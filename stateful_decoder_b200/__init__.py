@@ -35,6 +35,7 @@ MERGE_CONVEX = 1
 DTYPE_F32 = 0
 DTYPE_BF16 = 1
 STATE_ENCODER_CACHE = 1
+STATE_GRAPHS = 2
 
 READ_S, READ_E, READ_RING_K, READ_RING_V, READ_MEM_K, READ_MEM_V, READ_ENC_K, READ_ENC_V = range(8)
 

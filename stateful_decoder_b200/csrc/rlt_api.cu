@@ -25,7 +25,9 @@
 #include <cstring>
 #include <map>
 #include <mutex>
+#include <set>
 #include <string>
+#include <tuple>
 #include <vector>
 
 #include "internal.h"
@@ -143,6 +145,22 @@ struct rlt_state {
   float* gemm_ws = nullptr; size_t gemm_ws_floats = 0;  // split-K exchange of the decode GEMMs (bf16)
   int32_t* pending = nullptr;  // [B] last sampled x_{t+1}, not yet consumed (report App. A, pending token)
   bool has_pending = false;
+  // CUDA-graph replay of decoder steps (flag RLT_STATE_GRAPHS): one
+  // executable graph per step shape -- (encoder step: none / some / all
+  // sequences, its token source, decode-attention chunks) -- captured the
+  // second time the shape occurs and launched on a private stream that is
+  // ordered after the caller's stream by events.  A failed capture turns
+  // graphs off for the state (every step then launches its kernels).
+  using GraphKey = std::tuple<int, const void*, int>;
+  struct StepGraph {
+    cudaGraphExec_t exec;
+    int64_t kernels;
+  };
+  std::map<GraphKey, StepGraph> graphs;
+  std::set<GraphKey> graph_seen;
+  bool graph_ok = true;
+  cudaStream_t gstream = nullptr;
+  cudaEvent_t ev_in = nullptr, ev_out = nullptr;
   // encoder-prefill workspace, rows = sequences x tokens of one chunk
   int64_t pf_rows = 0;
   void* pf_x = nullptr; void* pf_big = nullptr; void* pf_q = nullptr; void* pf_k = nullptr; void* pf_v = nullptr;
@@ -805,16 +823,22 @@ int32_t transition_impl(rlt_model* m, rlt_state* S, bool masked, bool et_ready, 
                     st));
     RLT_TRY(gemm<T>(S, w.dw2, F, S->hbuf, F, d, B, F, EPI_RESID, cout_(epi_out(S->s, srow, 0), g_next), true, st));
   }
-  // positions (and, for idle sequences of a masked phase, their saved rows)
+  // positions (and, for idle sequences of a masked phase, their saved rows);
+  // the caller moves the host copies with advance_host
   RLT_CUDA(advance_positions(S->pos + B, S->pos, masked ? S->pos + 2 * B : nullptr, B, d, S->s,
                              masked ? S->s_save : nullptr, static_cast<bf16*>(S->zb),
                              static_cast<const bf16*>(S->zb_save), S->ss, S->ss_save, n_ss, st));
-  for (int b = 0; b < B; ++b) {
+  return RLT_OK;
+}
+
+// Host copies of the positions after a transition, as advance_kernel moves
+// the device copy.
+void advance_host(rlt_state* S, bool masked) {
+  for (int b = 0; b < S->B; ++b) {
     if (!active_h(S, masked, b)) continue;
     S->dec_h[b] += 1;
     S->enc_h[b] = std::max(S->enc_h[b], S->dec_h[b]);
   }
-  return RLT_OK;
 }
 
 // Readout (eq. 2.6) of s_t: logits = W_o RMSNorm_o(s_t), then the teacher
@@ -852,6 +876,57 @@ int32_t readout_impl(rlt_model* m, rlt_state* S, const int32_t* next, int64_t ne
 
 #define RLT_DISPATCH(m, fn, ...) \
   ((m)->cfg.dtype == RLT_DTYPE_BF16 ? fn<bf16>(__VA_ARGS__) : fn<float>(__VA_ARGS__))
+
+// The kernels of one decoder step (encoder step where needed, then the
+// transition), launched directly or, for states made with RLT_STATE_GRAPHS,
+// through the step graph of their shape.
+int32_t step_kernels(rlt_model* m, rlt_state* s, const int32_t* tok_src, bool any_enc, bool all_enc, cudaStream_t st) {
+  if (any_enc) RLT_TRY(RLT_DISPATCH(m, encode_step_impl, m, s, tok_src, false, st));
+  RLT_TRY(RLT_DISPATCH(m, transition_impl, m, s, false, any_enc && all_enc, st));
+  return RLT_OK;
+}
+
+int32_t step_launch(rlt_model* m, rlt_state* s, const int32_t* tok_src, bool any_enc, bool all_enc, cudaStream_t st) {
+  if (!(s->flags & RLT_STATE_GRAPHS) || !s->graph_ok || m->prof.on)
+    return step_kernels(m, s, tok_src, any_enc, all_enc, st);
+  int n_max = 1;
+  for (int b = 0; b < s->B; ++b) n_max = std::max(n_max, n_keys_h(s, false, b));
+  const rlt_state::GraphKey key{(any_enc ? 1 : 0) + (all_enc ? 2 : 0), tok_src, (n_max + kPrefixChunk - 1) / kPrefixChunk};
+  auto it = s->graphs.find(key);
+  if (it == s->graphs.end()) {
+    if (!s->graph_seen.count(key)) {  // first time: plain launches (one-time kernel setup happens outside a capture)
+      s->graph_seen.insert(key);
+      return step_kernels(m, s, tok_src, any_enc, all_enc, st);
+    }
+    if (!s->gstream) {
+      RLT_CUDA(cudaStreamCreateWithFlags(&s->gstream, cudaStreamNonBlocking));
+      RLT_CUDA(cudaEventCreateWithFlags(&s->ev_in, cudaEventDisableTiming));
+      RLT_CUDA(cudaEventCreateWithFlags(&s->ev_out, cudaEventDisableTiming));
+    }
+    cudaGraph_t g = nullptr;
+    const int64_t n0 = launch_count();
+    bool captured = cudaStreamBeginCapture(s->gstream, cudaStreamCaptureModeThreadLocal) == cudaSuccess;
+    const int32_t r = captured ? step_kernels(m, s, tok_src, any_enc, all_enc, s->gstream) : RLT_OK;
+    if (captured) captured = cudaStreamEndCapture(s->gstream, &g) == cudaSuccess && r == RLT_OK;
+    cudaGraphExec_t exec = nullptr;
+    if (captured) captured = cudaGraphInstantiate(&exec, g, 0) == cudaSuccess;
+    if (g) cudaGraphDestroy(g);
+    if (!captured) {  // graphs off for this state; this step launches its kernels
+      cudaGetLastError();
+      s->graph_ok = false;
+      return step_kernels(m, s, tok_src, any_enc, all_enc, st);
+    }
+    it = s->graphs.emplace(key, rlt_state::StepGraph{exec, launch_count() - n0}).first;
+  } else {
+    for (int64_t i = 0; i < it->second.kernels; ++i) note_launch();
+  }
+  RLT_CUDA(cudaEventRecord(s->ev_in, st));
+  RLT_CUDA(cudaStreamWaitEvent(s->gstream, s->ev_in, 0));
+  RLT_CUDA(cudaGraphLaunch(it->second.exec, s->gstream));
+  RLT_CUDA(cudaEventRecord(s->ev_out, s->gstream));
+  RLT_CUDA(cudaStreamWaitEvent(st, s->ev_out, 0));
+  return RLT_OK;
+}
 
 int32_t check_sampling(const rlt_sampling* samp, const rlt_readout_out* out) {
   if (!samp) return RLT_OK;
@@ -939,7 +1014,7 @@ int32_t rlt_model_free(rlt_model* m) {
 int32_t rlt_state_create(rlt_model* m, int32_t batch, int32_t max_len, int32_t flags, rlt_state** out) {
   if (!m || !out) return fail(RLT_E_INVAL, "null argument");
   *out = nullptr;
-  if (flags & ~RLT_STATE_ENCODER_CACHE) return fail(RLT_E_INVAL, "unknown flags");
+  if (flags & ~(RLT_STATE_ENCODER_CACHE | RLT_STATE_GRAPHS)) return fail(RLT_E_INVAL, "unknown flags");
   RLT_CUDA(cudaSetDevice(m->device));
   rlt_state* S = nullptr;
   RLT_TRY(make_state(m, batch, max_len, flags, &S));
@@ -963,6 +1038,10 @@ int32_t rlt_state_free(rlt_state* s) {
   if (s != s->m->replay) s->m->live_states -= 1;
   cudaSetDevice(s->m->device);
   cudaDeviceSynchronize();
+  for (auto& g : s->graphs) cudaGraphExecDestroy(g.second.exec);
+  if (s->gstream) cudaStreamDestroy(s->gstream);
+  if (s->ev_in) cudaEventDestroy(s->ev_in);
+  if (s->ev_out) cudaEventDestroy(s->ev_out);
   free_all(s->allocs);
   delete s;
   return ok();
@@ -1276,6 +1355,7 @@ int32_t rlt_append_spans(rlt_model* m, rlt_state* s, const int32_t* tok_dev, int
   for (int k = 1; k <= max_len_span; ++k) {
     StepRange range(m, max_of(s->dec_h) + 1);
     RLT_TRY(RLT_DISPATCH(m, transition_impl, m, s, true, false, st));
+    advance_host(s, true);
     if (logp_dev && k < max_len_span)
       RLT_TRY(RLT_DISPATCH(m, readout_impl, m, s, tok_dev + k, ld_tok, logp_dev + (k - 1), ld_logp,
                            (const rlt_sampling*)nullptr, (const rlt_readout_out*)nullptr, true, st));
@@ -1314,9 +1394,10 @@ int32_t rlt_decoder_step(rlt_model* m, rlt_state* s, const int32_t* tok_dev, con
     if (!(s->flags & RLT_STATE_ENCODER_CACHE)) return fail(RLT_E_STATE, "x_t not encoded and the state has no encoder cache");
     if (!tok_dev && !s->has_pending)
       return fail(RLT_E_STATE, "x_t must be given: it is not yet encoded and no sampled token is pending");
-    RLT_TRY(RLT_DISPATCH(m, encode_step_impl, m, s, tok_dev ? tok_dev : s->pending, false, st));
   }
-  RLT_TRY(RLT_DISPATCH(m, transition_impl, m, s, false, any_enc && all_enc, st));
+  const int32_t* tok_src = any_enc ? (tok_dev ? tok_dev : s->pending) : nullptr;
+  RLT_TRY(step_launch(m, s, tok_src, any_enc, all_enc, st));
+  advance_host(s, false);
   s->has_pending = false;
   if (next_dev || samp || (out && out->logits))
     RLT_TRY(RLT_DISPATCH(m, readout_impl, m, s, next_dev, (int64_t)1, out ? out->logp : nullptr, (int64_t)1, samp, out,
@@ -1334,6 +1415,7 @@ int32_t rlt_prefill(rlt_model* m, rlt_state* s, const int32_t* tok_dev, int32_t 
   for (int t = 1; t <= T; ++t) {
     StepRange range(m, t);
     RLT_TRY(RLT_DISPATCH(m, transition_impl, m, s, false, false, st));
+    advance_host(s, false);
     if (logp_dev && t < T)
       RLT_TRY(RLT_DISPATCH(m, readout_impl, m, s, tok_dev + t, (int64_t)T, logp_dev + (t - 1), (int64_t)(T - 1),
                            (const rlt_sampling*)nullptr, (const rlt_readout_out*)nullptr, false, st));
@@ -1357,6 +1439,7 @@ int32_t rlt_replay_logprobs(rlt_model* m, const int32_t* tok_dev, int32_t B, int
   for (int t = 1; t <= S - 1; ++t) {
     StepRange range(m, t);
     RLT_TRY(RLT_DISPATCH(m, transition_impl, m, st_, false, false, st));
+    advance_host(st_, false);
     RLT_TRY(RLT_DISPATCH(m, readout_impl, m, st_, tok_dev + t, (int64_t)S, logp_dev + (t - 1), (int64_t)(S - 1),
                          (const rlt_sampling*)nullptr, (const rlt_readout_out*)nullptr, false, st));
   }
