@@ -323,7 +323,7 @@ def run_gpu(args, w: dict, kind: str, peaks: dict, rank: int, world: int) -> dic
         launches_per_step = (w["n_layers"] * (S - 1), w["n_layers"] * (S - 1))
     elif kind == "generate":
         T, n_gen = w["prompt"], w["gen"]
-        state = rlt.rlt_state_create(model, B, T + n_gen, rlt.STATE_ENCODER_CACHE)
+        state = rlt.rlt_state_create(model, B, T + n_gen, rlt.STATE_ENCODER_CACHE | rlt.STATE_GRAPHS)
         tok_host = torch.from_numpy(shard_tokens(w, rank, world)).pin_memory()
         tok = tok_host.cuda()
         ids = torch.zeros(n_gen, B, dtype=torch.int32, device=dev)
@@ -353,7 +353,9 @@ def run_gpu(args, w: dict, kind: str, peaks: dict, rank: int, world: int) -> dic
         T, blk = w["prompt"], w["block"]
         n_blocks = args.warmup + args.steps + PROFILE_BLOCKS
         max_len = T + blk * n_blocks
-        state = rlt.rlt_state_create(model, B, max_len, rlt.STATE_ENCODER_CACHE)
+        # decoder steps replay one CUDA graph per step shape (bit-identical to
+        # plain launches)
+        state = rlt.rlt_state_create(model, B, max_len, rlt.STATE_ENCODER_CACHE | rlt.STATE_GRAPHS)
         tok = torch.from_numpy(shard_tokens(w, rank, world)).cuda()
         ids = torch.zeros(blk, B, dtype=torch.int32, device=dev)
         lmu = torch.zeros(blk, B, device=dev)

@@ -178,6 +178,7 @@ class Model:
     def __init__(self, handle: ctypes.c_void_p, cfg: dict):
         self.h = handle
         self.cfg = dict(cfg)
+        self._lib = _lib  # kept for __del__, which may run after module teardown
 
     def __del__(self):
         self.free()
@@ -186,7 +187,7 @@ class Model:
         """Frees the model; returns RLT_E_STATE (and keeps the model) while
         states made on it are alive."""
         if getattr(self, "h", None):
-            code = _lib.rlt_model_free(self.h)
+            code = self._lib.rlt_model_free(self.h)
             if code != RLT_OK:
                 return code
             self.h = None
@@ -227,13 +228,14 @@ class State:
         self.model = model
         self.batch = batch
         self.max_len = max_len
+        self._lib = _lib  # kept for __del__, which may run after module teardown
 
     def __del__(self):
         self.free()
 
     def free(self):
         if getattr(self, "h", None):
-            _lib.rlt_state_free(self.h)
+            self._lib.rlt_state_free(self.h)
             self.h = None
 
     def info(self) -> dict:

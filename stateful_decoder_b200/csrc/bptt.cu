@@ -1,6 +1,8 @@
-// bptt.cu -- CUDA backend of the full-BPTT engine (bptt_core.h).  Every
-// functor of the engine runs as a kernel with one thread per output index,
-// except the three contractions of a bf16 model: Y = X W^T (MmNT),
+// bptt.cu -- CUDA backend of the full-BPTT engine (bptt_core.h).  Most
+// functors of the engine run as a kernel with one thread per output index;
+// the readout loss runs one block per row, the RMSNorms and the three
+// attention functors one warp per row, query or key; and the three
+// contractions of a bf16 model: Y = X W^T (MmNT),
 // Y = D W (MmNN) and W_grad += D^T X (MmTN) run on the tensor cores through
 // the library's tcgen05 GEMM (C[n][m] = sum_k B[n][k] A[m][k], both operands
 // K-major bf16, fp32 accumulation), with the operands rounded to bf16 -- the
@@ -11,6 +13,8 @@
 // models keep the CUDA-core functors.
 // Also the widening of stored weights (fp32 or bf16, possibly pitched views)
 // into the fp32 copies the engine differentiates.
+#include <nvtx3/nvToolsExt.h>
+
 #include <map>
 #include <tuple>
 #include <vector>
@@ -51,6 +55,187 @@ __global__ void to_bf16_t_kernel(const float* __restrict__ src, int64_t ld, int 
   for (int y = threadIdx.y; y < 32; y += 8) {
     const int c = c0 + y, r = r0 + threadIdx.x;
     if (c < C && r < Rp) dst[(int64_t)c * Rp + r] = __float2bfloat16_rn(tile[threadIdx.x][y]);
+  }
+}
+
+// ---- row and attention functors with warp- or block-level parallelism: the
+// arithmetic of the bptt_core.h functors (up to the order of summation),
+// without one thread walking a whole row or key range alone.
+
+// Readout loss of row b (Xent): one block per row.
+__global__ void __launch_bounds__(256) xent_kernel(Xent<float> k) {
+  __shared__ float red[32];
+  const int b = blockIdx.x;
+  const float* l = k.logits + (int64_t)b * k.V;
+  float mx = -INFINITY;
+  for (int v = threadIdx.x; v < k.V; v += blockDim.x) mx = fmaxf(mx, l[v]);
+  mx = block_max(mx, red);
+  float den = 0.f;
+  for (int v = threadIdx.x; v < k.V; v += blockDim.x) den += expf(l[v] - mx);
+  den = block_sum(den, red);
+  const float lse = mx + logf(den);
+  const int y = k.tok[(int64_t)b * k.tok_sb + k.t + 1];
+  if (k.logp && threadIdx.x == 0) k.logp[(int64_t)b * k.w_sb + k.t] = l[y] - lse;
+  if (k.dlogits) {
+    const float w = k.wts[(int64_t)b * k.w_sb + k.t];
+    float* dl = k.dlogits + (int64_t)b * k.V;
+    for (int v = threadIdx.x; v < k.V; v += blockDim.x) dl[v] = w * (expf(l[v] - lse) - (v == y ? 1.f : 0.f));
+  }
+}
+
+// RMSNorm forward (RmsF) and its input adjoint (RmsBX): one warp per row.
+__global__ void __launch_bounds__(256) rmsf_kernel(RmsF<float> k, int64_t rows) {
+  const int64_t r = (int64_t)blockIdx.x * 8 + (threadIdx.x >> 5);
+  const int lane = threadIdx.x & 31;
+  if (r >= rows) return;
+  const float* x = k.X + r * k.ldx;
+  float ss = 0.f;
+  for (int j = lane; j < k.d; j += 32) ss += x[j] * x[j];
+  ss = warp_sum(ss);
+  const float ri = 1.0f / sqrtf(ss / (float)k.d + k.eps);
+  if (lane == 0) k.rinv[r] = ri;
+  float* y = k.Y + r * k.ldy;
+  for (int j = lane; j < k.d; j += 32) y[j] = x[j] * ri * k.g[j];
+}
+__global__ void __launch_bounds__(256) rmsbx_kernel(RmsBX<float> k, int64_t rows) {
+  const int64_t r = (int64_t)blockIdx.x * 8 + (threadIdx.x >> 5);
+  const int lane = threadIdx.x & 31;
+  if (r >= rows) return;
+  const float* dy = k.dY + r * k.ldd;
+  const float* x = k.X + r * k.ldx;
+  const float ri = k.rinv[r];
+  float dot = 0.f;
+  for (int j = lane; j < k.d; j += 32) dot += dy[j] * k.g[j] * x[j] * ri;
+  dot = warp_sum(dot) / (float)k.d;
+  float* dx = k.dX + r * k.lddx;
+  for (int j = lane; j < k.d; j += 32) dx[j] += ri * (dy[j] * k.g[j] - x[j] * ri * dot);
+}
+
+// Attention functors, one warp per (sequence, query or key, head); lane l
+// holds head dimensions l, l+32, ... (at most kMaxHead / 32 of them).
+constexpr int kLaneDims = kMaxHead / 32;
+
+__device__ __forceinline__ float lane_dot(const float* a, const float* b, int hd, int lane) {
+  float s = 0.f;
+#pragma unroll
+  for (int j = 0; j < kLaneDims; ++j) {
+    const int e = lane + 32 * j;
+    if (e < hd) s += a[e] * b[e];
+  }
+  return warp_sum(s);
+}
+
+// AttnF: online softmax over the query's keys.
+__global__ void __launch_bounds__(256) attnf_kernel(AttnF<float> k, int64_t n) {
+  const int64_t idx = (int64_t)blockIdx.x * 8 + (threadIdx.x >> 5);
+  const int lane = threadIdx.x & 31;
+  if (idx >= n) return;
+  const AttnGeom<float>& g = k.g;
+  const int h = (int)(idx % g.H);
+  const int64_t bi = idx / g.H;
+  const int i = (int)(bi % g.Tq);
+  const int64_t b = bi / g.Tq;
+  const float* q = k.Q + b * g.q_sb + i * g.q_si + (int64_t)h * g.hd;
+  float mx = -INFINITY, den = 0.f, acc[kLaneDims];
+#pragma unroll
+  for (int j = 0; j < kLaneDims; ++j) acc[j] = 0.f;
+  for (int p = g.lo(i); p <= g.hi(i); ++p) {
+    const float* kr = k.K + b * g.k_sb + p * g.k_sp + (int64_t)h * g.hd;
+    const float* vr = k.Vv + b * g.k_sb + p * g.k_sp + (int64_t)h * g.hd;
+    const float s = lane_dot(q, kr, g.hd, lane) * k.scale;
+    const float nm = fmaxf(mx, s);
+    const float c = expf(mx - nm), w = expf(s - nm);
+    den = den * c + w;
+#pragma unroll
+    for (int j = 0; j < kLaneDims; ++j) {
+      const int e = lane + 32 * j;
+      acc[j] = acc[j] * c + (e < g.hd ? w * vr[e] : 0.f);
+    }
+    mx = nm;
+  }
+  float* o = k.O + b * g.q_sb + i * g.q_si + (int64_t)h * g.hd;
+#pragma unroll
+  for (int j = 0; j < kLaneDims; ++j) {
+    const int e = lane + 32 * j;
+    if (e < g.hd) o[e] = acc[j] / den;
+  }
+  if (lane == 0) k.lse[b * g.l_sb + i * g.l_si + h] = mx + logf(den);
+}
+
+// AttnBQ: dq = scale * sum_p P_p (dO.v_p - dO.o) k_p (overwrites dQ).
+__global__ void __launch_bounds__(256) attnbq_kernel(AttnBQ<float> k, int64_t n) {
+  const int64_t idx = (int64_t)blockIdx.x * 8 + (threadIdx.x >> 5);
+  const int lane = threadIdx.x & 31;
+  if (idx >= n) return;
+  const AttnGeom<float>& g = k.g;
+  const int h = (int)(idx % g.H);
+  const int64_t bi = idx / g.H;
+  const int i = (int)(bi % g.Tq);
+  const int64_t b = bi / g.Tq;
+  const int64_t qo = b * g.q_sb + i * g.q_si + (int64_t)h * g.hd;
+  const float L = k.lse[b * g.l_sb + i * g.l_si + h];
+  const float Dv = lane_dot(k.dO + qo, k.O + qo, g.hd, lane);
+  float acc[kLaneDims];
+#pragma unroll
+  for (int j = 0; j < kLaneDims; ++j) acc[j] = 0.f;
+  for (int p = g.lo(i); p <= g.hi(i); ++p) {
+    const float* kr = k.K + b * g.k_sb + p * g.k_sp + (int64_t)h * g.hd;
+    const float* vr = k.Vv + b * g.k_sb + p * g.k_sp + (int64_t)h * g.hd;
+    const float s = lane_dot(k.Q + qo, kr, g.hd, lane);
+    const float dp = lane_dot(k.dO + qo, vr, g.hd, lane);
+    const float P = expf(s * k.scale - L);
+    const float ds = P * (dp - Dv) * k.scale;
+#pragma unroll
+    for (int j = 0; j < kLaneDims; ++j) {
+      const int e = lane + 32 * j;
+      if (e < g.hd) acc[j] += ds * kr[e];
+    }
+  }
+#pragma unroll
+  for (int j = 0; j < kLaneDims; ++j) {
+    const int e = lane + 32 * j;
+    if (e < g.hd) k.dQ[qo + e] = acc[j];
+  }
+}
+
+// AttnBKV: dK, dV of one key position (accumulated) over the queries that see it.
+__global__ void __launch_bounds__(256) attnbkv_kernel(AttnBKV<float> k, int64_t n) {
+  const int64_t idx = (int64_t)blockIdx.x * 8 + (threadIdx.x >> 5);
+  const int lane = threadIdx.x & 31;
+  if (idx >= n) return;
+  const AttnGeom<float>& g = k.g;
+  const int h = (int)(idx % g.H);
+  const int64_t bp = idx / g.H;
+  const int p = k.p0 + (int)(bp % k.np);
+  const int64_t b = bp / k.np;
+  const int64_t ko = b * g.k_sb + p * g.k_sp + (int64_t)h * g.hd;
+  float ak[kLaneDims], av[kLaneDims];
+#pragma unroll
+  for (int j = 0; j < kLaneDims; ++j) ak[j] = av[j] = 0.f;
+  for (int i = 0; i < g.Tq; ++i) {
+    if (p < g.lo(i) || p > g.hi(i)) continue;
+    const int64_t qo = b * g.q_sb + i * g.q_si + (int64_t)h * g.hd;
+    const float s = lane_dot(k.Q + qo, k.K + ko, g.hd, lane);
+    const float dp = lane_dot(k.dO + qo, k.Vv + ko, g.hd, lane);
+    const float Dv = lane_dot(k.dO + qo, k.O + qo, g.hd, lane);
+    const float P = expf(s * k.scale - k.lse[b * g.l_sb + i * g.l_si + h]);
+    const float ds = P * (dp - Dv) * k.scale;
+#pragma unroll
+    for (int j = 0; j < kLaneDims; ++j) {
+      const int e = lane + 32 * j;
+      if (e < g.hd) {
+        ak[j] += ds * k.Q[qo + e];
+        av[j] += P * k.dO[qo + e];
+      }
+    }
+  }
+#pragma unroll
+  for (int j = 0; j < kLaneDims; ++j) {
+    const int e = lane + 32 * j;
+    if (e < g.hd) {
+      k.dK[ko + e] += ak[j];
+      k.dV[ko + e] += av[j];
+    }
   }
 }
 
@@ -104,6 +289,27 @@ struct CudaBackend {
     err = cudaGetLastError();
   }
   int ok() const { return err == cudaSuccess ? 0 : -1; }
+  void range_push(const char* name) { nvtxRangePushA(name); }
+  void range_pop() { nvtxRangePop(); }
+
+  // ---- row and attention functors, warp or block per unit
+  template <class K> void launch_rows(void (*kern)(K, int64_t), const K& k, int64_t n) {
+    if (err != cudaSuccess || n <= 0) return;
+    kern<<<(unsigned)((n + 7) / 8), 256, 0, st>>>(k, n);
+    note_launch();
+    err = cudaGetLastError();
+  }
+  void launch(const Xent<float>& k, int64_t n) {
+    if (err != cudaSuccess || n <= 0) return;
+    xent_kernel<<<(unsigned)n, 256, 0, st>>>(k);
+    note_launch();
+    err = cudaGetLastError();
+  }
+  void launch(const RmsF<float>& k, int64_t n) { launch_rows(rmsf_kernel, k, n); }
+  void launch(const RmsBX<float>& k, int64_t n) { launch_rows(rmsbx_kernel, k, n); }
+  void launch(const AttnF<float>& k, int64_t n) { launch_rows(attnf_kernel, k, n); }
+  void launch(const AttnBQ<float>& k, int64_t n) { launch_rows(attnbq_kernel, k, n); }
+  void launch(const AttnBKV<float>& k, int64_t n) { launch_rows(attnbkv_kernel, k, n); }
 
   // ---- tensor-core contractions
   bf16* grow(bf16** p, size_t* cap, size_t n) {

@@ -499,7 +499,9 @@ template <class Real> struct Xent {
 // Backend concept: T* alloc<T>(n) (zeroed; null and ok() != 0 on failure),
 // zero(p, n), copy(dst, src, n) on the backend, upload(dst, host_src, n),
 // launch(functor, n) running functor(i) for i in [0, n), ok() (0 when every
-// operation so far succeeded; after a failure the backend runs nothing).
+// operation so far succeeded; after a failure the backend runs nothing),
+// range_push(name) / range_pop() marking a phase for a profiler (may do
+// nothing).
 template <class BK, class Real>
 class Engine {
  public:
@@ -540,7 +542,9 @@ class Engine {
         bk_.copy(s_cur_, rec(t - t0).zout, (size_t)D.B * D.d);
       }
       for (int t = t1 - 1; t >= t0; --t) step_backward(t, t - t0, tok, wts);
+      bk_.range_push("rlt_weight_grads");  // a profiler can select the segment's dW contractions
       segment_grads(t0, t1);
+      bk_.range_pop();
       memory_pass(t0, t1);
     }
     launch(ColSum<Real>{ds_, D.d, G(T_SSTAR), D.B}, D.d);

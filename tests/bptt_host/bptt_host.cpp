@@ -37,6 +37,8 @@ struct HostBackend {
     for (int64_t i = 0; i < n; ++i) k(i);
   }
   int ok() const { return 0; }
+  void range_push(const char*) {}
+  void range_pop() {}
 };
 
 static bool read_all(FILE* f, void* p, size_t bytes) { return fread(p, 1, bytes, f) == bytes; }

@@ -18,6 +18,9 @@ By Prop. 3.1 of the report (prefill and incremental schedules compute the
 same distributions), the oracle's replay of the whole sequence is the
 expected output of either GPU schedule.
 
+A second kind of golden (``bptt_hd128_long``) holds the full-BPTT gradient
+of the oracle on a long sequence (see GRAD_GOLDEN below).
+
     python tests/golden/make_goldens.py [name ...]     # default: all
 """
 from __future__ import annotations
@@ -51,6 +54,44 @@ GOLDENS = {
 }
 
 
+# Gradient golden of the full-BPTT backward (report §5.4): a bf16 model at
+# hd 128 over S = 600 tokens (the forward's decode attention spans three
+# 256-key chunks), weights of eq. 5.1, gradients of the oracle's autograd
+# (oracle/bptt.py).  Only the tensors in GRAD_NAMES are stored (float32).
+GRAD_GOLDEN = "bptt_hd128_long"
+GRAD_MODEL = dict(d=256, n_heads=2, n_layers=1, window=8, ffn=384, vocab=128, dtype=1, prompt=600, gen=0)
+GRAD_NAMES = ("s_star", "b_gate", "g_merge", "g_out", "w_gate", "w_state", "w_out", "wq.0", "wk.0", "w2.0",
+              "wq_mem.0", "wk_mem.0", "g_dsa.0", "g_ea.0")
+
+
+def grad_workload() -> dict:
+    return synth.workload("tiny", **GRAD_MODEL)
+
+
+def make_grad() -> None:
+    import oracle
+    from oracle import bptt
+    w = grad_workload()
+    tok = synth.tokens(w, batch=1)
+    S = tok.shape[1]
+    om = oracle.Model(synth.model_config(w), seed=synth.WEIGHT_SEED)
+    wts = np.full(S - 1, 1.0 / (S - 1))  # eq. 5.1
+    t0 = time.time()
+    loss, g = bptt.loss_and_grads(om, tok[0], wts)
+    print(f"{GRAD_GOLDEN}: {S} tokens in {time.time() - t0:.0f} s", flush=True)
+    lp = om.replay_logprobs(tok[0])
+    arrays = {"grad_" + n.replace(".", "_"): np.asarray(g[n], dtype=np.float32) for n in GRAD_NAMES}
+    tmp = path(GRAD_GOLDEN) + ".tmp.npz"
+    np.savez_compressed(tmp, logp=lp, loss=np.float64(loss), names=np.asarray(GRAD_NAMES), **arrays)
+    os.replace(tmp, path(GRAD_GOLDEN))
+
+
+def load_grad() -> dict:
+    z = np.load(path(GRAD_GOLDEN))
+    return {"logp": z["logp"], "loss": float(z["loss"]),
+            "grads": {n: z["grad_" + n.replace(".", "_")] for n in GRAD_NAMES}}
+
+
 def path(name: str) -> str:
     return os.path.join(HERE, name + ".npz")
 
@@ -79,5 +120,8 @@ def make(name: str) -> None:
 
 
 if __name__ == "__main__":
-    for n in (sys.argv[1:] or list(GOLDENS)):
-        make(n)
+    for n in (sys.argv[1:] or list(GOLDENS) + [GRAD_GOLDEN]):
+        if n == GRAD_GOLDEN:
+            make_grad()
+        else:
+            make(n)

@@ -32,3 +32,21 @@ def test_golden_is_the_oracle_output(oracle_lib, name):
     for i, r in enumerate(rows):
         want = om.replay_logprobs(tok[r, :N_CHECK + 1])
         assert np.max(np.abs(lp[i, :N_CHECK] - want)) <= 1e-12, (name, r)
+
+
+def test_gradient_golden_is_the_oracle_output(oracle_lib):
+    """The stored full-BPTT gradients (float32) equal a fresh run of the
+    gradient oracle on the same model, tokens and eq. 5.1 weights."""
+    from oracle import bptt
+    g = goldens.load_grad()
+    w = goldens.grad_workload()
+    tok = synth.tokens(w, batch=1)
+    S = tok.shape[1]
+    om = oracle_lib.Model(synth.model_config(w), seed=synth.WEIGHT_SEED)
+    loss, want = bptt.loss_and_grads(om, tok[0], np.full(S - 1, 1.0 / (S - 1)))
+    assert abs(loss - g["loss"]) <= 1e-12 * max(1.0, abs(loss))
+    assert np.max(np.abs(om.replay_logprobs(tok[0]) - g["logp"])) <= 1e-12
+    for name, stored in g["grads"].items():
+        ref = want[name]
+        assert stored.shape == ref.shape, name
+        assert np.max(np.abs(stored.astype(np.float64) - ref)) <= 1e-6 * max(1.0, float(np.max(np.abs(ref)))), name

@@ -141,3 +141,32 @@ def test_backward_on_a_side_stream(rlt, oracle_lib):
         ref = want[name]
         assert np.max(np.abs(m.grad(name) - ref)) <= 1e-4 * float(np.max(np.abs(ref))) + 1e-6, name
     rlt.rlt_check_device()
+
+
+def test_backward_long_sequence_hd128():
+    """A bf16 model at hd 128 over 600 tokens (the forward's decode attention
+    spans three 256-key chunks; the SWA window wraps 75 times; 19 segments
+    of 32): the log-probs and the gradients of the stored tensors against
+    the oracle's, kept as a golden (tests/golden/make_goldens.py, the
+    gradient oracle's autograd in fp64), at the bf16 bars above."""
+    import torch
+
+    import stateful_decoder_b200 as rlt
+    from tests.golden import make_goldens as goldens
+    g = goldens.load_grad()
+    w = goldens.grad_workload()
+    cfg = synth.model_config(w)
+    tok = synth.tokens(w, batch=1)
+    S = tok.shape[1]
+    m = rlt.rlt_init_weights(cfg, synth.WEIGHT_SEED)
+    wts = torch.full((1, S - 1), 1.0 / (S - 1), device="cuda")
+    lp = torch.zeros(1, S - 1, device="cuda")
+    rlt.rlt_replay_backward(m, torch.from_numpy(tok).cuda(), wts, segment=32, logp=lp)
+    torch.cuda.synchronize()
+    rlt.rlt_check_device()
+    assert np.max(np.abs(lp.cpu().numpy()[0] - g["logp"])) <= 5e-2
+    for name, ref in g["grads"].items():
+        ref = ref.astype(np.float64)
+        scale = float(np.max(np.abs(ref)))
+        err = float(np.max(np.abs(m.grad(name) - ref)))
+        assert err <= 5e-2 * scale + 1e-6, (name, err / scale)
