@@ -363,17 +363,21 @@ struct CudaBackend {
     cache.emplace(key, b);
     return b;
   }
-  // C[n][m] (+)= sum_k Bop[n][k] Aop[m][k] into fp32 rows `ldc` apart
+  // C[n][m] (+)= sum_k Bop[n][k] Aop[m][k] into fp32 rows `ldc` apart.  A
+  // grid of output tiles that already fills the GPU runs unsplit; smaller
+  // ones split K inside clusters (the decode plan).  The backward has no
+  // batch-invariance constraint, so the choice may follow N.
   void gemm(const bf16* Aop, int M, const bf16* Bop, int N, int K, float* C, int64_t ldc, bool acc) {
     if (err != cudaSuccess) return;
     EpiParams ep{};
     ep.out = C;
     ep.out_map = plain_rows(ldc);
     ep.aux0_map = plain_rows(0);
-    const size_t wsn = gemm_tc_workspace_floats(M, N, K, 1);
+    const int split = (int64_t)(M / 128) * ((N + 255) / 256) >= kSmCount ? 0 : 1;
+    const size_t wsn = gemm_tc_workspace_floats(M, N, K, split);
     float* w = wsn ? workspace(wsn) : nullptr;
     if (err != cudaSuccess) return;
-    err = gemm_tc(Aop, K, Bop, K, M, N, K, acc ? EPI_RESID : EPI_STORE, ep, 1, w, wsn, st);
+    err = gemm_tc(Aop, K, Bop, K, M, N, K, acc ? EPI_RESID : EPI_STORE, ep, split, w, wsn, st);
   }
   static int64_t round64(int64_t x) { return (x + 63) / 64 * 64; }
 

@@ -1414,7 +1414,7 @@ int32_t rlt_prefill(rlt_model* m, rlt_state* s, const int32_t* tok_dev, int32_t 
   RLT_TRY(RLT_DISPATCH(m, encode_prefix_impl, m, s, tok_dev, (int64_t)T, T, 0, s->B, 0, st));
   for (int t = 1; t <= T; ++t) {
     StepRange range(m, t);
-    RLT_TRY(RLT_DISPATCH(m, transition_impl, m, s, false, false, st));
+    RLT_TRY(step_launch(m, s, nullptr, false, false, st));
     advance_host(s, false);
     if (logp_dev && t < T)
       RLT_TRY(RLT_DISPATCH(m, readout_impl, m, s, tok_dev + t, (int64_t)T, logp_dev + (t - 1), (int64_t)(T - 1),
@@ -1431,14 +1431,14 @@ int32_t rlt_replay_logprobs(rlt_model* m, const int32_t* tok_dev, int32_t B, int
     rlt_state_free(m->replay);
     m->replay = nullptr;
   }
-  if (!m->replay) RLT_TRY(make_state(m, B, S, 0, &m->replay));
+  if (!m->replay) RLT_TRY(make_state(m, B, S, RLT_STATE_GRAPHS, &m->replay));
   rlt_state* st_ = m->replay;
   cudaStream_t st = (cudaStream_t)stream;
   RLT_TRY(RLT_DISPATCH(m, reset_state, st_, st));
   RLT_TRY(RLT_DISPATCH(m, encode_prefix_impl, m, st_, tok_dev, (int64_t)S, S, 0, B, 0, st));
   for (int t = 1; t <= S - 1; ++t) {
     StepRange range(m, t);
-    RLT_TRY(RLT_DISPATCH(m, transition_impl, m, st_, false, false, st));
+    RLT_TRY(step_launch(m, st_, nullptr, false, false, st));
     advance_host(st_, false);
     RLT_TRY(RLT_DISPATCH(m, readout_impl, m, st_, tok_dev + t, (int64_t)S, logp_dev + (t - 1), (int64_t)(S - 1),
                          (const rlt_sampling*)nullptr, (const rlt_readout_out*)nullptr, false, st));
