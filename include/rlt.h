@@ -353,18 +353,30 @@ int32_t rlt_replay_ratios(rlt_model* m, const int32_t* tok_dev, int32_t B, int32
  * arithmetic is fp32 on fp32 copies of the weights.  Gradients are
  * accumulated into fp32 buffers the model owns, one per stored tensor, read
  * with rlt_grad_read and cleared with rlt_grad_zero.  logp_dev [B][S-1]
- * (may be NULL) receives the log-probs the pass computed.  Device memory
- * is allocated inside the call and freed before it returns, in fp32: about
- * 4 * B * S * (L * (12d + 3F) + 4 G d + 13d + 3F) bytes for the encoder
- * activations, the decoder key/value history and their adjoints, plus
- * 4 * segment * B * (L * (11d + 3F) + 6d + V) bytes for one segment's
- * recomputed steps, plus the fp32 weight copies.  The stream is
- * synchronised.  Head size at most 128.  The token
- * ids are copied to the host and checked against the vocabulary before any
- * work is enqueued.  Errors: RLT_E_INVAL (arguments, a token id out of
- * range), RLT_E_OOM, RLT_E_CUDA. */
+ * (may be NULL) receives the log-probs the pass computed.
+ * Device memory, in fp32: about 4 * B * S * (L * (12d + 3F) + 4 G d + 13d +
+ * 3F) bytes for the encoder activations, the decoder key/value history and
+ * their adjoints, plus 4 * segment * B * (L * (11d + 3F) + 6d + V) bytes for
+ * one segment's recomputed steps, plus the fp32 weight copies.  It is
+ * allocated by the first call for a (B, S, segment) and kept by the model
+ * for the next calls of the same sizes (another size frees it first;
+ * rlt_backward_release and rlt_model_free free it).  The first call of a
+ * size launches its kernels one by one; the second captures the whole pass
+ * (weight copies included, so weights loaded between calls are used) as a
+ * CUDA graph, which later calls replay.  A pass of more than 400,000 kernels
+ * is never captured.  The work runs on a stream of the model's own, ordered
+ * after the work already on `stream`, and `stream` waits for it; the call
+ * returns once it is enqueued.  Head size at most 128.  The token ids are
+ * copied to the host and checked against the vocabulary before any work is
+ * enqueued (this waits for `stream`).  Errors: RLT_E_INVAL (arguments, a
+ * token id out of range), RLT_E_OOM, RLT_E_CUDA (the kept buffers are freed
+ * after an error). */
 int32_t rlt_replay_backward(rlt_model* m, const int32_t* tok_dev, int32_t B, int32_t S, const float* w_dev,
                             int32_t segment, float* logp_dev, void* stream);
+
+/* Frees the device memory and the graph rlt_replay_backward keeps between
+ * calls (after the device has finished its work).  Errors: RLT_E_INVAL. */
+int32_t rlt_backward_release(rlt_model* m);
 
 /* Copies the accumulated fp32 gradient of a stored tensor (rlt_tensor_info
  * names and shapes, [rows][cols] row-major) to host.  Before any

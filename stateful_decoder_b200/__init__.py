@@ -46,7 +46,7 @@ EXPORTED = (
     "rlt_last_error", "rlt_check_device", "rlt_profile_enable", "rlt_profile_read", "rlt_op_linear",
     "rlt_op_sample", "rlt_kernel_launches", "rlt_op_prefix_attention", "rlt_op_prefix_attention_noalloc",
     "rlt_state_export", "rlt_state_import", "rlt_replay_ratios", "rlt_replay_backward", "rlt_grad_read",
-    "rlt_grad_zero", "rlt_test_bounded_wait", "rlt_state_positions", "rlt_append_spans",
+    "rlt_grad_zero", "rlt_test_bounded_wait", "rlt_state_positions", "rlt_append_spans", "rlt_backward_release",
 )
 
 
@@ -107,6 +107,7 @@ _sig = {
     "rlt_replay_backward": [_vp, _vp, _i32, _i32, _vp, _i32, _vp, _vp],
     "rlt_grad_read": [_vp, ctypes.c_char_p, _vp, ctypes.c_size_t],
     "rlt_grad_zero": [_vp, _vp],
+    "rlt_backward_release": [_vp],
     "rlt_op_linear": [_vp, _vp, _vp, _i32, _i32, _i32, _i32, _i32, _vp],
     "rlt_op_prefix_attention": [_vp, _vp, _vp, ctypes.c_int64, _i32, _i32, _i32, _i32, _i32, _vp, _i32, _vp, _vp],
     "rlt_op_prefix_attention_noalloc": [_vp, _vp, _vp, ctypes.c_int64, _i32, _i32, _i32, _i32, _i32, _vp, _i32, _vp,
@@ -389,7 +390,9 @@ def rlt_replay_ratios(model: Model, tokens, logmu, action_mask, logp, ratio=None
 def rlt_replay_backward(model: Model, tokens, weights, segment: int = 32, logp=None, stream=None) -> None:
     """Full-BPTT gradient of -sum w[b][t] log p(x_{t+1} | x_1..t): tokens int32
     [B, S], weights float32 [B, S-1], optional logp float32 [B, S-1] (CUDA
-    tensors).  Gradients accumulate in the model (Model.grad, rlt_grad_zero)."""
+    tensors).  Gradients accumulate in the model (Model.grad, rlt_grad_zero).
+    The model keeps the pass's buffers (and, from the second call of a size,
+    a CUDA graph of the pass) until rlt_backward_release or another size."""
     B, S = tokens.shape
     _check(_lib.rlt_replay_backward(model.h, _dev(tokens, "torch.int32"), B, S,
                                     _dev(weights, "torch.float32", B * (S - 1)), segment,
@@ -398,6 +401,11 @@ def rlt_replay_backward(model: Model, tokens, weights, segment: int = 32, logp=N
 
 def rlt_grad_zero(model: Model, stream=None) -> None:
     _check(_lib.rlt_grad_zero(model.h, _stream(stream)))
+
+
+def rlt_backward_release(model: Model) -> None:
+    """Frees what rlt_replay_backward keeps between calls."""
+    _check(_lib.rlt_backward_release(model.h))
 
 
 def rlt_op_linear(w, x, y, use_tensor_cores: bool = True, stream=None) -> None:

@@ -28,6 +28,7 @@ namespace {
 
 template <class K>
 __global__ void __launch_bounds__(256) functor_kernel(K k, int64_t n) {
+  griddep_enter();
   const int64_t i = (int64_t)blockIdx.x * blockDim.x + threadIdx.x;
   if (i < n) k(i);
 }
@@ -45,6 +46,7 @@ struct ToBf16 {
 // [R][C] fp32 matrix transposed to [C][Rp] bf16 through 32 x 32 shared-memory
 // tiles (coalesced on both sides).  Grid (ceil(C/32), Rp/32), block (32, 8).
 __global__ void to_bf16_t_kernel(const float* __restrict__ src, int64_t ld, int R, int C, int Rp, bf16* dst) {
+  griddep_enter();
   __shared__ float tile[32][33];
   const int c0 = blockIdx.x * 32, r0 = blockIdx.y * 32;
   for (int y = threadIdx.y; y < 32; y += 8) {
@@ -64,6 +66,7 @@ __global__ void to_bf16_t_kernel(const float* __restrict__ src, int64_t ld, int 
 
 // Readout loss of row b (Xent): one block per row.
 __global__ void __launch_bounds__(256) xent_kernel(Xent<float> k) {
+  griddep_enter();
   __shared__ float red[32];
   const int b = blockIdx.x;
   const float* l = k.logits + (int64_t)b * k.V;
@@ -85,6 +88,7 @@ __global__ void __launch_bounds__(256) xent_kernel(Xent<float> k) {
 
 // RMSNorm forward (RmsF) and its input adjoint (RmsBX): one warp per row.
 __global__ void __launch_bounds__(256) rmsf_kernel(RmsF<float> k, int64_t rows) {
+  griddep_enter();
   const int64_t r = (int64_t)blockIdx.x * 8 + (threadIdx.x >> 5);
   const int lane = threadIdx.x & 31;
   if (r >= rows) return;
@@ -98,6 +102,7 @@ __global__ void __launch_bounds__(256) rmsf_kernel(RmsF<float> k, int64_t rows) 
   for (int j = lane; j < k.d; j += 32) y[j] = x[j] * ri * k.g[j];
 }
 __global__ void __launch_bounds__(256) rmsbx_kernel(RmsBX<float> k, int64_t rows) {
+  griddep_enter();
   const int64_t r = (int64_t)blockIdx.x * 8 + (threadIdx.x >> 5);
   const int lane = threadIdx.x & 31;
   if (r >= rows) return;
@@ -127,6 +132,7 @@ __device__ __forceinline__ float lane_dot(const float* a, const float* b, int hd
 
 // AttnF: online softmax over the query's keys.
 __global__ void __launch_bounds__(256) attnf_kernel(AttnF<float> k, int64_t n) {
+  griddep_enter();
   const int64_t idx = (int64_t)blockIdx.x * 8 + (threadIdx.x >> 5);
   const int lane = threadIdx.x & 31;
   if (idx >= n) return;
@@ -164,6 +170,7 @@ __global__ void __launch_bounds__(256) attnf_kernel(AttnF<float> k, int64_t n) {
 
 // AttnBQ: dq = scale * sum_p P_p (dO.v_p - dO.o) k_p (overwrites dQ).
 __global__ void __launch_bounds__(256) attnbq_kernel(AttnBQ<float> k, int64_t n) {
+  griddep_enter();
   const int64_t idx = (int64_t)blockIdx.x * 8 + (threadIdx.x >> 5);
   const int lane = threadIdx.x & 31;
   if (idx >= n) return;
@@ -200,6 +207,7 @@ __global__ void __launch_bounds__(256) attnbq_kernel(AttnBQ<float> k, int64_t n)
 
 // AttnBKV: dK, dV of one key position (accumulated) over the queries that see it.
 __global__ void __launch_bounds__(256) attnbkv_kernel(AttnBKV<float> k, int64_t n) {
+  griddep_enter();
   const int64_t idx = (int64_t)blockIdx.x * 8 + (threadIdx.x >> 5);
   const int lane = threadIdx.x & 31;
   if (idx >= n) return;
@@ -239,16 +247,25 @@ __global__ void __launch_bounds__(256) attnbkv_kernel(AttnBKV<float> k, int64_t 
   }
 }
 
-// Device backend of Engine: plain stream-ordered launches (no dependent
-// launch), buffers from cudaMalloc released after the stream drains.
+// Device backend of Engine: stream-ordered launches with programmatic
+// dependent launch (every kernel here waits for its predecessor at entry, then
+// releases its own dependents, so the next launch overlaps this one's tail;
+// the GEMM's pre-wait weight loads read operands made two or more kernels
+// back, which are complete by then), buffers from cudaMalloc released after
+// the stream drains.
 struct CudaBackend {
   cudaStream_t st;
   bool tc;  // bf16 model: contractions on the tensor cores
   std::vector<void*> allocs;
   cudaError_t err = cudaSuccess;
-  // bf16 weight copies (plain [M][K] and transposed [K][M]) by (address, pitch, rows, cols)
+  // bf16 weight copies (plain [M][K] and transposed [K][M]) by (address, pitch, rows, cols); a copy is
+  // remade at its first use in each pass (begin_pass), since the weights may change between passes
   using WKey = std::tuple<const float*, int64_t, int, int>;
-  std::map<WKey, bf16*> w_plain, w_trans;
+  struct WCopy {
+    bf16* p;
+    bool fresh;
+  };
+  std::map<WKey, WCopy> w_plain, w_trans;
   // per-contraction operand scratch and the split-K exchange area, grown on demand
   bf16* sa = nullptr; size_t sa_n = 0;
   bf16* sb = nullptr; size_t sb_n = 0;
@@ -284,9 +301,7 @@ struct CudaBackend {
   template <class K> void launch(const K& k, int64_t n) {
     if (err != cudaSuccess || n <= 0) return;
     const int64_t blocks = (n + 255) / 256;
-    functor_kernel<K><<<(unsigned)blocks, 256, 0, st>>>(k, n);
-    note_launch();
-    err = cudaGetLastError();
+    err = launch_pdl(functor_kernel<K>, dim3((unsigned)blocks), dim3(256), 0, st, k, n);
   }
   int ok() const { return err == cudaSuccess ? 0 : -1; }
   void range_push(const char* name) { nvtxRangePushA(name); }
@@ -295,15 +310,11 @@ struct CudaBackend {
   // ---- row and attention functors, warp or block per unit
   template <class K> void launch_rows(void (*kern)(K, int64_t), const K& k, int64_t n) {
     if (err != cudaSuccess || n <= 0) return;
-    kern<<<(unsigned)((n + 7) / 8), 256, 0, st>>>(k, n);
-    note_launch();
-    err = cudaGetLastError();
+    err = launch_pdl(kern, dim3((unsigned)((n + 7) / 8)), dim3(256), 0, st, k, n);
   }
   void launch(const Xent<float>& k, int64_t n) {
     if (err != cudaSuccess || n <= 0) return;
-    xent_kernel<<<(unsigned)n, 256, 0, st>>>(k);
-    note_launch();
-    err = cudaGetLastError();
+    err = launch_pdl(xent_kernel, dim3((unsigned)n), dim3(256), 0, st, k);
   }
   void launch(const RmsF<float>& k, int64_t n) { launch_rows(rmsf_kernel, k, n); }
   void launch(const RmsBX<float>& k, int64_t n) { launch_rows(rmsbx_kernel, k, n); }
@@ -341,26 +352,33 @@ struct CudaBackend {
   }
   void to_bf16_t(const float* src, int64_t ld, int R, int C, int Rp, bf16* dst) {
     if (err != cudaSuccess) return;
-    to_bf16_t_kernel<<<dim3((unsigned)((C + 31) / 32), (unsigned)(Rp / 32)), dim3(32, 8), 0, st>>>(src, ld, R, C, Rp,
-                                                                                                 dst);
-    note_launch();
-    err = cudaGetLastError();
+    err = launch_pdl(to_bf16_t_kernel, dim3((unsigned)((C + 31) / 32), (unsigned)(Rp / 32)), dim3(32, 8), 0, st, src,
+                     ld, R, C, Rp, dst);
   }
-  // bf16 copy of the weight block W[M][K] (pitch ldw), plain or transposed, once per call
+  void begin_pass() {
+    for (auto& e : w_plain) e.second.fresh = false;
+    for (auto& e : w_trans) e.second.fresh = false;
+  }
+  // bf16 copy of the weight block W[M][K] (pitch ldw), plain or transposed, once per pass
   const bf16* weight(const float* W, int64_t ldw, int M, int K, bool transposed) {
+    if (err != cudaSuccess) return nullptr;
     auto& cache = transposed ? w_trans : w_plain;
     const WKey key{W, ldw, M, K};
     auto it = cache.find(key);
-    if (it != cache.end()) return it->second;
-    void* q = nullptr;
-    if (err != cudaSuccess) return nullptr;
-    err = cudaMalloc(&q, (size_t)M * K * sizeof(bf16));
-    if (err != cudaSuccess) { cudaGetLastError(); return nullptr; }
-    allocs.push_back(q);
-    bf16* b = static_cast<bf16*>(q);
+    if (it != cache.end() && it->second.fresh) return it->second.p;
+    bf16* b = nullptr;
+    if (it != cache.end()) {
+      b = it->second.p;
+    } else {
+      void* q = nullptr;
+      err = cudaMalloc(&q, (size_t)M * K * sizeof(bf16));
+      if (err != cudaSuccess) { cudaGetLastError(); return nullptr; }
+      allocs.push_back(q);
+      b = static_cast<bf16*>(q);
+    }
     if (transposed) to_bf16_t(W, ldw, M, K, M, b);  // [K][M]; M % 64 == 0 where used
     else to_bf16(W, ldw, M, K, b);
-    cache.emplace(key, b);
+    cache[key] = WCopy{b, true};
     return b;
   }
   // C[n][m] (+)= sum_k Bop[n][k] Aop[m][k] into fp32 rows `ldc` apart.  A
@@ -439,17 +457,124 @@ cudaError_t widen_to_f32(const void* src, int dtype, int64_t rows, int64_t cols,
   return cudaGetLastError();
 }
 
-cudaError_t replay_backward_f32(const Dims& D, const float* const* W32, float* const* G32, const int32_t* tok,
-                                const float* wts, int seg, float* logp, bool tensor_cores, cudaStream_t st) {
-  cudaError_t e;
-  {
-    CudaBackend bk(st, tensor_cores);
-    Engine<CudaBackend, float> eng(bk, D, W32, G32);
-    eng.run(tok, wts, seg, logp);
-    e = bk.err;
-  }  // the backend drains the stream and frees the engine's buffers here
+// ---------------------------------------------------------------- runner
+namespace {
+// Above this many kernels a pass runs its launches directly: a graph of that
+// size costs more to instantiate and hold than its launches cost.
+constexpr int64_t kMaxGraphKernels = 400000;
+
+struct StreamSet {
+  cudaStream_t s = nullptr;
+  cudaEvent_t in = nullptr, out = nullptr;
+  ~StreamSet() {
+    if (in) cudaEventDestroy(in);
+    if (out) cudaEventDestroy(out);
+    if (s) cudaStreamDestroy(s);
+  }
+};
+}  // namespace
+
+struct Runner {
+  Dims D;
+  int seg;
+  StreamSet ss;  // destroyed after the backend below, which drains the stream
+  CudaBackend bk;
+  Engine<CudaBackend, float> eng;
+  int32_t* tok = nullptr;
+  float* wts = nullptr;
+  float* logp = nullptr;
+  int passes = 0;
+  bool graph_ok = true;
+  cudaGraphExec_t exec = nullptr;
+  int64_t kernels = 0;  // kernels of one pass
+  Runner(const Dims& d, int sg, cudaStream_t s, bool tc, const float* const* W32, float* const* G32)
+      : D(d), seg(sg), bk(s, tc), eng(bk, d, W32, G32) {}
+  ~Runner() {
+    if (exec) cudaGraphExecDestroy(exec);
+  }
+};
+
+cudaError_t runner_create(const Dims& D, int seg, bool tensor_cores, const float* const* W32, float* const* G32,
+                          Runner** out) {
+  *out = nullptr;
+  cudaStream_t s = nullptr;
+  cudaError_t e = cudaStreamCreateWithFlags(&s, cudaStreamNonBlocking);
   if (e != cudaSuccess) return e;
-  return cudaGetLastError();
+  Runner* r = new Runner(D, seg, s, tensor_cores, W32, G32);
+  r->ss.s = s;
+  e = cudaEventCreateWithFlags(&r->ss.in, cudaEventDisableTiming);
+  if (e == cudaSuccess) e = cudaEventCreateWithFlags(&r->ss.out, cudaEventDisableTiming);
+  if (e == cudaSuccess) {
+    r->tok = r->bk.alloc<int32_t>((size_t)D.B * D.S);
+    r->wts = r->bk.alloc<float>((size_t)D.B * (D.S - 1));
+    r->logp = r->bk.alloc<float>((size_t)D.B * (D.S - 1));
+    e = r->bk.err;
+  }
+  if (e != cudaSuccess) {
+    delete r;
+    return e;
+  }
+  *out = r;
+  return cudaSuccess;
+}
+
+void runner_free(Runner* r) { delete r; }
+
+cudaError_t runner_run(Runner* r, cudaError_t (*prologue)(void* ctx, cudaStream_t s), void* ctx, const int32_t* tok,
+                       const float* wts, float* logp, cudaStream_t st) {
+  const Dims& D = r->D;
+  cudaStream_t gs = r->ss.s;
+  cudaError_t e = cudaEventRecord(r->ss.in, st);
+  if (e == cudaSuccess) e = cudaStreamWaitEvent(gs, r->ss.in, 0);
+  if (e == cudaSuccess)
+    e = cudaMemcpyAsync(r->tok, tok, (size_t)D.B * D.S * 4, cudaMemcpyDeviceToDevice, gs);
+  if (e == cudaSuccess)
+    e = cudaMemcpyAsync(r->wts, wts, (size_t)D.B * (D.S - 1) * 4, cudaMemcpyDeviceToDevice, gs);
+  if (e != cudaSuccess) return e;
+  // the pass: widen the weights, then the engine (forward sweep, segments in reverse, encoder)
+  auto pass = [&]() -> cudaError_t {
+    cudaError_t pe = prologue(ctx, gs);
+    if (pe != cudaSuccess) return pe;
+    r->bk.begin_pass();
+    const int rc = r->eng.run(r->tok, r->wts, r->seg, r->logp);
+    if (r->bk.err != cudaSuccess) return r->bk.err;
+    return rc == 0 ? cudaSuccess : cudaErrorInvalidValue;
+  };
+  if (r->exec) {
+    for (int64_t i = 0; i < r->kernels; ++i) note_launch();
+    e = cudaGraphLaunch(r->exec, gs);
+  } else if (r->passes == 0 || !r->graph_ok || r->kernels > kMaxGraphKernels) {
+    const int64_t n0 = launch_count();
+    e = pass();
+    if (r->passes == 0) r->kernels = launch_count() - n0;
+  } else {
+    // second pass: capture it (every buffer and bf16 weight copy exists by
+    // now, so the pass allocates nothing), then launch the graph
+    cudaGraph_t g = nullptr;
+    bool ok = cudaStreamBeginCapture(gs, cudaStreamCaptureModeThreadLocal) == cudaSuccess;
+    const int64_t n0 = launch_count();
+    const cudaError_t pe = ok ? pass() : cudaSuccess;
+    const int64_t n1 = launch_count();
+    if (ok) ok = cudaStreamEndCapture(gs, &g) == cudaSuccess && pe == cudaSuccess;
+    if (ok) ok = cudaGraphInstantiate(&r->exec, g, 0) == cudaSuccess;
+    if (g) cudaGraphDestroy(g);
+    if (ok) {
+      r->kernels = n1 - n0;
+      e = cudaGraphLaunch(r->exec, gs);
+    } else {  // graphs off for this runner; this pass launches its kernels
+      cudaGetLastError();
+      r->exec = nullptr;
+      r->graph_ok = false;
+      r->bk.err = cudaSuccess;
+      e = pass();
+    }
+  }
+  if (e != cudaSuccess) return e;
+  ++r->passes;
+  if (logp) e = cudaMemcpyAsync(logp, r->logp, (size_t)D.B * (D.S - 1) * 4, cudaMemcpyDeviceToDevice, gs);
+  if (e == cudaSuccess) e = cudaEventRecord(r->ss.out, gs);
+  if (e == cudaSuccess) e = cudaStreamWaitEvent(st, r->ss.out, 0);
+  return e;
 }
 
 }  // namespace bptt

@@ -43,6 +43,7 @@
 #include <stdio.h>
 
 #include <string>
+#include <utility>
 #include <vector>
 
 #if defined(__CUDACC__)
@@ -510,12 +511,21 @@ class Engine {
   Engine(BK& bk, const Dims& D, const Real* const* Wt, Real* const* Gt) : bk_(bk), D_(D), Wt_(Wt), Gt_(Gt) {}
 
   // tok [B][S] and wts [B][S-1] on the backend; logp [B][S-1] (may be null).
+  // An engine may run several passes of the same sizes and segment length:
+  // the first allocates its buffers, later ones set every buffer back to
+  // zero, the state the first pass starts from (-1: another segment length).
   int run(const int32_t* tok, const Real* wts, int seg, Real* logp) {
     const Dims& D = D_;
     if (seg < 1) seg = 1;
     if (seg > D.S - 1) seg = D.S - 1;
-    seg_ = seg;
-    setup();
+    if (!ready_) {
+      seg_ = seg;
+      setup();
+      ready_ = true;
+    } else {
+      if (seg != seg_) return -1;
+      for (const auto& b : bufs_) bk_.zero(b.first, b.second);
+    }
     if (bk_.ok() != 0) return bk_.ok();
     encoder_forward(tok);
     copy2(Wt(T_SSTAR), 0, s_cur_, D.d, D.B, D.d);  // H_0: s_star in every sequence (eq. 2.3)
@@ -576,6 +586,8 @@ class Engine {
   const Real* const* Wt_;
   Real* const* Gt_;
   int seg_ = 1;
+  bool ready_ = false;
+  std::vector<std::pair<Real*, size_t>> bufs_;  // every buffer of setup(), zero at the start of a pass
   std::vector<double> inv_host_;
   double* inv_ = nullptr;
   std::vector<EncRec> enc_;
@@ -600,7 +612,11 @@ class Engine {
   StepRec& rec(int slot) { return recs_[slot]; }
   Real scale() const { return Real(1) / r_sqrt(Real(D_.hd())); }
 
-  Real* A(size_t n) { return bk_.template alloc<Real>(n); }
+  Real* A(size_t n) {
+    Real* p = bk_.template alloc<Real>(n);
+    bufs_.emplace_back(p, n);
+    return p;
+  }
 
   void setup() {
     const Dims& D = D_;

@@ -183,11 +183,24 @@ namespace bptt {
 cudaError_t widen_to_f32(const void* src, int dtype, int64_t rows, int64_t cols, int64_t pitch, float* dst,
                          cudaStream_t st);
 // Full-BPTT gradient of the weighted replay loss (bptt_core.h) on fp32
-// weights W32 into G32 (per catalogue index; null where a tensor is absent).
-// tensor_cores: run the contractions whose shapes allow it on tcgen05 with
-// bf16 operands (bf16 models).  Drains the stream before it returns.
-cudaError_t replay_backward_f32(const Dims& D, const float* const* W32, float* const* G32, const int32_t* tok,
-                                const float* wts, int seg, float* logp, bool tensor_cores, cudaStream_t st);
+// weights W32 into G32 (per catalogue index; null where a tensor is absent),
+// held for repeated calls of one size: the runner owns the engine's buffers,
+// staging copies of the inputs, its own stream and, from its second pass on,
+// a CUDA graph of the whole pass (prologue included) that later passes
+// replay.  The W32 and G32 arrays and the buffers they point to must outlive
+// the runner.  tensor_cores: run the contractions whose shapes allow it on
+// tcgen05 with bf16 operands (bf16 models).
+struct Runner;
+cudaError_t runner_create(const Dims& D, int seg, bool tensor_cores, const float* const* W32, float* const* G32,
+                          Runner** out);
+// One pass: waits for `st`, copies tok [B][S] and wts [B][S-1] to staging,
+// runs prologue(stream) (it fills W32) and the engine on the runner's
+// stream, copies the log-probs to logp (may be null), and makes `st` wait for
+// the pass.  Does not block the host.
+cudaError_t runner_run(Runner* r, cudaError_t (*prologue)(void* ctx, cudaStream_t s), void* ctx, const int32_t* tok,
+                       const float* wts, float* logp, cudaStream_t st);
+// Drains the runner's stream and frees everything it holds.
+void runner_free(Runner* r);
 }  // namespace bptt
 
 }  // namespace rlt

@@ -106,8 +106,24 @@ struct rlt_model {
   rlt_state* replay = nullptr;  // model-owned state of rlt_replay_logprobs
   int64_t live_states = 0;      // states made by rlt_state_create and not yet freed
   std::vector<float*> grad;     // fp32 gradient per catalogue index of bptt_core.h (rlt_replay_backward)
+  struct BackwardHold* bwd = nullptr;  // buffers of rlt_replay_backward, kept for calls of the same sizes
   ProfileRec prof;
 };
+
+// What rlt_replay_backward keeps between calls with the same (B, S, segment):
+// fp32 copies of the weights (refilled by every pass) and the runner
+// (engine buffers, staging inputs, its stream and its graph).
+struct BackwardHold {
+  int B = 0, S = 0, seg = 0, dtype = 0;
+  std::vector<float*> w32;
+  std::vector<const View*> views;
+  std::vector<void*> allocs;
+  bptt::Runner* runner = nullptr;
+};
+
+namespace {
+void release_backward(rlt_model* m);
+}  // namespace
 
 struct rlt_state {
   rlt_model* m = nullptr;
@@ -1005,6 +1021,7 @@ int32_t rlt_model_free(rlt_model* m) {
   cudaSetDevice(m->device);
   cudaDeviceSynchronize();
   if (m->replay) rlt_state_free(m->replay);
+  release_backward(m);
   for (cudaEvent_t e : m->prof.ev) cudaEventDestroy(e);
   free_all(m->allocs);
   delete m;
@@ -1554,6 +1571,29 @@ const View* bptt_view(const rlt_model* m, const bptt::Dims& D, int i) {
 // accumulates into them on the same stream.  The buffers join the model's
 // allocations only once all exist; a failure part-way frees those already
 // made, so a retry starts clean.
+// Frees what rlt_replay_backward keeps (after its work has drained).
+void release_backward(rlt_model* m) {
+  BackwardHold* h = m->bwd;
+  if (!h) return;
+  m->bwd = nullptr;
+  if (h->runner) bptt::runner_free(h->runner);
+  cudaDeviceSynchronize();
+  free_all(h->allocs);
+  delete h;
+}
+
+// The prologue of every backward pass: the fp32 copies of the current weights.
+cudaError_t widen_weights(void* ctx, cudaStream_t st) {
+  const BackwardHold* h = static_cast<const BackwardHold*>(ctx);
+  for (size_t i = 0; i < h->w32.size(); ++i) {
+    const View* v = h->views[i];
+    if (!v) continue;
+    const cudaError_t e = bptt::widen_to_f32(v->base, h->dtype, v->rows, v->cols, v->pitch, h->w32[i], st);
+    if (e != cudaSuccess) return e;
+  }
+  return cudaSuccess;
+}
+
 int32_t ensure_grads(rlt_model* m, const bptt::Dims& D, cudaStream_t st) {
   if (!m->grad.empty()) return RLT_OK;
   const int n = bptt::n_tensors(D);
@@ -1600,31 +1640,55 @@ int32_t rlt_replay_backward(rlt_model* m, const int32_t* tok_dev, int32_t B, int
       if (v < 0 || v >= m->cfg.vocab) return fail(RLT_E_INVAL, "token id " + std::to_string(v) + " out of range");
   }
   const bptt::Dims D = bptt_dims(m, B, S);
+  const int seg = std::min(segment, S - 1);
   RLT_TRY(ensure_grads(m, D, st));
-  // fp32 copies of the current weights, freed before returning
-  const int n = bptt::n_tensors(D);
-  std::vector<float*> w32(n, nullptr);
-  std::vector<void*> tmp;
-  int32_t r = RLT_OK;
-  for (int i = 0; i < n && r == RLT_OK; ++i) {
-    const View* v = bptt_view(m, D, i);
-    if (!v) continue;
-    void* p = nullptr;
-    r = dev_alloc(tmp, &p, (size_t)(v->rows * v->cols) * 4);
-    if (r != RLT_OK) break;
-    w32[i] = static_cast<float*>(p);
-    const cudaError_t e = bptt::widen_to_f32(v->base, m->cfg.dtype, v->rows, v->cols, v->pitch, w32[i], st);
-    if (e != cudaSuccess) r = fail(RLT_E_CUDA, std::string("widen: ") + cudaGetErrorString(e));
+  if (m->bwd && (m->bwd->B != B || m->bwd->S != S || m->bwd->seg != seg)) release_backward(m);
+  if (!m->bwd) {
+    BackwardHold* h = new BackwardHold();
+    h->B = B;
+    h->S = S;
+    h->seg = seg;
+    h->dtype = m->cfg.dtype;
+    const int n = bptt::n_tensors(D);
+    h->w32.assign(n, nullptr);
+    h->views.assign(n, nullptr);
+    int32_t r = RLT_OK;
+    for (int i = 0; i < n && r == RLT_OK; ++i) {
+      const View* v = bptt_view(m, D, i);
+      if (!v) continue;
+      void* p = nullptr;
+      r = dev_alloc(h->allocs, &p, (size_t)(v->rows * v->cols) * 4);
+      h->views[i] = v;
+      h->w32[i] = static_cast<float*>(p);
+    }
+    if (r == RLT_OK) {
+      const cudaError_t e = bptt::runner_create(D, seg, m->cfg.dtype == RLT_DTYPE_BF16, h->w32.data(),
+                                                m->grad.data(), &h->runner);
+      if (e == cudaErrorMemoryAllocation) r = fail(RLT_E_OOM, "backward buffers: out of device memory");
+      else if (e != cudaSuccess) r = fail(RLT_E_CUDA, std::string("backward setup: ") + cudaGetErrorString(e));
+    }
+    if (r != RLT_OK) {
+      free_all(h->allocs);
+      delete h;
+      return r;
+    }
+    m->bwd = h;
   }
-  if (r == RLT_OK) {
-    const cudaError_t e = bptt::replay_backward_f32(D, w32.data(), m->grad.data(), tok_dev, w_dev, segment, logp_dev,
-                                                    m->cfg.dtype == RLT_DTYPE_BF16, st);
-    if (e == cudaErrorMemoryAllocation) r = fail(RLT_E_OOM, "backward buffers: out of device memory");
-    else if (e != cudaSuccess) r = fail(RLT_E_CUDA, std::string("backward: ") + cudaGetErrorString(e));
+  const cudaError_t e = bptt::runner_run(m->bwd->runner, widen_weights, m->bwd, tok_dev, w_dev, logp_dev, st);
+  if (e != cudaSuccess) {
+    cudaGetLastError();
+    release_backward(m);
+    if (e == cudaErrorMemoryAllocation) return fail(RLT_E_OOM, "backward buffers: out of device memory");
+    return fail(RLT_E_CUDA, std::string("backward: ") + cudaGetErrorString(e));
   }
-  cudaStreamSynchronize(st);
-  free_all(tmp);
-  return r;
+  return ok();
+}
+
+int32_t rlt_backward_release(rlt_model* m) {
+  if (!m) return fail(RLT_E_INVAL, "null argument");
+  RLT_CUDA(cudaSetDevice(m->device));
+  release_backward(m);
+  return ok();
 }
 
 int32_t rlt_grad_read(const rlt_model* m, const char* name, float* host, size_t bytes) {

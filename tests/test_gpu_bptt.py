@@ -170,3 +170,53 @@ def test_backward_long_sequence_hd128():
         scale = float(np.max(np.abs(ref)))
         err = float(np.max(np.abs(m.grad(name) - ref)))
         assert err <= 5e-2 * scale + 1e-6, (name, err / scale)
+
+
+def test_backward_kept_between_calls_and_replayed(rlt, oracle_lib):
+    """The model keeps the backward's buffers between calls of one size: the
+    first call launches its kernels, the second captures the whole pass as a
+    CUDA graph, later ones replay it.  Every call below starts from zeroed
+    gradients and meets the oracle at the bf16 bars: four calls of one size
+    on different tokens and target weights, with a weight loaded between the
+    second and the third (the graph's prologue refreshes the fp32 weight
+    copies); then a call of another batch size (the kept buffers are
+    rebuilt); then one after rlt_backward_release."""
+    import torch
+
+    from oracle import bptt
+    w = synth.workload("tiny", d=128, n_heads=2, ffn=192, vocab=256, prompt=10, dtype=1, window=3)
+    cfg = synth.model_config(w)
+    m = rlt.rlt_init_weights(cfg, synth.WEIGHT_SEED)
+    om = oracle_lib.Model(cfg, seed=synth.WEIGHT_SEED)
+    rng = np.random.default_rng(11)
+
+    def check(tok, seg=4):
+        B, S = tok.shape
+        wts = rng.uniform(-1.0, 1.0, (B, S - 1)).astype(np.float32)
+        rlt.rlt_grad_zero(m)
+        lp = torch.zeros((B, S - 1), dtype=torch.float32, device="cuda")
+        rlt.rlt_replay_backward(m, torch.from_numpy(tok).cuda(), torch.from_numpy(wts).cuda(), segment=seg, logp=lp)
+        want = None
+        lp_err = 0.0
+        for b in range(B):
+            lp_err = max(lp_err, float(np.max(np.abs(lp[b].cpu().numpy() - om.replay_logprobs(tok[b])))))
+            _, g = bptt.loss_and_grads(om, tok[b], wts[b].astype(np.float64))
+            want = g if want is None else {k: want[k] + g[k] for k in want}
+        assert lp_err <= 5e-2
+        for name, ref in want.items():
+            scale = float(np.max(np.abs(ref)))
+            assert float(np.max(np.abs(m.grad(name) - ref))) <= 5e-2 * scale + 1e-6, name
+
+    base = synth.tokens(w, batch=2)
+    for i in range(4):
+        tok = base.copy() if i == 0 else rng.integers(0, cfg["vocab"], size=base.shape).astype(np.int32)
+        tok[:, 0] = base[:, 0]  # BOS
+        if i == 2:
+            ws = m.get_weights("w_state")[::-1].copy()
+            m.load_weights("w_state", ws)
+            om.set("w_state", ws)
+        check(tok)
+    check(synth.tokens(w, batch=3))
+    rlt.rlt_backward_release(m)
+    check(base)
+    rlt.rlt_check_device()

@@ -99,11 +99,13 @@ def test_weights_match_oracle_generator(rlt, oracle_lib):
 
 
 # ------------------------------------------------------------------ teacher-forced parity
+# W160_hd64: a ring of 159 entries takes the streamed SWA kernel (chunks of
+# 64 keys at hd 64 in fp32: 64 + 64 + 31) and wraps twice over 400 positions.
 TINY_VARIANTS = [dict(), dict(window=1), dict(window=32), dict(groups=2, merge_kind=1), dict(tied=0, window=3),
-                 dict(alpha=0.5, window=2)]
+                 dict(alpha=0.5, window=2), dict(window=160, n_heads=1, prompt=400)]
 
 
-@pytest.mark.parametrize("kw", TINY_VARIANTS, ids=["tiny", "W1", "Wfull", "G2_convex", "untied", "W2"])
+@pytest.mark.parametrize("kw", TINY_VARIANTS, ids=["tiny", "W1", "Wfull", "G2_convex", "untied", "W2", "W160_hd64"])
 def test_replay_parity_fp32(rlt, torch_mod, oracle_lib, kw):
     w, cfg = _tiny(**kw)
     tok = synth.tokens(w)
@@ -112,8 +114,9 @@ def test_replay_parity_fp32(rlt, torch_mod, oracle_lib, kw):
     assert np.max(np.abs(got - want)) <= TOL_F32
 
 
-@pytest.mark.parametrize("kw", [dict(), dict(n_heads=4), dict(groups=2, merge_kind=1), dict(window=1)],
-                         ids=["hd128", "hd64", "G2_convex", "W1"])
+@pytest.mark.parametrize("kw", [dict(), dict(n_heads=4), dict(groups=2, merge_kind=1), dict(window=1),
+                                dict(window=200, prompt=420)],
+                         ids=["hd128", "hd64", "G2_convex", "W1", "W200_wrap"])
 def test_replay_parity_bf16(rlt, torch_mod, oracle_lib, kw):
     w, cfg = _bf16_small(**kw)
     tok = synth.tokens(w)

@@ -29,6 +29,9 @@ pytestmark = pytest.mark.gpu
 PROMPTS = [37, 5, 100, 64]
 SPANS = [3, 0, 17, 9]
 GEN1, GEN2 = 6, 4
+# bf16_wide: a window of 160 (the streamed SWA kernel); two of the rings wrap
+# during the prompt, one during the steps, one never
+PROMPTS_WIDE = [190, 5, 230, 157]
 
 
 @pytest.fixture(scope="module")
@@ -44,14 +47,15 @@ def _model(kind):
         w = synth.workload("tiny", window=4, prompt=8, batch=4)
         tol = 1e-4
     else:
-        w = synth.workload("small", d=256, n_heads=2, n_layers=2, window=16, groups=1, ffn=512, vocab=1024, dtype=1,
-                           batch=4, prompt=8, gen=0, dist="zipf", data_seed=1201)
+        w = synth.workload("small", d=256, n_heads=2, n_layers=2, window=160 if kind == "bf16_wide" else 16,
+                           groups=1, ffn=512, vocab=1024, dtype=1, batch=4, prompt=8, gen=0, dist="zipf",
+                           data_seed=1201)
         tol = 5e-2
-    return w, synth.model_config(w), tol
+    return w, synth.model_config(w), tol, PROMPTS_WIDE if kind == "bf16_wide" else PROMPTS
 
 
-def _histories(w, rows):
-    n = max(PROMPTS) + GEN1 + max(SPANS) + GEN2 + 2
+def _histories(w, rows, prompts):
+    n = max(prompts) + GEN1 + max(SPANS) + GEN2 + 2
     tok = synth.tokens(w, batch=4, length=n)
     return tok[rows]
 
@@ -118,18 +122,18 @@ def _run(rlt, torch, m, hist, prompts, spans, snapshot_at_end=False):
     return out, phases, st
 
 
-@pytest.mark.parametrize("kind", ["f32", "bf16"])
+@pytest.mark.parametrize("kind", ["f32", "bf16", "bf16_wide"])
 def test_ragged_batch(rlt, oracle_lib, kind):
     import torch
-    w, cfg, tol = _model(kind)
-    hist = _histories(w, [0, 1, 2, 3])
+    w, cfg, tol, prompts = _model(kind)
+    hist = _histories(w, [0, 1, 2, 3], prompts)
     m = rlt.rlt_init_weights(cfg, synth.WEIGHT_SEED)
-    got, phases, st = _run(rlt, torch, m, hist, PROMPTS, SPANS)
+    got, phases, st = _run(rlt, torch, m, hist, prompts, SPANS)
 
     # per-sequence positions and ring bookkeeping, exact
     Wm1 = cfg["window"] - 1
-    want_dec = [np.array(PROMPTS), np.array(PROMPTS) + GEN1, np.array(PROMPTS) + GEN1 + np.array(SPANS),
-                np.array(PROMPTS) + GEN1 + np.array(SPANS) + GEN2]
+    want_dec = [np.array(prompts), np.array(prompts) + GEN1, np.array(prompts) + GEN1 + np.array(SPANS),
+                np.array(prompts) + GEN1 + np.array(SPANS) + GEN2]
     for ph, dec in zip(phases, want_dec):
         assert np.array_equal(ph["n_dec"], dec) and np.array_equal(ph["n_enc"], dec)
         assert np.array_equal(ph["ring_valid"], np.minimum(dec, Wm1))
@@ -149,7 +153,7 @@ def test_ragged_batch(rlt, oracle_lib, kind):
 
     # bit-identical to each sequence alone
     for b in range(4):
-        one, ph1, st1 = _run(rlt, torch, m, hist[b:b + 1], [PROMPTS[b]], [SPANS[b]])
+        one, ph1, st1 = _run(rlt, torch, m, hist[b:b + 1], [prompts[b]], [SPANS[b]])
         for (bb, t), v in one.items():
             assert got[(b, t)] == v, (kind, b, t, got[(b, t)], v)
         assert int(ph1[-1]["n_dec"][0]) == int(want_dec[-1][b])
