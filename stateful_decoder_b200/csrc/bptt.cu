@@ -64,25 +64,60 @@ __global__ void to_bf16_t_kernel(const float* __restrict__ src, int64_t ld, int 
 // arithmetic of the bptt_core.h functors (up to the order of summation),
 // without one thread walking a whole row or key range alone.
 
-// Readout loss of row b (Xent): one block per row.
-__global__ void __launch_bounds__(256) xent_kernel(Xent<float> k) {
+// Readout loss of row b (Xent): one block of 1024 threads per row.  One
+// pass keeps a running maximum and sum per thread (combined over the block),
+// a second writes the adjoint; rows of V % 4 == 0 move as float4.
+constexpr int kXentThreads = 1024;
+__device__ __forceinline__ void online_add(float x, float& mx, float& den) {
+  if (x > mx) {
+    den = den * expf(mx - x) + 1.f;
+    mx = x;
+  } else {
+    den += expf(x - mx);
+  }
+}
+__global__ void __launch_bounds__(kXentThreads) xent_kernel(Xent<float> k) {
   griddep_enter();
   __shared__ float red[32];
   const int b = blockIdx.x;
   const float* l = k.logits + (int64_t)b * k.V;
-  float mx = -INFINITY;
-  for (int v = threadIdx.x; v < k.V; v += blockDim.x) mx = fmaxf(mx, l[v]);
-  mx = block_max(mx, red);
-  float den = 0.f;
-  for (int v = threadIdx.x; v < k.V; v += blockDim.x) den += expf(l[v] - mx);
-  den = block_sum(den, red);
-  const float lse = mx + logf(den);
+  const bool vec = (k.V & 3) == 0;
+  float mx = -INFINITY, den = 0.f;
+  if (vec) {
+    const float4* l4 = reinterpret_cast<const float4*>(l);
+    for (int v = threadIdx.x; v < k.V / 4; v += kXentThreads) {
+      const float4 x = l4[v];
+      online_add(x.x, mx, den);
+      online_add(x.y, mx, den);
+      online_add(x.z, mx, den);
+      online_add(x.w, mx, den);
+    }
+  } else {
+    for (int v = threadIdx.x; v < k.V; v += kXentThreads) online_add(l[v], mx, den);
+  }
+  const float M = block_max(mx, red);
+  den = block_sum(mx == -INFINITY ? 0.f : den * expf(mx - M), red);
+  const float lse = M + logf(den);
   const int y = k.tok[(int64_t)b * k.tok_sb + k.t + 1];
   if (k.logp && threadIdx.x == 0) k.logp[(int64_t)b * k.w_sb + k.t] = l[y] - lse;
   if (k.dlogits) {
     const float w = k.wts[(int64_t)b * k.w_sb + k.t];
     float* dl = k.dlogits + (int64_t)b * k.V;
-    for (int v = threadIdx.x; v < k.V; v += blockDim.x) dl[v] = w * (expf(l[v] - lse) - (v == y ? 1.f : 0.f));
+    if (vec) {
+      const float4* l4 = reinterpret_cast<const float4*>(l);
+      float4* d4 = reinterpret_cast<float4*>(dl);
+      for (int v = threadIdx.x; v < k.V / 4; v += kXentThreads) {
+        const float4 x = l4[v];
+        float4 o;
+        o.x = w * (expf(x.x - lse) - (4 * v == y ? 1.f : 0.f));
+        o.y = w * (expf(x.y - lse) - (4 * v + 1 == y ? 1.f : 0.f));
+        o.z = w * (expf(x.z - lse) - (4 * v + 2 == y ? 1.f : 0.f));
+        o.w = w * (expf(x.w - lse) - (4 * v + 3 == y ? 1.f : 0.f));
+        d4[v] = o;
+      }
+    } else {
+      for (int v = threadIdx.x; v < k.V; v += kXentThreads) dl[v] = w * (expf(l[v] - lse) - (v == y ? 1.f : 0.f));
+    }
   }
 }
 
@@ -94,11 +129,13 @@ __global__ void __launch_bounds__(256) rmsf_kernel(RmsF<float> k, int64_t rows) 
   if (r >= rows) return;
   const float* x = k.X + r * k.ldx;
   float ss = 0.f;
+#pragma unroll 8
   for (int j = lane; j < k.d; j += 32) ss += x[j] * x[j];
   ss = warp_sum(ss);
   const float ri = 1.0f / sqrtf(ss / (float)k.d + k.eps);
   if (lane == 0) k.rinv[r] = ri;
   float* y = k.Y + r * k.ldy;
+#pragma unroll 8
   for (int j = lane; j < k.d; j += 32) y[j] = x[j] * ri * k.g[j];
 }
 __global__ void __launch_bounds__(256) rmsbx_kernel(RmsBX<float> k, int64_t rows) {
@@ -110,9 +147,11 @@ __global__ void __launch_bounds__(256) rmsbx_kernel(RmsBX<float> k, int64_t rows
   const float* x = k.X + r * k.ldx;
   const float ri = k.rinv[r];
   float dot = 0.f;
+#pragma unroll 8
   for (int j = lane; j < k.d; j += 32) dot += dy[j] * k.g[j] * x[j] * ri;
   dot = warp_sum(dot) / (float)k.d;
   float* dx = k.dX + r * k.lddx;
+#pragma unroll 8
   for (int j = lane; j < k.d; j += 32) dx[j] += ri * (dy[j] * k.g[j] - x[j] * ri * dot);
 }
 
@@ -130,7 +169,12 @@ __device__ __forceinline__ float lane_dot(const float* a, const float* b, int hd
   return warp_sum(s);
 }
 
-// AttnF: online softmax over the query's keys.
+// Keys per round of the attention loops: the round's key and value loads
+// are all issued before any is used, so a warp waits for one load latency per
+// round instead of one per key.
+constexpr int kKeyRound = 8;
+
+// AttnF: online softmax over the query's keys, kKeyRound keys per update.
 __global__ void __launch_bounds__(256) attnf_kernel(AttnF<float> k, int64_t n) {
   griddep_enter();
   const int64_t idx = (int64_t)blockIdx.x * 8 + (threadIdx.x >> 5);
@@ -142,20 +186,55 @@ __global__ void __launch_bounds__(256) attnf_kernel(AttnF<float> k, int64_t n) {
   const int i = (int)(bi % g.Tq);
   const int64_t b = bi / g.Tq;
   const float* q = k.Q + b * g.q_sb + i * g.q_si + (int64_t)h * g.hd;
+  float qd[kLaneDims];
+#pragma unroll
+  for (int j = 0; j < kLaneDims; ++j) qd[j] = lane + 32 * j < g.hd ? q[lane + 32 * j] : 0.f;
   float mx = -INFINITY, den = 0.f, acc[kLaneDims];
 #pragma unroll
   for (int j = 0; j < kLaneDims; ++j) acc[j] = 0.f;
-  for (int p = g.lo(i); p <= g.hi(i); ++p) {
-    const float* kr = k.K + b * g.k_sb + p * g.k_sp + (int64_t)h * g.hd;
-    const float* vr = k.Vv + b * g.k_sb + p * g.k_sp + (int64_t)h * g.hd;
-    const float s = lane_dot(q, kr, g.hd, lane) * k.scale;
-    const float nm = fmaxf(mx, s);
-    const float c = expf(mx - nm), w = expf(s - nm);
-    den = den * c + w;
+  const int lo = g.lo(i), hi = g.hi(i);
+  const float* kb = k.K + b * g.k_sb + (int64_t)h * g.hd;
+  const float* vb = k.Vv + b * g.k_sb + (int64_t)h * g.hd;
+  for (int p0 = lo; p0 <= hi; p0 += kKeyRound) {
+    float kk[kKeyRound][kLaneDims], vv[kKeyRound][kLaneDims];
 #pragma unroll
-    for (int j = 0; j < kLaneDims; ++j) {
-      const int e = lane + 32 * j;
-      acc[j] = acc[j] * c + (e < g.hd ? w * vr[e] : 0.f);
+    for (int u = 0; u < kKeyRound; ++u) {
+      const bool ok = p0 + u <= hi;
+#pragma unroll
+      for (int j = 0; j < kLaneDims; ++j) {
+        const int e = lane + 32 * j;
+        kk[u][j] = ok && e < g.hd ? kb[(int64_t)(p0 + u) * g.k_sp + e] : 0.f;
+        vv[u][j] = ok && e < g.hd ? vb[(int64_t)(p0 + u) * g.k_sp + e] : 0.f;
+      }
+    }
+    float sc[kKeyRound];
+#pragma unroll
+    for (int u = 0; u < kKeyRound; ++u) {
+      sc[u] = 0.f;
+#pragma unroll
+      for (int j = 0; j < kLaneDims; ++j) sc[u] += qd[j] * kk[u][j];
+    }
+#pragma unroll
+    for (int off = 16; off > 0; off >>= 1)
+#pragma unroll
+      for (int u = 0; u < kKeyRound; ++u) sc[u] += __shfl_xor_sync(0xffffffffu, sc[u], off);
+    float bm = -INFINITY;
+#pragma unroll
+    for (int u = 0; u < kKeyRound; ++u) {
+      sc[u] = p0 + u <= hi ? sc[u] * k.scale : -INFINITY;
+      bm = fmaxf(bm, sc[u]);
+    }
+    const float nm = fmaxf(mx, bm);
+    const float c = expf(mx - nm);
+    den *= c;
+#pragma unroll
+    for (int j = 0; j < kLaneDims; ++j) acc[j] *= c;
+#pragma unroll
+    for (int u = 0; u < kKeyRound; ++u) {
+      const float w = expf(sc[u] - nm);
+      den += w;
+#pragma unroll
+      for (int j = 0; j < kLaneDims; ++j) acc[j] += w * vv[u][j];
     }
     mx = nm;
   }
@@ -168,7 +247,8 @@ __global__ void __launch_bounds__(256) attnf_kernel(AttnF<float> k, int64_t n) {
   if (lane == 0) k.lse[b * g.l_sb + i * g.l_si + h] = mx + logf(den);
 }
 
-// AttnBQ: dq = scale * sum_p P_p (dO.v_p - dO.o) k_p (overwrites dQ).
+// AttnBQ: dq = scale * sum_p P_p (dO.v_p - dO.o) k_p (overwrites dQ),
+// kKeyRound keys per round.
 __global__ void __launch_bounds__(256) attnbq_kernel(AttnBQ<float> k, int64_t n) {
   griddep_enter();
   const int64_t idx = (int64_t)blockIdx.x * 8 + (threadIdx.x >> 5);
@@ -182,20 +262,53 @@ __global__ void __launch_bounds__(256) attnbq_kernel(AttnBQ<float> k, int64_t n)
   const int64_t qo = b * g.q_sb + i * g.q_si + (int64_t)h * g.hd;
   const float L = k.lse[b * g.l_sb + i * g.l_si + h];
   const float Dv = lane_dot(k.dO + qo, k.O + qo, g.hd, lane);
-  float acc[kLaneDims];
+  float qd[kLaneDims], dod[kLaneDims], acc[kLaneDims];
 #pragma unroll
-  for (int j = 0; j < kLaneDims; ++j) acc[j] = 0.f;
-  for (int p = g.lo(i); p <= g.hi(i); ++p) {
-    const float* kr = k.K + b * g.k_sb + p * g.k_sp + (int64_t)h * g.hd;
-    const float* vr = k.Vv + b * g.k_sb + p * g.k_sp + (int64_t)h * g.hd;
-    const float s = lane_dot(k.Q + qo, kr, g.hd, lane);
-    const float dp = lane_dot(k.dO + qo, vr, g.hd, lane);
-    const float P = expf(s * k.scale - L);
-    const float ds = P * (dp - Dv) * k.scale;
+  for (int j = 0; j < kLaneDims; ++j) {
+    const int e = lane + 32 * j;
+    qd[j] = e < g.hd ? k.Q[qo + e] : 0.f;
+    dod[j] = e < g.hd ? k.dO[qo + e] : 0.f;
+    acc[j] = 0.f;
+  }
+  const int lo = g.lo(i), hi = g.hi(i);
+  const float* kb = k.K + b * g.k_sb + (int64_t)h * g.hd;
+  const float* vb = k.Vv + b * g.k_sb + (int64_t)h * g.hd;
+  for (int p0 = lo; p0 <= hi; p0 += kKeyRound) {
+    float kk[kKeyRound][kLaneDims], vv[kKeyRound][kLaneDims];
 #pragma unroll
-    for (int j = 0; j < kLaneDims; ++j) {
-      const int e = lane + 32 * j;
-      if (e < g.hd) acc[j] += ds * kr[e];
+    for (int u = 0; u < kKeyRound; ++u) {
+      const bool ok = p0 + u <= hi;
+#pragma unroll
+      for (int j = 0; j < kLaneDims; ++j) {
+        const int e = lane + 32 * j;
+        kk[u][j] = ok && e < g.hd ? kb[(int64_t)(p0 + u) * g.k_sp + e] : 0.f;
+        vv[u][j] = ok && e < g.hd ? vb[(int64_t)(p0 + u) * g.k_sp + e] : 0.f;
+      }
+    }
+    float sc[kKeyRound], dp[kKeyRound];
+#pragma unroll
+    for (int u = 0; u < kKeyRound; ++u) {
+      sc[u] = dp[u] = 0.f;
+#pragma unroll
+      for (int j = 0; j < kLaneDims; ++j) {
+        sc[u] += qd[j] * kk[u][j];
+        dp[u] += dod[j] * vv[u][j];
+      }
+    }
+#pragma unroll
+    for (int off = 16; off > 0; off >>= 1)
+#pragma unroll
+      for (int u = 0; u < kKeyRound; ++u) {
+        sc[u] += __shfl_xor_sync(0xffffffffu, sc[u], off);
+        dp[u] += __shfl_xor_sync(0xffffffffu, dp[u], off);
+      }
+#pragma unroll
+    for (int u = 0; u < kKeyRound; ++u) {
+      if (p0 + u > hi) continue;
+      const float P = expf(sc[u] * k.scale - L);
+      const float ds = P * (dp[u] - Dv) * k.scale;
+#pragma unroll
+      for (int j = 0; j < kLaneDims; ++j) acc[j] += ds * kk[u][j];
     }
   }
 #pragma unroll
@@ -314,7 +427,7 @@ struct CudaBackend {
   }
   void launch(const Xent<float>& k, int64_t n) {
     if (err != cudaSuccess || n <= 0) return;
-    err = launch_pdl(xent_kernel, dim3((unsigned)n), dim3(256), 0, st, k);
+    err = launch_pdl(xent_kernel, dim3((unsigned)n), dim3(kXentThreads), 0, st, k);
   }
   void launch(const RmsF<float>& k, int64_t n) { launch_rows(rmsf_kernel, k, n); }
   void launch(const RmsBX<float>& k, int64_t n) { launch_rows(rmsbx_kernel, k, n); }
