@@ -152,7 +152,9 @@ int32_t rlt_init_weights(const rlt_config* cfg, uint64_t seed, rlt_model** out);
 
 /* Copies a whole tensor from host memory in the model's storage format (fp32,
  * or bf16 bit patterns) and bumps the model version.  bytes must equal
- * rows*cols*element size.  Errors: RLT_E_INVAL (unknown name, size). */
+ * rows*cols*element size.  Waits for the device first, so work enqueued
+ * before the call (on any stream) reads the old values.  Errors:
+ * RLT_E_INVAL (unknown name, size), RLT_E_CUDA. */
 int32_t rlt_load_weights(rlt_model* m, const char* name, const void* host, size_t bytes);
 
 /* Copies a whole tensor to host memory (storage format). */

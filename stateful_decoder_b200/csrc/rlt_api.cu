@@ -996,6 +996,9 @@ int32_t rlt_load_weights(rlt_model* m, const char* name, const void* host, size_
   const View& v = it->second;
   if (bytes != (size_t)(v.rows * v.cols) * m->esz) return fail(RLT_E_INVAL, "size mismatch for " + std::string(name));
   RLT_CUDA(cudaSetDevice(m->device));
+  // work still reading the weights may run on streams that do not order
+  // with this copy (the backward's own stream, a caller's non-blocking one)
+  RLT_CUDA(cudaDeviceSynchronize());
   RLT_CUDA(cudaMemcpy2D(v.base, v.pitch * m->esz, host, v.cols * m->esz, v.cols * m->esz, v.rows, cudaMemcpyHostToDevice));
   m->version += 1;
   return ok();
@@ -1566,11 +1569,6 @@ const View* bptt_view(const rlt_model* m, const bptt::Dims& D, int i) {
   return it == m->views.end() ? nullptr : &it->second;
 }
 
-// Allocates the model's gradient buffers on first use and zeroes them on the
-// caller's stream `st`, so the zeroing is ordered before the backward that
-// accumulates into them on the same stream.  The buffers join the model's
-// allocations only once all exist; a failure part-way frees those already
-// made, so a retry starts clean.
 // Frees what rlt_replay_backward keeps (after its work has drained).
 void release_backward(rlt_model* m) {
   BackwardHold* h = m->bwd;
@@ -1594,6 +1592,11 @@ cudaError_t widen_weights(void* ctx, cudaStream_t st) {
   return cudaSuccess;
 }
 
+// Allocates the model's gradient buffers on first use and zeroes them on the
+// caller's stream `st`, so the zeroing is ordered before the backward that
+// accumulates into them on the same stream.  The buffers join the model's
+// allocations only once all exist; a failure part-way frees those already
+// made, so a retry starts clean.
 int32_t ensure_grads(rlt_model* m, const bptt::Dims& D, cudaStream_t st) {
   if (!m->grad.empty()) return RLT_OK;
   const int n = bptt::n_tensors(D);
