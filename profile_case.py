@@ -20,9 +20,12 @@ shape of the workload's model but holds fewer layers' state.
       tokens of `batch` sequences (GEMMs with B*len activation rows, causal
       attention on the tensor cores).
 
-  python profile_case.py bptt --workload small --batch 16 --len 64 [--layers 2]
+  python profile_case.py bptt --workload small --batch 16 --len 64 [--layers 2] [--eager]
       Profiles one full-BPTT backward (rlt_replay_backward, eq. 5.1 weights,
-      segments of 32) of `batch` sequences of `len` tokens.
+      segments of 32) of `batch` sequences of `len` tokens: the second call
+      of its size (the replay of the captured graph), or with --eager a
+      first call again (direct launches; the NVTX range "rlt_weight_grads"
+      then marks each segment's weight-gradient contractions).
 
   python profile_case.py summarize launches.csv [S]
       Per-kernel summary of an ncu launch list (gpu__time_duration.sum, --csv)
@@ -129,6 +132,10 @@ def bptt(args) -> None:
     wts = torch.full((B, S - 1), 1.0 / (B * (S - 1)), device="cuda")
     rlt.rlt_replay_backward(m, tok, wts, segment=32)  # warm-up
     torch.cuda.synchronize()
+    if args.eager:
+        # the profiled call then launches its kernels one by one (a first call
+        # of its size), so NVTX ranges around a phase select its launches
+        rlt.rlt_backward_release(m)
     torch.cuda.cudart().cudaProfilerStart()
     rlt.rlt_replay_backward(m, tok, wts, segment=32)
     torch.cuda.synchronize()
@@ -191,6 +198,8 @@ def main() -> None:
     p.add_argument("--batch", type=int, default=16)
     p.add_argument("--len", type=int, default=64)
     p.add_argument("--layers", type=int, default=0)
+    p.add_argument("--eager", action="store_true",
+                   help="profile a first call of its size (direct launches) instead of the graph replay")
     b = sub.add_parser("summarize")
     b.add_argument("csv")
     b.add_argument("S", type=int, nargs="?", default=1024)
