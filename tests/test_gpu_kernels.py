@@ -1,8 +1,8 @@
 """Kernel-level numerics of the decode attention (eq. 2.15 / eq. 2.8) against
 a plain PyTorch fp32 reference of the same operation, through the C ABI's
 op-level entry point.  Cases span one key, exact chunk boundaries (256),
-ragged tails, several chunks, head sizes 16/64/128/256 and both storage types,
-with and without the rotary map on the query."""
+ragged tails, several chunks (up to nine), head sizes 16/32/64/128/256 and
+both storage types, with and without the rotary map on the query."""
 import math
 
 import numpy as np
@@ -48,6 +48,10 @@ CASES = [  # B, H, hd, n, ld_t, dtype, rope
     (2, 4, 16, 513, 600, "f32", True),
     (2, 2, 256, 300, 320, "bf16", True),
     (3, 1, 256, 100, 128, "f32", False),
+    (2, 2, 64, 512, 520, "bf16", False),
+    (2, 2, 64, 513, 520, "bf16", True),
+    (1, 4, 32, 1100, 1200, "bf16", True),
+    (1, 2, 16, 2100, 2200, "f32", True),
 ]
 
 
