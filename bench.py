@@ -337,8 +337,10 @@ def run_gpu(args, w: dict, kind: str, peaks: dict, rank: int, world: int) -> dic
             rlt.rlt_prefill(model, state, tok)
             rlt.rlt_readout(model, state, sampling=samp, sampled=ids[0], logp_sampled=lps[0], logmu=lmu[0])
             for i in range(1, n_gen):
-                rlt.rlt_decoder_step(model, state, tokens=ids[i - 1], sampling=samp, sampled=ids[i],
-                                     logp_sampled=lps[i], logmu=lmu[i])
+                # consumes the token the previous readout sampled (pending in
+                # the state), so every position shares one token source and
+                # the step graphs differ only by the attention chunk count
+                rlt.rlt_decoder_step(model, state, sampling=samp, sampled=ids[i], logp_sampled=lps[i], logmu=lmu[i])
 
         def step_e2e():
             tok.copy_(tok_host, non_blocking=True)
