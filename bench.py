@@ -458,6 +458,7 @@ def run_gpu(args, w: dict, kind: str, peaks: dict, rank: int, world: int) -> dic
     value = world * tokens_per_step * args.steps / (ms / 1e3)
     e2e = world * tokens_per_step * args.steps / (ms_e2e / 1e3)
     roof = step_roofline(w, kind, peaks, t_range)
+    free_b, total_b = torch.cuda.mem_get_info(dev)  # the state, weights and workspaces are all still held
     ms_step = ms / args.steps
 
     def share(ms_sampled, n_sampled, per_step):
@@ -475,6 +476,7 @@ def run_gpu(args, w: dict, kind: str, peaks: dict, rank: int, world: int) -> dic
         "swa": {"gbs": gbs(s_bytes, s_ms, s_n), "share": share(s_ms, s_n, launches_per_step[1])},
         "step_roofline": {"bound_ms": roof["bound_ms"], "frac": roof["bound_ms"] / ms_step},
         "tokens_per_step": tokens_per_step,
+        "memory": {"device_used_gib": (total_b - free_b) / 2**30, "device_total_gib": total_b / 2**30},
     }
 
 
@@ -524,8 +526,10 @@ def run_backward(args, w: dict, rank: int, world: int) -> dict:
     ms = max_over_ranks(e0.elapsed_time(e1), world, dev)
     clk = clocks.stop()
     rlt.rlt_check_device()
+    free_b, total_b = torch.cuda.mem_get_info(dev)  # the kept backward buffers are still held
     return {"value": world * B * (S - 1) * args.steps / (ms / 1e3), "ms_per_step": ms / args.steps,
-            "launches": launches, "clocks": clk, "B": B, "S": S}
+            "launches": launches, "clocks": clk, "B": B, "S": S,
+            "memory": {"device_used_gib": (total_b - free_b) / 2**30, "device_total_gib": total_b / 2**30}}
 
 
 def read_traffic_ratio() -> tuple[float | None, str]:
@@ -647,7 +651,8 @@ def main():
                                objective="eq. 5.1 weights",
                                arithmetic="contractions on tcgen05 with bf16 operands, fp32 accumulation; "
                                           "attention, norms and elementwise adjoints on CUDA cores in fp32"),
-                "roofline": roof, "gpu_launches": r["launches"], "clocks": r["clocks"]}), flush=True)
+                "roofline": roof, "gpu_launches": r["launches"], "clocks": r["clocks"],
+                "memory": r["memory"]}), flush=True)
         return
 
     r = run_gpu(args, w, kind, peaks, rank, world)
@@ -687,6 +692,7 @@ def main():
         "e2e": {"value": r["e2e"], "unit": "tokens/s", "h2d_bytes_per_step": r["h2d"], "d2h_bytes_per_step": r["d2h"]},
         "gpu_launches": r["launches"],
         "clocks": r["clocks"],
+        "memory": r["memory"],
     }
     print(json.dumps(line), flush=True)
 
