@@ -90,8 +90,8 @@ __global__ void rmsnorm_kernel(const float* __restrict__ x, RowMap x_map, const 
 
 // The same, one warp per row for d = 128 * NV: the row stays in registers
 // (NV float4 per lane), the sum of squares is a warp butterfly, and the
-// output is written with 16-byte stores.  Used for the token-parallel
-// encoder's many rows.
+// output is written with 16-byte stores.  Used for every row count at these
+// widths (rows 16-byte aligned).
 template <typename WT, typename OT, int NV>
 __global__ void __launch_bounds__(256) rmsnorm_warp_kernel(const float* __restrict__ x, RowMap x_map, int64_t rows,
                                                            const WT* __restrict__ gamma, float eps, OT* out,
@@ -564,10 +564,14 @@ cudaError_t embed(const int32_t* tok, int64_t n_rows, int tok_per_seq, int64_t t
   return cudaGetLastError();
 }
 
+// The kernel (and with it the order of the sum of squares) is chosen from the
+// row width and layout alone, never from the number of rows, so a row's
+// result does not depend on how many rows share the launch (the batch).
 template <typename WT, typename OT>
 cudaError_t rmsnorm(const float* x, RowMap x_map, const WT* gamma, int64_t rows, int d, float eps, OT* out,
                     int64_t ld_out, cudaStream_t st) {
-  if (rows >= 4096 && ld_out % 4 == 0 && (d == 256 || d == 512 || d == 1024 || d == 2048)) {
+  const bool rows16 = x_map.ld % 4 == 0 && (x_map.per_group <= 0 || x_map.group_stride % 4 == 0) && ld_out % 4 == 0;
+  if (rows16 && (d == 256 || d == 512 || d == 1024 || d == 2048)) {
     const dim3 grid((unsigned)((rows + 7) / 8));
     cudaError_t e_l;
     switch (d) {

@@ -346,8 +346,9 @@ def test_replay_full_size_sampled(rlt, torch_mod, oracle_lib):
 
 def test_batched_equals_single_wide_tiles(rlt, torch_mod):
     """At the reference width the decode GEMMs pick wider activation tiles for
-    B=256 than for B=1 (and the LM head differs too); a sequence's log-probs
-    must still be bit-identical (no batch-dependent reduction order)."""
+    B=256 than for B=100 or B=1 (and the LM head differs too); a sequence's
+    log-probs must still be bit-identical (no batch-dependent reduction
+    order)."""
     w = synth.workload("replay", n_layers=1, batch=256, prompt=24)
     cfg = synth.model_config(w)
     tok = synth.tokens(w)
@@ -356,6 +357,9 @@ def test_batched_equals_single_wide_tiles(rlt, torch_mod):
     for b in (0, 131, 255):
         one, _ = _gpu_replay(rlt, torch_mod, cfg, tok[b:b + 1].copy(), model=m)
         assert np.array_equal(one[0], full[b]), (b, np.max(np.abs(one[0] - full[b])))
+    # 65..128 rows take two 64-wide tiles where the plan has 128-wide ones
+    mid, _ = _gpu_replay(rlt, torch_mod, cfg, tok[:100].copy(), model=m)
+    assert np.array_equal(mid, full[:100])
 
 
 # ------------------------------------------------------------------ RL replay ratios
