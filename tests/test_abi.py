@@ -87,6 +87,7 @@ def test_backward_arguments_validated_on_host():
     lib = rlt._lib
     assert lib.rlt_replay_backward(None, None, 1, 2, None, 4, None, None) == rlt.RLT_E_INVAL
     assert lib.rlt_grad_zero(None, None) == rlt.RLT_E_INVAL
+    assert lib.rlt_backward_release(None) == rlt.RLT_E_INVAL
     buf = (ctypes.c_float * 4)()
     assert lib.rlt_grad_read(None, b"emb", buf, 16) == rlt.RLT_E_INVAL
 
