@@ -461,9 +461,23 @@ def run_gpu(args, w: dict, kind: str, peaks: dict, rank: int, world: int) -> dic
     free_b, total_b = torch.cuda.mem_get_info(dev)  # the state, weights and workspaces are all still held
     ms_step = ms / args.steps
 
-    def share(ms_sampled, n_sampled, per_step):
+    def share(ms_sampled, n_sampled, per_step, scale=1.0):
         # mean sampled launch time x launches of one step / step time
-        return (ms_sampled / n_sampled) * per_step / ms_step if n_sampled else None
+        return (ms_sampled / n_sampled) * per_step / ms_step * scale if n_sampled else None
+
+    # The block workload profiles the blocks after the timed ones, where every
+    # prefix-attention launch reads more keys (t of them: C^E_<=t and
+    # M_<=t); its share is scaled to the timed positions by the ratio of mean
+    # key counts.  The SWA ring is full at both, and the other workloads
+    # profile the same schedule they time.
+    key_scale, share_note = 1.0, "profiled and timed positions are the same schedule"
+    if kind == "block":
+        t_hi = t_range[1]
+        prof_t = [t for t in range(t_hi + 1, t_hi + w["block"] * n_prof + 1) if t % PROFILE_STRIDE == 0]
+        timed_mean = (t_range[0] + t_range[1]) / 2
+        key_scale = timed_mean / (sum(prof_t) / len(prof_t))
+        share_note = (f"profiled launches at t={prof_t[0]}..{prof_t[-1]} (every {PROFILE_STRIDE}th), scaled by "
+                      f"{key_scale:.4f} = mean attended keys at the timed t={t_range[0]}..{t_range[1]} / at the profiled t")
 
     def gbs(nbytes, ms_sampled, n_sampled):
         return (nbytes / n_sampled) / ((ms_sampled / n_sampled) / 1e3) / 1e9 if n_sampled else None
@@ -472,7 +486,7 @@ def run_gpu(args, w: dict, kind: str, peaks: dict, rank: int, world: int) -> dic
         "value": value, "ms_per_step": ms_step, "e2e": e2e, "h2d": h2d, "d2h": d2h, "launches": launches,
         "clocks": clk, "t_range": t_range,
         "attn": {"ms": a_ms, "n": a_n, "bytes": a_bytes, "gbs": gbs(a_bytes, a_ms, a_n),
-                 "share": share(a_ms, a_n, launches_per_step[0])},
+                 "share": share(a_ms, a_n, launches_per_step[0], key_scale), "share_note": share_note},
         "swa": {"gbs": gbs(s_bytes, s_ms, s_n), "share": share(s_ms, s_n, launches_per_step[1])},
         "step_roofline": {"bound_ms": roof["bound_ms"], "frac": roof["bound_ms"] / ms_step},
         "tokens_per_step": tokens_per_step,
@@ -685,7 +699,7 @@ def main():
                      "peak_source": peaks["source"] + " (copy bandwidth)",
                      "profiled_launches": a["n"],
                      "sampling": f"separate untimed pass: launches at every {PROFILE_STRIDE}th position, CUDA events",
-                     "share_of_step": a["share"]},
+                     "share_of_step": a["share"], "share_note": a["share_note"]},
         "swa_attn": {"achieved_gbs": r["swa"]["gbs"], "share_of_step": r["swa"]["share"]},
         "step_roofline": r["step_roofline"],
         "cpu_baseline": cpu,
