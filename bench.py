@@ -162,6 +162,21 @@ def max_over_ranks(ms: float, world: int, device=None) -> float:
     return float(t.item())
 
 
+def gather_rows(x, world: int):
+    """The optional end-of-run collective of the sharded path: every rank's
+    per-sequence results (rows, dim 0) gathered, in rank order, into one
+    [world * rows, ...] tensor on every rank (NCCL on GPUs, gloo on CPU).
+    Nothing is exchanged during the timed steps."""
+    if world <= 1:
+        return x
+    import torch
+    import torch.distributed as dist
+    x = x.contiguous()
+    parts = [torch.empty_like(x) for _ in range(world)]
+    dist.all_gather(parts, x)
+    return torch.cat(parts)
+
+
 # ---------------------------------------------------------------- clocks
 class ClockSampler:
     FIELDS = ("index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
@@ -319,6 +334,7 @@ def run_gpu(args, w: dict, kind: str, peaks: dict, rank: int, world: int) -> dic
 
         h2d, d2h = tok_host.numel() * 4, logp_host.numel() * 4
         n_prof = 1
+        result = lambda: (logp, "teacher-forced log-probs [B, S-1] fp32")  # noqa: E731
         # decode-attention launches of one step: prefix (memory), SWA
         launches_per_step = (w["n_layers"] * (S - 1), w["n_layers"] * (S - 1))
     elif kind == "generate":
@@ -349,6 +365,7 @@ def run_gpu(args, w: dict, kind: str, peaks: dict, rank: int, world: int) -> dic
 
         h2d, d2h = tok_host.numel() * 4, ids_host.numel() * 4
         n_prof = 1
+        result = lambda: (ids.t(), "sampled token ids [B, generated] int32")  # noqa: E731
         n_dec = T + n_gen - 1
         launches_per_step = (w["n_layers"] * n_dec + w["n_layers"] * (n_gen - 1), w["n_layers"] * n_dec)
     else:  # block: prompt prefilled untimed, then blocks of sampled transitions
@@ -399,6 +416,7 @@ def run_gpu(args, w: dict, kind: str, peaks: dict, rank: int, world: int) -> dic
 
         h2d, d2h = first.numel() * 4, ids_host.numel() * 4 + lmu_host.numel() * 4
         n_prof = PROFILE_BLOCKS
+        result = lambda: (ids.t(), "last block's sampled token ids [B, 32] int32")  # noqa: E731
         # prefix attention: encoder step over C^E and cross-attention over M; SWA
         launches_per_step = (2 * w["n_layers"] * blk, w["n_layers"] * blk)
 
@@ -455,6 +473,13 @@ def run_gpu(args, w: dict, kind: str, peaks: dict, rank: int, world: int) -> dic
     ms_e2e, _ = timed(step_e2e, args.steps)
     rlt.rlt_check_device()
 
+    # untimed: the shards' results gathered once at the end of the run
+    res, what = result()
+    gathered = gather_rows(res, world)
+    collective = None if world <= 1 else {
+        "end_of_run_all_gather": what, "rows": int(gathered.shape[0]),
+        "bytes": int(gathered.numel() * gathered.element_size())}
+
     value = world * tokens_per_step * args.steps / (ms / 1e3)
     e2e = world * tokens_per_step * args.steps / (ms_e2e / 1e3)
     roof = step_roofline(w, kind, peaks, t_range)
@@ -491,6 +516,7 @@ def run_gpu(args, w: dict, kind: str, peaks: dict, rank: int, world: int) -> dic
         "step_roofline": {"bound_ms": roof["bound_ms"], "frac": roof["bound_ms"] / ms_step},
         "tokens_per_step": tokens_per_step,
         "memory": {"device_used_gib": (total_b - free_b) / 2**30, "device_total_gib": total_b / 2**30},
+        "collective": collective,
     }
 
 
@@ -707,6 +733,7 @@ def main():
         "gpu_launches": r["launches"],
         "clocks": r["clocks"],
         "memory": r["memory"],
+        "collective": r["collective"],
     }
     print(json.dumps(line), flush=True)
 

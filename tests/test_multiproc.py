@@ -1,7 +1,8 @@
 """The N>1 path on CPU: two gloo ranks each take their shard of the global
 batch (bench.shard_tokens), score it independently (here with the oracle, the
-device path being absent on CPU) and the gathered shards equal the unsharded
-run; the job time is the max over ranks."""
+device path being absent on CPU), and the shards gathered by the bench's
+end-of-run collective (bench.gather_rows) equal the unsharded run; the job
+time is the max over ranks."""
 import os
 import socket
 
@@ -33,11 +34,10 @@ def _worker(rank, world, port, out_dir):
     tok = bench.shard_tokens(w, rank, world)
     om = oracle.Model(synth.model_config(w), seed=synth.WEIGHT_SEED)
     mine = torch.from_numpy(np.stack([om.replay_logprobs(t) for t in tok]))
-    parts = [torch.zeros_like(mine) for _ in range(world)]
-    dist.all_gather(parts, mine)
+    gathered = bench.gather_rows(mine, world)  # the bench's end-of-run collective
     slowest = bench.max_over_ranks(float(rank + 1), world)
     if rank == 0:
-        np.save(os.path.join(out_dir, "gathered.npy"), torch.cat(parts).numpy())
+        np.save(os.path.join(out_dir, "gathered.npy"), gathered.numpy())
         np.save(os.path.join(out_dir, "slowest.npy"), np.array([slowest]))
     dist.barrier()
     dist.destroy_process_group()
