@@ -16,7 +16,7 @@ reached here stay well inside it.
 Other workloads (--workload): `replay` (the reference width at L = 24,
 B = 256 x 1024 tokens, one rlt_replay_logprobs call per step), `layerwise`,
 `small`, `refdepth-b64` (one whole prefill + generation per step) and
-`bptt-small` (full-BPTT backward).
+`bptt-small` and `bptt-replay` (full-BPTT backward).
 
 Multi-GPU (torchrun): sequences shard across ranks with no data-path
 collective (weak scaling, B sequences per rank); timing is the max over ranks.
@@ -51,6 +51,8 @@ BENCH_WORKLOADS = {
     "refdepth-b64": ("refdepth", {"batch": 64}, "generate"),
     # full-BPTT forward + backward (rlt_replay_backward) of the small model
     "bptt-small": ("small", {"prompt": 256, "gen": 0}, "backward"),
+    # the same at the reference width (d=2048, 24+24 layers), 16 sequences
+    "bptt-replay": ("replay", {"batch": 16, "prompt": 256, "gen": 0}, "backward"),
 }
 DEFAULT_WORKLOAD = "refdepth"
 BPTT_METRIC = "RLT full-BPTT tokens/s (replay forward + backward through the whole history) on 1 B200"
