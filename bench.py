@@ -19,7 +19,9 @@ B = 256 x 1024 tokens, one rlt_replay_logprobs call per step), `layerwise`,
 `bptt-small` and `bptt-replay` (full-BPTT backward).
 
 Multi-GPU (torchrun): sequences shard across ranks with no data-path
-collective (weak scaling, B sequences per rank); timing is the max over ranks.
+collective during the timed steps (weak scaling, B sequences per rank);
+timing is the max over ranks, and the shards' results are all-gathered once
+at the end of the run.
 
   python bench.py [--gpus N] [--steps K] [--warmup W] [--workload NAME] [--impl reference]
 """
