@@ -383,6 +383,16 @@ struct CudaBackend {
   bf16* sa = nullptr; size_t sa_n = 0;
   bf16* sb = nullptr; size_t sb_n = 0;
   float* ws = nullptr; size_t ws_n = 0;
+  // Operations issued so far, and which fp32 rows the bf16 activation copy
+  // in `sb` holds (the operand of the contraction issued as operation `at`):
+  // a contraction that directly follows one of the same rows reuses it.
+  int64_t ops = 0;
+  struct XCopy {
+    const float* x;
+    int64_t ld, rows;
+    int cols;
+    int64_t at;
+  } xc{nullptr, 0, 0, 0, -2};
   CudaBackend(cudaStream_t s, bool use_tc) : st(s), tc(use_tc) {}
   ~CudaBackend() {
     cudaStreamSynchronize(st);
@@ -402,16 +412,23 @@ struct CudaBackend {
     return static_cast<T*>(p);
   }
   template <class T> void zero(T* p, size_t n) {
+    ++ops;
     if (err == cudaSuccess && n) err = cudaMemsetAsync(p, 0, n * sizeof(T), st);
   }
   template <class T> void copy(T* dst, const T* src, size_t n) {
+    ++ops;
     if (err == cudaSuccess && n) err = cudaMemcpyAsync(dst, src, n * sizeof(T), cudaMemcpyDeviceToDevice, st);
   }
   template <class T> void upload(T* dst, const T* src, size_t n) {
+    ++ops;
     if (err == cudaSuccess && n) err = cudaMemcpyAsync(dst, src, n * sizeof(T), cudaMemcpyHostToDevice, st);
     if (err == cudaSuccess) err = cudaStreamSynchronize(st);  // the host source is the engine's own vector
   }
   template <class K> void launch(const K& k, int64_t n) {
+    ++ops;
+    launch_impl(k, n);
+  }
+  template <class K> void launch_impl(const K& k, int64_t n) {
     if (err != cudaSuccess || n <= 0) return;
     const int64_t blocks = (n + 255) / 256;
     err = launch_pdl(functor_kernel<K>, dim3((unsigned)blocks), dim3(256), 0, st, k, n);
@@ -422,10 +439,12 @@ struct CudaBackend {
 
   // ---- row and attention functors, warp or block per unit
   template <class K> void launch_rows(void (*kern)(K, int64_t), const K& k, int64_t n) {
+    ++ops;
     if (err != cudaSuccess || n <= 0) return;
     err = launch_pdl(kern, dim3((unsigned)((n + 7) / 8)), dim3(256), 0, st, k, n);
   }
   void launch(const Xent<float>& k, int64_t n) {
+    ++ops;
     if (err != cudaSuccess || n <= 0) return;
     err = launch_pdl(xent_kernel, dim3((unsigned)n), dim3(kXentThreads), 0, st, k);
   }
@@ -461,7 +480,7 @@ struct CudaBackend {
     return ws;
   }
   void to_bf16(const float* src, int64_t ld, int64_t rows, int64_t cols, bf16* dst) {
-    launch(ToBf16{src, ld, dst, cols}, rows * cols);
+    launch_impl(ToBf16{src, ld, dst, cols}, rows * cols);
   }
   void to_bf16_t(const float* src, int64_t ld, int R, int C, int Rp, bf16* dst) {
     if (err != cudaSuccess) return;
@@ -512,20 +531,34 @@ struct CudaBackend {
   }
   static int64_t round64(int64_t x) { return (x + 63) / 64 * 64; }
 
+  // true when the rows [a, a + (ra-1)*lda + ca) and [b, b + (rb-1)*ldb + cb) share memory
+  static bool spans_overlap(const float* a, int64_t lda, int64_t ra, int64_t ca, const float* b, int64_t ldb,
+                            int64_t rb, int64_t cb) {
+    const float* a1 = a + (ra - 1) * lda + ca;
+    const float* b1 = b + (rb - 1) * ldb + cb;
+    return a < b1 && b < a1;
+  }
   // Y[r][m] (+)= sum_k X[r][k] W[m][k]
   void launch(const MmNT<float>& k, int64_t n) {
+    const int64_t op = ++ops;
     const int64_t R = n / k.M;
-    if (!tc || k.M % 128 || k.K % 64) return launch<MmNT<float>>(k, n);
+    if (!tc || k.M % 128 || k.K % 64) return launch_impl<MmNT<float>>(k, n);
     const bf16* Wb = weight(k.Wm, k.ldw, k.M, k.K, false);
     bf16* Xb = grow(&sb, &sb_n, (size_t)R * k.K);
     if (!Wb || !Xb) return;
-    to_bf16(k.X, k.ldx, R, k.K, Xb);
+    // the operation just before was a contraction of the same rows, whose
+    // bf16 copy is still in sb (the q/k/v and W1/W3 projections of one input)
+    const bool reuse = xc.at == op - 1 && xc.x == k.X && xc.ld == k.ldx && xc.rows == R && xc.cols == k.K;
+    if (!reuse) to_bf16(k.X, k.ldx, R, k.K, Xb);
     gemm(Wb, k.M, Xb, (int)R, k.K, k.Y, k.ldy, k.acc != 0);
+    const bool wrote_source = spans_overlap(k.Y, k.ldy, R, k.M, k.X, k.ldx, R, k.K);
+    xc = XCopy{k.X, k.ldx, R, k.K, wrote_source ? -2 : op};
   }
   // Y[r][c] (+)= sum_m D[r][m] W[m][c]   (c < K)
   void launch(const MmNN<float>& k, int64_t n) {
+    ++ops;
     const int64_t R = n / k.K;
-    if (!tc || k.K % 128 || k.M % 64) return launch<MmNN<float>>(k, n);
+    if (!tc || k.K % 128 || k.M % 64) return launch_impl<MmNN<float>>(k, n);
     const bf16* Wt = weight(k.Wm, k.ldw, k.M, k.K, true);  // [K][M]
     bf16* Db = grow(&sb, &sb_n, (size_t)R * k.M);
     if (!Wt || !Db) return;
@@ -534,8 +567,9 @@ struct CudaBackend {
   }
   // G[m][c] += sum_r D[r][m] X[r][c]   (m < M = n / K, c < K), reduction padded to 64
   void launch(const MmTN<float>& k, int64_t n) {
+    ++ops;
     const int64_t M = n / k.K;
-    if (!tc || k.K % 128) return launch<MmTN<float>>(k, n);
+    if (!tc || k.K % 128) return launch_impl<MmTN<float>>(k, n);
     const int Rp = (int)round64(k.R);
     bf16* Xt = grow(&sa, &sa_n, (size_t)k.K * Rp);
     bf16* Dt = grow(&sb, &sb_n, (size_t)M * Rp);
