@@ -501,12 +501,7 @@ def run_gpu(args, w: dict, kind: str, peaks: dict, rank: int, world: int) -> dic
     # profile the same schedule they time.
     key_scale, share_note = 1.0, "profiled and timed positions are the same schedule"
     if kind == "block":
-        t_hi = t_range[1]
-        prof_t = [t for t in range(t_hi + 1, t_hi + w["block"] * n_prof + 1) if t % PROFILE_STRIDE == 0]
-        timed_mean = (t_range[0] + t_range[1]) / 2
-        key_scale = timed_mean / (sum(prof_t) / len(prof_t))
-        share_note = (f"profiled launches at t={prof_t[0]}..{prof_t[-1]} (every {PROFILE_STRIDE}th), scaled by "
-                      f"{key_scale:.4f} = mean attended keys at the timed t={t_range[0]}..{t_range[1]} / at the profiled t")
+        key_scale, share_note = block_share_scale(t_range, w["block"], n_prof)
 
     def gbs(nbytes, ms_sampled, n_sampled):
         return (nbytes / n_sampled) / ((ms_sampled / n_sampled) / 1e3) / 1e9 if n_sampled else None
@@ -522,6 +517,19 @@ def run_gpu(args, w: dict, kind: str, peaks: dict, rank: int, world: int) -> dic
         "memory": {"device_used_gib": (total_b - free_b) / 2**30, "device_total_gib": total_b / 2**30},
         "collective": collective,
     }
+
+
+def block_share_scale(t_range: tuple[int, int], blk: int, n_prof: int) -> tuple[float, str]:
+    """Factor from the profiled to the timed positions of the block workload
+    for the prefix-attention share: the profiling pass runs the n_prof blocks
+    after the timed positions t_range, sampling every PROFILE_STRIDE-th
+    position, and a launch at position t reads t keys (C^E_<=t, M_<=t)."""
+    t_hi = t_range[1]
+    prof_t = [t for t in range(t_hi + 1, t_hi + blk * n_prof + 1) if t % PROFILE_STRIDE == 0]
+    scale = ((t_range[0] + t_range[1]) / 2) / (sum(prof_t) / len(prof_t))
+    note = (f"profiled launches at t={prof_t[0]}..{prof_t[-1]} (every {PROFILE_STRIDE}th), scaled by "
+            f"{scale:.4f} = mean attended keys at the timed t={t_range[0]}..{t_range[1]} / at the profiled t")
+    return scale, note
 
 
 def backward_flops(w: dict, B: int, S: int) -> float:

@@ -89,3 +89,14 @@ def test_traffic_ratio_only_for_the_captured_source(tmp_path, monkeypatch):
     (src / "attn_decode.cu").write_bytes(b"// kernel v2\n")
     ratio, note = bench.read_traffic_ratio()
     assert ratio is None and "changed" in note
+
+
+def test_block_share_scale():
+    """The prefix-attention share of the block step is measured on the two
+    blocks after the timed ones and scaled by the ratio of mean attended keys
+    (a launch at position t reads t keys)."""
+    import bench
+    scale, note = bench.block_share_scale((2209, 2848), 32, 2)
+    prof = list(range(2852, 2913, 4))  # every 4th of t = 2849..2912
+    assert abs(scale - 2528.5 / (sum(prof) / len(prof))) < 1e-12
+    assert "t=2852..2912" in note and "t=2209..2848" in note
