@@ -6,11 +6,13 @@
 //
 //   bptt_host names B S d H L W G F V tied merge_kind
 //       prints "index name rows cols" for every stored tensor;
-//   bptt_host run in.bin out.bin
+//   bptt_host run in.bin out.bin [passes]
 //       in:  int32 B S d H L W G F V tied merge_kind seg; float64 alpha eps
 //            rope_base; int32 tok[B*S]; float64 wts[B*(S-1)]; float64 of every
 //            stored tensor in index order;
 //       out: float64 logp[B*(S-1)], then the gradient of every stored tensor.
+//       passes (default 1): run the pass that many times on one engine (the
+//       way the library keeps it between calls); gradients accumulate.
 #include <cstdio>
 #include <cstdlib>
 #include <cstring>
@@ -58,10 +60,12 @@ int main(int argc, char** argv) {
     }
     return 0;
   }
-  if (argc != 4 || strcmp(argv[1], "run")) {
-    fprintf(stderr, "usage: bptt_host names B S d H L W G F V tied merge_kind | run in.bin out.bin\n");
+  if ((argc != 4 && argc != 5) || strcmp(argv[1], "run")) {
+    fprintf(stderr, "usage: bptt_host names B S d H L W G F V tied merge_kind | run in.bin out.bin [passes]\n");
     return 2;
   }
+  const int passes = argc == 5 ? atoi(argv[4]) : 1;
+  if (passes < 1) return 2;
   FILE* f = fopen(argv[2], "rb");
   if (!f) return 3;
   int32_t h[12];
@@ -91,7 +95,8 @@ int main(int argc, char** argv) {
   std::vector<double> logp(wts.size(), 0.0);
   HostBackend bk;
   Engine<HostBackend, double> eng(bk, D, wp.data(), gp.data());
-  if (eng.run(tok.data(), wts.data(), seg, logp.data()) != 0) return 6;
+  for (int p = 0; p < passes; ++p)
+    if (eng.run(tok.data(), wts.data(), seg, logp.data()) != 0) return 6;
   FILE* o = fopen(argv[3], "wb");
   if (!o) return 3;
   fwrite(logp.data(), 8, logp.size(), o);

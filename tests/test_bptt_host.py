@@ -55,7 +55,7 @@ def _names(exe, cfg, B, S):
     return [(ln.split()[1], int(ln.split()[2]), int(ln.split()[3])) for ln in out.strip().splitlines()]
 
 
-def _run_host(exe, tmp_path, cfg, P, tok, wts, seg):
+def _run_host(exe, tmp_path, cfg, P, tok, wts, seg, passes=1):
     B, S = tok.shape
     names = _names(exe, cfg, B, S)
     inp, outp = str(tmp_path / "in.bin"), str(tmp_path / "out.bin")
@@ -69,7 +69,7 @@ def _run_host(exe, tmp_path, cfg, P, tok, wts, seg):
             assert a.shape == (r, c), name
             f.write(np.ascontiguousarray(a, dtype=np.float64).tobytes())
     env = dict(os.environ, ASAN_OPTIONS="detect_leaks=1:abort_on_error=0", UBSAN_OPTIONS="halt_on_error=1")
-    r = subprocess.run([exe, "run", inp, outp], capture_output=True, text=True, env=env, timeout=600)
+    r = subprocess.run([exe, "run", inp, outp, str(passes)], capture_output=True, text=True, env=env, timeout=600)
     assert r.returncode == 0, r.stderr[-4000:]
     raw = np.fromfile(outp, dtype=np.float64)
     n_lp = B * (S - 1)
@@ -119,3 +119,26 @@ def test_host_engine_equals_gradient_oracle(oracle_lib, host_exe, tmp_path, kw, 
     for k in want:
         scale = max(1.0, np.max(np.abs(want[k])))
         assert np.max(np.abs(grads[k] - want[k])) < 1e-10 * scale, k
+
+
+def test_host_engine_reused_for_more_passes(oracle_lib, host_exe, tmp_path):
+    """One engine running three passes (as the library keeps it between calls
+    of one size): every pass starts from zeroed buffers, so the gradients are
+    exactly three times one pass's and the log-probs the oracle's."""
+    from oracle import bptt
+    w = synth.workload("tiny", d=32, n_heads=4, ffn=48, vocab=40, prompt=12, window=3)
+    cfg = synth.model_config(w)
+    m = oracle_lib.Model(cfg, seed=42)
+    rng = np.random.default_rng(13)
+    tok = synth.tokens(w, batch=2)
+    B, S = tok.shape
+    wts = rng.uniform(-1.0, 1.0, (B, S - 1))
+    P = {k: v.detach().numpy() for k, v in bptt.parameters(m).items()}
+    logp1, g1 = _run_host(host_exe, tmp_path, cfg, P, tok, wts, 4)
+    logp3, g3 = _run_host(host_exe, tmp_path, cfg, P, tok, wts, 4, passes=3)
+    assert np.array_equal(logp1, logp3)
+    for b in range(B):
+        assert np.max(np.abs(logp3[b] - m.replay_logprobs(tok[b]))) < 1e-11
+    for k in g1:
+        scale = max(1.0, np.max(np.abs(g1[k])))
+        assert np.max(np.abs(g3[k] - 3.0 * g1[k])) < 1e-12 * scale, k
